@@ -1,0 +1,466 @@
+/*
+ * mx_oracle.c -- plain, slow, obviously-correct CPU oracle for microscaling
+ * quantization (MXFP8 E4M3/E5M2, MXFP4, NVFP4) and the block-scaled GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, the package's smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA implementation.
+ *
+ * Every decision is made in fp64 on exactly-representable values, element by
+ * element, in the order the pages describe.  Sources (page title, section):
+ *
+ *   [MXFP4-page]  "Microscaling MXFP4/NVFP4 on Blackwell for reasoning LLMs"
+ *                 (produtoramaxvision.com.br blog).  Sections "Fundamentos
+ *                 matemáticos do formato MXFP4 e E8M0" (E2M1 value set, E8M0
+ *                 formula, dequantization by multiplication, 4.25 bits/element,
+ *                 format table with the E4M3 range [-448, 448]) and the FAQ entry
+ *                 on how E8M0 computes the block's shared exponent (the ceil
+ *                 scale rule).
+ *   [NVFP4-news]  "NVIDIA's FP4 format delivers 1.68x speedup" (zubnet.ai):
+ *                 NVFP4 = E2M1 elements in 16-element blocks; MXFP8 = E4M3/E5M2
+ *                 elements in 32-element blocks (OCP standard).
+ *   [OAS/MBS]     "Unveiling the Potential of Quantization with MXFP4:
+ *                 Strategies for Quantization Error Reduction" (gist.science),
+ *                 section "Metodologia e Propostas" A: the standard MX mapping
+ *                 puts the block maximum into (3, 6] of the E2M1 range.
+ *
+ * Readings taken where the pages are silent (each listed in the design doc):
+ *   R1  rounding of elements is round-to-nearest, ties to the even code, and
+ *       saturating ("satfinite") at the format's largest finite magnitude;
+ *   R2  the sign of a value that rounds to zero is kept (-0 -> 0x8 / 0x80);
+ *   R3  an all-zero MX block gets E8M0 byte 0 (the ceil rule's limit, clamped);
+ *       E8M0 0xFF is NaN and never produced;
+ *   R4  NVFP4 global scale g = amax_t / (6 * 448) rounded UP to fp32
+ *       (amax_t == 0 -> g = 1); g is a decode multiplier like the E8M0 scale;
+ *   R5  NVFP4 block scale s = the smallest positive finite E4M3 value with
+ *       amax_b <= 6 * g * s (the ceil rule carried to an E4M3 scale); an
+ *       all-zero block gets s = 0 (code 0x00) and all-zero codes;
+ *   R6  FP4 packing: byte j of a row = code[2j] | code[2j+1] << 4;
+ *   R7  block-scale byte (r, c) of an [R x C] scale matrix lives at
+ *       ((r/128) * ceil(C/4) + c/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4,
+ *       padding bytes are 0.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <float.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_MXFP8_E4M3 = 0, ORC_MXFP8_E5M2 = 1, ORC_MXFP4 = 2, ORC_NVFP4 = 3 };
+enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_ENONFINITE = 2 };
+
+/* ------------------------------------------------------------------------- */
+/* threads                                                                   */
+/* ------------------------------------------------------------------------- */
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int orc_get_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------- */
+/* bf16                                                                      */
+/* ------------------------------------------------------------------------- */
+
+/* bf16 is the top half of an IEEE binary32. */
+double orc_bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round an fp64 value to bf16 with round-to-nearest-even, in one rounding.
+ * Finite values at or above the midpoint between the largest finite bf16 and
+ * 2^128 go to infinity, as IEEE RNE overflow does. */
+uint16_t orc_double_to_bf16_rne(double v) {
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    const double overflow_mid = ldexp(2.0 - ldexp(1.0, -8), 127);
+    if (a >= overflow_mid) return sign | 0x7F80;
+    int ex;
+    frexp(a, &ex);              /* a = f * 2^ex, f in [0.5, 1) */
+    int e = ex - 1;             /* a in [2^e, 2^(e+1)) */
+    if (e < -126) e = -126;     /* subnormal range has the quantum of 2^-126 * 2^-7 */
+    double quantum = ldexp(1.0, e - 7);
+    double n = a / quantum;     /* exact: power-of-two scaling */
+    double r = rint(n);         /* default rounding mode: nearest, ties to even */
+    double val = r * quantum;   /* exactly a bf16 value */
+    float f = (float)val;       /* exact */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------- */
+/* element and scale formats, decoded bit by bit                             */
+/* ------------------------------------------------------------------------- */
+
+/* E2M1 [MXFP4-page, Fundamentos]: bit 3 sign, bits 2-1 exponent with bias 1,
+ * bit 0 mantissa.  Exponent field 0 is subnormal: 0 or 0.5. */
+double orc_e2m1_decode(uint8_t code) {
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* E4M3 (OCP "fn" variant named by the MXFP8 definition): bias 7, no infinities,
+ * S.1111.111 is NaN, largest finite 448 = 1.75 * 2^8 [MXFP4-page table, FP8 (E4M3)
+ * range [-448, 448]]. */
+double orc_e4m3_decode(uint8_t code) {
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* E5M2: bias 15, IEEE-style infinities and NaNs, largest finite 57344. */
+double orc_e5m2_decode(uint8_t code) {
+    int s = (code >> 7) & 1, e = (code >> 2) & 31, m = code & 3;
+    double mag;
+    if (e == 31) {
+        if (m != 0) return NAN;
+        mag = INFINITY;
+    } else if (e == 0) {
+        mag = ldexp((double)m, -16);
+    } else {
+        mag = ldexp(1.0 + m / 4.0, e - 15);
+    }
+    return s ? -mag : mag;
+}
+
+/* E8M0 [MXFP4-page, Fundamentos]: Escala = 2^(E - 127); 0xFF is NaN. */
+double orc_e8m0_decode(uint8_t code) {
+    if (code == 0xFF) return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* Sorted tables of the non-negative finite values of each element format,
+ * indexed by code.  Built from the decoders above. */
+static double g_e2m1_pos[8];
+static double g_e4m3_pos[127];   /* codes 0x00 .. 0x7E */
+static double g_e5m2_pos[124];   /* codes 0x00 .. 0x7B */
+static int g_tables_ready = 0;
+
+static void build_tables(void) {
+    if (g_tables_ready) return;
+    for (int c = 0; c < 8; ++c) g_e2m1_pos[c] = orc_e2m1_decode((uint8_t)c);
+    for (int c = 0; c < 127; ++c) g_e4m3_pos[c] = orc_e4m3_decode((uint8_t)c);
+    for (int c = 0; c < 124; ++c) g_e5m2_pos[c] = orc_e5m2_decode((uint8_t)c);
+    g_tables_ready = 1;
+}
+
+/* Round |v| onto a sorted table with round-to-nearest, ties to the even code
+ * (consecutive codes differ in their mantissa LSB, so "even code" is "even
+ * mantissa"), saturating at the last entry [reading R1]. */
+static int rne_index(const double *tab, int n, double a) {
+    if (a >= tab[n - 1]) return n - 1;
+    int lo = 0, hi = n - 1;           /* invariant: tab[lo] <= a < tab[hi] */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (tab[mid] <= a) lo = mid; else hi = mid;
+    }
+    double midpoint = 0.5 * (tab[lo] + tab[hi]);   /* exact in fp64 */
+    if (a < midpoint) return lo;
+    if (a > midpoint) return hi;
+    return (lo % 2 == 0) ? lo : hi;
+}
+
+/* Encoders: sign kept even when the magnitude rounds to zero [reading R2]. */
+uint8_t orc_e2m1_encode(double v) {
+    build_tables();
+    int c = rne_index(g_e2m1_pos, 8, fabs(v));
+    return (uint8_t)(c | (signbit(v) ? 0x8 : 0));
+}
+
+uint8_t orc_e4m3_encode(double v) {
+    build_tables();
+    if (isnan(v)) return 0x7F;
+    int c = rne_index(g_e4m3_pos, 127, fabs(v));
+    return (uint8_t)(c | (signbit(v) ? 0x80 : 0));
+}
+
+uint8_t orc_e5m2_encode(double v) {
+    build_tables();
+    if (isnan(v)) return 0x7F;
+    int c = rne_index(g_e5m2_pos, 124, fabs(v));
+    return (uint8_t)(c | (signbit(v) ? 0x80 : 0));
+}
+
+/* ------------------------------------------------------------------------- */
+/* format parameters                                                         */
+/* ------------------------------------------------------------------------- */
+static int fmt_block(int fmt) { return fmt == ORC_NVFP4 ? 16 : 32; }
+static int fmt_bits(int fmt) { return (fmt == ORC_MXFP4 || fmt == ORC_NVFP4) ? 4 : 8; }
+static double fmt_maxelem(int fmt) {
+    switch (fmt) {
+    case ORC_MXFP8_E4M3: return 448.0;
+    case ORC_MXFP8_E5M2: return 57344.0;
+    default: return 6.0;
+    }
+}
+static double fmt_decode(int fmt, uint8_t code) {
+    switch (fmt) {
+    case ORC_MXFP8_E4M3: return orc_e4m3_decode(code);
+    case ORC_MXFP8_E5M2: return orc_e5m2_decode(code);
+    default: return orc_e2m1_decode(code & 0xF);
+    }
+}
+static uint8_t fmt_encode(int fmt, double v) {
+    switch (fmt) {
+    case ORC_MXFP8_E4M3: return orc_e4m3_encode(v);
+    case ORC_MXFP8_E5M2: return orc_e5m2_encode(v);
+    default: return orc_e2m1_encode(v);
+    }
+}
+
+int orc_block_size(int fmt) { return fmt_block(fmt); }
+double orc_max_element(int fmt) { return fmt_maxelem(fmt); }
+
+/* ------------------------------------------------------------------------- */
+/* storage: packed codes and the 128x4-tiled block-scale layout              */
+/* ------------------------------------------------------------------------- */
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+size_t orc_codes_bytes(int fmt, int64_t rows, int64_t cols) {
+    return (size_t)(rows * cols * fmt_bits(fmt) / 8);
+}
+
+size_t orc_scales_bytes(int fmt, int64_t rows, int64_t cols) {
+    int64_t sc = cols / fmt_block(fmt);
+    return (size_t)(ceil_div(rows, 128) * 128 * ceil_div(sc, 4) * 4);
+}
+
+/* [reading R7] position of scale (r, c) in a scale matrix with sf_cols columns */
+size_t orc_sf_offset(int64_t r, int64_t c, int64_t sf_cols) {
+    int64_t tiles_per_row = ceil_div(sf_cols, 4);
+    int64_t tile = (r / 128) * tiles_per_row + c / 4;
+    return (size_t)(tile * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4));
+}
+
+/* ------------------------------------------------------------------------- */
+/* scale rules                                                               */
+/* ------------------------------------------------------------------------- */
+
+/* MX block exponent [MXFP4-page, FAQ on E8M0]:
+ *   E = ceil(log2(max_val / max_elem)) + 127,
+ * i.e. the smallest integer e with max_val <= max_elem * 2^e, found exactly by
+ * comparing against ldexp (never a floating log2).  Clamped to [0, 254]
+ * [reading R3]; max_val == 0 gives 0. */
+int orc_mx_scale_byte(double amax, double maxelem) {
+    if (!(amax > 0.0)) return 0;
+    int e = ilogb(amax) - ilogb(maxelem);
+    while (amax > ldexp(maxelem, e)) ++e;
+    while (amax <= ldexp(maxelem, e - 1)) --e;
+    int E = e + 127;
+    if (E < 0) E = 0;
+    if (E > 254) E = 254;
+    return E;
+}
+
+/* [reading R4] g = RU_fp32(amax_t / 2688); the real quotient is bracketed by
+ * exact fp64 products f * 2688 (f has 24 significant bits, 2688 = 21 * 2^7). */
+float orc_nvfp4_global_scale(double amax_t) {
+    if (!(amax_t > 0.0)) return 1.0f;
+    float f = (float)(amax_t / 2688.0);
+    while ((double)f * 2688.0 < amax_t) f = nextafterf(f, INFINITY);
+    for (;;) {
+        float p = nextafterf(f, 0.0f);
+        if (p > 0.0f && (double)p * 2688.0 >= amax_t) f = p; else break;
+    }
+    return f;
+}
+
+/* [reading R5] smallest positive finite E4M3 s with amax_b <= 6 * g * s.
+ * 6 * g * s has at most 24 + 4 + 2 significant bits: exact in fp64. */
+uint8_t orc_nvfp4_block_scale(double amax_b, float g) {
+    build_tables();
+    if (!(amax_b > 0.0)) return 0x00;
+    for (int c = 1; c <= 126; ++c)
+        if (amax_b <= 6.0 * (double)g * g_e4m3_pos[c]) return (uint8_t)c;
+    return 0x7E;
+}
+
+/* ------------------------------------------------------------------------- */
+/* quantize / dequantize                                                     */
+/* ------------------------------------------------------------------------- */
+
+static void put_code(int fmt, uint8_t *codes, int64_t K, int64_t r, int64_t k, uint8_t q) {
+    if (fmt_bits(fmt) == 8) {
+        codes[r * K + k] = q;
+    } else {
+        uint8_t *byte = &codes[r * (K / 2) + k / 2];
+        if (k % 2 == 0) *byte = (uint8_t)((*byte & 0xF0) | (q & 0xF));      /* [reading R6] */
+        else            *byte = (uint8_t)((*byte & 0x0F) | ((q & 0xF) << 4));
+    }
+}
+
+static uint8_t get_code(int fmt, const uint8_t *codes, int64_t K, int64_t r, int64_t k) {
+    if (fmt_bits(fmt) == 8) return codes[r * K + k];
+    uint8_t byte = codes[r * (K / 2) + k / 2];
+    return (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+}
+
+/* Largest |x| over a bf16 tensor (fp64). */
+double orc_amax_bf16(const uint16_t *src, int64_t M, int64_t K, int64_t ld) {
+    double amax = 0.0;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double a = fabs(orc_bf16_to_double(src[r * ld + k]));
+            if (a > amax) amax = a;
+        }
+    return amax;
+}
+
+/* Quantize a row-major bf16 [M x K] matrix (row pitch ld elements).
+ * codes: orc_codes_bytes bytes; scales: orc_scales_bytes bytes (fully written,
+ * padding 0).  NVFP4: if gscale_given, *gscale is used as g, else g is computed
+ * and stored to *gscale.  Non-finite input is outside the contract: returns
+ * ORC_ENONFINITE. */
+int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
+                 uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
+    build_tables();
+    int bs = fmt_block(fmt);
+    if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            if (!isfinite(orc_bf16_to_double(src[r * ld + k]))) return ORC_ENONFINITE;
+    int64_t sf_cols = K / bs;
+    memset(scales, 0, orc_scales_bytes(fmt, M, K));
+    memset(codes, 0, orc_codes_bytes(fmt, M, K));
+    double maxelem = fmt_maxelem(fmt);
+    float g = 1.0f;
+    if (fmt == ORC_NVFP4) {
+        if (gscale_given) g = *gscale;
+        else { g = orc_nvfp4_global_scale(orc_amax_bf16(src, M, K, ld)); *gscale = g; }
+    }
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t j = 0; j < sf_cols; ++j) {
+            double amax = 0.0;
+            for (int i = 0; i < bs; ++i) {
+                double a = fabs(orc_bf16_to_double(src[r * ld + j * bs + i]));
+                if (a > amax) amax = a;
+            }
+            uint8_t sbyte;
+            double denom;            /* the real number each element is divided by */
+            if (fmt == ORC_NVFP4) {
+                sbyte = orc_nvfp4_block_scale(amax, g);
+                denom = (double)g * orc_e4m3_decode(sbyte);   /* exact product */
+            } else {
+                sbyte = (uint8_t)orc_mx_scale_byte(amax, maxelem);
+                denom = orc_e8m0_decode(sbyte);
+            }
+            scales[orc_sf_offset(r, j, sf_cols)] = sbyte;
+            for (int i = 0; i < bs; ++i) {
+                double x = orc_bf16_to_double(src[r * ld + j * bs + i]);
+                uint8_t q;
+                if (denom == 0.0) {
+                    q = fmt_encode(fmt, signbit(x) ? -0.0 : 0.0);  /* all-zero NVFP4 block */
+                } else {
+                    /* MX: division by a power of two is exact.  NVFP4: if x/denom
+                     * is not a midpoint of the E2M1 grid it is at least 2^-31
+                     * (relative) away from every midpoint (x has 8 significant
+                     * bits, denom 28), far above the fp64 rounding error, and an
+                     * exact midpoint is returned exactly; so the fp64 quotient
+                     * rounds exactly as the real one does. */
+                    q = fmt_encode(fmt, x / denom);
+                }
+                put_code(fmt, codes, K, r, j * bs + i, q);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* Dequantize to fp64: x = g * s * q (g = 1 for MX) [MXFP4-page, Fundamentos:
+ * x_real = S_E8M0 * x_E2M1].  The products are exact in fp64. */
+int orc_dequantize_f64(int fmt, const uint8_t *codes, const uint8_t *scales, float gscale,
+                       int64_t M, int64_t K, double *dst) {
+    int bs = fmt_block(fmt);
+    if (fmt < 0 || fmt > 3 || K % bs != 0) return ORC_EINVAL;
+    int64_t sf_cols = K / bs;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t sb = scales[orc_sf_offset(r, k / bs, sf_cols)];
+            double s = (fmt == ORC_NVFP4) ? (double)gscale * orc_e4m3_decode(sb)
+                                          : orc_e8m0_decode(sb);
+            dst[r * K + k] = s * fmt_decode(fmt, get_code(fmt, codes, K, r, k));
+        }
+    }
+    return ORC_OK;
+}
+
+/* Dequantize to bf16 with one RNE rounding of the exact value. */
+int orc_dequantize_bf16(int fmt, const uint8_t *codes, const uint8_t *scales, float gscale,
+                        int64_t M, int64_t K, uint16_t *dst, int64_t ld) {
+    int bs = fmt_block(fmt);
+    if (fmt < 0 || fmt > 3 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    int64_t sf_cols = K / bs;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t sb = scales[orc_sf_offset(r, k / bs, sf_cols)];
+            double s = (fmt == ORC_NVFP4) ? (double)gscale * orc_e4m3_decode(sb)
+                                          : orc_e8m0_decode(sb);
+            dst[r * ld + k] = orc_double_to_bf16_rne(s * fmt_decode(fmt, get_code(fmt, codes, K, r, k)));
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* GEMM on dequantized operands                                              */
+/* ------------------------------------------------------------------------- */
+
+/* C[i][j] = sum_k A[i][k] * B[j][k] in fp64, and Cabs = sum_k |A||B| (for the
+ * tolerance), for the listed rows of A only (rows == NULL: all M rows).
+ * Output row t corresponds to A row rows[t]. */
+int orc_gemm_f64(const double *A, const double *B, const int64_t *rows, int64_t nrows,
+                 int64_t N, int64_t K, double *C, double *Cabs) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t i = rows ? rows[t] : t;
+        const double *a = A + i * K;
+        for (int64_t j = 0; j < N; ++j) {
+            const double *b = B + j * K;
+            double acc = 0.0, accabs = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = a[k] * b[k];
+                acc += p;
+                accabs += fabs(p);
+            }
+            C[t * N + j] = acc;
+            if (Cabs) Cabs[t * N + j] = accabs;
+        }
+    }
+    return ORC_OK;
+}
+
+/* GELU with the exact erf form (the pages give no GELU; PyTorch's default form
+ * is taken): 0.5 * x * (1 + erf(x / sqrt(2))). */
+double orc_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }
+
+void orc_gelu_array(const double *x, double *y, int64_t n) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) y[i] = orc_gelu(x[i]);
+}
