@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark of the microscaling hot path on B200: activation quantize + block-
+scaled GEMM, reported as TFLOP/s with the roofline of the dominant kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload dit_mxfp8|mlp_nvfp4|skinny_nvfp4|quant_sweep]
+                    [--no-extras]
+
+Default workload (the configuration the headline metric is quoted on): the
+DiT-like MXFP8 E4M3 W8A8 Linear, X bf16 [4096 x 3072] (N(0,1), 8 outlier
+channels x30) times W [3072 x 3072] (N(0, 0.02^2), pre-quantized).  One step =
+quantize X to MXFP8 (codes + tensor-core-tiled E8M0 scales) and run the
+block-scaled GEMM to bf16 C.  Inputs are resident in HBM; each step uses the
+next of several input sets whose total size exceeds the 126 MB L2, so every
+step starts cold.  Multi-GPU runs are independent replicas (weak scaling: the
+path has no collective).
+
+--impl reference times the CPU oracle (the plain fp64 C implementation) on a
+bounded row sample of the same workload, per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 2 ** 20
+# Page-quoted spec peaks (Microscaling MXFP4/NVFP4 page, section "Arquitetura
+# Blackwell SM100"), reported beside the measured ones.
+SPEC = {"hbm_gbs": 8000.0, "fp8_tflops": 2250.0, "fp4_tflops": 4500.0}
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    "dit_mxfp8": dict(fmt=0, M=4096, N=3072, K=3072, x="dit", wseed=2, name="dit_mxfp8_w8a8_linear_4096x3072x3072"),
+    "mlp_nvfp4": dict(fmt=3, M=4608, N=12288, K=3072, x="student_t", wseed=4,
+                      name="mlp_nvfp4_w4a4_gemm1_4608x12288x3072"),
+    "skinny_nvfp4": dict(fmt=3, M=16, N=28672, K=8192, x="normal", wseed=7, name="skinny_nvfp4_16x28672x8192"),
+}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def tensor_peak(fmt: int, peaks: dict, sustained: bool):
+    """Dense block-scaled peak for the element type: the measured bf16 GEMM peak
+    times the nominal ratio (fp8 = 2x bf16, fp4 = 4x bf16)."""
+    base = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    return base * (2.0 if fmt in (0, 1) else 4.0)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx_, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx_ = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx_, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ inputs
+def make_inputs(wl: dict):
+    from fp8_quantization_block_b200 import synth
+    if wl["x"] == "dit":
+        X = synth.dit_activations(1, wl["M"], wl["K"])
+    elif wl["x"] == "student_t":
+        X = synth.student_t(3, wl["M"], wl["K"])
+    else:
+        X = synth.to_bf16_bits(np.random.default_rng(200 + wl["M"]).standard_normal((wl["M"], wl["K"])))
+    W = synth.gaussian_weights(wl["wseed"], wl["N"], wl["K"])
+    return X, W
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, wl, rank, world, device):
+    import torch
+    from fp8_quantization_block_b200 import mx, synth
+
+    fmt, M, N, K = wl["fmt"], wl["M"], wl["N"], wl["K"]
+    X_bits, W_bits = make_inputs(wl)
+    X0 = synth.bits_to_tensor(X_bits).to(device)
+    W0 = synth.bits_to_tensor(W_bits).to(device)
+    per_set = M * K * 2 + mx.mx_codes_bytes(fmt, N, K) + mx.mx_scales_bytes(fmt, N, K) + M * N * 2 + \
+        mx.mx_codes_bytes(fmt, M, K) + mx.mx_scales_bytes(fmt, M, K)
+    n_sets = max(2, int(np.ceil(3 * L2_BYTES / per_set)))
+    sets = []
+    for i in range(n_sets):
+        X = X0.clone()
+        Wq = mx.quantize(W0, fmt)               # weights pre-quantized (outside the step)
+        Xq = mx.empty(fmt, M, K)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        sets.append((X, Wq, Xq, C))
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        X, Wq, Xq, C = sets[i % n_sets]
+        if ev is not None:
+            ev[0].record(stream)
+        mx.quantize(X, fmt, out=Xq)
+        if ev is not None:
+            ev[1].record(stream)
+        mx.gemm(Xq, Wq, out=C)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    clocks = clk.summary()
+    mx.check_device_error()
+    ms = t0.elapsed_time(t1)
+    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    g_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end-to-end through the C ABI with host buffers: H2D of X, quantize, GEMM, D2H of C
+    X_host = synth.bits_to_tensor(X_bits).pin_memory()
+    C_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd, Wq, Xq, Cd = sets[0]
+
+    def e2e_step():
+        Xd.copy_(X_host, non_blocking=True)
+        mx.quantize(Xd, fmt, out=Xq)
+        mx.gemm(Xq, Wq, out=Cd)
+        C_host.copy_(Cd, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    del sets
+    torch.cuda.empty_cache()
+    return dict(ms=ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, clocks=clocks, n_sets=n_sets, per_set=per_set,
+                h2d=M * K * 2, d2h=M * N * 2)
+
+
+def quant_bytes_per_elem(fmt):
+    return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625}[fmt]
+
+
+def extras_gpu(device):
+    """Short measurements of the other hot-path rows (quantize sweep, NVFP4
+    MLP GEMM, skinny weight-stream GEMM), each on rotating buffers > L2."""
+    import torch
+    from fp8_quantization_block_b200 import mx
+
+    peaks, _ = measured_peaks()
+    out = {}
+
+    def timed(fn, n, reps=20, warm=3):
+        for i in range(warm):
+            fn(i)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for i in range(reps):
+            fn(warm + i)
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / reps
+
+    g = torch.Generator(device=device).manual_seed(100)
+    # quantize sweep (K = 4096): a few points of the curve
+    sweep = {}
+    for M in (4096, 65536, 262144):
+        K = 4096
+        n = max(2, int(np.ceil(2 * L2_BYTES / (M * K * 2))))
+        xs = [torch.randn((M, K), generator=g, device=device).to(torch.bfloat16) for _ in range(min(n, 8))]
+        for fmt in (0, 2, 3):
+            qs = [mx.empty(fmt, M, K) for _ in xs]
+            gs = torch.ones(1, device=device)
+            ms = timed(lambda i: mx.quantize(xs[i % len(xs)], fmt, out=qs[i % len(xs)],
+                                             gscale=gs if fmt == 3 else None), len(xs))
+            gbs = M * K * quant_bytes_per_elem(fmt) / (ms * 1e-3) / 1e9
+            sweep[f"{['mxfp8_e4m3', 'e5m2', 'mxfp4', 'nvfp4'][fmt]}_M{M}"] = {
+                "us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+            if fmt == 3:
+                ms2 = timed(lambda i: mx.quantize(xs[i % len(xs)], fmt, out=qs[i % len(xs)]), len(xs))
+                gbs2 = M * K * quant_bytes_per_elem(fmt) / (ms2 * 1e-3) / 1e9
+                sweep[f"nvfp4_with_amax_prepass_M{M}"] = {"us": round(ms2 * 1e3, 2), "GB/s": round(gbs2, 1),
+                                                          "frac_hbm": round(gbs2 / peaks["hbm_gbs"], 3)}
+            del qs
+        del xs
+    out["quantize_sweep"] = sweep
+    # GEMMs
+    for name, (fmt, M, N, K) in {"mlp_nvfp4_gemm1": (3, 4608, 12288, 3072), "mlp_nvfp4_gemm2": (3, 4608, 3072, 12288),
+                                 "skinny_nvfp4_M16": (3, 16, 28672, 8192), "skinny_mxfp4_M16": (2, 16, 28672, 8192),
+                                 "skinny_nvfp4_M128": (3, 128, 28672, 8192)}.items():
+        a = torch.randn((M, K), generator=g, device=device).to(torch.bfloat16)
+        w = (torch.randn((N, K), generator=g, device=device) * 0.02).to(torch.bfloat16)
+        qa = mx.quantize(a, fmt)
+        wbytes = mx.mx_codes_bytes(fmt, N, K) + mx.mx_scales_bytes(fmt, N, K)
+        nw = max(2, int(np.ceil(2 * L2_BYTES / wbytes)))
+        qws = [mx.quantize(w, fmt) for _ in range(nw)]
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        ms = timed(lambda i: mx.gemm(qa, qws[i % nw], out=C), nw)
+        tf = 2 * M * N * K / (ms * 1e-3) / 1e12
+        bytes_ = wbytes + mx.mx_codes_bytes(fmt, M, K) + mx.mx_scales_bytes(fmt, M, K) + M * N * 2
+        gbs = bytes_ / (ms * 1e-3) / 1e9
+        out[name] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1),
+                     "frac_tensor": round(tf / tensor_peak(fmt, peaks, False), 3),
+                     "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        del a, w, qa, qws, C
+    torch.cuda.empty_cache()
+    mx.check_device_error()
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle arm
+def oracle_sample(wl, X_bits, W_bits, rows: int):
+    """Time the oracle's quantize of `rows` rows of X and its fp64 GEMM of those
+    rows against the whole (pre-quantized) W.  Returns seconds."""
+    import oracle
+    fmt, N, K = wl["fmt"], wl["N"], wl["K"]
+    cw, sw, gw = oracle.quantize(fmt, W_bits)             # weights: pre-quantized, untimed
+    Wd = oracle.dequantize_f64(fmt, cw, sw, gw, N, K)
+    t = time.perf_counter()
+    xs = np.ascontiguousarray(X_bits[:rows])
+    g = oracle.nvfp4_global_scale(oracle.amax_bf16(X_bits)) if fmt == 3 else None
+    cx, sx, gx = oracle.quantize(fmt, xs, gscale=g)
+    Xd = oracle.dequantize_f64(fmt, cx, sx, gx, rows, K)
+    oracle.gemm_f64(Xd, Wd)
+    return time.perf_counter() - t
+
+
+def pick_sample_rows(wl, X_bits, W_bits, target_s: float):
+    rows = 8
+    t = oracle_sample(wl, X_bits, W_bits, rows)
+    rows = int(min(wl["M"], max(8, rows * target_s / max(t, 1e-3))))
+    return rows
+
+
+def cpu_baseline(wl, X_bits, W_bits, target_s=12.0):
+    import oracle
+    rows = pick_sample_rows(wl, X_bits, W_bits, target_s)
+    secs = oracle_sample(wl, X_bits, W_bits, rows)
+    flops = 2.0 * rows * wl["N"] * wl["K"]
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} of {wl['M']} activation rows: quantize + fp64 GEMM vs all {wl['N']} weight rows "
+                      f"({secs:.1f} s), throughput scaled per FLOP"}
+
+
+def run_reference(args, wl):
+    import oracle
+    X_bits, W_bits = make_inputs(wl)
+    target = max(1.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    rows = pick_sample_rows(wl, X_bits, W_bits, target)
+    for _ in range(args.warmup):
+        oracle_sample(wl, X_bits, W_bits, rows)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(wl, X_bits, W_bits, rows)
+    secs = time.perf_counter() - t
+    flops = 2.0 * rows * wl["N"] * wl["K"] * args.steps
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl["name"], "format": FMT_NAMES[wl["fmt"]], "M": wl["M"], "N": wl["N"], "K": wl["K"],
+                   "sample_rows": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(), "kind": "oracle",
+                         "sample": f"{rows} activation rows per step (quantize + fp64 GEMM), scaled per FLOP"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
+FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dit_mxfp8", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        return
+
+    import torch
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    from fp8_quantization_block_b200 import build as mxbuild
+    if rank == 0:
+        mxbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+
+    r = run_gpu(args, wl, rank, world, device)
+    peaks, peak_src = measured_peaks()
+    fmt, M, N, K = wl["fmt"], wl["M"], wl["N"], wl["K"]
+    flops = 2.0 * M * N * K
+    ms_step = r["ms"] / args.steps
+    value = world * flops * args.steps / (r["ms"] * 1e-3) / 1e12
+    g_avg = sum(r["g_ms"]) / len(r["g_ms"])
+    q_avg = sum(r["q_ms"]) / len(r["q_ms"])
+    g_tf = flops / (g_avg * 1e-3) / 1e12
+    tpeak = tensor_peak(fmt, peaks, sustained=False)
+    q_bytes = M * K * quant_bytes_per_elem(fmt)
+    q_gbs = q_bytes / (q_avg * 1e-3) / 1e9
+    e2e_value = world * flops * args.steps / (r["e2e_ms"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": FMT_NAMES[fmt], "data": "synthetic",
+        "config": {"workload": wl["name"], "format": FMT_NAMES[fmt], "M": M, "N": N, "K": K,
+                   "step": "mx_quantize(X) + mx_gemm(Xq, Wq pre-quantized)",
+                   "l2": f"inputs larger than L2: {r['n_sets']} rotating input sets x {r['per_set'] / 2**20:.1f} MB",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel<{FMT_NAMES[fmt]}>", "achieved": round(g_tf, 1),
+                     "peak": round(tpeak, 1), "unit": "TFLOP/s", "frac": round(g_tf / tpeak, 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16 x {2 if fmt < 2 else 4} (nominal dtype ratio)",
+                     "frac_of_page_spec": round(g_tf / SPEC["fp8_tflops" if fmt < 2 else "fp4_tflops"], 4),
+                     "kernel_us": round(g_avg * 1e3, 2)},
+        "quantize": {"kernel": f"quantize_kernel<{FMT_NAMES[fmt]}>", "us": round(q_avg * 1e3, 2),
+                     "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
+                     "bytes_per_elem": quant_bytes_per_elem(fmt)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_quantize -> mx_gemm -> D2H C"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_extras:
+        line["extras"] = extras_gpu(device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        X_bits, W_bits = make_inputs(wl)
+        line["cpu_baseline"] = cpu_baseline(wl, X_bits, W_bits)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

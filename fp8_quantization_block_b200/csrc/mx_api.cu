@@ -1,0 +1,313 @@
+// mx_api.cu -- the C ABI of libmx.so (declared in include/mx.h): host-side
+// argument checks, TMA descriptor encoding and kernel launches.  The kernels
+// themselves live in quantize.cuh and gemm_sm100.cuh; this file is the single
+// translation unit of the library.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "mx.h"
+#include "mx_common.cuh"
+#include "quantize.cuh"
+#include "gemm_sm100.cuh"
+
+namespace {
+
+using namespace mx;
+
+std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
+std::atomic<int> g_skip_producer{0};
+
+bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 3; }
+int fmt_block(int fmt) { return fmt == MX_NVFP4 ? 16 : 32; }
+int fmt_bits(int fmt) { return (fmt == MX_MXFP4 || fmt == MX_NVFP4) ? 4 : 8; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mx_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
+
+mx_status last_launch() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        fprintf(stderr, "libmx: launch failed: %s\n", cudaGetErrorString(e));
+        return MX_ERR_CUDA;
+    }
+    return MX_OK;
+}
+
+// --- cuTensorMapEncodeTiled through the runtime's driver entry point ---------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2D uint8 tensor [rows x row_bytes] (row pitch = row_bytes), box 128 bytes x box_rows, 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap *m, const void *base, int64_t rows, int64_t row_bytes, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// --- quantize ------------------------------------------------------------
+template <int FMT>
+void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
+                     const float *g_in, float *g_out, cudaStream_t st) {
+    const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    dim3 grid((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows));
+    quantize_kernel<FMT><<<grid, kQThreads, 0, st>>>(src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
+                                                      sf_tiles_k, g_in, g_out);
+}
+
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+// amax(|src|) -> slot (float bits), then g = RU(amax / 2688) in place.
+mx_status nvfp4_gscale_prepass(const uint16_t *src, int64_t M, int64_t K, int64_t ld, float *slot, cudaStream_t st) {
+    if (cudaMemsetAsync(slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
+    const int64_t vecs = M * (K / 8);
+    int64_t blocks = cdiv(vecs, 256 * 8);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    amax_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, M, K, ld, reinterpret_cast<unsigned int *>(slot));
+    gscale_from_amax_kernel<<<1, 1, 0, st>>>(slot);
+    return last_launch();
+}
+
+mx_status check_tensor(const mx_tensor *t, bool need_codes) {
+    if (!t || !valid_fmt(t->fmt) || t->rows < 0 || t->cols < 0) return MX_ERR_INVALID_ARG;
+    if (t->cols % fmt_block(t->fmt) != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (t->rows > 0 && t->cols > 0) {
+        if (need_codes && (!t->codes || !t->scales)) return MX_ERR_INVALID_ARG;
+        if (!aligned16(t->codes) || !aligned16(t->scales)) return MX_ERR_MISALIGNED;
+        if (t->fmt == MX_NVFP4 && !t->gscale) return MX_ERR_INVALID_ARG;
+    }
+    return MX_OK;
+}
+
+// --- GEMM ----------------------------------------------------------------
+template <int FMT, int BN, int STAGES>
+mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
+                        const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
+    using L = GemmSmem<FMT, BN, STAGES>;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    const int64_t M = A->rows, N = B->rows, K = A->cols;
+    const int64_t kbytes = K * fmt_bits(FMT) / 8;
+    CUtensorMap ta, tb;
+    if (!make_tmap_u8(&ta, a_codes, M, kbytes, kBM)) return MX_ERR_CUDA;
+    if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN)) return MX_ERR_CUDA;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_kernel<FMT, BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        L::kAlloc);
+    });
+    if (attr_err != cudaSuccess) return MX_ERR_CUDA;
+    GemmParams p;
+    p.sfa = a_scales;
+    p.sfb = B->scales;
+    p.sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    p.C = C;
+    p.ldc = ldc;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.num_kt = (int)cdiv(kbytes, kStageKBytes);
+    p.ga = ga;
+    p.gb = B->gscale;
+    p.amax_out = amax_out;
+    p.epilogue = epilogue;
+    p.skip_producer = g_skip_producer.load();
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, kBM));
+    gemm_kernel<FMT, BN, STAGES><<<grid, kGemmThreads, L::kAlloc, st>>>(ta, tb, p);
+    return last_launch();
+}
+
+template <int FMT>
+mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
+                          const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
+    if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+}
+
+mx_status launch_gemm(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
+                      const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
+    switch (A->fmt) {
+    case MX_MXFP8_E4M3: return launch_gemm_fmt<0>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    case MX_MXFP8_E5M2: return launch_gemm_fmt<1>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    case MX_MXFP4: return launch_gemm_fmt<2>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    default: return launch_gemm_fmt<3>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    }
+}
+
+// Byte budget of the fused call's workspace header (X's global-scale slot).
+constexpr size_t kFusedWsHeader = 256;
+
+}  // namespace
+
+extern "C" {
+
+size_t mx_codes_bytes(int fmt, int64_t rows, int64_t cols) {
+    if (!valid_fmt(fmt) || rows < 0 || cols < 0) return 0;
+    return (size_t)(rows * cols * fmt_bits(fmt) / 8);
+}
+
+size_t mx_scales_bytes(int fmt, int64_t rows, int64_t cols) {
+    if (!valid_fmt(fmt) || rows < 0 || cols < 0) return 0;
+    return (size_t)(cdiv(rows, 128) * 128 * cdiv(cols / fmt_block(fmt), 4) * 4);
+}
+
+int mx_block_size(int fmt) { return valid_fmt(fmt) ? fmt_block(fmt) : 0; }
+
+int mx_version(void) { return 100; }
+
+const char *mx_status_string(mx_status s) {
+    switch (s) {
+    case MX_OK: return "MX_OK";
+    case MX_ERR_INVALID_ARG: return "MX_ERR_INVALID_ARG";
+    case MX_ERR_UNSUPPORTED_SHAPE: return "MX_ERR_UNSUPPORTED_SHAPE";
+    case MX_ERR_MISALIGNED: return "MX_ERR_MISALIGNED";
+    case MX_ERR_CUDA: return "MX_ERR_CUDA";
+    case MX_ERR_TIMEOUT: return "MX_ERR_TIMEOUT";
+    case MX_ERR_DEVICE: return "MX_ERR_DEVICE";
+    }
+    return "MX_ERR_UNKNOWN";
+}
+
+mx_status mx_debug_set(int key, uint64_t value) {
+    switch (key) {
+    case MX_DEBUG_WAIT_LIMIT_NS: g_wait_limit_ns.store(value ? value : 1); return MX_OK;
+    case MX_DEBUG_SKIP_PRODUCER: g_skip_producer.store(value ? 1 : 0); return MX_OK;
+    default: return MX_ERR_INVALID_ARG;
+    }
+}
+
+mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
+                      const float *gscale_in, void *stream) {
+    if (!valid_fmt(fmt) || !dst || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    if (dst->fmt != fmt || dst->rows != M || dst->cols != K) return MX_ERR_INVALID_ARG;
+    if (K % fmt_block(fmt) != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || K == 0) return MX_OK;
+    if (!src_bf16 || !dst->codes || !dst->scales) return MX_ERR_INVALID_ARG;
+    if (fmt == MX_NVFP4 && !dst->gscale) return MX_ERR_INVALID_ARG;
+    if (ld_src < K || (ld_src & 7) != 0) return MX_ERR_MISALIGNED;
+    if (!aligned16(src_bf16) || !aligned16(dst->codes) || !aligned16(dst->scales)) return MX_ERR_MISALIGNED;
+    if (cdiv(M, kQTileRows) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint16_t *src = static_cast<const uint16_t *>(src_bf16);
+    switch (fmt) {
+    case MX_MXFP8_E4M3: launch_quantize<0>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP8_E5M2: launch_quantize<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP4: launch_quantize<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    default: {
+        if (gscale_in == nullptr) {
+            mx_status s = nvfp4_gscale_prepass(src, M, K, ld_src, dst->gscale, st);
+            if (s != MX_OK) return s;
+            launch_quantize<3>(src, M, K, ld_src, dst, dst->gscale, nullptr, st);
+        } else {
+            launch_quantize<3>(src, M, K, ld_src, dst, gscale_in, gscale_in == dst->gscale ? nullptr : dst->gscale,
+                               st);
+        }
+    }
+    }
+    return last_launch();
+}
+
+mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, void *stream) {
+    mx_status s = check_tensor(src, true);
+    if (s != MX_OK) return s;
+    if (src->rows == 0 || src->cols == 0) return MX_OK;
+    if (!dst_bf16) return MX_ERR_INVALID_ARG;
+    if (ld_dst < src->cols || (ld_dst & 7) != 0 || !aligned16(dst_bf16)) return MX_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n = src->rows * (src->cols / 8);
+    const unsigned blocks = (unsigned)cdiv(n, 256);
+    const uint8_t *c = static_cast<const uint8_t *>(src->codes);
+    uint16_t *d = static_cast<uint16_t *>(dst_bf16);
+    switch (src->fmt) {
+    case MX_MXFP8_E4M3: dequantize_kernel<0><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP8_E5M2: dequantize_kernel<1><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP4: dequantize_kernel<2><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
+    default: dequantize_kernel<3><<<blocks, 256, 0, st>>>(c, src->scales, src->gscale, src->rows, src->cols, d, ld_dst);
+    }
+    return last_launch();
+}
+
+mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t ldc, void *stream) {
+    mx_status s = check_tensor(A, true);
+    if (s != MX_OK) return s;
+    s = check_tensor(B, true);
+    if (s != MX_OK) return s;
+    if (A->fmt != B->fmt || A->cols != B->cols) return MX_ERR_INVALID_ARG;
+    const int64_t M = A->rows, N = B->rows, K = A->cols;
+    if (M == 0 || N == 0) return MX_OK;
+    if (!C_bf16) return MX_ERR_INVALID_ARG;
+    if (ldc < N) return MX_ERR_INVALID_ARG;
+    if (!aligned16(C_bf16)) return MX_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) return cuda_status(cudaMemset2DAsync(C_bf16, ldc * 2, 0, N * 2, M, st));
+    if (K % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || cdiv(M, kBM) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
+    return launch_gemm(A, B, A->codes, A->scales, A->gscale, static_cast<uint16_t *>(C_bf16), ldc, 0, nullptr, st);
+}
+
+size_t mx_fused_workspace_bytes(void) { return kFusedWsHeader; }
+
+mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx, const mx_tensor *W,
+                            void *C_bf16, int64_t ldc, int epilogue, float *amax_out, const float *x_gscale,
+                            const float *x_amax, void *workspace, size_t workspace_bytes, void *stream) {
+    (void)fmt; (void)X_bf16; (void)M; (void)K; (void)ldx; (void)W; (void)C_bf16; (void)ldc; (void)epilogue;
+    (void)amax_out; (void)x_gscale; (void)x_amax; (void)workspace; (void)workspace_bytes; (void)stream;
+    return MX_ERR_UNSUPPORTED_SHAPE;  // provided by the fused kernel
+}
+
+mx_status mx_check_device_error(void *stream, uint32_t info[4]) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        fprintf(stderr, "libmx: stream error: %s\n", cudaGetErrorString(e));
+        return MX_ERR_CUDA;
+    }
+    uint32_t w[4] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(w, g_error_word, sizeof(w)) != cudaSuccess) return MX_ERR_CUDA;
+    const uint32_t zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(g_error_word, zero, sizeof(zero)) != cudaSuccess) return MX_ERR_CUDA;
+    if (info) memcpy(info, w, sizeof(w));
+    if (w[0] & DEVERR_TIMEOUT) return MX_ERR_TIMEOUT;
+    if (w[0] & DEVERR_BOUNDS) return MX_ERR_DEVICE;
+    return MX_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,170 @@
+/*
+ * mx.h -- C ABI of libmx.so: microscaling quantization (MXFP8 E4M3/E5M2, MXFP4,
+ * NVFP4) and the block-scaled matrix multiply that consumes it, on one NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources for what each call computes (page title, section):
+ *   [MX]    "Microscaling MXFP4/NVFP4 on Blackwell for reasoning LLMs"
+ *           (produtoramaxvision.com.br), sections "Fundamentos matemáticos do
+ *           formato MXFP4 e E8M0" (E2M1 values, E8M0 = 2^(E-127), x = S * x_elem,
+ *           4.25 bits/element, E4M3 range [-448, 448]), "Arquitetura Blackwell
+ *           SM100 e aceleração nativa de NVFP4" (the tensor core applies the
+ *           block scales during FP32 accumulation) and the FAQ entry on how E8M0
+ *           picks the block exponent (E = ceil(log2(max|x| / max_elem)) + 127).
+ *   [NEWS]  "NVIDIA's FP4 format delivers 1.68x speedup" (zubnet.ai): NVFP4 is
+ *           E2M1 in 16-element blocks; MXFP8 is E4M3/E5M2 in 32-element blocks.
+ *   [IMPL]  "Implementação da quantização NVFP4 e MXFP8" (matsubara.tec.br):
+ *           Linear layers with both operands quantized, the quantize kernel as a
+ *           bottleneck for small tensors, CUDA Graphs for batch-1 launches.
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses; the caller allocates and
+ *     owns every buffer.  The library allocates nothing.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Nothing blocks the host except mx_check_device_error.
+ *   - Errors are returned as mx_status; nothing throws across the ABI.
+ *     Argument errors are detected on the host before any launch.  Faults the
+ *     GPU detects (a bounded wait that ran out, a bounds check) are recorded in
+ *     a per-process device error word read by mx_check_device_error.
+ *   - All device pointers must be 16-byte aligned (TMA and vector accesses).
+ *   - Matrices are row-major; the reduction dimension K is contiguous.
+ */
+#ifndef MX_H_
+#define MX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element formats.  Block size 32 with an E8M0 scale for the three MX formats;
+ * block size 16 with an E4M3 scale plus one FP32 per-tensor scale for NVFP4. */
+typedef enum {
+    MX_MXFP8_E4M3 = 0,
+    MX_MXFP8_E5M2 = 1,
+    MX_MXFP4 = 2,
+    MX_NVFP4 = 3
+} mx_format;
+
+typedef enum {
+    MX_OK = 0,
+    MX_ERR_INVALID_ARG = 1,       /* NULL pointer, bad enum, negative size, ... */
+    MX_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of what the call needs    */
+    MX_ERR_MISALIGNED = 3,        /* pointer or leading dimension not 16-B aligned */
+    MX_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, ...)   */
+    MX_ERR_TIMEOUT = 5,           /* a bounded device-side wait ran out         */
+    MX_ERR_DEVICE = 6             /* a device-side bounds/consistency check hit */
+} mx_status;
+
+/* A quantized [rows x cols] matrix (cols = K, the blocked dimension).
+ *   codes : device, mx_codes_bytes(fmt, rows, cols) bytes.  FP8: one code per
+ *           byte, row-major.  FP4: two codes per byte, byte j of a row holds
+ *           code 2j in its low nibble and code 2j+1 in its high nibble.
+ *   scales: device, mx_scales_bytes(fmt, rows, cols) bytes.  One scale byte per
+ *           block (E8M0 for MX, E4M3 for NVFP4), laid out in 512-byte tiles of
+ *           128 rows x 4 scale columns: scale (r, c) of a matrix with C scale
+ *           columns is at ((r/128)*ceil(C/4) + c/4)*512 + (r%32)*16
+ *           + ((r%128)/32)*4 + c%4 -- the layout the sm_100 tensor core reads.
+ *           Padding bytes (rows >= rows, columns >= C) are 0.
+ *   gscale: device, one float (NVFP4 only; NULL otherwise): the per-tensor
+ *           decode multiplier g.  Real value = g * scale * element.           */
+typedef struct {
+    int32_t fmt;
+    int32_t reserved;
+    int64_t rows;
+    int64_t cols;
+    void *codes;
+    uint8_t *scales;
+    float *gscale;
+} mx_tensor;
+
+/* Sizes in bytes of the two buffers of an mx_tensor.  0 for a bad format. */
+size_t mx_codes_bytes(int fmt, int64_t rows, int64_t cols);
+size_t mx_scales_bytes(int fmt, int64_t rows, int64_t cols);
+/* Elements per scale block: 32 (MX formats) or 16 (NVFP4); 0 for a bad format. */
+int mx_block_size(int fmt);
+
+/* Quantize a bf16 matrix src [M x K] (row pitch ld_src elements, ld_src >= K,
+ * ld_src % 8 == 0) into dst ([MX] "Fundamentos" and FAQ; [NEWS]).
+ *   MX formats: per block, E = ceil(log2(max|x| / max_elem)) + 127 clamped to
+ *     [0, 254] (0 for an all-zero block), elements = RNE(x / 2^(E-127))
+ *     saturating to the element format (max_elem = 448 / 57344 / 6).
+ *   NVFP4: g = the FP32 value *gscale_in if gscale_in != NULL, else
+ *     amax(|src|) / 2688 rounded up to FP32 (1.0 for an all-zero tensor),
+ *     computed on the device (an extra read of src).  g is written to
+ *     *dst->gscale.  Block scale s = smallest positive finite E4M3 with
+ *     max|x| <= 6*g*s (0 for an all-zero block); element = RNE of the exact
+ *     quotient x / (g*s) onto E2M1, saturating at 6.
+ * Rounding is to nearest, ties to even; a value that rounds to zero keeps its
+ * sign.  K must be a multiple of the block size (32, or 16 for NVFP4).
+ * dst->rows/cols must equal M/K and dst->fmt must equal fmt.  Non-finite
+ * inputs are outside the contract (their block's codes are unspecified). */
+mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64_t ld_src,
+                      mx_tensor *dst, const float *gscale_in, void *stream);
+
+/* Dequantize: dst[r][k] = RNE_bf16(g * scale * element), computed exactly
+ * before the single rounding ([MX] "Fundamentos": x_real = S * x_elem).
+ * ld_dst >= cols, ld_dst % 8 == 0. */
+mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, void *stream);
+
+/* Block-scaled GEMM on the tensor cores ([MX] "Arquitetura Blackwell SM100"):
+ *   C[i][j] = RNE_bf16( sum_k A_dq[i][k] * B_dq[j][k] ),  A [M x K], B [N x K],
+ * A_dq / B_dq the dequantized operands (the scales are applied inside the
+ * tensor core during FP32 accumulation; NVFP4 also multiplies by gA * gB in
+ * the epilogue).  A->fmt == B->fmt, A->cols == B->cols == K, K % 128 == 0.
+ * C is bf16 [M x N] with row pitch ldc (ldc >= N).  Accuracy contract:
+ *   |C - C_ref| <= 2^-8 |C_ref| + 1e-4 (|A_dq| |B_dq|^T)  elementwise.       */
+mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t ldc, void *stream);
+
+/* Epilogues of the fused call. */
+typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
+
+/* Fused activation-quantize + GEMM: X is bf16 [M x K] (row pitch ldx), W a
+ * pre-quantized [N x K] mx_tensor of format fmt.  X is quantized exactly as
+ * mx_quantize would (same codes and scales, bit for bit) inside the GEMM's
+ * producer, never written to memory, and C = X_dq * W_dq^T as in mx_gemm.
+ *   epilogue : MX_EPI_NONE, or MX_EPI_GELU (exact erf form, applied in FP32
+ *              before the bf16 rounding).
+ *   amax_out : NULL, or a device float that receives max |C| over the bf16
+ *              outputs (it is zeroed by this call first).  Feeding it to the
+ *              next call's x_amax chains two NVFP4 GEMMs without a host sync.
+ *   NVFP4 only, how g of X is found (first non-NULL wins):
+ *     x_gscale : device float holding g itself;
+ *     x_amax   : device float holding amax(|X|); g = RU_fp32(amax / 2688);
+ *     neither  : amax(|X|) is computed by a pre-pass into `workspace`, which
+ *                must then be a device buffer of at least
+ *                mx_fused_workspace_bytes() bytes (unused otherwise).
+ * K % 128 == 0, ldx % 8 == 0. */
+mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx,
+                            const mx_tensor *W, void *C_bf16, int64_t ldc, int epilogue,
+                            float *amax_out, const float *x_gscale, const float *x_amax,
+                            void *workspace, size_t workspace_bytes, void *stream);
+size_t mx_fused_workspace_bytes(void);
+
+/* Synchronize `stream`, then read and clear the device error word.  Returns
+ * MX_OK, MX_ERR_TIMEOUT (a bounded wait inside a kernel gave up: the kernel
+ * returned early and its outputs are unspecified) or MX_ERR_DEVICE.  If info is
+ * non-NULL it receives {flags, first site id, first block id, count}. */
+mx_status mx_check_device_error(void *stream, uint32_t info[4]);
+
+/* Human-readable name of a status. */
+const char *mx_status_string(mx_status s);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int mx_version(void);
+
+/* Test hooks (host-side settings read at each launch):
+ *   MX_DEBUG_WAIT_LIMIT_NS : limit of every device-side wait (default 1e9 ns).
+ *   MX_DEBUG_SKIP_PRODUCER : 1 = GEMM producers skip their loads, so the
+ *                            consumers' bounded waits run out (fault test);
+ *                            never set in normal use.
+ * Returns MX_ERR_INVALID_ARG for an unknown key. */
+typedef enum { MX_DEBUG_WAIT_LIMIT_NS = 1, MX_DEBUG_SKIP_PRODUCER = 2 } mx_debug_key;
+mx_status mx_debug_set(int key, uint64_t value);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MX_H_ */
