@@ -175,7 +175,19 @@ def run_gpu(args, wl, rank, world, device):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+    # estimate the step time, so the clock sampler sees ~1.5 s of the same load
+    # immediately before (and including) the timed region
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_a.record(stream)
+    for i in range(10):
+        step(i)
+    e_b.record(stream)
+    torch.cuda.synchronize()
+    est_ms = max(e_a.elapsed_time(e_b) / 10, 1e-3)
+    n_load = int(min(200000, max(0, args.load_window_s * 1000.0 / est_ms)))
     with ClockSampler(device.index if device.index is not None else 0) as clk:
+        for i in range(n_load):
+            step(i)
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
@@ -199,10 +211,11 @@ def run_gpu(args, wl, rank, world, device):
     C_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     Xd, Wq, Xq, Cd = sets[0]
 
+    ws = mx.fused_workspace(fmt, M, K, device)
+
     def e2e_step():
         Xd.copy_(X_host, non_blocking=True)
-        mx.quantize(Xd, fmt, out=Xq)
-        mx.gemm(Xq, Wq, out=Cd)
+        mx.gemm_fused_act(Xd, Wq, out=Cd, workspace=ws)
         C_host.copy_(Cd, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -223,6 +236,7 @@ def run_gpu(args, wl, rank, world, device):
         e2e_ms = float(t.item())
     del sets
     torch.cuda.empty_cache()
+    clocks["window"] = f"{n_load} untimed steps (~{args.load_window_s} s) then the {args.steps} timed steps"
     return dict(ms=ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, clocks=clocks, n_sets=n_sets, per_set=per_set,
                 h2d=M * K * 2, d2h=M * N * 2)
 
@@ -360,6 +374,43 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_CASES = {
+    # name: (kind, fmt, M, N, K)
+    "gemm_dit_mxfp8": ("gemm", 0, 4096, 3072, 3072),
+    "gemm_mlp1_nvfp4": ("gemm", 3, 4608, 12288, 3072),
+    "gemm_mlp2_nvfp4": ("gemm", 3, 4608, 3072, 12288),
+    "gemm_skinny_nvfp4": ("gemm", 3, 16, 28672, 8192),
+    "quant_mxfp8_32768x4096": ("quant", 0, 32768, 0, 4096),
+    "quant_mxfp4_32768x4096": ("quant", 2, 32768, 0, 4096),
+    "quant_nvfp4_32768x4096": ("quant", 3, 32768, 0, 4096),
+}
+
+
+def run_profile_case(name: str, reps: int = 4):
+    """Run one kernel case a few times (for ncu captures; nothing is timed)."""
+    import torch
+    from fp8_quantization_block_b200 import build as mxbuild
+    from fp8_quantization_block_b200 import mx
+    mxbuild.build()
+    kind, fmt, M, N, K = PROFILE_CASES[name]
+    g = torch.Generator(device="cuda").manual_seed(1)
+    x = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    if kind == "quant":
+        q = mx.empty(fmt, M, K)
+        gs = torch.ones(1, device="cuda")
+        for _ in range(reps):
+            mx.quantize(x, fmt, out=q, gscale=gs if fmt == 3 else None)
+    else:
+        w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        qa, qw = mx.quantize(x, fmt), mx.quantize(w, fmt)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(reps):
+            mx.gemm(qa, qw, out=C)
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    print(f"profile case {name}: {reps} launches done", flush=True)
+
+
 METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
 FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4"}
 
@@ -373,7 +424,14 @@ def main():
     ap.add_argument("--workload", default="dit_mxfp8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--load-window-s", type=float, default=1.5,
+                    help="seconds of untimed steps run under the clock sampler right before the timed steps")
+    ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
+                    help="run one kernel case a few times for an ncu capture, then exit")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args.profile)
+        return
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
@@ -429,7 +487,7 @@ def main():
                      "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
                      "bytes_per_elem": quant_bytes_per_elem(fmt)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
-                "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_quantize -> mx_gemm -> D2H C"},
+                "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_gemm_fused_act -> D2H C"},
         "gpu_launches": 2 * args.steps,
         "clocks": r["clocks"],
     }

@@ -6,16 +6,28 @@
 // NVFP4": the 5th-generation tensor core consumes the block codes directly and
 // applies the block scale during FP32 accumulation).
 //
-// One CTA computes one 128 x BN output tile with four warp roles:
+// Persistent kernel: one CTA per SM walks output tiles of 128 x BN (tile t,
+// t + gridDim.x, ...) with five warp roles:
 //   warp 0     TMA producer: code tiles of A and B (128-byte swizzled, K-major)
-//              plus their 512-byte scale tiles into a STAGES-deep smem ring;
-//   warp 1     TMEM owner and MMA issuer: tcgen05.cp moves each stage's scale
-//              tiles into TMEM, then one thread issues the block-scaled
+//              plus their 512-byte scale tiles into a STAGES-deep smem ring
+//              that runs continuously across tiles;
+//   warps 6-9  scale warps (one per TMEM lane quadrant): copy each stage's
+//              scale tiles from shared memory into TMEM with tcgen05.st, into
+//              one of two TMEM slots, one stage ahead of the MMAs.  (Staging the
+//              scales with tcgen05.cp instead costs tensor-pipe cycles that do
+//              not overlap the MMAs; register stores from other warps do.)
+//   warp 1     TMEM owner and MMA issuer: one lane issues the block-scaled
 //              tcgen05.mma instructions (4 per stage, 32 bytes of K each) into
-//              an FP32 accumulator in TMEM, and tcgen05.commit frees the stage;
+//              an FP32 accumulator in TMEM; tcgen05.commit frees the smem stage
+//              and the scale slot;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (one row per thread),
-//              x gA*gB for NVFP4, optional GELU and |C| max, bf16 RNE, stores.
-// Every mbarrier wait is bounded (mx_common.cuh).
+//              x gA*gB for NVFP4, optional GELU and |C| max, bf16 RNE, staged
+//              in shared memory and written with TMA bulk-tensor stores.
+// The two accumulators alternate between tiles so that the epilogue of one
+// tile overlaps the MMAs of the next.  TMEM has 512 columns: the accumulators
+// sit at [0, BN) and [S, S + BN) and share BN - S columns, which the epilogue
+// drains first and then releases; the two scale slots take the columns from
+// S + BN up.  Every mbarrier wait is bounded (mx_common.cuh).
 #pragma once
 
 #include "mx_common.cuh"
@@ -49,20 +61,25 @@ struct GemmFmt<3> {  // NVFP4: kind::mxf4nvf4, scale_vec 4X (16-element blocks),
 
 constexpr int kBM = 128;
 constexpr int kStageKBytes = 128;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
+constexpr int kSfSlots = 4;
+constexpr int kEpiWarps = 4;
+constexpr int kEpiChunkBytes = 32 * 32 * 2;  // 32 rows x 32 bf16 columns per epilogue warp
 
 struct GemmParams {
     const uint8_t *sfa;
     const uint8_t *sfb;
     int64_t sf_tiles_k;  // 512-byte scale tiles per 128-row band (= ceil(K / block / 4))
-    uint16_t *C;
+    uint16_t *C;         // used by the direct-store epilogue (when TMA stores are not possible)
     int64_t ldc;
     int M, N, K;
     int num_kt;           // stages along K = ceil(K_bytes / 128)
+    int m_blocks, n_blocks;
     const float *ga;      // NVFP4 per-tensor scales (nullptr for MX)
     const float *gb;
     float *amax_out;      // nullable: max |C| (bf16) via atomicMax on float bits
     int epilogue;         // 0 none, 1 GELU
+    int use_tma_store;    // 1: C via TMA bulk-tensor stores (ldc % 8 == 0, C 16-B aligned)
     int skip_producer;    // test hook: never issue loads
     uint64_t wait_limit_ns;
 };
@@ -77,19 +94,24 @@ struct GemmSmem {
     static constexpr int kSfbBytes = F::kChunks * 512 * kBBands;
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + STAGES * kABytes;
-    static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
+    static constexpr int kOffEpi = kOffB + STAGES * kBBytes;
+    static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiChunkBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
     static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
-    static constexpr int kNumBars = 2 * STAGES + 1;
+    // full[S], empty[S], acc_full[2], acc_empty, mma_done, sf_full[2], sf_empty[2]
+    static constexpr int kNumBars = 2 * STAGES + 4 + 2 * kSfSlots;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
-    // TMEM columns: accumulator, then scale tiles of A and B for one stage.
-    static constexpr int kTmemSfa = BN;
-    static constexpr int kTmemSfb = BN + 4 * F::kChunks;
-    static constexpr int kTmemUsed = kTmemSfb + 4 * F::kChunks * kBBands;
-    static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
-                                   : kTmemUsed <= 256 ? 256 : 512;
+    // TMEM: two accumulators at columns 0 and kAccStride (sharing BN - kAccStride
+    // columns), then kSfSlots scale slots of kSfSlotCols columns each.
+    static constexpr int kTmemCols = 512;
+    static constexpr int kSfSlotCols = 4 * F::kChunks * (1 + kBBands);
+    static constexpr int kAccRoom = kTmemCols - BN - kSfSlots * kSfSlotCols;
+    static constexpr int kAccStride = (kAccRoom >= BN ? BN : kAccRoom) / 32 * 32;
+    static constexpr int kTmemSf = kAccStride + BN;
+    static_assert(kAccStride >= 32, "accumulator double buffering needs TMEM room");
+    static_assert(kTmemSf + kSfSlots * kSfSlotCols <= kTmemCols, "TMEM budget");
 };
 
 // Instruction descriptor of the block-scaled MMA (M = 128, K-major A and B).
@@ -108,6 +130,14 @@ MX_DEVICE_INLINE void gemm_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t ides
     else tc_mma_nvf4(d, a, b, idesc, sfa, sfb, acc);
 }
 
+template <int FMT>
+MX_DEVICE_INLINE void gemm_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                  uint32_t acc, uint32_t issue) {
+    if (FMT <= 1) tc_mma_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+    else if (FMT == 2) tc_mma_mxf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+    else tc_mma_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+}
+
 MX_DEVICE_INLINE float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752440f)); }
 
 // Number of valid 32-byte MMA steps and 512-byte scale chunks in stage kt.
@@ -121,32 +151,95 @@ MX_DEVICE_INLINE void stage_extent(int kt, int K, int &n_mma, int &n_chunk) {
     n_chunk = (n_mma + F::kMmaPerChunk - 1) / F::kMmaPerChunk;
 }
 
+
+// Scale warps: move one stage's scale tiles from shared memory into a TMEM
+// slot of this warp's 32 lanes.  Lane r loads row r (16 bytes = 4 columns) of
+// every 512-byte tile first, then writes them with wide tcgen05.st.  Slot
+// layout: A tiles c at columns 4c; B tiles (c, band h) at 4*kChunks + 4*(c*bands + h).
+// smem B tiles are stored band-major: (h * kChunks + c) * 512.
+template <int CHUNKS, int BANDS>
+MX_DEVICE_INLINE void stage_scales_to_tmem(const uint8_t *sfa_stage, const uint8_t *sfb_stage, uint32_t t_slot,
+                                           int lane) {
+    uint32_t a[4 * CHUNKS];
+    uint32_t b[4 * CHUNKS * BANDS];
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(sfa_stage + c * 512 + lane * 16);
+        a[4 * c] = v.x, a[4 * c + 1] = v.y, a[4 * c + 2] = v.z, a[4 * c + 3] = v.w;
+#pragma unroll
+        for (int h = 0; h < BANDS; ++h) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(sfb_stage + (h * CHUNKS + c) * 512 + lane * 16);
+            const int o = 4 * (c * BANDS + h);
+            b[o] = w.x, b[o + 1] = w.y, b[o + 2] = w.z, b[o + 3] = w.w;
+        }
+    }
+    if (CHUNKS == 4) {
+        tmem_st16(t_slot, *reinterpret_cast<const uint32_t(*)[16]>(&a[0]));
+    } else if (CHUNKS == 2) {
+        tmem_st8(t_slot, *reinterpret_cast<const uint32_t(*)[8]>(&a[0]));
+    } else {
+        tmem_st4(t_slot, a[0], a[1], a[2], a[3]);
+    }
+    constexpr int kB = 4 * CHUNKS * BANDS;  // 4, 8, 16 or 32 columns
+    const uint32_t tb = t_slot + 4 * CHUNKS;
+    if (kB == 32) {
+        tmem_st16(tb, *reinterpret_cast<const uint32_t(*)[16]>(&b[0]));
+        tmem_st16(tb + 16, *reinterpret_cast<const uint32_t(*)[16]>(&b[(kB == 32) ? 16 : 0]));
+    } else if (kB == 16) {
+        tmem_st16(tb, *reinterpret_cast<const uint32_t(*)[16]>(&b[0]));
+    } else if (kB == 8) {
+        tmem_st8(tb, *reinterpret_cast<const uint32_t(*)[8]>(&b[0]));
+    } else {
+        tmem_st4(tb, b[0], b[1], b[2], b[3]);
+    }
+    tmem_wait_st();
+}
+
+MX_DEVICE_INLINE void tile_coords(int tile, int m_blocks, int &m0, int &n0, int bn) {
+    m0 = (tile % m_blocks) * kBM;
+    n0 = (tile / m_blocks) * bn;
+}
+
 template <int FMT, int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = GemmSmem<FMT, BN, STAGES>;
+    static_assert(STAGES >= kSfSlots, "scale slots are recycled through the stage barriers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *empty = full + STAGES;
-    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_full = empty + STAGES;  // [2]
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *mma_done = acc_empty + 1;
+    uint64_t *sf_full = mma_done + 1;      // [kSfSlots]
+    uint64_t *sf_empty = sf_full + kSfSlots;  // [kSfSlots]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * BN;
+    const int num_tiles = p.m_blocks * p.n_blocks;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        mbar_init(&acc_full[0], 1);
+        mbar_init(&acc_full[1], 1);
+        mbar_init(acc_empty, kEpiWarps);
+        mbar_init(mma_done, 1);
+        for (int i = 0; i < kSfSlots; ++i) {
+            mbar_init(&sf_full[i], 4);
+            mbar_init(&sf_empty[i], 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.use_tma_store) tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, L::kTmemCols);
@@ -159,83 +252,179 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0 && !p.skip_producer) {
+        // The whole warp walks the loop (all values warp-uniform); lane 0
+        // issues the copies.
+        if (!p.skip_producer) {
             const int n_bands_total = (p.N + 127) / 128;
-            int last_round[STAGES];
-            for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
-            for (int kt = 0; kt < p.num_kt; ++kt) {
-                const int s = kt % STAGES, round = kt / STAGES;
-                if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY,
-                                       abort_flag))
-                    break;
-                int n_mma, n_chunk;
-                stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
+            int last_kg = -1;
+            int kg = 0;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+                int m0, n0;
+                tile_coords(tile, p.m_blocks, m0, n0, BN);
                 const int bands = min(L::kBBands, n_bands_total - n0 / 128);
-                const uint32_t bytes = L::kABytes + L::kBBytes + (uint32_t)n_chunk * 512u * (1u + (uint32_t)bands);
-                mbar_arrive_expect_tx(&full[s], bytes);
-                tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, kt * kStageKBytes, m0, &full[s]);
-                tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, kt * kStageKBytes, n0, &full[s]);
-                const int64_t sf_k = (int64_t)kt * F::kChunks;
-                bulk_load(smem + L::kOffSfa + s * L::kSfaBytes, p.sfa + ((int64_t)(m0 / 128) * p.sf_tiles_k + sf_k) * 512,
-                          (uint32_t)n_chunk * 512u, &full[s]);
-                for (int h = 0; h < bands; ++h)
-                    bulk_load(smem + L::kOffSfb + s * L::kSfbBytes + h * F::kChunks * 512,
-                              p.sfb + ((int64_t)(n0 / 128 + h) * p.sf_tiles_k + sf_k) * 512, (uint32_t)n_chunk * 512u,
-                              &full[s]);
-                last_round[s] = round;
+                const uint8_t *sfa_row = p.sfa + (int64_t)(m0 / 128) * p.sf_tiles_k * 512;
+                const uint8_t *sfb_row = p.sfb + (int64_t)(n0 / 128) * p.sf_tiles_k * 512;
+                for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
+                    const int s = kg % STAGES, round = kg / STAGES;
+                    if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY,
+                                           abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    int n_mma, n_chunk;
+                    stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
+                    const uint32_t sf_bytes = (uint32_t)n_chunk * 512u;
+                    const uint32_t bytes = L::kABytes + L::kBBytes + sf_bytes * (1u + (uint32_t)bands);
+                    const int64_t sf_k = (int64_t)kt * F::kChunks * 512;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, kt * kStageKBytes, m0, &full[s]);
+                        tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, kt * kStageKBytes, n0, &full[s]);
+                        bulk_load(smem + L::kOffSfa + s * L::kSfaBytes, sfa_row + sf_k, sf_bytes, &full[s]);
+                        for (int h = 0; h < bands; ++h)
+                            bulk_load(smem + L::kOffSfb + s * L::kSfbBytes + h * F::kChunks * 512,
+                                      sfb_row + (int64_t)h * p.sf_tiles_k * 512 + sf_k, sf_bytes, &full[s]);
+                    }
+                    __syncwarp();
+                    last_kg = kg;
+                }
             }
-            // Do not leave while copies into this CTA's shared memory are in flight.
-            for (int s = 0; s < STAGES; ++s)
-                if (last_round[s] >= 0)
-                    mbar_wait_bounded(&full[s], last_round[s] & 1, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
+            // Do not leave while copies into this CTA's shared memory are in flight:
+            // wait for the last fill of every stage that was used.
+            for (int k = max(0, last_kg - STAGES + 1); k <= last_kg; ++k)
+                mbar_wait_bounded(&full[k % STAGES], (k / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t t_acc = tmem, t_sfa = tmem + L::kTmemSfa, t_sfb = tmem + L::kTmemSfb;
-            const uint32_t a_base = smem_u32(smem + L::kOffA), b_base = smem_u32(smem + L::kOffB);
-            const uint32_t sfa_base = smem_u32(smem + L::kOffSfa), sfb_base = smem_u32(smem + L::kOffSfb);
-            for (int kt = 0; kt < p.num_kt; ++kt) {
-                const int s = kt % STAGES, round = kt / STAGES;
-                if (!mbar_wait_bounded(&full[s], round & 1, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag)) break;
+        // All 32 lanes walk the loop with warp-uniform operands; the tcgen05
+        // instructions are predicated on lane 0, so the same thread issues every
+        // MMA and the commits that track them, without a divergent branch.
+        const uint32_t a_base = smem_u32(smem + L::kOffA), b_base = smem_u32(smem + L::kOffB);
+        const uint64_t desc_ab = smem_desc(0, 16, 1024, 2);
+        const uint32_t leader = lane == 0 ? 1u : 0u;
+        int kg = 0;
+        bool stop = false;
+        bool ready = false;  // result of the last peek at stage kg's barriers
+        int it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++it) {
+            const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
+            for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
+                const int s = kg % STAGES;
+                const int slot = kg % kSfSlots;
+                // sf_full of a stage implies its code tiles have landed: the scale warps
+                // arrive only after observing the stage's load barrier.
+                if (!ready && !mbar_wait_bounded(&sf_full[slot], (kg / kSfSlots) & 1, p.wait_limit_ns,
+                                                 SITE_GEMM_MMA_SF, abort_flag)) {
+                    stop = true;
+                    break;
+                }
                 tc_fence_after();
+                if (kt == 0 && it > 0) {
+                    // the epilogue has released the columns this accumulator shares
+                    if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY,
+                                           abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                }
                 int n_mma, n_chunk;
                 stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                for (int c = 0; c < n_chunk; ++c) {
-                    tc_cp_sf(t_sfa + 4 * c, smem_desc(sfa_base + s * L::kSfaBytes + c * 512, 0, 128, 0));
-#pragma unroll
-                    for (int h = 0; h < L::kBBands; ++h)
-                        tc_cp_sf(t_sfb + 4 * (c * L::kBBands + h),
-                                 smem_desc(sfb_base + s * L::kSfbBytes + (h * F::kChunks + c) * 512, 0, 128, 0));
-                }
                 const uint32_t a_stage = a_base + s * L::kABytes, b_stage = b_base + s * L::kBBytes;
+                const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
+                const uint32_t t_sfb = t_sfa + 4 * F::kChunks;
                 for (int j = 0; j < n_mma; ++j) {
                     const int chunk = j / F::kMmaPerChunk;
                     const uint32_t sf_id = (uint32_t)((j % F::kMmaPerChunk) * F::kSfPerMma);
-                    const uint64_t ad = smem_desc(a_stage + 32 * j, 16, 1024, 2);
-                    const uint64_t bd = smem_desc(b_stage + 32 * j, 16, 1024, 2);
-                    gemm_mma<FMT>(t_acc, ad, bd, gemm_idesc<FMT, BN>(sf_id), t_sfa + 4 * chunk,
-                                  t_sfb + 4 * L::kBBands * chunk, (kt > 0 || j > 0) ? 1u : 0u);
+                    const uint64_t ad = desc_ab | (uint64_t)(((a_stage + 32 * j) >> 4) & 0x3FFFu);
+                    const uint64_t bd = desc_ab | (uint64_t)(((b_stage + 32 * j) >> 4) & 0x3FFFu);
+                    gemm_mma_if<FMT>(t_acc, ad, bd, gemm_idesc<FMT, BN>(sf_id), t_sfa + 4 * chunk,
+                                     t_sfb + 4 * L::kBBands * chunk, (kt > 0 || j > 0) ? 1u : 0u, leader);
                 }
-                tc_commit(&empty[s]);
+                // frees the smem stage and (for the scale warps) the scale slot
+                tc_commit_if(&empty[s], leader);
+                // peek, without blocking, at the next stage while these MMAs run
+                {
+                    const int k1 = kg + 1;
+                    ready = mbar_test_wait(&sf_full[k1 % kSfSlots], (k1 / kSfSlots) & 1);
+                }
             }
-            tc_commit(acc_full);
+            if (!stop) tc_commit_if(&acc_full[it & 1], leader);
+        }
+        tc_commit_if(mma_done, leader);
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ scale warps
+        // Each warp owns one TMEM lane quadrant.  A 512-byte scale tile is 32
+        // rows of 16 bytes; row r holds the 4 scale columns of tile rows r,
+        // r+32, r+64, r+96 -- exactly TMEM lane r's 4 columns, which the MMA
+        // expects in every quadrant.  So every warp loads the same rows and
+        // stores them into its own 32 lanes.
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int kg = 0;
+        bool stop = false;
+        for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+            for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
+                const int s = kg % STAGES, slot = kg % kSfSlots;
+                if (!mbar_wait_bounded(&full[s], (kg / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_SF_FULL, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                // the slot's previous stage (kg - kSfSlots) has been consumed once its
+                // MMAs completed, which the commit on that stage's empty barrier signals
+                if (kg >= kSfSlots &&
+                    !mbar_wait_bounded(&empty[(kg - kSfSlots) % STAGES], ((kg - kSfSlots) / STAGES) & 1,
+                                       p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                int n_mma, n_chunk;
+                stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
+                (void)n_chunk;  // tiles past the K tail carry stale scales the MMAs never read
+                stage_scales_to_tmem<F::kChunks, L::kBBands>(smem + L::kOffSfa + s * L::kSfaBytes,
+                                                             smem + L::kOffSfb + s * L::kSfbBytes,
+                                                             tmem + lane_base + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols),
+                                                             lane);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_full[slot]);
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
-        const bool ok = mbar_wait_bounded(acc_full, 0, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag);
-        tc_fence_after();
-        if (ok && !*abort_flag) {
+        uint8_t *stage_buf = smem + L::kOffEpi + (warp - 2) * kEpiChunkBytes;
+        uint32_t amax = 0;
+        float scale = 1.0f;
+        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        int it = 0;
+        constexpr int kChunksPerTile = BN / 32;
+        constexpr int kOverlapChunks = (BN - L::kAccStride) / 32;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+            int m0, n0;
+            tile_coords(tile, p.m_blocks, m0, n0, BN);
+            const int b = it & 1;
+            if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
+            tc_fence_after();
             const int row = m0 + 32 * q + lane;
-            float scale = 1.0f;
-            if (FMT == 3) scale = (*p.ga) * (*p.gb);
-            uint32_t amax = 0;
-            const bool vec_ok = ((p.ldc & 7) == 0) && ((reinterpret_cast<uintptr_t>(p.C) & 15) == 0);
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                if (n0 + c0 >= p.N) break;  // warp-uniform
+            const int n_valid = p.N - n0;
+            const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
+            for (int idx = 0; idx < kChunksPerTile; ++idx) {
+                if (idx == kOverlapChunks) {
+                    // the shared columns are in registers: let the next tile's MMAs start
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acc_empty);
+                }
+                // buffer 0 drains its tail (shared with buffer 1) first
+                const int c = (b == 0) ? (idx + (kChunksPerTile - kOverlapChunks)) % kChunksPerTile : idx;
+                const int col = 32 * c;
+                if (col >= n_valid) continue;  // warp-uniform
                 uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, r);
+                tmem_ld32(t_acc + (uint32_t)col, r);
                 tmem_wait_ld();
                 uint32_t packed[16];
 #pragma unroll
@@ -249,29 +438,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     packed[i] = *reinterpret_cast<const uint32_t *>(&h);
                 }
                 if (p.amax_out != nullptr && row < p.M) {
-                    const int valid = min(32, p.N - (n0 + c0));
+                    const int valid = min(32, n_valid - col);
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (i < valid) amax = max(amax, (packed[i >> 1] >> (16 * (i & 1))) & 0x7FFFu);
                 }
-                if (row < p.M) {
-                    uint16_t *dst = p.C + (int64_t)row * p.ldc + n0 + c0;
-                    if (vec_ok && n0 + c0 + 32 <= p.N) {
+                if (m0 + 32 * q >= p.M) continue;  // warp-uniform: no rows of this quadrant exist
+                if (p.use_tma_store) {
+                    if (lane == 0) bulk_wait_group_read<0>();  // staging buffer free again
+                    __syncwarp();
+                    uint4 *dst = reinterpret_cast<uint4 *>(stage_buf + lane * 64);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            reinterpret_cast<uint4 *>(dst)[v] =
-                                make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                    } else {
-                        for (int i = 0; i < 32 && n0 + c0 + i < p.N; ++i)
-                            dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, n0 + col, m0 + 32 * q, stage_buf);
+                        bulk_commit_group();
                     }
+                } else if (row < p.M) {
+                    uint16_t *dst = p.C + (int64_t)row * p.ldc + n0 + col;
+                    for (int i = 0; i < 32 && col + i < n_valid; ++i) dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
                 }
             }
-            if (p.amax_out != nullptr) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                if (lane == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int *>(p.amax_out), amax << 16);
+            if (kOverlapChunks >= kChunksPerTile) {  // (not reached for the tile shapes used)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
             }
+        }
+        if (lane == 0) bulk_wait_group_all();
+        if (p.amax_out != nullptr) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if (lane == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int *>(p.amax_out), amax << 16);
         }
     }
 
@@ -279,8 +480,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        // All MMAs issued by this CTA have completed once acc_full has fired.
-        mbar_wait_bounded(acc_full, 0, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
+        // every MMA this CTA issued has completed once mma_done has fired
+        mbar_wait_bounded(mma_done, 0, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
         tmem_dealloc(tmem, L::kTmemCols);
     }
 }

@@ -14,6 +14,7 @@
 #include "mx_common.cuh"
 #include "quantize.cuh"
 #include "gemm_sm100.cuh"
+#include "gemm_pair_sm100.cuh"
 
 namespace {
 
@@ -21,6 +22,7 @@ using namespace mx;
 
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<int> g_skip_producer{0};
+std::atomic<int> g_pair_enabled{1};
 
 bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 3; }
 int fmt_block(int fmt) { return fmt == MX_NVFP4 ? 16 : 32; }
@@ -74,11 +76,11 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, int64_t rows, int64_t row_by
 // --- quantize ------------------------------------------------------------
 template <int FMT>
 void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
-                     const float *g_in, float *g_out, cudaStream_t st) {
+                     const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     dim3 grid((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows));
     quantize_kernel<FMT><<<grid, kQThreads, 0, st>>>(src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
-                                                      sf_tiles_k, g_in, g_out);
+                                                      sf_tiles_k, g_in, g_out, g_from_amax);
 }
 
 int num_sms() {
@@ -117,6 +119,20 @@ mx_status check_tensor(const mx_tensor *t, bool need_codes) {
 }
 
 // --- GEMM ----------------------------------------------------------------
+// bf16 [rows x cols] output (row pitch ld elements), box 32 x 32, no swizzle.
+bool make_tmap_c(CUtensorMap *m, void *base, int64_t rows, int64_t cols, int64_t ld) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int FMT, int BN, int STAGES>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                         const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
@@ -124,9 +140,12 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K * fmt_bits(FMT) / 8;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     if (!make_tmap_u8(&ta, a_codes, M, kbytes, kBM)) return MX_ERR_CUDA;
     if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN)) return MX_ERR_CUDA;
+    const bool tma_store = (ldc % 8 == 0) && aligned16(C);
+    memset(&tc, 0, sizeof(tc));
+    if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -144,20 +163,87 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.N = (int)N;
     p.K = (int)K;
     p.num_kt = (int)cdiv(kbytes, kStageKBytes);
+    p.m_blocks = (int)cdiv(M, kBM);
+    p.n_blocks = (int)cdiv(N, BN);
     p.ga = ga;
     p.gb = B->gscale;
     p.amax_out = amax_out;
     p.epilogue = epilogue;
+    p.use_tma_store = tma_store ? 1 : 0;
     p.skip_producer = g_skip_producer.load();
     p.wait_limit_ns = g_wait_limit_ns.load();
-    dim3 grid((unsigned)cdiv(N, BN), (unsigned)cdiv(M, kBM));
-    gemm_kernel<FMT, BN, STAGES><<<grid, kGemmThreads, L::kAlloc, st>>>(ta, tb, p);
+    const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
+    gemm_kernel<FMT, BN, STAGES><<<grid, kGemmThreads, L::kAlloc, st>>>(ta, tb, tc, p);
+    return last_launch();
+}
+
+// CTA-pair kernel: 256 x 256 tiles on clusters of two CTAs (M > 128).
+template <int FMT, int STAGES>
+mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
+                             const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out,
+                             cudaStream_t st) {
+    using L = PairSmem<FMT, STAGES>;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    const int64_t M = A->rows, N = B->rows, K = A->cols;
+    const int64_t kbytes = K * fmt_bits(FMT) / 8;
+    CUtensorMap ta, tb, tc;
+    if (!make_tmap_u8(&ta, a_codes, M, kbytes, 128)) return MX_ERR_CUDA;
+    if (!make_tmap_u8(&tb, B->codes, N, kbytes, 128)) return MX_ERR_CUDA;
+    const bool tma_store = (ldc % 8 == 0) && aligned16(C);
+    memset(&tc, 0, sizeof(tc));
+    if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_pair_kernel<FMT, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        L::kAlloc);
+    });
+    if (attr_err != cudaSuccess) return MX_ERR_CUDA;
+    GemmParams p;
+    p.sfa = a_scales;
+    p.sfb = B->scales;
+    p.sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    p.C = C;
+    p.ldc = ldc;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.num_kt = (int)cdiv(kbytes, kStageKBytes);
+    p.m_blocks = (int)cdiv(M, 256);
+    p.n_blocks = (int)cdiv(N, 256);
+    p.ga = ga;
+    p.gb = B->gscale;
+    p.amax_out = amax_out;
+    p.epilogue = epilogue;
+    p.use_tma_store = tma_store ? 1 : 0;
+    p.skip_producer = g_skip_producer.load();
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    const int64_t max_pairs = num_sms() / 2;
+    const unsigned pairs = (unsigned)(tiles < max_pairs ? tiles : max_pairs);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES>, ta, tb, tc, p) != cudaSuccess) return last_launch();
     return last_launch();
 }
 
 template <int FMT>
 mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                           const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
+    if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load())
+        return launch_gemm_pair_t<FMT, FMT == 3 ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
 }
@@ -172,8 +258,56 @@ mx_status launch_gemm(const mx_tensor *A, const mx_tensor *B, const void *a_code
     }
 }
 
-// Byte budget of the fused call's workspace header (X's global-scale slot).
+// The fused call's workspace: a 256-byte header (g, amax of X), then X's codes
+// and scales, each starting on a 256-byte boundary.
 constexpr size_t kFusedWsHeader = 256;
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t fused_ws_bytes(int fmt, int64_t M, int64_t K) {
+    return kFusedWsHeader + align256((size_t)(M * K * fmt_bits(fmt) / 8)) +
+           align256((size_t)(cdiv(M, 128) * 128 * cdiv(K / fmt_block(fmt), 4) * 4));
+}
+
+// Quantize X into the workspace as the A operand of the GEMM.  Returns the
+// device pointer of X's g (NVFP4) through *ga.
+mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int64_t ldx, uint8_t *ws,
+                           const float *x_gscale, const float *x_amax, mx_tensor *xa, const float **ga,
+                           cudaStream_t st) {
+    float *g_slot = reinterpret_cast<float *>(ws);
+    float *amax_slot = reinterpret_cast<float *>(ws + 4);
+    xa->fmt = fmt;
+    xa->reserved = 0;
+    xa->rows = M;
+    xa->cols = K;
+    xa->codes = ws + kFusedWsHeader;
+    xa->scales = ws + kFusedWsHeader + align256((size_t)(M * K * fmt_bits(fmt) / 8));
+    xa->gscale = g_slot;
+    *ga = nullptr;
+    switch (fmt) {
+    case MX_MXFP8_E4M3: launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP8_E5M2: launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP4: launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    default:
+        if (x_gscale != nullptr) {
+            launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st);
+            *ga = x_gscale;
+        } else {
+            const float *amax = x_amax;
+            if (amax == nullptr) {
+                if (cudaMemsetAsync(amax_slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
+                const int64_t vecs = M * (K / 8);
+                int64_t blocks = cdiv(vecs, 256 * 8);
+                const int64_t cap = (int64_t)num_sms() * 8;
+                if (blocks > cap) blocks = cap;
+                if (blocks < 1) blocks = 1;
+                amax_kernel<<<(unsigned)blocks, 256, 0, st>>>(X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
+                amax = amax_slot;
+            }
+            launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1);
+            *ga = g_slot;
+        }
+    }
+    return last_launch();
+}
 
 }  // namespace
 
@@ -210,6 +344,7 @@ mx_status mx_debug_set(int key, uint64_t value) {
     switch (key) {
     case MX_DEBUG_WAIT_LIMIT_NS: g_wait_limit_ns.store(value ? value : 1); return MX_OK;
     case MX_DEBUG_SKIP_PRODUCER: g_skip_producer.store(value ? 1 : 0); return MX_OK;
+    case MX_DEBUG_PAIR_GEMM: g_pair_enabled.store(value ? 1 : 0); return MX_OK;
     default: return MX_ERR_INVALID_ARG;
     }
 }
@@ -283,14 +418,41 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
     return launch_gemm(A, B, A->codes, A->scales, A->gscale, static_cast<uint16_t *>(C_bf16), ldc, 0, nullptr, st);
 }
 
-size_t mx_fused_workspace_bytes(void) { return kFusedWsHeader; }
+size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K) {
+    if (!valid_fmt(fmt) || M < 0 || K < 0) return 0;
+    return fused_ws_bytes(fmt, M, K);
+}
 
 mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx, const mx_tensor *W,
                             void *C_bf16, int64_t ldc, int epilogue, float *amax_out, const float *x_gscale,
                             const float *x_amax, void *workspace, size_t workspace_bytes, void *stream) {
-    (void)fmt; (void)X_bf16; (void)M; (void)K; (void)ldx; (void)W; (void)C_bf16; (void)ldc; (void)epilogue;
-    (void)amax_out; (void)x_gscale; (void)x_amax; (void)workspace; (void)workspace_bytes; (void)stream;
-    return MX_ERR_UNSUPPORTED_SHAPE;  // provided by the fused kernel
+    if (!valid_fmt(fmt) || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    mx_status s = check_tensor(W, true);
+    if (s != MX_OK) return s;
+    if (W->fmt != fmt || W->cols != K) return MX_ERR_INVALID_ARG;
+    if (epilogue != MX_EPI_NONE && epilogue != MX_EPI_GELU) return MX_ERR_INVALID_ARG;
+    const int64_t N = W->rows;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (amax_out != nullptr) {
+        if (!aligned16(amax_out) && (reinterpret_cast<uintptr_t>(amax_out) & 3u)) return MX_ERR_MISALIGNED;
+        if (cudaMemsetAsync(amax_out, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
+    }
+    if (M == 0 || N == 0) return MX_OK;
+    if (!X_bf16 || !C_bf16) return MX_ERR_INVALID_ARG;
+    if (ldc < N) return MX_ERR_INVALID_ARG;
+    if (!aligned16(C_bf16) || !aligned16(X_bf16) || ldx < K || (ldx & 7) != 0) return MX_ERR_MISALIGNED;
+    if (K == 0) return cuda_status(cudaMemset2DAsync(C_bf16, ldc * 2, 0, N * 2, M, st));
+    if (K % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || cdiv(M, kBM) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (!workspace) return MX_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MX_ERR_MISALIGNED;
+    if (workspace_bytes < fused_ws_bytes(fmt, M, K)) return MX_ERR_INVALID_ARG;
+    mx_tensor xa;
+    const float *ga = nullptr;
+    s = fused_quantize_x(fmt, static_cast<const uint16_t *>(X_bf16), M, K, ldx, static_cast<uint8_t *>(workspace),
+                         x_gscale, x_amax, &xa, &ga, st);
+    if (s != MX_OK) return s;
+    return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out, st);
 }
 
 mx_status mx_check_device_error(void *stream, uint32_t info[4]) {

@@ -29,6 +29,11 @@ enum : unsigned {
     SITE_GEMM_MMA_ACC_EMPTY = 4,
     SITE_GEMM_TAIL = 5,
     SITE_FUSED_PRODUCER_EMPTY = 6,
+    SITE_GEMM_EPI_DRAIN = 7,
+    SITE_GEMM_SF_FULL = 8,
+    SITE_GEMM_SF_EMPTY = 9,
+    SITE_GEMM_MMA_SF = 10,
+    SITE_GEMM_SF_LOAD = 11,
 };
 
 // {flags, first site, first block, count}
@@ -87,6 +92,20 @@ MX_DEVICE_INLINE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+
+// Non-blocking test of an mbarrier phase (no suspension).
+MX_DEVICE_INLINE bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most limit_ns.
 // Returns false (and records a timeout) if it did not, or if *abort is set by
 // another role of the same CTA that already gave up.
@@ -129,6 +148,23 @@ MX_DEVICE_INLINE void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes
         "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+
+
+// 2D tiled TMA store (bulk-group completion) from this CTA's shared memory.
+MX_DEVICE_INLINE void tma_store_2d(const void *tmap, int32_t x, int32_t y, const void *smem_src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(smem_u32(smem_src))
+                 : "memory");
+}
+MX_DEVICE_INLINE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups still read shared memory.
+template <int N>
+MX_DEVICE_INLINE void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until all committed bulk groups have completed (writes performed).
+MX_DEVICE_INLINE void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- tcgen05
 MX_DEVICE_INLINE void tmem_alloc(uint32_t *smem_slot, uint32_t ncols) {
@@ -199,6 +235,141 @@ MX_DEVICE_INLINE void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 MX_DEVICE_INLINE void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Store 16 consecutive 32-bit TMEM columns of this warp's 32 lanes (one register
+// per lane and column), then wait for the stores to complete.
+MX_DEVICE_INLINE void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+MX_DEVICE_INLINE void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+MX_DEVICE_INLINE void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+MX_DEVICE_INLINE void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+
+// ---------------------------------------------------------------- clusters (CTA pairs)
+MX_DEVICE_INLINE uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+MX_DEVICE_INLINE void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of this cluster.
+MX_DEVICE_INLINE uint32_t mapa_shared(uint32_t local_saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(rank));
+    return r;
+}
+// Arrive (relaxed, cluster scope) on an mbarrier given by its shared::cluster
+// address.  Callers order their tcgen05 stores before it with tcgen05.wait::st
+// and tcgen05.fence::before_thread_sync; a release at cluster scope costs
+// about a thousand cycles per arrive here and is not needed for that order.
+MX_DEVICE_INLINE void mbar_arrive_cluster(uint32_t cluster_saddr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_saddr) : "memory");
+}
+// 2D tiled TMA load into this CTA's shared memory whose completion is signalled
+// on an mbarrier of the pair's leader CTA (cta_group::2 form, no multicast).
+MX_DEVICE_INLINE void tma_load_2d_pair(void *smem_dst, const void *tmap, int32_t x, int32_t y, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+MX_DEVICE_INLINE void tmem_alloc_pair(uint32_t *smem_slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+MX_DEVICE_INLINE void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+MX_DEVICE_INLINE void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive on the mbarrier at this offset in every CTA of `cta_mask` once all prior
+// tcgen05 operations of this thread (issued for the CTA pair) complete.
+MX_DEVICE_INLINE void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                     smem_u32(bar)),
+                 "h"(cta_mask)
+                 : "memory");
+}
+// Block-scaled MMAs of a CTA pair (M = 256 across the two CTAs' TMEM).
+MX_DEVICE_INLINE void tc_mma_pair_mxf8f6f4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                           uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+MX_DEVICE_INLINE void tc_mma_pair_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+MX_DEVICE_INLINE void tc_mma_pair_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+
+// ---------------------------------------------------------------- predicated tcgen05 issue
+// The whole warp executes these with warp-uniform operands; only threads whose
+// `issue` flag is set perform the operation.  (No branch: operands stay uniform.)
+MX_DEVICE_INLINE void tc_commit_if(uint64_t *bar, uint32_t issue) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "@p tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(issue)
+        : "memory");
+}
+MX_DEVICE_INLINE void tc_commit_pair_if(uint64_t *bar, uint16_t cta_mask, uint32_t issue) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
+        "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask), "r"(issue)
+        : "memory");
+}
+#define MX_DEFINE_MMA_IF(NAME, GROUP, KIND)                                                                        \
+    MX_DEVICE_INLINE void NAME(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,          \
+                               uint32_t sfb, uint32_t accumulate, uint32_t issue) {                                 \
+        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %7, 0;\n\t"                   \
+                     "@q tcgen05.mma.cta_group::" GROUP ".kind::" KIND " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d), \
+                     "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb), "r"(issue)             \
+                     : "memory");                                                                                   \
+    }
+MX_DEFINE_MMA_IF(tc_mma_mxf8f6f4_if, "1", "mxf8f6f4.block_scale")
+MX_DEFINE_MMA_IF(tc_mma_mxf4_if, "1", "mxf4.block_scale.block32")
+MX_DEFINE_MMA_IF(tc_mma_nvf4_if, "1", "mxf4nvf4.block_scale.block16")
+MX_DEFINE_MMA_IF(tc_mma_pair_mxf8f6f4_if, "2", "mxf8f6f4.block_scale")
+MX_DEFINE_MMA_IF(tc_mma_pair_mxf4_if, "2", "mxf4.block_scale.block32")
+MX_DEFINE_MMA_IF(tc_mma_pair_nvf4_if, "2", "mxf4nvf4.block_scale.block16")
+#undef MX_DEFINE_MMA_IF
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (sm_100 form): start >> 4 in bits [0,14),

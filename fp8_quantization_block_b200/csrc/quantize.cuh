@@ -10,11 +10,12 @@
 //          q = RNE_sat(x / (g s)) of the exact quotient.
 //
 // Kernel shape: one CTA quantizes a 128-row x 128-column tile of the bf16 input
-// (32 KB), 8 warps x 16 rows; every thread issues its eight 16-byte loads up
-// front.  A 32-element MX block is held by 4 neighbouring lanes, a 16-element
-// NVFP4 block by 2, and its max |x| is a warp-shuffle reduction of integer
-// maxima of the bf16 magnitude bits.  The scale bytes of the tile (one or two
-// 512-byte tensor-core tiles of 128 rows x 4 scale columns) are assembled in
+// (32 KB).  Each thread owns 16 consecutive elements of a row (32 bytes, two
+// 16-byte loads) per pass, 8 threads per row, 4 passes; all eight loads of a
+// thread are issued up front.  A 16-element NVFP4 block is one thread's, a
+// 32-element MX block two neighbouring lanes' (one shuffle).  Block maxima use
+// packed bf16x2 max on the magnitude bits.  The scale bytes of the tile (one or
+// two 512-byte tensor-core tiles of 128 rows x 4 scale columns) are assembled in
 // shared memory and written out with 16-byte stores.
 #pragma once
 
@@ -71,15 +72,14 @@ MX_DEVICE_INLINE float e4m3_pos_value(uint32_t c) {
 
 // Does 6 * g * s >= amax hold exactly?  fma rounds once, so the sign of
 // fma(6s, g, -amax) is the sign of the exact difference (6s is exact in fp32).
-MX_DEVICE_INLINE bool nv_scale_ok(uint32_t c, float g, float amax) {
-    return __fmaf_rn(6.0f * e4m3_pos_value(c), g, -amax) >= 0.0f;
-}
+MX_DEVICE_INLINE bool nv_scale_ok(float s, float g, float amax) { return __fmaf_rn(6.0f * s, g, -amax) >= 0.0f; }
 
 // NVFP4 block scale: smallest positive finite E4M3 s with amax <= 6 g s,
-// 0 for an all-zero block, 0x7E (448) if none suffices.
-MX_DEVICE_INLINE uint32_t nv_block_scale(float amax, float g) {
+// 0 for an all-zero block, 0x7E (448) if none suffices.  inv6g ~ 1/(6g) only
+// seeds the search; the exact comparisons decide.
+MX_DEVICE_INLINE uint32_t nv_block_scale(float amax, float g, float inv6g, const float *val) {
     if (!(amax > 0.0f)) return 0u;
-    float approx = amax / (6.0f * g);
+    const float approx = amax * inv6g;
     uint32_t c;
     asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %1;\n\tcvt.u32.u16 %0, h;\n\t}"
         : "=r"(c)
@@ -88,8 +88,8 @@ MX_DEVICE_INLINE uint32_t nv_block_scale(float amax, float g) {
     if (c == 0x7Fu) c = 0x7Eu;  // NaN (g not positive): saturate
     if (c == 0u) c = 1u;
     // At most a step or two from the answer; the loops are bounded by the code range.
-    while (c < 0x7Eu && !nv_scale_ok(c, g, amax)) ++c;
-    while (c > 1u && nv_scale_ok(c - 1u, g, amax)) --c;
+    while (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ++c;
+    while (c > 1u && nv_scale_ok(val[c - 1u], g, amax)) --c;
     return c;
 }
 
@@ -133,58 +133,77 @@ MX_DEVICE_INLINE uint32_t cvt8_e2m1(const float (&a)[8]) {
 MX_DEVICE_INLINE float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 MX_DEVICE_INLINE float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Sign bits of the 8 bf16 values in v, moved to the sign bit (bit 3) of each nibble.
-MX_DEVICE_INLINE uint32_t nibble_signs(const uint4 &v) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t s = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s |= (((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u)) << (8 * i);
-    return s;
-}
-
 // E2M1 magnitude of code c (0..7).
 MX_DEVICE_INLINE float e2m1_mag(uint32_t c) {
     return c < 2u ? 0.5f * (float)c : __uint_as_float(((c >> 1) + 126u) << 23) * (1.0f + 0.5f * (float)(c & 1u));
 }
 
-// NVFP4 elements: codes of |x| / (g s) for 8 values, exact RNE of the real
-// quotient.  Two fp32 evaluations with directed rounding bracket the exact
-// quotient; where both round to the same E2M1 code that code is exact (RNE is
-// monotone).  Where they differ the quotient is within a few ulps of the
-// midpoint between two neighbouring codes, and the sign of |x| - g*s*mid,
-// computed exactly by one fma, decides (ties to the even code).
-MX_DEVICE_INLINE uint32_t nv_codes8(const uint4 &v, float g, float s, float r_lo, float r_hi) {
-    const uint32_t w[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
-    float mag[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        mag[2 * i] = bf16lo(w[i]);
-        mag[2 * i + 1] = bf16hi(w[i]);
-    }
-    float lo[8], hi[8];
+// Eight fp32 -> eight E2M1 codes packed (element i in nibble i), RNE, saturating;
+// a value that rounds to zero keeps its sign (the conversion does this).
+// (cvt8_e2m1 above.)
+
+// NVFP4 elements: codes of x / (g s) for 16 values, the exact RNE of the real
+// quotient.  r_lo <= 1/(g s) <= r_hi.  lo = x * r_lo rounded toward zero keeps
+// the sign and bounds |x| / (g s) from below; hi = |x| * r_hi rounded up bounds
+// it from above.  Where the two give the same E2M1 magnitude, that code (with
+// lo's sign) is exact, because RNE is monotone.  Elsewhere the magnitude is
+// walked up from lo's, deciding each midpoint m by the sign of |x| - g*s*m,
+// which one fma computes exactly (s*m is exact in fp32); ties go to the even
+// code.  The walk uses registers only.
+MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, float s, float r_lo, float r_hi,
+                                 uint32_t &out0, uint32_t &out1) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float x[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        lo[i] = __fmul_rd(mag[i], r_lo);
-        hi[i] = __fmul_ru(mag[i], r_hi);
+        x[2 * i] = bf16lo(w[i]);
+        x[2 * i + 1] = bf16hi(w[i]);
     }
-    uint32_t clo = cvt8_e2m1(lo);
-    uint32_t chi = cvt8_e2m1(hi);
-    if (clo != chi) {
-        uint32_t fixed = 0;
+    float lo[16], hi[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t a = (clo >> (4 * i)) & 7u, b = (chi >> (4 * i)) & 7u, c = a;
-            if (a != b) {
-                float mid = 0.5f * (e2m1_mag(a) + e2m1_mag(b));     // exact, 3 significant bits
-                float d = __fmaf_rn(-g, s * mid, mag[i]);           // sign(|x| - g*s*mid), exact
-                c = d > 0.0f ? b : (d < 0.0f ? a : ((a & 1u) ? b : a));
-            }
-            fixed |= c << (4 * i);
-        }
-        clo = fixed;
+    for (int i = 0; i < 16; ++i) {
+        lo[i] = __fmul_rz(x[i], r_lo);
+        hi[i] = __fmul_ru(fabsf(x[i]), r_hi);
     }
-    return clo;
+    const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
+    const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
+    const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
+    const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
+    uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
+    const uint32_t h0 = cvt8_e2m1(hi0), h1 = cvt8_e2m1(hi1);
+    if (((c0 & 0x77777777u) != h0) || ((c1 & 0x77777777u) != h1)) {
+        uint32_t f0 = 0, f1 = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t cl = i < 8 ? c0 : c1, ch = i < 8 ? h0 : h1;
+            const int sh = 4 * (i & 7);
+            uint32_t c = (cl >> sh) & 7u;
+            const uint32_t b = (ch >> sh) & 7u;
+            const float ax = fabsf(x[i]);
+            while (c < b) {
+                const float mid = 0.5f * (e2m1_mag(c) + e2m1_mag(c + 1u));   // 3 significant bits
+                const float d = __fmaf_rn(-g, s * mid, ax);                   // sign(|x| - g*s*mid)
+                if (d > 0.0f || (d == 0.0f && (c & 1u))) ++c;
+                else break;
+            }
+            const uint32_t nib = (c | ((cl >> sh) & 8u)) << sh;
+            if (i < 8) f0 |= nib;
+            else f1 |= nib;
+        }
+        c0 = f0;
+        c1 = f1;
+    }
+    out0 = c0;
+    out1 = c1;
 }
+
+// Per-CTA tables for NVFP4, indexed by positive E4M3 code c (1..126):
+// the value s, and 1/s rounded down and up.
+struct NvTables {
+    float val[128];
+    float inv_lo[128];
+    float inv_hi[128];
+};
 
 // ------------------------------------------------------------------ loads / stores
 MX_DEVICE_INLINE uint4 ldg_stream(const void *p) {
@@ -206,99 +225,140 @@ constexpr int kQTileRows = 128;
 constexpr int kQTileCols = 128;
 constexpr int kQThreads = 256;
 
+// Largest bf16 magnitude (as its bit pattern) among the 16 values of v0, v1.
+MX_DEVICE_INLINE uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    __nv_bfloat162 m[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t a = w[2 * i] & 0x7FFF7FFFu, b = w[2 * i + 1] & 0x7FFF7FFFu;
+        m[i] = __hmax2(*reinterpret_cast<const __nv_bfloat162 *>(&a), *reinterpret_cast<const __nv_bfloat162 *>(&b));
+    }
+    const __nv_bfloat162 r = __hmax2(__hmax2(m[0], m[1]), __hmax2(m[2], m[3]));
+    const uint32_t rb = *reinterpret_cast<const uint32_t *>(&r);
+    return max(rb & 0xFFFFu, rb >> 16);
+}
+
 // src bf16 [M x K] (row pitch ld).  codes / scales as in mx.h.  sf_tiles_k =
-// ceil((K / block) / 4) 512-byte tiles per 128-row band.  gscale: NVFP4 g
-// (read), or for gscale_out != nullptr the value is also stored there by CTA 0.
+// ceil((K / block) / 4) 512-byte tiles per 128-row band.  NVFP4: *gscale_in
+// is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
+// if gscale_out != nullptr, CTA 0 also stores g there.
 template <int FMT>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
                                                              int64_t ld, uint8_t *__restrict__ codes,
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
                                                              const float *__restrict__ gscale_in,
-                                                             float *__restrict__ gscale_out) {
+                                                             float *__restrict__ gscale_out, int g_from_amax) {
     using T = FmtTraits<FMT>;
     constexpr int kBlocksPerRow = kQTileCols / T::kBlock;  // 4 (MX) or 8 (NVFP4)
     constexpr int kSfBytes = kQTileRows * kBlocksPerRow;   // 512 or 1024
+    constexpr int kPasses = kQTileRows / 32;               // 32 rows per pass (8 warps x 4 rows)
     __shared__ __align__(16) uint8_t sf_tile[kSfBytes];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row0 = (int64_t)blockIdx.y * kQTileRows;
     const int64_t col0 = (int64_t)blockIdx.x * kQTileCols;
-    const int cl = (lane & 15) * 8;                 // column of this lane's 8 elements inside the tile
+    const int cl = (lane & 7) * 16;                 // first of this lane's 16 columns inside the tile
     const int64_t col = col0 + cl;
-    const bool col_ok = col < K;                    // K % 8 == 0: all 8 or none
+    const bool col_ok = col < K;                    // K % 16 == 0: all 16 or none
+    const int jb = cl / T::kBlock;                  // block index inside the tile row
 
-    float g = 1.0f;
+    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f;
+    __shared__ NvTables nvt;
     if (FMT == FMT_NVFP4) {
         g = *gscale_in;
+        if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;   // g = RU(amax / (6 * 448))
         if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
+        rg_lo = __frcp_rd(g);
+        rg_hi = __frcp_ru(g);
+        inv6g = 1.0f / (6.0f * g);
+        if (threadIdx.x < 128) {
+            const uint32_t c = threadIdx.x;
+            const float v = (c == 0u || c == 127u) ? 0.0f : e4m3_pos_value(c);
+            nvt.val[c] = v;
+            nvt.inv_lo[c] = v > 0.0f ? __frcp_rd(v) : 0.0f;
+            nvt.inv_hi[c] = v > 0.0f ? __frcp_ru(v) : 0.0f;
+        }
+        __syncthreads();
     }
 
-    uint4 v[8];
+    uint4 v[kPasses][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rl = warp * 16 + 2 * i + (lane >> 4);
+    for (int i = 0; i < kPasses; ++i) {
+        const int rl = i * 32 + warp * 4 + (lane >> 3);
         const int64_t row = row0 + rl;
-        if (row < M && col_ok) v[i] = ldg_stream(src + row * ld + col);
-        else v[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (row < M && col_ok) {
+            const uint16_t *p = src + row * ld + col;
+            v[i][0] = ldg_stream(p);
+            v[i][1] = ldg_stream(p + 8);
+        } else {
+            v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
 
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rl = warp * 16 + 2 * i + (lane >> 4);
+    for (int i = 0; i < kPasses; ++i) {
+        const int rl = i * 32 + warp * 4 + (lane >> 3);
         const int64_t row = row0 + rl;
-        uint32_t m = 0;
-        m = bf16x2_absmax(m, v[i].x);
-        m = bf16x2_absmax(m, v[i].y);
-        m = bf16x2_absmax(m, v[i].z);
-        m = bf16x2_absmax(m, v[i].w);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        if (T::kBlock == 32) m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const int jb = (lane & 15) / (T::kBlock / 8);   // block index inside the tile row
+        const bool ok = row < M && col_ok;
+        uint32_t m = absmax16(v[i][0], v[i][1]);
+        if (T::kBlock == 32) m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         uint32_t sbyte;
         if (FMT == FMT_NVFP4) {
-            const float amax = __uint_as_float(m << 16);
-            sbyte = nv_block_scale(amax, g);
-            if (row < M && col_ok) {
-                uint32_t q;
+            sbyte = nv_block_scale(__uint_as_float(m << 16), g, inv6g, nvt.val);
+            if (ok) {
+                uint32_t q0 = 0, q1 = 0;
                 if (sbyte == 0u) {
-                    q = 0u;
+                    // all-zero block: codes are the signs of the zeros
+                    const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w,
+                                           v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint32_t sgn = (w[e >> 1] >> (16 * (e & 1) + 15)) & 1u;
+                        if (e < 8) q0 |= sgn << (4 * e + 3);
+                        else q1 |= sgn << (4 * (e - 8) + 3);
+                    }
                 } else {
-                    const float s = e4m3_pos_value(sbyte);
-                    const float G_lo = __fmul_rd(g, s), G_hi = __fmul_ru(g, s);
-                    const float r_lo = __frcp_rd(G_hi), r_hi = __frcp_ru(G_lo);
-                    q = nv_codes8(v[i], g, s, r_lo, r_hi);
+                    // r_lo <= 1/(g s) <= r_hi: products of one-sided bounds, rounded outward
+                    const float r_lo = __fmul_rd(rg_lo, nvt.inv_lo[sbyte]);
+                    const float r_hi = __fmul_ru(rg_hi, nvt.inv_hi[sbyte]);
+                    nv_codes16(v[i][0], v[i][1], g, nvt.val[sbyte], r_lo, r_hi, q0, q1);
                 }
-                q |= nibble_signs(v[i]);
-                *reinterpret_cast<uint32_t *>(codes + row * (K / 2) + col / 2) = q;
+                *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
             }
         } else {
             const int E = mx_scale_byte<FMT>(m);
             sbyte = (uint32_t)E;
-            if (row < M && col_ok) {
+            if (ok) {
                 const float inv = mx_inv_scale(E);
-                const uint4 w = v[i];
+                const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w,
+                                       v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
+                float f[16];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    f[2 * e] = bf16lo(w[e]) * inv;
+                    f[2 * e + 1] = bf16hi(w[e]) * inv;
+                }
                 if (T::kBits == 8) {
-                    uint2 q;
-                    q.x = cvt4_fp8<FMT>(bf16lo(w.x) * inv, bf16hi(w.x) * inv, bf16lo(w.y) * inv, bf16hi(w.y) * inv);
-                    q.y = cvt4_fp8<FMT>(bf16lo(w.z) * inv, bf16hi(w.z) * inv, bf16lo(w.w) * inv, bf16hi(w.w) * inv);
-                    *reinterpret_cast<uint2 *>(codes + row * K + col) = q;
+                    uint4 q;
+                    q.x = cvt4_fp8<FMT>(f[0], f[1], f[2], f[3]);
+                    q.y = cvt4_fp8<FMT>(f[4], f[5], f[6], f[7]);
+                    q.z = cvt4_fp8<FMT>(f[8], f[9], f[10], f[11]);
+                    q.w = cvt4_fp8<FMT>(f[12], f[13], f[14], f[15]);
+                    *reinterpret_cast<uint4 *>(codes + row * K + col) = q;
                 } else {
-                    const uint4 a = make_uint4(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu, w.z & 0x7FFF7FFFu,
-                                               w.w & 0x7FFF7FFFu);
-                    float f[8] = {bf16lo(a.x) * inv, bf16hi(a.x) * inv, bf16lo(a.y) * inv, bf16hi(a.y) * inv,
-                                  bf16lo(a.z) * inv, bf16hi(a.z) * inv, bf16lo(a.w) * inv, bf16hi(a.w) * inv};
-                    const uint32_t q = cvt8_e2m1(f) | nibble_signs(w);
-                    *reinterpret_cast<uint32_t *>(codes + row * (K / 2) + col / 2) = q;
+                    const float(&f0)[8] = *reinterpret_cast<const float(*)[8]>(&f[0]);
+                    const float(&f1)[8] = *reinterpret_cast<const float(*)[8]>(&f[8]);
+                    *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(cvt8_e2m1(f0), cvt8_e2m1(f1));
                 }
             }
         }
         // Scale byte of (rl, jb) inside the tile's 512-byte tensor-core tiles.
-        const bool owner = (lane & ((T::kBlock / 8) - 1)) == 0;
+        const bool owner = T::kBlock == 16 || (lane & 1) == 0;
         if (owner) {
             const int64_t jglob = col0 / T::kBlock + jb;
             if (!(row < M) || jglob >= K / T::kBlock) sbyte = 0u;   // padding bytes are 0
-            const int chunk = jb >> 2;
-            sf_tile[chunk * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (jb & 3)] = (uint8_t)sbyte;
+            sf_tile[(jb >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (jb & 3)] = (uint8_t)sbyte;
         }
     }
     __syncthreads();

@@ -26,7 +26,7 @@ FORMATS = {"mxfp8_e4m3": 0, "mxfp8_e5m2": 1, "mxfp4": 2, "nvfp4": 3}
 MX_OK, MX_ERR_INVALID_ARG, MX_ERR_UNSUPPORTED_SHAPE, MX_ERR_MISALIGNED = 0, 1, 2, 3
 MX_ERR_CUDA, MX_ERR_TIMEOUT, MX_ERR_DEVICE = 4, 5, 6
 MX_EPI_NONE, MX_EPI_GELU = 0, 1
-MX_DEBUG_WAIT_LIMIT_NS, MX_DEBUG_SKIP_PRODUCER = 1, 2
+MX_DEBUG_WAIT_LIMIT_NS, MX_DEBUG_SKIP_PRODUCER, MX_DEBUG_PAIR_GEMM = 1, 2, 3
 
 EXPORTED = [
     "mx_codes_bytes", "mx_scales_bytes", "mx_block_size", "mx_quantize", "mx_dequantize", "mx_gemm",
@@ -68,7 +68,7 @@ def lib() -> ctypes.CDLL:
                 "mx_dequantize": (i32, [T, P, i64, P]),
                 "mx_gemm": (i32, [T, T, P, i64, P]),
                 "mx_gemm_fused_act": (i32, [i32, P, i64, i64, i64, T, P, i64, i32, P, P, P, P, sz, P]),
-                "mx_fused_workspace_bytes": (sz, []),
+                "mx_fused_workspace_bytes": (sz, [i32, i64, i64]),
                 "mx_check_device_error": (i32, [P, ctypes.POINTER(ctypes.c_uint32)]),
                 "mx_status_string": (ctypes.c_char_p, [i32]),
                 "mx_version": (i32, []),
@@ -113,8 +113,8 @@ def mx_gemm_fused_act(fmt, X_ptr, M, K, ldx, W: MxTensorC, C_ptr, ldc, epilogue,
                                        x_gscale_ptr, x_amax_ptr, ws_ptr, ws_bytes, stream))
 
 
-def mx_fused_workspace_bytes() -> int:
-    return int(lib().mx_fused_workspace_bytes())
+def mx_fused_workspace_bytes(fmt: int, M: int, K: int) -> int:
+    return int(lib().mx_fused_workspace_bytes(fmt, M, K))
 
 
 def mx_check_device_error(stream=None):
@@ -207,11 +207,18 @@ def gemm_fused_act(x: torch.Tensor, W: MxTensor, out: torch.Tensor | None = None
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     M, K = x.shape
     out = out if out is not None else torch.empty((M, W.rows), dtype=torch.bfloat16, device=x.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is None:
+        workspace = fused_workspace(W.fmt, M, K, x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
     check(mx_gemm_fused_act(W.fmt, x.data_ptr(), M, K, x.stride(0), W.c(), out.data_ptr(), out.stride(0), epilogue,
                             _ptr(amax_out), _ptr(x_gscale), _ptr(x_amax), _ptr(workspace), ws_bytes,
                             _stream(stream)), "mx_gemm_fused_act")
     return out
+
+
+def fused_workspace(fmt: int, M: int, K: int, device="cuda") -> torch.Tensor:
+    """A workspace for gemm_fused_act (torch's allocator hands out 256-B aligned blocks)."""
+    return torch.empty(mx_fused_workspace_bytes(fmt, M, K), dtype=torch.uint8, device=device)
 
 
 def check_device_error(stream=None) -> None:

@@ -123,8 +123,12 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
 
 /* Fused activation-quantize + GEMM: X is bf16 [M x K] (row pitch ldx), W a
  * pre-quantized [N x K] mx_tensor of format fmt.  X is quantized exactly as
- * mx_quantize would (same codes and scales, bit for bit) inside the GEMM's
- * producer, never written to memory, and C = X_dq * W_dq^T as in mx_gemm.
+ * mx_quantize would (same codes and scales, bit for bit) once, into the
+ * caller's `workspace` (which stays resident in L2 at these sizes), and the
+ * block-scaled GEMM consumes it in the same stream: C = X_dq * W_dq^T as in
+ * mx_gemm.  X's quantized form is not an output of this call.
+ *   workspace: device buffer of at least mx_fused_workspace_bytes(fmt, M, K)
+ *              bytes, 256-byte aligned; its contents are scratch.
  *   epilogue : MX_EPI_NONE, or MX_EPI_GELU (exact erf form, applied in FP32
  *              before the bf16 rounding).
  *   amax_out : NULL, or a device float that receives max |C| over the bf16
@@ -133,15 +137,15 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  *   NVFP4 only, how g of X is found (first non-NULL wins):
  *     x_gscale : device float holding g itself;
  *     x_amax   : device float holding amax(|X|); g = RU_fp32(amax / 2688);
- *     neither  : amax(|X|) is computed by a pre-pass into `workspace`, which
- *                must then be a device buffer of at least
- *                mx_fused_workspace_bytes() bytes (unused otherwise).
+ *     neither  : amax(|X|) is computed by a pre-pass over X.
  * K % 128 == 0, ldx % 8 == 0. */
 mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx,
                             const mx_tensor *W, void *C_bf16, int64_t ldc, int epilogue,
                             float *amax_out, const float *x_gscale, const float *x_amax,
                             void *workspace, size_t workspace_bytes, void *stream);
-size_t mx_fused_workspace_bytes(void);
+/* Workspace bytes mx_gemm_fused_act needs for an [M x K] activation of format
+ * fmt (a 256-byte header, then X's codes and scales); 0 for a bad format. */
+size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K);
 
 /* Synchronize `stream`, then read and clear the device error word.  Returns
  * MX_OK, MX_ERR_TIMEOUT (a bounded wait inside a kernel gave up: the kernel
@@ -160,8 +164,11 @@ int mx_version(void);
  *   MX_DEBUG_SKIP_PRODUCER : 1 = GEMM producers skip their loads, so the
  *                            consumers' bounded waits run out (fault test);
  *                            never set in normal use.
+ *   MX_DEBUG_PAIR_GEMM     : 1 (default) = GEMMs with M > 128 and N > 128 run
+ *                            on CTA pairs (256 x 256 tiles); 0 = single-CTA
+ *                            128 x 256 tiles for every shape.
  * Returns MX_ERR_INVALID_ARG for an unknown key. */
-typedef enum { MX_DEBUG_WAIT_LIMIT_NS = 1, MX_DEBUG_SKIP_PRODUCER = 2 } mx_debug_key;
+typedef enum { MX_DEBUG_WAIT_LIMIT_NS = 1, MX_DEBUG_SKIP_PRODUCER = 2, MX_DEBUG_PAIR_GEMM = 3 } mx_debug_key;
 mx_status mx_debug_set(int key, uint64_t value);
 
 #ifdef __cplusplus

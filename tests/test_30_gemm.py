@@ -159,3 +159,24 @@ def test_gemm_is_deterministic():
     c2 = mx.gemm(qa, qb)
     torch.cuda.synchronize()
     assert torch.equal(c1.view(torch.int16), c2.view(torch.int16))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("pair", [0, 1])
+def test_pair_and_single_cta_kernels(fmt, pair):
+    """M > 128 runs on CTA pairs (256 x 256 tiles) by default; the single-CTA
+    kernel (128 x 256 tiles) stays available.  Both against the oracle,
+    including ragged M and N tails and a K tail inside a stage."""
+    M, N, K = 333, 520, 640
+    A_bits = synth.sweep_tensor(3000 + fmt, M, K)
+    B_bits = synth.gaussian_weights(4000 + fmt, N, K)
+    qa, qb, Ad, Bd = quantized_pair(fmt, A_bits, B_bits)
+    try:
+        assert mx.mx_debug_set(mx.MX_DEBUG_PAIR_GEMM, pair) == mx.MX_OK
+        C = mx.gemm(qa, qb)
+        torch.cuda.synchronize()
+        mx.check_device_error()
+    finally:
+        mx.mx_debug_set(mx.MX_DEBUG_PAIR_GEMM, 1)
+    ok, worst = gemm_check(C, Ad, Bd)
+    assert ok, worst

@@ -1,0 +1,114 @@
+"""Fused activation-quantize + GEMM: bitwise equal to mx_quantize + mx_gemm,
+GELU / |C| max epilogue against the fp64 oracle, and the NVFP4 MLP chain
+(GEMM1 -> GELU -> amax -> GEMM2) without a host sync."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_quantization_block_b200 import mx, synth
+from gpu_helpers import gemm_check, host, to_dev
+
+pytestmark = pytest.mark.gpu
+FMTS = [0, 1, 2, 3]
+
+
+def bits16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,N,K", [(64, 64, 256), (200, 300, 384), (512, 768, 1024)])
+def test_fused_equals_unfused(fmt, M, N, K):
+    X_bits = synth.sweep_tensor(300 + M, M, K)
+    W_bits = synth.gaussian_weights(400 + N, N, K)
+    X, Wt = to_dev(X_bits), to_dev(W_bits)
+    W = mx.quantize(Wt, fmt)
+    C_f = mx.gemm_fused_act(X, W)
+    C_u = mx.gemm(mx.quantize(X, fmt), W)
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    assert torch.equal(C_f.view(torch.int16), C_u.view(torch.int16))
+
+
+def test_nvfp4_gscale_sources_agree():
+    M, N, K = 256, 512, 768
+    X = to_dev(synth.student_t(50, M, K))
+    W = mx.quantize(to_dev(synth.gaussian_weights(51, N, K)), 3)
+    C_pre = mx.gemm_fused_act(X, W)                                       # amax pre-pass
+    amax = X.abs().max().float().reshape(1)
+    C_amax = mx.gemm_fused_act(X, W, x_amax=amax)                         # g from amax
+    g = mx.quantize(X, 3).gscale
+    C_g = mx.gemm_fused_act(X, W, x_gscale=g)                             # g given
+    torch.cuda.synchronize()
+    assert torch.equal(C_pre.view(torch.int16), C_amax.view(torch.int16))
+    assert torch.equal(C_pre.view(torch.int16), C_g.view(torch.int16))
+    assert float(g.cpu()[0]) == oracle.nvfp4_global_scale(float(amax.cpu()[0]))
+
+
+@pytest.mark.parametrize("fmt", [0, 3])
+def test_gelu_and_amax_epilogue(fmt):
+    M, N, K = 192, 320, 512
+    X_bits = synth.student_t(60, M, K)
+    W_bits = synth.gaussian_weights(61, N, K)
+    X = to_dev(X_bits)
+    W = mx.quantize(to_dev(W_bits), fmt)
+    amax = torch.full((1,), 123.0, device="cuda")
+    H = mx.gemm_fused_act(X, W, epilogue=mx.MX_EPI_GELU, amax_out=amax)
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    # oracle: quantize X and W on the host, fp64 GEMM, fp64 GELU
+    cx, sx, gx = oracle.quantize(fmt, X_bits)
+    cw, sw, gw = host(W)
+    Xd = oracle.dequantize_f64(fmt, cx, sx, gx, M, K)
+    Wd = oracle.dequantize_f64(fmt, cw, sw, gw, N, K)
+    Cref, Cabs = oracle.gemm_f64(Xd, Wd)
+    Href = oracle.gelu(Cref)
+    Hg = H.float().cpu().double().numpy()
+    bound = 1.13 * (2.0 ** -8 * np.abs(Cref) + 1e-4 * Cabs) + 2.0 ** -8 * np.abs(Href) + 1e-30
+    assert np.all(np.abs(Hg - Href) <= bound), float(np.max(np.abs(Hg - Href) / bound))
+    assert float(amax.cpu()[0]) == float(H.abs().max().float().cpu())     # zeroed, then max |H|
+
+
+def test_nvfp4_mlp_chain_without_host_sync():
+    M, D, F = 256, 512, 1024
+    X = to_dev(synth.student_t(70, M, D))
+    W1 = mx.quantize(to_dev(synth.gaussian_weights(71, F, D)), 3)
+    W2 = mx.quantize(to_dev(synth.gaussian_weights(72, D, F)), 3)
+    aH = torch.empty(1, device="cuda")
+    H = mx.gemm_fused_act(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=aH)
+    Y = mx.gemm_fused_act(H, W2, x_amax=aH)
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    # the same chain unfused: quantize H (g from its own amax) then GEMM
+    qH = mx.quantize(H, 3)
+    Y_u = mx.gemm(qH, W2)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y_u.view(torch.int16))
+    # and against the oracle on H as produced by the GPU
+    H_bits = bits16(H)
+    ch, sh, gh = oracle.quantize(3, H_bits)
+    assert np.array_equal(qH.codes.cpu().numpy(), ch) and np.array_equal(qH.scales.cpu().numpy(), sh)
+    cw, sw, gw = host(W2)
+    Hd = oracle.dequantize_f64(3, ch, sh, gh, M, F)
+    W2d = oracle.dequantize_f64(3, cw, sw, gw, D, F)
+    ok, worst = gemm_check(Y, Hd, W2d)
+    assert ok, worst
+
+
+def test_workspace_checks():
+    X = torch.zeros((64, 256), dtype=torch.bfloat16, device="cuda")
+    W = mx.quantize(torch.zeros((64, 256), dtype=torch.bfloat16, device="cuda"), 0)
+    C = torch.empty((64, 64), dtype=torch.bfloat16, device="cuda")
+    need = mx.mx_fused_workspace_bytes(0, 64, 256)
+    ws = torch.empty(need + 512, dtype=torch.uint8, device="cuda")
+    s = mx.mx_gemm_fused_act(0, X.data_ptr(), 64, 256, 256, W.c(), C.data_ptr(), 64, 0, None, None, None,
+                             ws.data_ptr(), need - 1, None)
+    assert s == mx.MX_ERR_INVALID_ARG
+    s = mx.mx_gemm_fused_act(0, X.data_ptr(), 64, 256, 256, W.c(), C.data_ptr(), 64, 0, None, None, None,
+                             ws.data_ptr() + 16, need, None)
+    assert s == mx.MX_ERR_MISALIGNED
+    s = mx.mx_gemm_fused_act(2, X.data_ptr(), 64, 256, 256, W.c(), C.data_ptr(), 64, 0, None, None, None,
+                             ws.data_ptr(), need, None)
+    assert s == mx.MX_ERR_INVALID_ARG                                      # W format differs
+    torch.cuda.synchronize()
