@@ -455,6 +455,49 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out, st);
 }
 
+}  // extern "C"
+
+// --- mx_gemm_fused_act_noalloc: scratch without allocation -------------------
+// The scratch lives in this file-scope device array.  Host code must not pass
+// the symbol itself to a kernel (on the host it is only a stand-in, not a
+// device address): its device address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MX_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (set up on first use).
+mx_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MX_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MX_ERR_UNSUPPORTED_SHAPE;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MX_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MX_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mx_status mx_gemm_fused_act_noalloc(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx,
+                                    const mx_tensor *W, void *C_bf16, int64_t ldc, int epilogue, float *amax_out,
+                                    const float *x_gscale, const float *x_amax, void *stream) {
+    if (!valid_fmt(fmt) || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    if (fused_ws_bytes(fmt, M, K) > MX_NOALLOC_SCRATCH_BYTES) return MX_ERR_UNSUPPORTED_SHAPE;
+    void *scratch = nullptr;
+    const mx_status s = noalloc_scratch(&scratch);
+    if (s != MX_OK) return s;
+    return mx_gemm_fused_act(fmt, X_bf16, M, K, ldx, W, C_bf16, ldc, epilogue, amax_out, x_gscale, x_amax, scratch,
+                             MX_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 mx_status mx_check_device_error(void *stream, uint32_t info[4]) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);

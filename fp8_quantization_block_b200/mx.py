@@ -31,8 +31,9 @@ MX_DEBUG_WAIT_LIMIT_NS, MX_DEBUG_SKIP_PRODUCER, MX_DEBUG_PAIR_GEMM = 1, 2, 3
 EXPORTED = [
     "mx_codes_bytes", "mx_scales_bytes", "mx_block_size", "mx_quantize", "mx_dequantize", "mx_gemm",
     "mx_gemm_fused_act", "mx_fused_workspace_bytes", "mx_check_device_error", "mx_status_string",
-    "mx_version", "mx_debug_set",
+    "mx_version", "mx_debug_set", "mx_gemm_fused_act_noalloc",
 ]
+MX_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class MxError(RuntimeError):
@@ -69,6 +70,7 @@ def lib() -> ctypes.CDLL:
                 "mx_gemm": (i32, [T, T, P, i64, P]),
                 "mx_gemm_fused_act": (i32, [i32, P, i64, i64, i64, T, P, i64, i32, P, P, P, P, sz, P]),
                 "mx_fused_workspace_bytes": (sz, [i32, i64, i64]),
+                "mx_gemm_fused_act_noalloc": (i32, [i32, P, i64, i64, i64, T, P, i64, i32, P, P, P, P]),
                 "mx_check_device_error": (i32, [P, ctypes.POINTER(ctypes.c_uint32)]),
                 "mx_status_string": (ctypes.c_char_p, [i32]),
                 "mx_version": (i32, []),
@@ -111,6 +113,13 @@ def mx_gemm_fused_act(fmt, X_ptr, M, K, ldx, W: MxTensorC, C_ptr, ldc, epilogue,
                       x_amax_ptr, ws_ptr, ws_bytes, stream) -> int:
     return int(lib().mx_gemm_fused_act(fmt, X_ptr, M, K, ldx, ctypes.byref(W), C_ptr, ldc, epilogue, amax_out_ptr,
                                        x_gscale_ptr, x_amax_ptr, ws_ptr, ws_bytes, stream))
+
+
+def mx_gemm_fused_act_noalloc(fmt, X_ptr, M, K, ldx, W: MxTensorC, C_ptr, ldc, epilogue, amax_out_ptr, x_gscale_ptr,
+                              x_amax_ptr, stream) -> int:
+    """The fused call with the library's own fixed scratch (no workspace; allocates nothing)."""
+    return int(lib().mx_gemm_fused_act_noalloc(fmt, X_ptr, M, K, ldx, ctypes.byref(W), C_ptr, ldc, epilogue,
+                                               amax_out_ptr, x_gscale_ptr, x_amax_ptr, stream))
 
 
 def mx_fused_workspace_bytes(fmt: int, M: int, K: int) -> int:

@@ -147,6 +147,31 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
  * fmt (a 256-byte header, then X's codes and scales); 0 for a bad format. */
 size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K);
 
+/* mx_gemm_fused_act without a workspace argument, for callers that cannot
+ * allocate device memory: code running while a stream is being captured or
+ * inside an engine's enqueue/plugin callback where allocation is forbidden,
+ * latency-critical paths that must not pay for cudaMalloc's implicit device
+ * synchronization, and runtimes with a fixed memory budget.  The pages have no
+ * counterpart to this call; it exists for those callers only.
+ *   Scratch: a fixed array of MX_NOALLOC_SCRATCH_BYTES inside libmx.so itself,
+ *   one per GPU that loads the library, kept until the process exits.  The
+ *   call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *   routine).  Shapes whose mx_fused_workspace_bytes(fmt, M, K) exceeds the
+ *   array are rejected with MX_ERR_UNSUPPORTED_SHAPE before any launch.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, once per device, with that device current); make
+ *   that first call before any stream capture.
+ *   Every call uses the same array and leaves its contents behind (whatever
+ *   must start at zero is cleared by the call).  Calls that overlap on the GPU
+ *   -- on different streams, or from several host threads -- race on it and
+ *   must be serialized by the caller.
+ * All other arguments, results and errors are those of mx_gemm_fused_act. */
+#define MX_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+mx_status mx_gemm_fused_act_noalloc(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx,
+                                    const mx_tensor *W, void *C_bf16, int64_t ldc, int epilogue,
+                                    float *amax_out, const float *x_gscale, const float *x_amax,
+                                    void *stream);
+
 /* Synchronize `stream`, then read and clear the device error word.  Returns
  * MX_OK, MX_ERR_TIMEOUT (a bounded wait inside a kernel gave up: the kernel
  * returned early and its outputs are unspecified) or MX_ERR_DEVICE.  If info is
