@@ -38,7 +38,10 @@ struct PairSmem {
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + STAGES * kABytes;
     static constexpr int kOffEpi = kOffB + STAGES * kBBytes;
-    static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiChunkBytes;
+    static constexpr int kNoEpi = STAGES * (kABytes + kBBytes + kSfaBytes + kSfbBytes) + (3 * STAGES + 4 + 2 * kSfSlots) * 8 +
+                                  16 + 1024;
+    static constexpr int kEpiBufs = (kNoEpi + kEpiWarps * 2 * kEpiChunkBytes <= kSmemLimit) ? 2 : 1;
+    static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiBufs * kEpiChunkBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
     static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
     // full[S] (leader's counts both CTAs' code tiles), empty[S], sfload[S],
@@ -280,14 +283,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue (this CTA's 128 rows)
         const int q = warp & 3;
-        uint8_t *stage_buf = smem + L::kOffEpi + (warp - 2) * kEpiChunkBytes;
+        uint8_t *bufs = smem + L::kOffEpi + (warp - 2) * L::kEpiBufs * kEpiChunkBytes;
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-        uint32_t amax = 0;
+        uint32_t amax = 0, nstore = 0;
         float scale = 1.0f;
         if (FMT == 3) scale = (*p.ga) * (*p.gb);
         int it = 0;
-        constexpr int kChunksPerTile = 256 / 32;
-        constexpr int kOverlapChunks = (256 - L::kAccStride) / 32;
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             int m0, n0;
             tile_coords(tile, p.m_blocks, m0, n0, 256);
@@ -295,64 +296,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
-            const int row = m0 + 32 * q + lane;
-            const int n_valid = p.N - n0;
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
-            for (int idx = 0; idx < kChunksPerTile; ++idx) {
-                if (idx == kOverlapChunks) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-                }
-                const int c = (b == 0) ? (idx + (kChunksPerTile - kOverlapChunks)) % kChunksPerTile : idx;
-                const int col = 32 * c;
-                if (col >= n_valid) continue;  // warp-uniform
-                uint32_t r[32];
-                tmem_ld32(t_acc + (uint32_t)col, r);
-                tmem_wait_ld();
-                uint32_t packed[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float x0 = __uint_as_float(r[2 * i]) * scale, x1 = __uint_as_float(r[2 * i + 1]) * scale;
-                    if (p.epilogue == 1) {
-                        x0 = gelu_erf(x0);
-                        x1 = gelu_erf(x1);
-                    }
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-                    packed[i] = *reinterpret_cast<const uint32_t *>(&h);
-                }
-                if (p.amax_out != nullptr && row < p.M) {
-                    const int valid = min(32, n_valid - col);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < valid) amax = max(amax, (packed[i >> 1] >> (16 * (i & 1))) & 0x7FFFu);
-                }
-                if (m0 + 32 * q >= p.M) continue;  // warp-uniform
-                if (p.use_tma_store) {
-                    if (lane == 0) bulk_wait_group_read<0>();
-                    __syncwarp();
-                    uint4 *dst = reinterpret_cast<uint4 *>(stage_buf + lane * 64);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmC, n0 + col, m0 + 32 * q, stage_buf);
-                        bulk_commit_group();
-                    }
-                } else if (row < p.M) {
-                    uint16_t *dst = p.C + (int64_t)row * p.ldc + n0 + col;
-                    for (int i = 0; i < 32 && col + i < n_valid; ++i) dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
-                }
-            }
+            epilogue_tile<256, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
+                                              [&] {
+                                                  if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+                                              });
         }
-        if (lane == 0) bulk_wait_group_all();
-        if (p.amax_out != nullptr) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            if (lane == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int *>(p.amax_out), amax << 16);
-        }
+        epilogue_finish(p, lane, amax);
     }
 
     tc_fence_before();

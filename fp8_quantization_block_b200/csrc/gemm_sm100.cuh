@@ -65,6 +65,7 @@ constexpr int kGemmThreads = 320;
 constexpr int kSfSlots = 4;
 constexpr int kEpiWarps = 4;
 constexpr int kEpiChunkBytes = 32 * 32 * 2;  // 32 rows x 32 bf16 columns per epilogue warp
+constexpr int kSmemLimit = 232448;           // dynamic shared memory per CTA (opt-in maximum)
 
 struct GemmParams {
     const uint8_t *sfa;
@@ -95,7 +96,11 @@ struct GemmSmem {
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + STAGES * kABytes;
     static constexpr int kOffEpi = kOffB + STAGES * kBBytes;
-    static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiChunkBytes;
+    // two staging buffers per epilogue warp where shared memory allows, else one
+    static constexpr int kNoEpi = STAGES * (kABytes + kBBytes + kSfaBytes + kSfbBytes) + (2 * STAGES + 4 + 2 * kSfSlots) * 8 +
+                                  16 + 1024;
+    static constexpr int kEpiBufs = (kNoEpi + kEpiWarps * 2 * kEpiChunkBytes <= kSmemLimit) ? 2 : 1;
+    static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiBufs * kEpiChunkBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
     static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
     // full[S], empty[S], acc_full[2], acc_empty, mma_done, sf_full[2], sf_empty[2]
@@ -198,6 +203,152 @@ MX_DEVICE_INLINE void stage_scales_to_tmem(const uint8_t *sfa_stage, const uint8
 MX_DEVICE_INLINE void tile_coords(int tile, int m_blocks, int &m0, int &n0, int bn) {
     m0 = (tile % m_blocks) * kBM;
     n0 = (tile / m_blocks) * bn;
+}
+
+// ---------------------------------------------------------------- epilogue
+// One 32-column chunk of this warp's 32 accumulator rows: TMEM -> registers,
+// x scale (NVFP4: gA * gB), optional GELU, bf16 round-to-nearest-even.  The
+// options are template parameters so that the unused paths cost no issue
+// slots (the epilogue warps share schedulers with the MMA and scale warps).
+template <bool SCALED, bool GELU>
+MX_DEVICE_INLINE void epi_load_convert(uint32_t t_addr, float scale, uint32_t (&packed)[16]) {
+    uint32_t r[32];
+    tmem_ld32(t_addr, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float x0 = __uint_as_float(r[2 * i]), x1 = __uint_as_float(r[2 * i + 1]);
+        if (SCALED) {
+            x0 *= scale;
+            x1 *= scale;
+        }
+        if (GELU) {
+            x0 = gelu_erf(x0);
+            x1 = gelu_erf(x1);
+        }
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+        packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+}
+
+// Write one converted chunk (rows m0q + lane, columns n0 + col ..) and fold
+// it into the running |C| maximum.  TMA stores go through NBUF staging
+// buffers of this warp, so a store only waits for the one issued NBUF
+// chunks earlier to have finished reading shared memory.
+template <int NBUF>
+MX_DEVICE_INLINE void epi_emit(const GemmParams &p, const CUtensorMap *tmC, const uint32_t (&packed)[16], int m0q,
+                               int n0, int col, int lane, uint8_t *bufs, uint32_t &nstore, uint32_t &amax) {
+    const int row = m0q + lane;
+    const int n_valid = p.N - n0;
+    if (p.amax_out != nullptr && row < p.M) {
+        const int valid = min(32, n_valid - col);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < valid) amax = max(amax, (packed[i >> 1] >> (16 * (i & 1))) & 0x7FFFu);
+    }
+    if (m0q >= p.M) return;  // warp-uniform: no rows of this quadrant exist
+    if (p.use_tma_store) {
+        uint8_t *buf = bufs + (nstore % NBUF) * kEpiChunkBytes;
+        if (lane == 0) bulk_wait_group_read<NBUF - 1>();  // this buffer's previous store has read it
+        __syncwarp();
+        uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * 64);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmC, n0 + col, m0q, buf);
+            bulk_commit_group();
+        }
+        ++nstore;
+    } else if (row < p.M) {
+        uint16_t *dst = p.C + (int64_t)row * p.ldc + n0 + col;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (col + i < n_valid) dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
+    }
+}
+
+// Drain one accumulator tile (BN columns) for this warp's TMEM quadrant.  The
+// two accumulator buffers share BN - ACC_STRIDE columns (buffer 0's tail is
+// buffer 1's head), and the next tile's MMAs wait for release().  Without
+// GELU those chunks are pulled into registers first, so release() runs
+// before any store is issued and the tensor pipe idles only for the TMEM
+// reads.
+template <int BN, int ACC_STRIDE, int NBUF, bool SCALED, bool GELU, typename Release>
+MX_DEVICE_INLINE void epilogue_tile_t(const GemmParams &p, const CUtensorMap *tmC, uint32_t t_acc, int b, int m0q,
+                                      int n0, int lane, uint8_t *bufs, uint32_t &nstore, uint32_t &amax, float scale,
+                                      Release release) {
+    constexpr int kChunks = BN / 32;
+    constexpr int kOv = (BN - ACC_STRIDE) / 32;
+    static_assert(kOv >= 0 && kOv <= kChunks, "accumulator overlap");
+    const int n_valid = p.N - n0;
+    if (GELU) {
+        // GELU needs more live registers per chunk: drain in order, releasing
+        // after the shared chunks have been written out.
+        for (int idx = 0; idx < kChunks; ++idx) {
+            if (idx == kOv) {
+                tc_fence_before();
+                __syncwarp();
+                release();
+            }
+            const int col = 32 * ((b == 0) ? (idx + (kChunks - kOv)) % kChunks : idx);
+            if (col >= n_valid) continue;  // warp-uniform
+            uint32_t packed[16];
+            epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
+            epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+        }
+        if (kOv == kChunks) {
+            tc_fence_before();
+            __syncwarp();
+            release();
+        }
+        return;
+    }
+    uint32_t ov[kOv > 0 ? kOv : 1][16];
+#pragma unroll
+    for (int i = 0; i < kOv; ++i) {
+        const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
+        if (col < n_valid) epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, ov[i]);
+    }
+    tc_fence_before();
+    __syncwarp();
+    release();
+#pragma unroll
+    for (int i = 0; i < kOv; ++i) {
+        const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
+        if (col < n_valid) epi_emit<NBUF>(p, tmC, ov[i], m0q, n0, col, lane, bufs, nstore, amax);
+    }
+    for (int i = 0; i < kChunks - kOv; ++i) {
+        const int col = 32 * ((b == 0) ? i : (kOv + i));
+        if (col >= n_valid) break;  // warp-uniform; columns ascend
+        uint32_t packed[16];
+        epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
+        epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+    }
+}
+
+template <int BN, int ACC_STRIDE, int NBUF, bool SCALED, typename Release>
+MX_DEVICE_INLINE void epilogue_tile(const GemmParams &p, const CUtensorMap *tmC, uint32_t t_acc, int b, int m0q,
+                                    int n0, int lane, uint8_t *bufs, uint32_t &nstore, uint32_t &amax, float scale,
+                                    Release release) {
+    if (p.epilogue == 1)
+        epilogue_tile_t<BN, ACC_STRIDE, NBUF, SCALED, true>(p, tmC, t_acc, b, m0q, n0, lane, bufs, nstore, amax, scale,
+                                                            release);
+    else
+        epilogue_tile_t<BN, ACC_STRIDE, NBUF, SCALED, false>(p, tmC, t_acc, b, m0q, n0, lane, bufs, nstore, amax, scale,
+                                                             release);
+}
+
+// Flush this warp's stores and publish its |C| maximum.
+MX_DEVICE_INLINE void epilogue_finish(const GemmParams &p, int lane, uint32_t amax) {
+    if (lane == 0) bulk_wait_group_all();
+    if (p.amax_out != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int *>(p.amax_out), amax << 16);
+    }
 }
 
 template <int FMT, int BN, int STAGES>
@@ -396,84 +547,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
-        uint8_t *stage_buf = smem + L::kOffEpi + (warp - 2) * kEpiChunkBytes;
-        uint32_t amax = 0;
+        uint8_t *bufs = smem + L::kOffEpi + (warp - 2) * L::kEpiBufs * kEpiChunkBytes;
+        uint32_t amax = 0, nstore = 0;
         float scale = 1.0f;
         if (FMT == 3) scale = (*p.ga) * (*p.gb);
         int it = 0;
-        constexpr int kChunksPerTile = BN / 32;
-        constexpr int kOverlapChunks = (BN - L::kAccStride) / 32;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             int m0, n0;
             tile_coords(tile, p.m_blocks, m0, n0, BN);
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
-            const int row = m0 + 32 * q + lane;
-            const int n_valid = p.N - n0;
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
-            for (int idx = 0; idx < kChunksPerTile; ++idx) {
-                if (idx == kOverlapChunks) {
-                    // the shared columns are in registers: let the next tile's MMAs start
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(acc_empty);
-                }
-                // buffer 0 drains its tail (shared with buffer 1) first
-                const int c = (b == 0) ? (idx + (kChunksPerTile - kOverlapChunks)) % kChunksPerTile : idx;
-                const int col = 32 * c;
-                if (col >= n_valid) continue;  // warp-uniform
-                uint32_t r[32];
-                tmem_ld32(t_acc + (uint32_t)col, r);
-                tmem_wait_ld();
-                uint32_t packed[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float x0 = __uint_as_float(r[2 * i]) * scale, x1 = __uint_as_float(r[2 * i + 1]) * scale;
-                    if (p.epilogue == 1) {
-                        x0 = gelu_erf(x0);
-                        x1 = gelu_erf(x1);
-                    }
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-                    packed[i] = *reinterpret_cast<const uint32_t *>(&h);
-                }
-                if (p.amax_out != nullptr && row < p.M) {
-                    const int valid = min(32, n_valid - col);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < valid) amax = max(amax, (packed[i >> 1] >> (16 * (i & 1))) & 0x7FFFu);
-                }
-                if (m0 + 32 * q >= p.M) continue;  // warp-uniform: no rows of this quadrant exist
-                if (p.use_tma_store) {
-                    if (lane == 0) bulk_wait_group_read<0>();  // staging buffer free again
-                    __syncwarp();
-                    uint4 *dst = reinterpret_cast<uint4 *>(stage_buf + lane * 64);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmC, n0 + col, m0 + 32 * q, stage_buf);
-                        bulk_commit_group();
-                    }
-                } else if (row < p.M) {
-                    uint16_t *dst = p.C + (int64_t)row * p.ldc + n0 + col;
-                    for (int i = 0; i < 32 && col + i < n_valid; ++i) dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
-                }
-            }
-            if (kOverlapChunks >= kChunksPerTile) {  // (not reached for the tile shapes used)
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
-            }
+            epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
+                                             [&] {
+                                                 if (lane == 0) mbar_arrive(acc_empty);
+                                             });
         }
-        if (lane == 0) bulk_wait_group_all();
-        if (p.amax_out != nullptr) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            if (lane == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int *>(p.amax_out), amax << 16);
-        }
+        epilogue_finish(p, lane, amax);
     }
 
     tc_fence_before();

@@ -137,7 +137,7 @@ template <int FMT, int BN, int STAGES>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                         const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
     using L = GemmSmem<FMT, BN, STAGES>;
-    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K * fmt_bits(FMT) / 8;
     CUtensorMap ta, tb, tc;
@@ -184,7 +184,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
                              const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out,
                              cudaStream_t st) {
     using L = PairSmem<FMT, STAGES>;
-    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K * fmt_bits(FMT) / 8;
     CUtensorMap ta, tb, tc;
@@ -243,7 +243,7 @@ template <int FMT>
 mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                           const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
     if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load())
-        return launch_gemm_pair_t<FMT, FMT == 3 ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+        return launch_gemm_pair_t<FMT, (FMT == 2 || FMT == 3) ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
 }
