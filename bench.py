@@ -275,9 +275,14 @@ def extras_gpu(device):
         xs = [torch.randn((M, K), generator=g, device=device).to(torch.bfloat16) for _ in range(min(n, 8))]
         for fmt in (0, 2, 3):
             qs = [mx.empty(fmt, M, K) for _ in xs]
-            gs = torch.ones(1, device=device)
-            ms = timed(lambda i: mx.quantize(xs[i % len(xs)], fmt, out=qs[i % len(xs)],
-                                             gscale=gs if fmt == 3 else None), len(xs))
+            # NVFP4 with its per-tensor scale known (as for weights): g = RU(amax / 2688)
+            # of each input, from one untimed call with the amax pre-pass
+            gss = [None] * len(xs)
+            if fmt == 3:
+                for i, x in enumerate(xs):
+                    gss[i] = mx.quantize(x, fmt, out=qs[i]).gscale.clone()
+            ms = timed(lambda i: mx.quantize(xs[i % len(xs)], fmt, out=qs[i % len(xs)], gscale=gss[i % len(xs)]),
+                       len(xs))
             gbs = M * K * quant_bytes_per_elem(fmt) / (ms * 1e-3) / 1e9
             sweep[f"{['mxfp8_e4m3', 'e5m2', 'mxfp4', 'nvfp4'][fmt]}_M{M}"] = {
                 "us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
@@ -397,9 +402,9 @@ def run_profile_case(name: str, reps: int = 4):
     x = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
     if kind == "quant":
         q = mx.empty(fmt, M, K)
-        gs = torch.ones(1, device="cuda")
+        gs = mx.quantize(x, fmt, out=q).gscale.clone() if fmt == 3 else None   # NVFP4: g of this input
         for _ in range(reps):
-            mx.quantize(x, fmt, out=q, gscale=gs if fmt == 3 else None)
+            mx.quantize(x, fmt, out=q, gscale=gs)
     else:
         w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
         qa, qw = mx.quantize(x, fmt), mx.quantize(w, fmt)

@@ -138,60 +138,60 @@ MX_DEVICE_INLINE float e2m1_mag(uint32_t c) {
     return c < 2u ? 0.5f * (float)c : __uint_as_float(((c >> 1) + 126u) << 23) * (1.0f + 0.5f * (float)(c & 1u));
 }
 
-// Eight fp32 -> eight E2M1 codes packed (element i in nibble i), RNE, saturating;
-// a value that rounds to zero keeps its sign (the conversion does this).
-// (cvt8_e2m1 above.)
-
 // NVFP4 elements: codes of x / (g s) for 16 values, the exact RNE of the real
-// quotient.  r_lo <= 1/(g s) <= r_hi.  lo = x * r_lo rounded toward zero keeps
-// the sign and bounds |x| / (g s) from below; hi = |x| * r_hi rounded up bounds
-// it from above.  Where the two give the same E2M1 magnitude, that code (with
-// lo's sign) is exact, because RNE is monotone.  Elsewhere the magnitude is
-// walked up from lo's, deciding each midpoint m by the sign of |x| - g*s*m,
-// which one fma computes exactly (s*m is exact in fp32); ties go to the even
-// code.  The walk uses registers only.
+// quotient q.  r_lo <= 1/(g s) <= r_hi.  lo = x * r_lo rounded toward zero
+// keeps the sign and bounds |q| from below; hi = |x| * r_hi rounded up bounds
+// it from above.  RNE is monotone, so the code lies between lo's and hi's;
+// the bracket is a few ulps wide, so they differ by at most one step, and
+// only when a midpoint m between the two codes lies inside it.  Such an
+// element (typically a tie: bf16 inputs divided by a short scale often land
+// exactly on a midpoint) is settled by the sign of |x| - g*s*m, which one fma
+// computes exactly (s*m is exact in fp32); a tie goes to the even code.
+
+// Midpoint between E2M1 magnitudes c and c + 1 (c = 0..6).
+MX_DEVICE_INLINE float e2m1_mid(uint32_t c) {
+    return c < 4u ? 0.25f + 0.5f * (float)c : (c < 6u ? (float)c - 1.5f : 5.0f);
+}
+
+// Settle the elements of one packed word (8 codes) whose bracket straddles a
+// midpoint.  diff has a nonzero nibble where lo's and hi's magnitudes differ;
+// w0..w3 hold the word's 8 bf16 inputs (element 2j in the low half of wj).
+MX_DEVICE_INLINE uint32_t nv_settle(uint32_t code, uint32_t diff, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                    float g, float s) {
+    while (diff != 0u) {
+        const int nib = (__ffs(diff) - 1) >> 2;
+        diff &= ~(0xFu << (4 * nib));
+        const int j = nib >> 1;
+        const uint32_t wj = j == 0 ? w0 : (j == 1 ? w1 : (j == 2 ? w2 : w3));
+        const float ax = fabsf((nib & 1) ? __uint_as_float(wj & 0xFFFF0000u) : __uint_as_float(wj << 16));
+        const uint32_t c = (code >> (4 * nib)) & 7u;                  // lo's magnitude, < hi's <= 7
+        const float d = __fmaf_rn(-g, s * e2m1_mid(c), ax);           // sign(|x| - g*s*mid)
+        if (d > 0.0f || (d == 0.0f && (c & 1u))) code += 1u << (4 * nib);
+    }
+    return code;
+}
+
 MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, float s, float r_lo, float r_hi,
                                  uint32_t &out0, uint32_t &out1) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        x[2 * i] = bf16lo(w[i]);
-        x[2 * i + 1] = bf16hi(w[i]);
-    }
     float lo[16], hi[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        lo[i] = __fmul_rz(x[i], r_lo);
-        hi[i] = __fmul_ru(fabsf(x[i]), r_hi);
+    for (int i = 0; i < 8; ++i) {
+        const float a = bf16lo(w[i]), b = bf16hi(w[i]);
+        lo[2 * i] = __fmul_rz(a, r_lo);
+        lo[2 * i + 1] = __fmul_rz(b, r_lo);
+        hi[2 * i] = __fmul_ru(fabsf(a), r_hi);
+        hi[2 * i + 1] = __fmul_ru(fabsf(b), r_hi);
     }
     const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
     const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
     const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
     const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
     uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
-    const uint32_t h0 = cvt8_e2m1(hi0), h1 = cvt8_e2m1(hi1);
-    if (((c0 & 0x77777777u) != h0) || ((c1 & 0x77777777u) != h1)) {
-        uint32_t f0 = 0, f1 = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t cl = i < 8 ? c0 : c1, ch = i < 8 ? h0 : h1;
-            const int sh = 4 * (i & 7);
-            uint32_t c = (cl >> sh) & 7u;
-            const uint32_t b = (ch >> sh) & 7u;
-            const float ax = fabsf(x[i]);
-            while (c < b) {
-                const float mid = 0.5f * (e2m1_mag(c) + e2m1_mag(c + 1u));   // 3 significant bits
-                const float d = __fmaf_rn(-g, s * mid, ax);                   // sign(|x| - g*s*mid)
-                if (d > 0.0f || (d == 0.0f && (c & 1u))) ++c;
-                else break;
-            }
-            const uint32_t nib = (c | ((cl >> sh) & 8u)) << sh;
-            if (i < 8) f0 |= nib;
-            else f1 |= nib;
-        }
-        c0 = f0;
-        c1 = f1;
+    const uint32_t d0 = (c0 & 0x77777777u) ^ cvt8_e2m1(hi0), d1 = (c1 & 0x77777777u) ^ cvt8_e2m1(hi1);
+    if ((d0 | d1) != 0u) {
+        c0 = nv_settle(c0, d0, w[0], w[1], w[2], w[3], g, s);
+        c1 = nv_settle(c1, d1, w[4], w[5], w[6], w[7], g, s);
     }
     out0 = c0;
     out1 = c1;
