@@ -6,17 +6,17 @@
 // (a cluster of 2) compute a 256 x 256 output tile with M = 256 MMAs: each CTA
 // loads its own 128 rows of A and its own 128-row half of B, and the tensor
 // core reads B from both CTAs' shared memory.  Per SM that is half the B
-// traffic of a 128 x 256 tile for the same MMA work, which keeps the L2 -> SM
-// traffic under the fabric's bandwidth at full MMA rate.  No load is multicast.
+// traffic of a 128 x 256 tile for the same MMA work.  No load is multicast.
 //
-// Roles per CTA (10 warps), as in the single-CTA kernel:
-//   warp 0     TMA producer: own A rows and B half (completion counted on the
-//              leader CTA's barrier), own scale tiles (local barrier);
-//   warps 6-9  scale warps: this CTA's TMEM gets the scales of its 128 A rows
-//              and of all 256 B rows, via tcgen05.st, ahead of the MMAs; the
-//              leader's also wait for the pair's code tiles, so the MMA thread
-//              checks one barrier per stage;
-//   warp 1     leader CTA only: issues the pair's MMAs; commits fan out to the
+// Roles per CTA (11 warps), as in the single-CTA kernel:
+//   warp 0     code-tile producer: own A rows and B half, completion counted
+//              on the leader CTA's barrier;
+//   warp 10    scale-tile producer: own A band and both B bands (this CTA's
+//              TMEM needs the scales of all 256 B rows), local barriers;
+//   warps 6-9  scale warps: this CTA's TMEM slot, then an arrive on the
+//              leader's slot barrier (8 arrivals: both CTAs' scale warps);
+//   warp 1     leader CTA only: issues the pair's MMAs once the pair's code
+//              tiles and both CTAs' scale slots are in; commits fan out to the
 //              barriers of both CTAs;
 //   warps 2-5  epilogue for this CTA's 128 rows of the tile.
 // Every mbarrier wait is bounded; both CTAs meet at a cluster barrier before
@@ -27,77 +27,30 @@
 
 namespace mx {
 
+// Per CTA: 128 rows of A and 128 rows of B in smem per stage, scale tiles of
+// two B bands, a 256-column accumulator.
 template <int FMT, int STAGES>
-struct PairSmem {
-    using F = GemmFmt<FMT>;
-    static constexpr int BN = 256;  // pair tile is 256 x 256
-    static constexpr int kABytes = 128 * kStageKBytes;
-    static constexpr int kBBytes = 128 * kStageKBytes;
-    static constexpr int kSfaBytes = F::kChunks * 512;
-    static constexpr int kSfbBytes = F::kChunks * 512 * 2;
-    static constexpr int kOffA = 0;
-    static constexpr int kOffB = kOffA + STAGES * kABytes;
-    static constexpr int kOffEpi = kOffB + STAGES * kBBytes;
-    static constexpr int kNoEpi = STAGES * (kABytes + kBBytes + kSfaBytes + kSfbBytes) + (3 * STAGES + 4 + 2 * kSfSlots) * 8 +
-                                  16 + 1024;
-    static constexpr int kEpiBufs = (kNoEpi + kEpiWarps * 2 * kEpiChunkBytes <= kSmemLimit) ? 2 : 1;
-    static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiBufs * kEpiChunkBytes;
-    static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
-    static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
-    // full[S] (leader's counts both CTAs' code tiles), empty[S], sfload[S],
-    // acc_full[2], acc_empty, mma_done, sf_full[slots], sf_empty[slots]
-    static constexpr int kNumBars = 3 * STAGES + 4 + 2 * kSfSlots;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kBytes = kOffMisc + 16;
-    static constexpr int kAlloc = kBytes + 1024;
-    // TMEM (per CTA) as in the single-CTA kernel with BN = 256.
-    using T = GemmSmem<FMT, 256, 1>;
-    static constexpr int kTmemCols = 512;
-    static constexpr int kSfSlotCols = T::kSfSlotCols;
-    static constexpr int kAccStride = T::kAccStride;
-    static constexpr int kTmemSf = T::kTmemSf;
-};
-
-template <int FMT>
-MX_DEVICE_INLINE uint32_t pair_idesc(uint32_t sf_id) {
-    using F = GemmFmt<FMT>;
-    return (sf_id << 4) | (F::kAFmt << 7) | (F::kAFmt << 10) | ((uint32_t)(256 >> 3) << 17) |
-           (F::kScaleUE8M0 << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
-}
-
-template <int FMT>
-MX_DEVICE_INLINE void pair_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
-                               uint32_t acc) {
-    if (FMT <= 1) tc_mma_pair_mxf8f6f4(d, a, b, idesc, sfa, sfb, acc);
-    else if (FMT == 2) tc_mma_pair_mxf4(d, a, b, idesc, sfa, sfb, acc);
-    else tc_mma_pair_nvf4(d, a, b, idesc, sfa, sfb, acc);
-}
-
-template <int FMT>
-MX_DEVICE_INLINE void pair_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
-                                  uint32_t acc, uint32_t issue) {
-    if (FMT <= 1) tc_mma_pair_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
-    else if (FMT == 2) tc_mma_pair_mxf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
-    else tc_mma_pair_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
-}
+using PairSmem = GemmLayout<FMT, 2, 128, STAGES>;
 
 template <int FMT, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSfa,
+                     const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = PairSmem<FMT, STAGES>;
     static_assert(STAGES >= kSfSlots, "scale slots are recycled through the stage barriers");
+    static_assert((kSfSlots & (kSfSlots - 1)) == 0, "scale slots: a power of two");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);  // leader's count both CTAs' code tiles
     uint64_t *empty = full + STAGES;
-    uint64_t *sfload = empty + STAGES;
-    uint64_t *acc_full = sfload + STAGES;  // [2]
+    uint64_t *sfload = empty + STAGES;          // [kSfGroups]
+    uint64_t *sfree = sfload + L::kSfGroups;    // [kSfGroups]
+    uint64_t *acc_full = sfree + L::kSfGroups;  // [2]
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *mma_done = acc_empty + 1;
-    uint64_t *sf_full = mma_done + 1;         // [kSfSlots]
-    uint64_t *sf_empty = sf_full + kSfSlots;  // [kSfSlots]
+    uint64_t *sf_full = mma_done + 1;           // [kSfSlots], leader's count both CTAs' scale warps
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -110,20 +63,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&sfload[s], 1);
+        }
+        for (int g = 0; g < L::kSfGroups; ++g) {
+            mbar_init(&sfload[g], 1);
+            mbar_init(&sfree[g], 4);
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         mbar_init(acc_empty, 2 * kEpiWarps);
         mbar_init(mma_done, 1);
-        for (int i = 0; i < kSfSlots; ++i) {
-            mbar_init(&sf_full[i], 8);
-            mbar_init(&sf_empty[i], 1);
-        }
+        for (int i = 0; i < kSfSlots; ++i) mbar_init(&sf_full[i], 8);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmSfa);
+        tma_prefetch_desc(&tmSfb);
         if (p.use_tma_store) tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
@@ -137,77 +92,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ code-tile producer
         if (!p.skip_producer) {
-            const int n_bands_total = (p.N + 127) / 128;
-            const int m_bands_total = (p.M + 127) / 128;
-            int last_kg = -1;
-            int kg = 0;
+            const uint32_t full_leader0 = mapa_shared(smem_u32(&full[0]), 0);
+            int used = 0, s = 0;
+            uint32_t ph = 0;
             bool stop = false;
             for (int tile = pair; tile < num_tiles && !stop; tile += npairs) {
                 int m0, n0;
                 tile_coords(tile, p.m_blocks, m0, n0, 256);
                 m0 = (tile % p.m_blocks) * 256;
                 const int my_m = m0 + 128 * (int)rank, my_n = n0 + 128 * (int)rank;
-                const bool sfa_exists = my_m / 128 < m_bands_total;
-                const int bands = min(2, n_bands_total - n0 / 128);
-                const uint8_t *sfa_row = p.sfa + (int64_t)(my_m / 128) * p.sf_tiles_k * 512;
-                const uint8_t *sfb_row = p.sfb + (int64_t)(n0 / 128) * p.sf_tiles_k * 512;
-                for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
-                    const int s = kg % STAGES, round = kg / STAGES;
-                    if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY,
-                                           abort_flag)) {
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY, abort_flag)) {
                         stop = true;
                         break;
                     }
-                    int n_mma, n_chunk;
-                    stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                    const uint32_t sf_bytes = (uint32_t)n_chunk * 512u;
-                    const int64_t sf_k = (int64_t)kt * F::kChunks * 512;
                     if (lane == 0) {
-                        const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
+                        const uint32_t full_leader = full_leader0 + 8u * (uint32_t)s;
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (L::kABytes + L::kBBytes));
                         tma_load_2d_pair(smem + L::kOffA + s * L::kABytes, &tmA, kt * kStageKBytes, my_m, full_leader);
                         tma_load_2d_pair(smem + L::kOffB + s * L::kBBytes, &tmB, kt * kStageKBytes, my_n, full_leader);
-                        mbar_arrive_expect_tx(&sfload[s], sf_bytes * ((sfa_exists ? 1u : 0u) + (uint32_t)bands));
-                        if (sfa_exists)
-                            bulk_load(smem + L::kOffSfa + s * L::kSfaBytes, sfa_row + sf_k, sf_bytes, &sfload[s]);
-                        for (int h = 0; h < bands; ++h)
-                            bulk_load(smem + L::kOffSfb + s * L::kSfbBytes + h * F::kChunks * 512,
-                                      sfb_row + (int64_t)h * p.sf_tiles_k * 512 + sf_k, sf_bytes, &sfload[s]);
                     }
                     __syncwarp();
-                    last_kg = kg;
+                    ++used;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             // Do not leave while copies into shared memory are in flight.  The
-            // leader's full barriers count both CTAs' code tiles.
-            for (int k = max(0, last_kg - STAGES + 1); k <= last_kg; ++k) {
-                if (rank == 0)
-                    mbar_wait_bounded(&full[k % STAGES], (k / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
-                mbar_wait_bounded(&sfload[k % STAGES], (k / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
-            }
+            // leader's full barriers count both CTAs' code tiles; the other CTA
+            // stays until the closing cluster barrier, which the leader reaches
+            // only after these waits.
+            if (rank == 0)
+                for (int u = max(0, used - STAGES); u < used; ++u)
+                    mbar_wait_bounded(&full[u % STAGES], (uint32_t)((u / STAGES) & 1), p.wait_limit_ns, SITE_GEMM_TAIL,
+                                      nullptr);
         }
+    } else if (warp == kSfWarp) {
+        // ------------------------------------------------------------ scale-tile producer
+        if (!p.skip_producer)
+            sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, pair, npairs, num_tiles,
+                                [&](int tile, int &a_band, int &b_band) {
+                                    int m0, n0;
+                                    tile_coords(tile, p.m_blocks, m0, n0, 256);
+                                    a_band = (tile % p.m_blocks) * 2 + (int)rank;
+                                    b_band = n0 / 128;
+                                },
+                                lane, abort_flag);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader)
         // As in the single-CTA kernel: all lanes walk the loop, lane 0 issues.
         if (rank == 0) {
-            const uint32_t a_base = smem_u32(smem + L::kOffA), b_base = smem_u32(smem + L::kOffB);
             const uint64_t desc_ab = smem_desc(0, 16, 1024, 2);
+            const uint64_t ad0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffA) >> 4) & 0x3FFFu);
+            const uint64_t bd0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffB) >> 4) & 0x3FFFu);
             const uint32_t leader = lane == 0 ? 1u : 0u;
-            int kg = 0;
+            int last_n_mma, last_n_chunk;
+            stage_extent<FMT>(p.num_kt - 1, p.K, last_n_mma, last_n_chunk);
+            int s = 0, slot = 0;        // stage and scale-slot ring positions
+            uint32_t fph = 0, sph = 0;  // parities of the current phases of full[s] and sf_full[slot]
             bool stop = false;
-            bool ready = false;  // result of the last peek at stage kg's barriers
+            bool ready = false;         // result of the last peek at both barriers
             int it = 0;
             for (int tile = pair; tile < num_tiles && !stop; tile += npairs, ++it) {
                 const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
-                for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
-                    const int s = kg % STAGES;
-                    const int slot = kg % kSfSlots;
-                    // sf_full of a stage implies its code tiles have landed: the scale warps
-                    // arrive only after observing the stage's load barrier.
-                    if (!ready && !mbar_wait_bounded(&sf_full[slot], (kg / kSfSlots) & 1, p.wait_limit_ns,
-                                                     SITE_GEMM_MMA_SF, abort_flag)) {
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!ready &&
+                        (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
+                         !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))) {
                         stop = true;
                         break;
                     }
@@ -220,25 +175,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                         tc_fence_after();
                     }
-                    int n_mma, n_chunk;
-                    stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                    const uint32_t a_stage = a_base + s * L::kABytes, b_stage = b_base + s * L::kBBytes;
                     const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
-                    const uint32_t t_sfb = t_sfa + 4 * F::kChunks;
-                    for (int j = 0; j < n_mma; ++j) {
-                        const int chunk = j / F::kMmaPerChunk;
-                        const uint32_t sf_id = (uint32_t)((j % F::kMmaPerChunk) * F::kSfPerMma);
-                        const uint64_t ad = desc_ab | (uint64_t)(((a_stage + 32 * j) >> 4) & 0x3FFFu);
-                        const uint64_t bd = desc_ab | (uint64_t)(((b_stage + 32 * j) >> 4) & 0x3FFFu);
-                        pair_mma_if<FMT>(t_acc, ad, bd, pair_idesc<FMT>(sf_id), t_sfa + 4 * chunk, t_sfb + 8 * chunk,
-                                         (kt > 0 || j > 0) ? 1u : 0u, leader);
-                    }
+                    issue_stage<FMT, true, 256, 8>(kt + 1 < p.num_kt ? 4 : last_n_mma, t_acc,
+                                                   ad0 + (uint64_t)(s * (L::kABytes >> 4)),
+                                                   bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa,
+                                                   t_sfa + 4 * F::kChunks, kt > 0 ? 1u : 0u, leader);
                     // frees both CTAs' smem stage and, for their scale warps, the scale slot
                     tc_commit_pair_if(&empty[s], 0x3, leader);
-                    {
-                        const int k1 = kg + 1;
-                        ready = mbar_test_wait(&sf_full[k1 % kSfSlots], (k1 / kSfSlots) & 1);
+                    if (++s == STAGES) {
+                        s = 0;
+                        fph ^= 1u;
                     }
+                    slot = (slot + 1) & (kSfSlots - 1);
+                    sph ^= (slot == 0) ? 1u : 0u;
+                    ready = mbar_test_wait(&full[s], fph) && mbar_test_wait(&sf_full[slot], sph);
                 }
                 if (!stop) tc_commit_pair_if(&acc_full[it & 1], 0x3, leader);
             }
@@ -248,38 +198,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps
         const int q = warp & 3;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const uint32_t sf_full_leader0 = mapa_shared(smem_u32(&sf_full[0]), 0);
-        int kg = 0;
-        bool stop = false;
-        for (int tile = pair; tile < num_tiles && !stop; tile += npairs) {
-            for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
-                const int s = kg % STAGES, slot = kg % kSfSlots;
-                if (!mbar_wait_bounded(&sfload[s], (kg / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_SF_LOAD, abort_flag) ||
-                    (rank == 0 &&
-                     !mbar_wait_bounded(&full[s], (kg / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_SF_FULL, abort_flag))) {
-                    stop = true;
-                    break;
-                }
-                if (kg >= kSfSlots &&
-                    !mbar_wait_bounded(&empty[(kg - kSfSlots) % STAGES], ((kg - kSfSlots) / STAGES) & 1,
-                                       p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                tc_fence_after();
-                int n_mma, n_chunk;
-                stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                (void)n_chunk;  // tiles past the K tail carry stale scales the MMAs never read
-                stage_scales_to_tmem<F::kChunks, 2>(smem + L::kOffSfa + s * L::kSfaBytes,
-                                                    smem + L::kOffSfb + s * L::kSfbBytes,
-                                                    tmem + lane_base + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols),
-                                                    lane);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot);
-            }
-        }
+        int my_tiles = 0;
+        for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
+        scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
+                              my_tiles, lane, abort_flag,
+                              [&](int slot) { mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot); });
     } else {
         // ------------------------------------------------------------ epilogue (this CTA's 128 rows)
         const int q = warp & 3;
@@ -297,10 +221,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
-            epilogue_tile<256, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
-                                              [&] {
-                                                  if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-                                              });
+            epilogue_tile<256, L::kAccStride, L::kEpiBufs, FMT == 3>(
+                p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
+                [&] {
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+                });
         }
         epilogue_finish(p, lane, amax);
     }

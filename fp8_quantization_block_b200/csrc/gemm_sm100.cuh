@@ -7,26 +7,30 @@
 // applies the block scale during FP32 accumulation).
 //
 // Persistent kernel: one CTA per SM walks output tiles of 128 x BN (tile t,
-// t + gridDim.x, ...) with five warp roles:
-//   warp 0     TMA producer: code tiles of A and B (128-byte swizzled, K-major)
-//              plus their 512-byte scale tiles into a STAGES-deep smem ring
-//              that runs continuously across tiles;
+// t + gridDim.x, ...) with six warp roles:
+//   warp 0     TMA producer of the code tiles of A and B (128-byte swizzled,
+//              K-major) into a STAGES-deep smem ring that runs continuously
+//              across tiles;
+//   warp 10    TMA producer of the 512-byte scale tiles: one 3D copy per
+//              operand brings kSfGroup stages' tiles (all of B's bands) into
+//              a ring of its own, ahead of the scale warps;
 //   warps 6-9  scale warps (one per TMEM lane quadrant): copy each stage's
-//              scale tiles from shared memory into TMEM with tcgen05.st, into
-//              one of two TMEM slots, one stage ahead of the MMAs.  (Staging the
-//              scales with tcgen05.cp instead costs tensor-pipe cycles that do
-//              not overlap the MMAs; register stores from other warps do.)
+//              scale tiles from shared memory into one of kSfSlots TMEM slots
+//              with tcgen05.st, as soon as the MMAs that read the slot's
+//              previous contents have completed.  (Staging the scales with
+//              tcgen05.cp instead costs tensor-pipe cycles that do not overlap
+//              the MMAs; register stores from other warps do.)
 //   warp 1     TMEM owner and MMA issuer: one lane issues the block-scaled
 //              tcgen05.mma instructions (4 per stage, 32 bytes of K each) into
-//              an FP32 accumulator in TMEM; tcgen05.commit frees the smem stage
-//              and the scale slot;
+//              an FP32 accumulator in TMEM once a stage's code tiles and scale
+//              slot are ready; tcgen05.commit frees the smem stage and the slot;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (one row per thread),
 //              x gA*gB for NVFP4, optional GELU and |C| max, bf16 RNE, staged
 //              in shared memory and written with TMA bulk-tensor stores.
 // The two accumulators alternate between tiles so that the epilogue of one
 // tile overlaps the MMAs of the next.  TMEM has 512 columns: the accumulators
 // sit at [0, BN) and [S, S + BN) and share BN - S columns, which the epilogue
-// drains first and then releases; the two scale slots take the columns from
+// drains first and then releases; the scale slots take the columns from
 // S + BN up.  Every mbarrier wait is bounded (mx_common.cuh).
 #pragma once
 
@@ -61,17 +65,17 @@ struct GemmFmt<3> {  // NVFP4: kind::mxf4nvf4, scale_vec 4X (16-element blocks),
 
 constexpr int kBM = 128;
 constexpr int kStageKBytes = 128;
-constexpr int kGemmThreads = 320;
-constexpr int kSfSlots = 4;
+constexpr int kGemmThreads = 352;  // 11 warps
+constexpr int kSfWarp = 10;        // the scale-tile producer
+constexpr int kSfSlots = 4;        // TMEM scale slots (a power of two)
+constexpr int kSfGroup = 2;        // stages per scale-tile copy
 constexpr int kEpiWarps = 4;
 constexpr int kEpiChunkBytes = 32 * 32 * 2;  // 32 rows x 32 bf16 columns per epilogue warp
 constexpr int kSmemLimit = 232448;           // dynamic shared memory per CTA (opt-in maximum)
 
 struct GemmParams {
-    const uint8_t *sfa;
-    const uint8_t *sfb;
-    int64_t sf_tiles_k;  // 512-byte scale tiles per 128-row band (= ceil(K / block / 4))
-    uint16_t *C;         // used by the direct-store epilogue (when TMA stores are not possible)
+    int64_t sf_tiles_k;   // 512-byte scale tiles per 128-row band (= ceil(K / block / 4))
+    uint16_t *C;          // used by the direct-store epilogue (when TMA stores are not possible)
     int64_t ldc;
     int M, N, K;
     int num_kt;           // stages along K = ceil(K_bytes / 128)
@@ -85,39 +89,52 @@ struct GemmParams {
     uint64_t wait_limit_ns;
 };
 
-template <int FMT, int BN, int STAGES>
-struct GemmSmem {
+// Shared-memory and TMEM plan of a CTA whose MMAs read a 128-row A tile and
+// B_BANDS 128-row bands of B per stage (B_ROWS rows of B in this CTA's smem).
+template <int FMT, int B_BANDS, int B_ROWS, int STAGES>
+struct GemmLayout {
     using F = GemmFmt<FMT>;
-    static constexpr int kBBands = BN / 128;
+    static constexpr int kBBands = B_BANDS;
     static constexpr int kABytes = kBM * kStageKBytes;
-    static constexpr int kBBytes = BN * kStageKBytes;
-    static constexpr int kSfaBytes = F::kChunks * 512;
-    static constexpr int kSfbBytes = F::kChunks * 512 * kBBands;
+    static constexpr int kBBytes = B_ROWS * kStageKBytes;
+    // scale tiles of one group: kSfGroup stages x kChunks 512-byte tiles of A's
+    // band, and the same for each of B's bands (band-major)
+    static constexpr int kSfaGroupBytes = kSfGroup * F::kChunks * 512;
+    static constexpr int kSfbGroupBytes = kSfaGroupBytes * B_BANDS;
+    static constexpr int kSfBandStride = kSfaGroupBytes;
+    // full[S], empty[S], sfload[G], sfree[G], acc_full[2], acc_empty, mma_done, sf_full[slots]
+    static constexpr int bytes_for(int groups, int bufs) {
+        return STAGES * (kABytes + kBBytes) + groups * (kSfaGroupBytes + kSfbGroupBytes) +
+               kEpiWarps * bufs * kEpiChunkBytes + (2 * STAGES + 2 * groups + 4 + kSfSlots) * 8 + 16 + 1024;
+    }
+    // as many scale groups in flight, then epilogue staging buffers, as fit
+    static constexpr int kSfGroups = bytes_for(4, 2) <= kSmemLimit ? 4 : (bytes_for(3, 1) <= kSmemLimit ? 3 : 2);
+    static constexpr int kEpiBufs = bytes_for(kSfGroups, 2) <= kSmemLimit ? 2 : 1;
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + STAGES * kABytes;
     static constexpr int kOffEpi = kOffB + STAGES * kBBytes;
-    // two staging buffers per epilogue warp where shared memory allows, else one
-    static constexpr int kNoEpi = STAGES * (kABytes + kBBytes + kSfaBytes + kSfbBytes) + (2 * STAGES + 4 + 2 * kSfSlots) * 8 +
-                                  16 + 1024;
-    static constexpr int kEpiBufs = (kNoEpi + kEpiWarps * 2 * kEpiChunkBytes <= kSmemLimit) ? 2 : 1;
     static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiBufs * kEpiChunkBytes;
-    static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
-    static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
-    // full[S], empty[S], acc_full[2], acc_empty, mma_done, sf_full[2], sf_empty[2]
-    static constexpr int kNumBars = 2 * STAGES + 4 + 2 * kSfSlots;
+    static constexpr int kOffSfb = kOffSfa + kSfGroups * kSfaGroupBytes;
+    static constexpr int kOffBar = kOffSfb + kSfGroups * kSfbGroupBytes;
+    static constexpr int kNumBars = 2 * STAGES + 2 * kSfGroups + 4 + kSfSlots;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+    static_assert(kAlloc <= kSmemLimit, "shared memory budget");
     // TMEM: two accumulators at columns 0 and kAccStride (sharing BN - kAccStride
     // columns), then kSfSlots scale slots of kSfSlotCols columns each.
+    static constexpr int kAccCols = 128 * B_BANDS;  // accumulator columns = N of the MMA
     static constexpr int kTmemCols = 512;
-    static constexpr int kSfSlotCols = 4 * F::kChunks * (1 + kBBands);
-    static constexpr int kAccRoom = kTmemCols - BN - kSfSlots * kSfSlotCols;
-    static constexpr int kAccStride = (kAccRoom >= BN ? BN : kAccRoom) / 32 * 32;
-    static constexpr int kTmemSf = kAccStride + BN;
+    static constexpr int kSfSlotCols = 4 * F::kChunks * (1 + B_BANDS);
+    static constexpr int kAccRoom = kTmemCols - kAccCols - kSfSlots * kSfSlotCols;
+    static constexpr int kAccStride = (kAccRoom >= kAccCols ? kAccCols : kAccRoom) / 32 * 32;
+    static constexpr int kTmemSf = kAccStride + kAccCols;
     static_assert(kAccStride >= 32, "accumulator double buffering needs TMEM room");
     static_assert(kTmemSf + kSfSlots * kSfSlotCols <= kTmemCols, "TMEM budget");
 };
+
+template <int FMT, int BN, int STAGES>
+using GemmSmem = GemmLayout<FMT, BN / 128, BN, STAGES>;
 
 // Instruction descriptor of the block-scaled MMA (M = 128, K-major A and B).
 template <int FMT, int BN>
@@ -143,6 +160,55 @@ MX_DEVICE_INLINE void gemm_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t i
     else tc_mma_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
 }
 
+// Instruction descriptor of the CTA-pair MMA (M = 256 over two CTAs, N = 256).
+template <int FMT>
+MX_DEVICE_INLINE uint32_t pair_idesc(uint32_t sf_id) {
+    using F = GemmFmt<FMT>;
+    return (sf_id << 4) | (F::kAFmt << 7) | (F::kAFmt << 10) | ((uint32_t)(256 >> 3) << 17) |
+           (F::kScaleUE8M0 << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
+}
+
+template <int FMT>
+MX_DEVICE_INLINE void pair_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                  uint32_t acc, uint32_t issue) {
+    if (FMT <= 1) tc_mma_pair_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+    else if (FMT == 2) tc_mma_pair_mxf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+    else tc_mma_pair_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+}
+
+// Issue the MMAs of one stage (n_mma 32-byte K steps: 4, fewer only in a
+// ragged last stage).  ad / bd: descriptors of the stage's A / B tiles;
+// consecutive K steps are 32 bytes (2 descriptor units) apart inside the
+// 128-byte swizzle atom.  SFB_STEP: TMEM columns per scale chunk of B (4 per
+// 128-row band).  With n_mma == 4 the loop unrolls and every operand but the
+// stage's bases folds to a constant, keeping the issuing thread's per-stage
+// instruction chain short.
+template <int FMT, bool PAIR, int BN, int SFB_STEP>
+MX_DEVICE_INLINE void issue_one(int j, uint32_t t_acc, uint64_t ad, uint64_t bd, uint32_t t_sfa, uint32_t t_sfb,
+                                uint32_t acc, uint32_t issue) {
+    using F = GemmFmt<FMT>;
+    const int chunk = j / F::kMmaPerChunk;
+    const uint32_t sf_id = (uint32_t)((j % F::kMmaPerChunk) * F::kSfPerMma);
+    const uint32_t a = acc | (j > 0 ? 1u : 0u);
+    if (PAIR)
+        pair_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, pair_idesc<FMT>(sf_id), t_sfa + 4 * chunk,
+                         t_sfb + SFB_STEP * chunk, a, issue);
+    else
+        gemm_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, gemm_idesc<FMT, BN>(sf_id), t_sfa + 4 * chunk,
+                         t_sfb + SFB_STEP * chunk, a, issue);
+}
+
+template <int FMT, bool PAIR, int BN, int SFB_STEP>
+MX_DEVICE_INLINE void issue_stage(int n_mma, uint32_t t_acc, uint64_t ad, uint64_t bd, uint32_t t_sfa, uint32_t t_sfb,
+                                  uint32_t acc, uint32_t issue) {
+    if (n_mma == 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) issue_one<FMT, PAIR, BN, SFB_STEP>(j, t_acc, ad, bd, t_sfa, t_sfb, acc, issue);
+    } else {
+        for (int j = 0; j < n_mma; ++j) issue_one<FMT, PAIR, BN, SFB_STEP>(j, t_acc, ad, bd, t_sfa, t_sfb, acc, issue);
+    }
+}
+
 MX_DEVICE_INLINE float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752440f)); }
 
 // Number of valid 32-byte MMA steps and 512-byte scale chunks in stage kt.
@@ -161,8 +227,8 @@ MX_DEVICE_INLINE void stage_extent(int kt, int K, int &n_mma, int &n_chunk) {
 // slot of this warp's 32 lanes.  Lane r loads row r (16 bytes = 4 columns) of
 // every 512-byte tile first, then writes them with wide tcgen05.st.  Slot
 // layout: A tiles c at columns 4c; B tiles (c, band h) at 4*kChunks + 4*(c*bands + h).
-// smem B tiles are stored band-major: (h * kChunks + c) * 512.
-template <int CHUNKS, int BANDS>
+// smem B tiles of band h start BAND_STRIDE bytes after those of band h - 1.
+template <int CHUNKS, int BANDS, int BAND_STRIDE>
 MX_DEVICE_INLINE void stage_scales_to_tmem(const uint8_t *sfa_stage, const uint8_t *sfb_stage, uint32_t t_slot,
                                            int lane) {
     uint32_t a[4 * CHUNKS];
@@ -173,7 +239,7 @@ MX_DEVICE_INLINE void stage_scales_to_tmem(const uint8_t *sfa_stage, const uint8
         a[4 * c] = v.x, a[4 * c + 1] = v.y, a[4 * c + 2] = v.z, a[4 * c + 3] = v.w;
 #pragma unroll
         for (int h = 0; h < BANDS; ++h) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(sfb_stage + (h * CHUNKS + c) * 512 + lane * 16);
+            const uint4 w = *reinterpret_cast<const uint4 *>(sfb_stage + h * BAND_STRIDE + c * 512 + lane * 16);
             const int o = 4 * (c * BANDS + h);
             b[o] = w.x, b[o + 1] = w.y, b[o + 2] = w.z, b[o + 3] = w.w;
         }
@@ -198,6 +264,98 @@ MX_DEVICE_INLINE void stage_scales_to_tmem(const uint8_t *sfa_stage, const uint8
         tmem_st4(tb, b[0], b[1], b[2], b[3]);
     }
     tmem_wait_st();
+}
+
+// ---------------------------------------------------------------- scale-tile roles
+// Producer of scale tiles (one warp; lane 0 issues): for each tile of this CTA
+// (bands_of(tile, a_band, b_band)), one 3D TMA copy per operand and group of
+// kSfGroup stages into ring slot g, once the scale warps have freed it.
+// Coordinates past the scale buffer (a ragged K or N) read zeros.
+template <typename L, typename BandsOf>
+MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *tmSfa, const CUtensorMap *tmSfb,
+                                       uint8_t *smem, uint64_t *sfload, uint64_t *sfree, int tile0, int tile_step,
+                                       int num_tiles, BandsOf bands_of, int lane, volatile int *abort_flag) {
+    constexpr int NG = L::kSfGroups;
+    constexpr int kChunks = L::F::kChunks;
+    int used = 0, g = 0;
+    uint32_t ph = 0;
+    bool stop = false;
+    for (int tile = tile0; tile < num_tiles && !stop; tile += tile_step) {
+        int a_band, b_band;
+        bands_of(tile, a_band, b_band);
+        for (int kt0 = 0; kt0 < p.num_kt; kt0 += kSfGroup) {
+            if (!mbar_wait_bounded(&sfree[g], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_SF_FREE, abort_flag)) {
+                stop = true;
+                break;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sfload[g], (uint32_t)(L::kSfaGroupBytes + L::kSfbGroupBytes));
+                tma_load_3d(smem + L::kOffSfa + g * L::kSfaGroupBytes, tmSfa, 0, kt0 * kChunks, a_band, &sfload[g]);
+                tma_load_3d(smem + L::kOffSfb + g * L::kSfbGroupBytes, tmSfb, 0, kt0 * kChunks, b_band, &sfload[g]);
+            }
+            __syncwarp();
+            ++used;
+            if (++g == NG) {
+                g = 0;
+                ph ^= 1u;
+            }
+        }
+    }
+    // Do not leave while copies into shared memory are in flight.
+    for (int u = max(0, used - NG); u < used; ++u)
+        mbar_wait_bounded(&sfload[u % NG], (uint32_t)((u / NG) & 1), p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
+}
+
+// Scale warps (one per TMEM lane quadrant; lane r handles TMEM lane 32q + r):
+// for every stage of this CTA's tiles, wait for its scale group in smem and
+// for the MMAs that last read the TMEM slot (stage kg - kSfSlots, whose
+// commit completes empty[]), then write the slot and report it with
+// arrive_full(slot).  After a group's last stage the warp frees the group.
+template <typename L, int STAGES, typename ArriveFull>
+MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *sfload, uint64_t *sfree, uint64_t *empty,
+                                 uint32_t t_sf0, int my_tiles, int lane, volatile int *abort_flag,
+                                 ArriveFull arrive_full) {
+    constexpr int NG = L::kSfGroups;
+    constexpr int kChunks = L::F::kChunks;
+    int g = 0, slot = 0, e = 0;
+    uint32_t gph = 0, eph = 0;
+    int kg = 0;
+    bool stop = false;
+    for (int t = 0; t < my_tiles && !stop; ++t) {
+        for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
+            const int gi = kt % kSfGroup;
+            if (gi == 0 && !mbar_wait_bounded(&sfload[g], gph, p.wait_limit_ns, SITE_GEMM_SF_LOAD, abort_flag)) {
+                stop = true;
+                break;
+            }
+            if (kg >= kSfSlots) {
+                if (!mbar_wait_bounded(&empty[e], eph, p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (++e == STAGES) {
+                    e = 0;
+                    eph ^= 1u;
+                }
+            }
+            tc_fence_after();
+            stage_scales_to_tmem<kChunks, L::kBBands, L::kSfBandStride>(
+                smem + L::kOffSfa + g * L::kSfaGroupBytes + gi * kChunks * 512,
+                smem + L::kOffSfb + g * L::kSfbGroupBytes + gi * kChunks * 512, t_sf0 + (uint32_t)(slot * L::kSfSlotCols),
+                lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_full(slot);
+            slot = (slot + 1) & (kSfSlots - 1);
+            if (gi == kSfGroup - 1 || kt == p.num_kt - 1) {
+                if (lane == 0) mbar_arrive(&sfree[g]);
+                if (++g == NG) {
+                    g = 0;
+                    gph ^= 1u;
+                }
+            }
+        }
+    }
 }
 
 MX_DEVICE_INLINE void tile_coords(int tile, int m_blocks, int &m0, int &n0, int bn) {
@@ -284,7 +442,7 @@ MX_DEVICE_INLINE void epilogue_tile_t(const GemmParams &p, const CUtensorMap *tm
     constexpr int kOv = (BN - ACC_STRIDE) / 32;
     static_assert(kOv >= 0 && kOv <= kChunks, "accumulator overlap");
     const int n_valid = p.N - n0;
-    if (GELU) {
+    if constexpr (GELU) {
         // GELU needs more live registers per chunk: drain in order, releasing
         // after the shared chunks have been written out.
         for (int idx = 0; idx < kChunks; ++idx) {
@@ -304,28 +462,28 @@ MX_DEVICE_INLINE void epilogue_tile_t(const GemmParams &p, const CUtensorMap *tm
             __syncwarp();
             release();
         }
-        return;
-    }
-    uint32_t ov[kOv > 0 ? kOv : 1][16];
+    } else {
+        uint32_t ov[kOv > 0 ? kOv : 1][16];
 #pragma unroll
-    for (int i = 0; i < kOv; ++i) {
-        const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
-        if (col < n_valid) epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, ov[i]);
-    }
-    tc_fence_before();
-    __syncwarp();
-    release();
+        for (int i = 0; i < kOv; ++i) {
+            const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
+            if (col < n_valid) epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, ov[i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        release();
 #pragma unroll
-    for (int i = 0; i < kOv; ++i) {
-        const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
-        if (col < n_valid) epi_emit<NBUF>(p, tmC, ov[i], m0q, n0, col, lane, bufs, nstore, amax);
-    }
-    for (int i = 0; i < kChunks - kOv; ++i) {
-        const int col = 32 * ((b == 0) ? i : (kOv + i));
-        if (col >= n_valid) break;  // warp-uniform; columns ascend
-        uint32_t packed[16];
-        epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
-        epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+        for (int i = 0; i < kOv; ++i) {
+            const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
+            if (col < n_valid) epi_emit<NBUF>(p, tmC, ov[i], m0q, n0, col, lane, bufs, nstore, amax);
+        }
+        for (int i = 0; i < kChunks - kOv; ++i) {
+            const int col = 32 * ((b == 0) ? i : (kOv + i));
+            if (col >= n_valid) break;  // warp-uniform; columns ascend
+            uint32_t packed[16];
+            epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
+            epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+        }
     }
 }
 
@@ -354,19 +512,22 @@ MX_DEVICE_INLINE void epilogue_finish(const GemmParams &p, int lane, uint32_t am
 template <int FMT, int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmC, GemmParams p) {
+                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSfa,
+                const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = GemmSmem<FMT, BN, STAGES>;
     static_assert(STAGES >= kSfSlots, "scale slots are recycled through the stage barriers");
+    static_assert((kSfSlots & (kSfSlots - 1)) == 0, "scale slots: a power of two");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *empty = full + STAGES;
-    uint64_t *acc_full = empty + STAGES;  // [2]
+    uint64_t *sfload = empty + STAGES;           // [kSfGroups]
+    uint64_t *sfree = sfload + L::kSfGroups;     // [kSfGroups]
+    uint64_t *acc_full = sfree + L::kSfGroups;   // [2]
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *mma_done = acc_empty + 1;
-    uint64_t *sf_full = mma_done + 1;      // [kSfSlots]
-    uint64_t *sf_empty = sf_full + kSfSlots;  // [kSfSlots]
+    uint64_t *sf_full = mma_done + 1;            // [kSfSlots]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -378,18 +539,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int g = 0; g < L::kSfGroups; ++g) {
+            mbar_init(&sfload[g], 1);
+            mbar_init(&sfree[g], 4);
+        }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         mbar_init(acc_empty, kEpiWarps);
         mbar_init(mma_done, 1);
-        for (int i = 0; i < kSfSlots; ++i) {
-            mbar_init(&sf_full[i], 4);
-            mbar_init(&sf_empty[i], 1);
-        }
+        for (int i = 0; i < kSfSlots; ++i) mbar_init(&sf_full[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmSfa);
+        tma_prefetch_desc(&tmSfb);
         if (p.use_tma_store) tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
@@ -402,71 +566,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ code-tile producer
         // The whole warp walks the loop (all values warp-uniform); lane 0
         // issues the copies.
         if (!p.skip_producer) {
-            const int n_bands_total = (p.N + 127) / 128;
-            int last_kg = -1;
-            int kg = 0;
+            int used = 0, s = 0;
+            uint32_t ph = 0;
             bool stop = false;
             for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
                 int m0, n0;
                 tile_coords(tile, p.m_blocks, m0, n0, BN);
-                const int bands = min(L::kBBands, n_bands_total - n0 / 128);
-                const uint8_t *sfa_row = p.sfa + (int64_t)(m0 / 128) * p.sf_tiles_k * 512;
-                const uint8_t *sfb_row = p.sfb + (int64_t)(n0 / 128) * p.sf_tiles_k * 512;
-                for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
-                    const int s = kg % STAGES, round = kg / STAGES;
-                    if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY,
-                                           abort_flag)) {
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY, abort_flag)) {
                         stop = true;
                         break;
                     }
-                    int n_mma, n_chunk;
-                    stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                    const uint32_t sf_bytes = (uint32_t)n_chunk * 512u;
-                    const uint32_t bytes = L::kABytes + L::kBBytes + sf_bytes * (1u + (uint32_t)bands);
-                    const int64_t sf_k = (int64_t)kt * F::kChunks * 512;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&full[s], bytes);
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)(L::kABytes + L::kBBytes));
                         tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, kt * kStageKBytes, m0, &full[s]);
                         tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, kt * kStageKBytes, n0, &full[s]);
-                        bulk_load(smem + L::kOffSfa + s * L::kSfaBytes, sfa_row + sf_k, sf_bytes, &full[s]);
-                        for (int h = 0; h < bands; ++h)
-                            bulk_load(smem + L::kOffSfb + s * L::kSfbBytes + h * F::kChunks * 512,
-                                      sfb_row + (int64_t)h * p.sf_tiles_k * 512 + sf_k, sf_bytes, &full[s]);
                     }
                     __syncwarp();
-                    last_kg = kg;
+                    ++used;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             // Do not leave while copies into this CTA's shared memory are in flight:
             // wait for the last fill of every stage that was used.
-            for (int k = max(0, last_kg - STAGES + 1); k <= last_kg; ++k)
-                mbar_wait_bounded(&full[k % STAGES], (k / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
+            for (int u = max(0, used - STAGES); u < used; ++u)
+                mbar_wait_bounded(&full[u % STAGES], (uint32_t)((u / STAGES) & 1), p.wait_limit_ns, SITE_GEMM_TAIL,
+                                  nullptr);
         }
+    } else if (warp == kSfWarp) {
+        // ------------------------------------------------------------ scale-tile producer
+        if (!p.skip_producer)
+            sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, blockIdx.x, gridDim.x, num_tiles,
+                                [&](int tile, int &a_band, int &b_band) {
+                                    int m0, n0;
+                                    tile_coords(tile, p.m_blocks, m0, n0, BN);
+                                    a_band = m0 / 128;
+                                    b_band = n0 / 128;
+                                },
+                                lane, abort_flag);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // All 32 lanes walk the loop with warp-uniform operands; the tcgen05
         // instructions are predicated on lane 0, so the same thread issues every
         // MMA and the commits that track them, without a divergent branch.
-        const uint32_t a_base = smem_u32(smem + L::kOffA), b_base = smem_u32(smem + L::kOffB);
+        // Ring positions advance incrementally and the descriptors of a stage
+        // are one add from a base: the loop is a short dependent chain per stage.
         const uint64_t desc_ab = smem_desc(0, 16, 1024, 2);
+        const uint64_t ad0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffA) >> 4) & 0x3FFFu);
+        const uint64_t bd0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffB) >> 4) & 0x3FFFu);
         const uint32_t leader = lane == 0 ? 1u : 0u;
-        int kg = 0;
+        int last_n_mma, last_n_chunk;
+        stage_extent<FMT>(p.num_kt - 1, p.K, last_n_mma, last_n_chunk);
+        int s = 0, slot = 0;    // stage and scale-slot ring positions
+        uint32_t fph = 0, sph = 0;  // parities of the current phases of full[s] and sf_full[slot]
         bool stop = false;
-        bool ready = false;  // result of the last peek at stage kg's barriers
+        bool ready = false;     // result of the last peek at both barriers
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++it) {
             const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
-            for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
-                const int s = kg % STAGES;
-                const int slot = kg % kSfSlots;
-                // sf_full of a stage implies its code tiles have landed: the scale warps
-                // arrive only after observing the stage's load barrier.
-                if (!ready && !mbar_wait_bounded(&sf_full[slot], (kg / kSfSlots) & 1, p.wait_limit_ns,
-                                                 SITE_GEMM_MMA_SF, abort_flag)) {
+            for (int kt = 0; kt < p.num_kt; ++kt) {
+                if (!ready &&
+                    (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
+                     !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))) {
                     stop = true;
                     break;
                 }
@@ -480,26 +648,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     tc_fence_after();
                 }
-                int n_mma, n_chunk;
-                stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                const uint32_t a_stage = a_base + s * L::kABytes, b_stage = b_base + s * L::kBBytes;
                 const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
-                const uint32_t t_sfb = t_sfa + 4 * F::kChunks;
-                for (int j = 0; j < n_mma; ++j) {
-                    const int chunk = j / F::kMmaPerChunk;
-                    const uint32_t sf_id = (uint32_t)((j % F::kMmaPerChunk) * F::kSfPerMma);
-                    const uint64_t ad = desc_ab | (uint64_t)(((a_stage + 32 * j) >> 4) & 0x3FFFu);
-                    const uint64_t bd = desc_ab | (uint64_t)(((b_stage + 32 * j) >> 4) & 0x3FFFu);
-                    gemm_mma_if<FMT>(t_acc, ad, bd, gemm_idesc<FMT, BN>(sf_id), t_sfa + 4 * chunk,
-                                     t_sfb + 4 * L::kBBands * chunk, (kt > 0 || j > 0) ? 1u : 0u, leader);
-                }
+                issue_stage<FMT, false, BN, 4 * L::kBBands>(kt + 1 < p.num_kt ? 4 : last_n_mma, t_acc,
+                                                            ad0 + (uint64_t)(s * (L::kABytes >> 4)),
+                                                            bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa,
+                                                            t_sfa + 4 * F::kChunks, kt > 0 ? 1u : 0u, leader);
                 // frees the smem stage and (for the scale warps) the scale slot
                 tc_commit_if(&empty[s], leader);
-                // peek, without blocking, at the next stage while these MMAs run
-                {
-                    const int k1 = kg + 1;
-                    ready = mbar_test_wait(&sf_full[k1 % kSfSlots], (k1 / kSfSlots) & 1);
+                if (++s == STAGES) {
+                    s = 0;
+                    fph ^= 1u;
                 }
+                slot = (slot + 1) & (kSfSlots - 1);
+                sph ^= (slot == 0) ? 1u : 0u;
+                // peek, without blocking, at the next stage while these MMAs run
+                ready = mbar_test_wait(&full[s], fph) && mbar_test_wait(&sf_full[slot], sph);
             }
             if (!stop) tc_commit_if(&acc_full[it & 1], leader);
         }
@@ -507,43 +670,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps
-        // Each warp owns one TMEM lane quadrant.  A 512-byte scale tile is 32
-        // rows of 16 bytes; row r holds the 4 scale columns of tile rows r,
-        // r+32, r+64, r+96 -- exactly TMEM lane r's 4 columns, which the MMA
-        // expects in every quadrant.  So every warp loads the same rows and
-        // stores them into its own 32 lanes.
         const int q = warp & 3;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        int kg = 0;
-        bool stop = false;
-        for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
-            for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
-                const int s = kg % STAGES, slot = kg % kSfSlots;
-                if (!mbar_wait_bounded(&full[s], (kg / STAGES) & 1, p.wait_limit_ns, SITE_GEMM_SF_FULL, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                // the slot's previous stage (kg - kSfSlots) has been consumed once its
-                // MMAs completed, which the commit on that stage's empty barrier signals
-                if (kg >= kSfSlots &&
-                    !mbar_wait_bounded(&empty[(kg - kSfSlots) % STAGES], ((kg - kSfSlots) / STAGES) & 1,
-                                       p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                tc_fence_after();
-                int n_mma, n_chunk;
-                stage_extent<FMT>(kt, p.K, n_mma, n_chunk);
-                (void)n_chunk;  // tiles past the K tail carry stale scales the MMAs never read
-                stage_scales_to_tmem<F::kChunks, L::kBBands>(smem + L::kOffSfa + s * L::kSfaBytes,
-                                                             smem + L::kOffSfb + s * L::kSfbBytes,
-                                                             tmem + lane_base + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols),
-                                                             lane);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_full[slot]);
-            }
-        }
+        int my_tiles = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
+        scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
+                              my_tiles, lane, abort_flag, [&](int slot) { mbar_arrive(&sf_full[slot]); });
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
@@ -559,10 +690,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
-            epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
-                                             [&] {
-                                                 if (lane == 0) mbar_arrive(acc_empty);
-                                             });
+            epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs,
+                                                                     nstore, amax, scale, [&] {
+                                                                         if (lane == 0) mbar_arrive(acc_empty);
+                                                                     });
         }
         epilogue_finish(p, lane, amax);
     }
@@ -571,7 +702,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        // every MMA this CTA issued has completed once mma_done has fired
+        // every MMA has completed once mma_done has fired
         mbar_wait_bounded(mma_done, 0, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
         tmem_dealloc(tmem, L::kTmemCols);
     }

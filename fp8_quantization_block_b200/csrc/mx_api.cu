@@ -133,6 +133,23 @@ bool make_tmap_c(CUtensorMap *m, void *base, int64_t rows, int64_t cols, int64_t
     return r == CUDA_SUCCESS;
 }
 
+// Scale tiles as a 3D tensor of 8-byte words: [bands][sf_tiles_k][64] (one
+// 512-byte tile = 64 words), box = box_chunks tiles of box_bands bands.  Reads
+// past either end (a ragged K or N) return zeros.
+bool make_tmap_sf(CUtensorMap *m, const uint8_t *scales, int64_t bands, int64_t sf_tiles_k, int box_chunks,
+                  int box_bands) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64u, (cuuint64_t)sf_tiles_k, (cuuint64_t)bands};
+    cuuint64_t strides[2] = {512u, (cuuint64_t)(sf_tiles_k * 512)};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_chunks, (cuuint32_t)box_bands};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<uint8_t *>(scales), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int FMT, int BN, int STAGES>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                         const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
@@ -140,9 +157,13 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K * fmt_bits(FMT) / 8;
-    CUtensorMap ta, tb, tc;
+    const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    CUtensorMap ta, tb, tc, tsa, tsb;
     if (!make_tmap_u8(&ta, a_codes, M, kbytes, kBM)) return MX_ERR_CUDA;
     if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN)) return MX_ERR_CUDA;
+    if (!make_tmap_sf(&tsa, a_scales, cdiv(M, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 1)) return MX_ERR_CUDA;
+    if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, L::kBBands))
+        return MX_ERR_CUDA;
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
@@ -154,9 +175,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     });
     if (attr_err != cudaSuccess) return MX_ERR_CUDA;
     GemmParams p;
-    p.sfa = a_scales;
-    p.sfb = B->scales;
-    p.sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    p.sf_tiles_k = sf_tiles_k;
     p.C = C;
     p.ldc = ldc;
     p.M = (int)M;
@@ -174,7 +193,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
-    gemm_kernel<FMT, BN, STAGES><<<grid, kGemmThreads, L::kAlloc, st>>>(ta, tb, tc, p);
+    gemm_kernel<FMT, BN, STAGES><<<grid, kGemmThreads, L::kAlloc, st>>>(ta, tb, tc, tsa, tsb, p);
     return last_launch();
 }
 
@@ -187,9 +206,13 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K * fmt_bits(FMT) / 8;
-    CUtensorMap ta, tb, tc;
+    const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    CUtensorMap ta, tb, tc, tsa, tsb;
     if (!make_tmap_u8(&ta, a_codes, M, kbytes, 128)) return MX_ERR_CUDA;
     if (!make_tmap_u8(&tb, B->codes, N, kbytes, 128)) return MX_ERR_CUDA;
+    if (!make_tmap_sf(&tsa, a_scales, cdiv(M, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 1)) return MX_ERR_CUDA;
+    if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 2))
+        return MX_ERR_CUDA;
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
@@ -201,9 +224,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     });
     if (attr_err != cudaSuccess) return MX_ERR_CUDA;
     GemmParams p;
-    p.sfa = a_scales;
-    p.sfb = B->scales;
-    p.sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    p.sf_tiles_k = sf_tiles_k;
     p.C = C;
     p.ldc = ldc;
     p.M = (int)M;
@@ -235,7 +256,8 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES>, ta, tb, tc, p) != cudaSuccess) return last_launch();
+    if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
+        return last_launch();
     return last_launch();
 }
 

@@ -34,6 +34,7 @@ enum : unsigned {
     SITE_GEMM_SF_EMPTY = 9,
     SITE_GEMM_MMA_SF = 10,
     SITE_GEMM_SF_LOAD = 11,
+    SITE_GEMM_SF_FREE = 12,
 };
 
 // {flags, first site, first block, count}
@@ -137,6 +138,15 @@ MX_DEVICE_INLINE void tma_load_2d(void *smem_dst, const void *tmap, int32_t x, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
             smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 3D tiled TMA load (no multicast) into this CTA's shared memory.
+MX_DEVICE_INLINE void tma_load_3d(void *smem_dst, const void *tmap, int32_t x, int32_t y, int32_t z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
 
