@@ -417,6 +417,39 @@ def run_profile_case(name: str, reps: int = 4):
 
 
 METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
+
+# DRAM bytes (read + write) per launch of the roofline kernel on each workload,
+# from one ncu capture (the summary under profiles/ named for the kernel and
+# workload gives the command); reported only while the kernel sources still
+# hash to `src`, i.e. the counters were taken on the code that runs.
+NCU_TRAFFIC = {
+    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6>", "bytes": 22778368 + 66560, "src": "af22953946a39d50"},
+}
+
+
+def csrc_hash() -> str:
+    import hashlib
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "fp8_quantization_block_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_bytes(workload_key: str, kernel: str):
+    rec = NCU_TRAFFIC.get(workload_key)
+    if rec is None or rec["kernel"] != kernel or rec["src"] != csrc_hash():
+        return None
+    return rec["bytes"]
+
+
+def gemm_kernel_name(fmt: int, M: int, N: int) -> str:
+    """The GEMM kernel mx_gemm dispatches to for this shape."""
+    if M > 128 and N > 128:
+        return f"gemm_pair_kernel<{fmt}, {6 if fmt < 2 else 5}>"
+    return f"gemm_kernel<{fmt}, {128 if N <= 128 else 256}, 4>"
 FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4"}
 
 
@@ -483,8 +516,9 @@ def main():
                    "step": "mx_quantize(X) + mx_gemm(Xq, Wq pre-quantized)",
                    "l2": f"inputs larger than L2: {r['n_sets']} rotating input sets x {r['per_set'] / 2**20:.1f} MB",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel<{FMT_NAMES[fmt]}>", "achieved": round(g_tf, 1),
-                     "peak": round(tpeak, 1), "unit": "TFLOP/s", "frac": round(g_tf / tpeak, 4), "traffic": None,
+        "roofline": {"bound": "tensor", "kernel": gemm_kernel_name(fmt, M, N), "achieved": round(g_tf, 1),
+                     "peak": round(tpeak, 1), "unit": "TFLOP/s", "frac": round(g_tf / tpeak, 4),
+                     "traffic": traffic_bytes(args.workload, gemm_kernel_name(fmt, M, N)),
                      "peak_source": f"{peak_src} bf16 x {2 if fmt < 2 else 4} (nominal dtype ratio)",
                      "frac_of_page_spec": round(g_tf / SPEC["fp8_tflops" if fmt < 2 else "fp4_tflops"], 4),
                      "kernel_us": round(g_avg * 1e3, 2)},
