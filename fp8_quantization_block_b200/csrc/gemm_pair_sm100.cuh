@@ -8,16 +8,17 @@
 // core reads B from both CTAs' shared memory.  Per SM that is half the B
 // traffic of a 128 x 256 tile for the same MMA work.  No load is multicast.
 //
-// Roles per CTA (11 warps), as in the single-CTA kernel:
+// Roles per CTA (12 warps), as in the single-CTA kernel:
 //   warp 0     code-tile producer: own A rows and B half, completion counted
 //              on the leader CTA's barrier;
 //   warp 10    scale-tile producer: own A band and both B bands (this CTA's
 //              TMEM needs the scales of all 256 B rows), local barriers;
 //   warps 6-9  scale warps: this CTA's TMEM slot, then an arrive on the
 //              leader's slot barrier (8 arrivals: both CTAs' scale warps);
-//   warp 1     leader CTA only: issues the pair's MMAs once the pair's code
-//              tiles and both CTAs' scale slots are in; commits fan out to the
-//              barriers of both CTAs;
+//   warp 11    leader CTA only: gate, counts the stages whose code tiles (both
+//              CTAs') and scale slots (both CTAs') are in;
+//   warp 1     leader CTA only: issues the pair's MMAs for the stages the gate
+//              reports; commits fan out to the barriers of both CTAs;
 //   warps 2-5  epilogue for this CTA's 128 rows of the tile.
 // Every mbarrier wait is bounded; both CTAs meet at a cluster barrier before
 // exit, so no CTA leaves while its partner may still signal it.
@@ -53,6 +54,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *sf_full = mma_done + 1;           // [kSfSlots], leader's count both CTAs' scale warps
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+    uint32_t *ready_count = reinterpret_cast<uint32_t *>(smem + L::kOffMisc + 8);  // gate -> MMA issuer
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs)
@@ -74,6 +76,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_init(mma_done, 1);
         for (int i = 0; i < kSfSlots; ++i) mbar_init(&sf_full[i], 8);
         *abort_flag = 0;
+        *ready_count = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -152,21 +155,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t leader = lane == 0 ? 1u : 0u;
             int last_n_mma, last_n_chunk;
             stage_extent<FMT>(p.num_kt - 1, p.K, last_n_mma, last_n_chunk);
-            int s = 0, slot = 0;        // stage and scale-slot ring positions
-            uint32_t fph = 0, sph = 0;  // parities of the current phases of full[s] and sf_full[slot]
+            int s = 0, slot = 0;  // stage and scale-slot ring positions
+            uint32_t kg = 0;      // stages consumed
+            uint32_t avail = 0;   // stages the gate warp has reported ready
             bool stop = false;
-            bool ready = false;         // result of the last peek at both barriers
             int it = 0;
             for (int tile = pair; tile < num_tiles && !stop; tile += npairs, ++it) {
                 const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
                 for (int kt = 0; kt < p.num_kt; ++kt) {
-                    if (!ready &&
-                        (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
-                         !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))) {
-                        stop = true;
-                        break;
+                    // the gate warp publishes how many stages have their code tiles and
+                    // scale slots in; read it only when the stages known ready run out
+                    if (kg >= avail) {
+                        avail = wait_counter_above(ready_count, kg, p.wait_limit_ns, SITE_GEMM_MMA_READY, abort_flag);
+                        if (avail == 0u) {
+                            stop = true;
+                            break;
+                        }
+                        tc_fence_after();
                     }
-                    tc_fence_after();
                     if (kt == 0 && it > 0) {
                         if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY,
                                                abort_flag)) {
@@ -182,18 +188,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                    t_sfa + 4 * F::kChunks, kt > 0 ? 1u : 0u, leader);
                     // frees both CTAs' smem stage and, for their scale warps, the scale slot
                     tc_commit_pair_if(&empty[s], 0x3, leader);
-                    if (++s == STAGES) {
-                        s = 0;
-                        fph ^= 1u;
-                    }
+                    s = (s + 1 == STAGES) ? 0 : s + 1;
                     slot = (slot + 1) & (kSfSlots - 1);
-                    sph ^= (slot == 0) ? 1u : 0u;
-                    ready = mbar_test_wait(&full[s], fph) && mbar_test_wait(&sf_full[slot], sph);
+                    ++kg;
                 }
                 if (!stop) tc_commit_pair_if(&acc_full[it & 1], 0x3, leader);
             }
             tc_commit_pair_if(mma_done, 0x3, leader);
             __syncwarp();
+        }
+    } else if (warp == kGateWarp) {
+        // ------------------------------------------------------------ gate (leader)
+        if (rank == 0) {
+            int my_tiles = 0;
+            for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
+            gate_role<STAGES>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
         }
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps

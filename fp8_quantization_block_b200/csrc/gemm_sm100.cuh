@@ -20,6 +20,11 @@
 //              previous contents have completed.  (Staging the scales with
 //              tcgen05.cp instead costs tensor-pipe cycles that do not overlap
 //              the MMAs; register stores from other warps do.)
+//   warp 11    gate: waits for each stage's code tiles and scale slot and
+//              publishes the count of ready stages in shared memory, so that
+//              the MMA issuer reads one word (rarely, as it runs behind)
+//              instead of waiting on two mbarriers per stage, whose latency
+//              would leave the tensor pipe idle between stages;
 //   warp 1     TMEM owner and MMA issuer: one lane issues the block-scaled
 //              tcgen05.mma instructions (4 per stage, 32 bytes of K each) into
 //              an FP32 accumulator in TMEM once a stage's code tiles and scale
@@ -65,8 +70,9 @@ struct GemmFmt<3> {  // NVFP4: kind::mxf4nvf4, scale_vec 4X (16-element blocks),
 
 constexpr int kBM = 128;
 constexpr int kStageKBytes = 128;
-constexpr int kGemmThreads = 352;  // 11 warps
+constexpr int kGemmThreads = 384;  // 12 warps
 constexpr int kSfWarp = 10;        // the scale-tile producer
+constexpr int kGateWarp = 11;      // publishes how many stages the MMA issuer may consume
 constexpr int kSfSlots = 4;        // TMEM scale slots (a power of two)
 constexpr int kSfGroup = 2;        // stages per scale-tile copy
 constexpr int kEpiWarps = 4;
@@ -363,6 +369,32 @@ MX_DEVICE_INLINE void tile_coords(int tile, int m_blocks, int &m0, int &n0, int 
     n0 = (tile / m_blocks) * bn;
 }
 
+// Gate warp: for every stage of this CTA's tiles, in order, wait for its code
+// tiles (full) and its scale slot (sf_full), then publish the number of
+// stages ready so far.
+template <int STAGES>
+MX_DEVICE_INLINE void gate_role(const GemmParams &p, uint64_t *full, uint64_t *sf_full, uint32_t *ready, int my_tiles,
+                                int lane, volatile int *abort_flag) {
+    int s = 0, slot = 0;
+    uint32_t fph = 0, sph = 0, k = 0;
+    for (int t = 0; t < my_tiles; ++t) {
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+            if (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
+                !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))
+                return;
+            ++k;
+            __syncwarp();
+            if (lane == 0) st_release_shared(ready, k);
+            if (++s == STAGES) {
+                s = 0;
+                fph ^= 1u;
+            }
+            slot = (slot + 1) & (kSfSlots - 1);
+            sph ^= (slot == 0) ? 1u : 0u;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- epilogue
 // One 32-column chunk of this warp's 32 accumulator rows: TMEM -> registers,
 // x scale (NVFP4: gA * gB), optional GELU, bf16 round-to-nearest-even.  The
@@ -530,6 +562,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *sf_full = mma_done + 1;            // [kSfSlots]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+    uint32_t *ready_count = reinterpret_cast<uint32_t *>(smem + L::kOffMisc + 8);  // gate -> MMA issuer
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = p.m_blocks * p.n_blocks;
@@ -549,6 +582,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_init(mma_done, 1);
         for (int i = 0; i < kSfSlots; ++i) mbar_init(&sf_full[i], 4);
         *abort_flag = 0;
+        *ready_count = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -624,21 +658,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t leader = lane == 0 ? 1u : 0u;
         int last_n_mma, last_n_chunk;
         stage_extent<FMT>(p.num_kt - 1, p.K, last_n_mma, last_n_chunk);
-        int s = 0, slot = 0;    // stage and scale-slot ring positions
-        uint32_t fph = 0, sph = 0;  // parities of the current phases of full[s] and sf_full[slot]
+        int s = 0, slot = 0;  // stage and scale-slot ring positions
+        uint32_t kg = 0;      // stages consumed
+        uint32_t avail = 0;   // stages the gate warp has reported ready
         bool stop = false;
-        bool ready = false;     // result of the last peek at both barriers
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++it) {
             const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
             for (int kt = 0; kt < p.num_kt; ++kt) {
-                if (!ready &&
-                    (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
-                     !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))) {
-                    stop = true;
-                    break;
+                // the gate warp publishes how many stages have their code tiles and
+                // scale slot in; read it only when the stages known ready run out
+                if (kg >= avail) {
+                    avail = wait_counter_above(ready_count, kg, p.wait_limit_ns, SITE_GEMM_MMA_READY, abort_flag);
+                    if (avail == 0u) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
                 }
-                tc_fence_after();
                 if (kt == 0 && it > 0) {
                     // the epilogue has released the columns this accumulator shares
                     if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY,
@@ -655,19 +692,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                             t_sfa + 4 * F::kChunks, kt > 0 ? 1u : 0u, leader);
                 // frees the smem stage and (for the scale warps) the scale slot
                 tc_commit_if(&empty[s], leader);
-                if (++s == STAGES) {
-                    s = 0;
-                    fph ^= 1u;
-                }
+                s = (s + 1 == STAGES) ? 0 : s + 1;
                 slot = (slot + 1) & (kSfSlots - 1);
-                sph ^= (slot == 0) ? 1u : 0u;
-                // peek, without blocking, at the next stage while these MMAs run
-                ready = mbar_test_wait(&full[s], fph) && mbar_test_wait(&sf_full[slot], sph);
+                ++kg;
             }
             if (!stop) tc_commit_if(&acc_full[it & 1], leader);
         }
         tc_commit_if(mma_done, leader);
         __syncwarp();
+    } else if (warp == kGateWarp) {
+        // ------------------------------------------------------------ gate
+        int my_tiles = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
+        gate_role<STAGES>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps
         const int q = warp & 3;

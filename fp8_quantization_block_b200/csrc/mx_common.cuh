@@ -35,6 +35,7 @@ enum : unsigned {
     SITE_GEMM_MMA_SF = 10,
     SITE_GEMM_SF_LOAD = 11,
     SITE_GEMM_SF_FREE = 12,
+    SITE_GEMM_MMA_READY = 13,
 };
 
 // {flags, first site, first block, count}
@@ -122,6 +123,39 @@ MX_DEVICE_INLINE bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t
                 record_error(DEVERR_TIMEOUT, site);
                 if (abort != nullptr) *abort = 1;
                 return false;
+            }
+        }
+    }
+}
+
+// A shared-memory counter published by one warp (release) and polled by
+// another (acquire): cheaper to read than an mbarrier when the reader only
+// needs to know how far the writer has got.
+MX_DEVICE_INLINE void st_release_shared(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+MX_DEVICE_INLINE uint32_t ld_acquire_shared(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
+// Poll *counter until it exceeds `need` (bounded like the mbarrier waits).
+// Returns the value seen, or 0 after recording a timeout.
+MX_DEVICE_INLINE uint32_t wait_counter_above(const uint32_t *counter, uint32_t need, uint64_t limit_ns, unsigned site,
+                                             volatile int *abort) {
+    uint32_t v = ld_acquire_shared(counter);
+    if (v > need) return v;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        v = ld_acquire_shared(counter);
+        if (v > need) return v;
+        if ((i & 15u) == 0u) {
+            if (abort != nullptr && *abort) return 0u;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                record_error(DEVERR_TIMEOUT, site);
+                if (abort != nullptr) *abort = 1;
+                return 0u;
             }
         }
     }
