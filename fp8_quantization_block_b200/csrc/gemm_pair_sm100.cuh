@@ -162,11 +162,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int it = 0;
             for (int tile = pair; tile < num_tiles && !stop; tile += npairs, ++it) {
                 const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
-                for (int kt = 0; kt < p.num_kt; ++kt) {
+                // One stage: its MMAs, then a commit that frees the smem stage and the
+                // scale slot once they have completed.
+                auto run_stage = [&](int k, uint32_t acc) {
+                    const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
+                    issue_stage<FMT, true, 256, 8>(k + 1 < p.num_kt ? 4 : last_n_mma, t_acc, ad0 + (uint64_t)(s * (L::kABytes >> 4)),
+                        bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader);
+                    tc_commit_pair_if(&empty[s], 0x3, leader);
+                    s = (s + 1 == STAGES) ? 0 : s + 1;
+                    slot = (slot + 1) & (kSfSlots - 1);
+                    ++kg;
+                };
+                // Two stages per iteration: the loop's own instructions then fall between
+                // MMAs only every other stage.
+                for (int kt = 0; kt < p.num_kt; kt += 2) {
+                    const bool two = kt + 1 < p.num_kt;
                     // the gate warp publishes how many stages have their code tiles and
                     // scale slots in; read it only when the stages known ready run out
-                    if (kg >= avail) {
-                        avail = wait_counter_above(ready_count, kg, p.wait_limit_ns, SITE_GEMM_MMA_READY, abort_flag);
+                    const uint32_t need = kg + (two ? 1u : 0u);
+                    if (need >= avail) {
+                        avail = wait_counter_above(ready_count, need, p.wait_limit_ns, SITE_GEMM_MMA_READY, abort_flag);
                         if (avail == 0u) {
                             stop = true;
                             break;
@@ -174,23 +189,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tc_fence_after();
                     }
                     if (kt == 0 && it > 0) {
-                        if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY,
-                                               abort_flag)) {
+                        // the epilogue has released the columns this accumulator shares
+                        if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY, abort_flag)) {
                             stop = true;
                             break;
                         }
                         tc_fence_after();
                     }
-                    const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
-                    issue_stage<FMT, true, 256, 8>(kt + 1 < p.num_kt ? 4 : last_n_mma, t_acc,
-                                                   ad0 + (uint64_t)(s * (L::kABytes >> 4)),
-                                                   bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa,
-                                                   t_sfa + 4 * F::kChunks, kt > 0 ? 1u : 0u, leader);
-                    // frees both CTAs' smem stage and, for their scale warps, the scale slot
-                    tc_commit_pair_if(&empty[s], 0x3, leader);
-                    s = (s + 1 == STAGES) ? 0 : s + 1;
-                    slot = (slot + 1) & (kSfSlots - 1);
-                    ++kg;
+                    run_stage(kt, kt > 0 ? 1u : 0u);
+                    if (two) run_stage(kt + 1, 1u);
                 }
                 if (!stop) tc_commit_pair_if(&acc_full[it & 1], 0x3, leader);
             }
