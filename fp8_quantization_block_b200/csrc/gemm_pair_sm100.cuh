@@ -93,6 +93,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     cluster_sync();  // both CTAs' barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // The setup above overlaps the previous kernel in the stream; its outputs
+    // (our operands, NVFP4 scales, C's prior contents) are read only after this.
+    griddep_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ code-tile producer
@@ -254,6 +257,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait_bounded(mma_done, 0, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
         tmem_dealloc_pair(tmem, L::kTmemCols);
     }
+    // the next kernel in the stream may start its setup now (it still waits
+    // for this grid's completion before reading anything)
+    griddep_launch_dependents();
     cluster_sync();
 }
 

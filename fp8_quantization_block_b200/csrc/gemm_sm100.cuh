@@ -598,6 +598,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // The setup above overlaps the previous kernel in the stream; its outputs
+    // (our operands, NVFP4 scales, C's prior contents) are read only after this.
+    griddep_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ code-tile producer
@@ -749,6 +752,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait_bounded(mma_done, 0, p.wait_limit_ns, SITE_GEMM_TAIL, nullptr);
         tmem_dealloc(tmem, L::kTmemCols);
     }
+    // the next kernel in the stream may start its setup now (it still waits
+    // for this grid's completion before reading anything)
+    griddep_launch_dependents();
 }
 
 }  // namespace mx

@@ -23,6 +23,16 @@ using namespace mx;
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<int> g_skip_producer{0};
 std::atomic<int> g_pair_enabled{1};
+std::atomic<int> g_pdl_enabled{1};
+
+// Launch attributes shared by the kernels that may overlap the previous kernel
+// in the stream (they call griddep_wait() before reading any input).
+int pdl_attr(cudaLaunchAttribute *a) {
+    if (!g_pdl_enabled.load()) return 0;
+    a->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a->val.programmaticStreamSerializationAllowed = 1;
+    return 1;
+}
 
 bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 3; }
 int fmt_block(int fmt) { return fmt == MX_NVFP4 ? 16 : 32; }
@@ -78,9 +88,16 @@ template <int FMT>
 void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
                      const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
-    dim3 grid((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows));
-    quantize_kernel<FMT><<<grid, kQThreads, 0, st>>>(src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
-                                                      sf_tiles_k, g_in, g_out, g_from_amax);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows), 1);
+    cfg.blockDim = dim3(kQThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    cudaLaunchKernelEx(&cfg, quantize_kernel<FMT>, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
+                       sf_tiles_k, g_in, g_out, g_from_amax);
 }
 
 int num_sms() {
@@ -193,7 +210,17 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
-    gemm_kernel<FMT, BN, STAGES><<<grid, kGemmThreads, L::kAlloc, st>>>(ta, tb, tc, tsa, tsb, p);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, BN, STAGES>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
+        return last_launch();
     return last_launch();
 }
 
@@ -249,13 +276,13 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kAlloc;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1 + (unsigned)pdl_attr(&attr[1]);
     if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
         return last_launch();
     return last_launch();
@@ -367,6 +394,7 @@ mx_status mx_debug_set(int key, uint64_t value) {
     case MX_DEBUG_WAIT_LIMIT_NS: g_wait_limit_ns.store(value ? value : 1); return MX_OK;
     case MX_DEBUG_SKIP_PRODUCER: g_skip_producer.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_PAIR_GEMM: g_pair_enabled.store(value ? 1 : 0); return MX_OK;
+    case MX_DEBUG_OVERLAP_LAUNCH: g_pdl_enabled.store(value ? 1 : 0); return MX_OK;
     default: return MX_ERR_INVALID_ARG;
     }
 }

@@ -128,6 +128,16 @@ MX_DEVICE_INLINE bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t
     }
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still
+// running; griddep_wait() returns once that kernel has completed and its
+// memory is visible, so everything before it must not read the previous
+// kernel's outputs.  griddep_launch_dependents() lets the next such kernel be
+// scheduled early (it still waits for this one's completion in its own
+// griddep_wait()).  Both are no-ops for kernels launched without the attribute.
+MX_DEVICE_INLINE void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MX_DEVICE_INLINE void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // A shared-memory counter published by one warp (release) and polled by
 // another (acquire): cheaper to read than an mbarrier when the reader only
 // needs to know how far the writer has got.

@@ -265,6 +265,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
 
     float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f;
     __shared__ NvTables nvt;
+    // src and g may come from the previous kernel in the stream
+    griddep_wait();
     if (FMT == FMT_NVFP4) {
         g = *gscale_in;
         if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;   // g = RU(amax / (6 * 448))
@@ -373,6 +375,9 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
             *reinterpret_cast<uint4 *>(scales + chunk0 * 512 + threadIdx.x * 16) = val;
         }
     }
+    // the next kernel in the stream may start its setup now (it still waits
+    // for this grid's completion before reading anything)
+    griddep_launch_dependents();
 }
 
 // max |x| over a bf16 tensor -> atomicMax on the float bits of *amax (init 0).

@@ -192,8 +192,19 @@ int mx_version(void);
  *   MX_DEBUG_PAIR_GEMM     : 1 (default) = GEMMs with M > 128 and N > 128 run
  *                            on CTA pairs (256 x 256 tiles); 0 = single-CTA
  *                            128 x 256 tiles for every shape.
+ *   MX_DEBUG_OVERLAP_LAUNCH: 1 (default) = quantize and GEMM kernels are
+ *                            launched with programmatic stream serialization:
+ *                            their setup (barriers, TMEM, descriptors) overlaps
+ *                            the tail of the previous kernel in the stream, and
+ *                            they read no input before that kernel completes.
+ *                            0 = ordinary stream order.
  * Returns MX_ERR_INVALID_ARG for an unknown key. */
-typedef enum { MX_DEBUG_WAIT_LIMIT_NS = 1, MX_DEBUG_SKIP_PRODUCER = 2, MX_DEBUG_PAIR_GEMM = 3 } mx_debug_key;
+typedef enum {
+    MX_DEBUG_WAIT_LIMIT_NS = 1,
+    MX_DEBUG_SKIP_PRODUCER = 2,
+    MX_DEBUG_PAIR_GEMM = 3,
+    MX_DEBUG_OVERLAP_LAUNCH = 4
+} mx_debug_key;
 mx_status mx_debug_set(int key, uint64_t value);
 
 #ifdef __cplusplus
