@@ -419,9 +419,9 @@ def run_profile_case(name: str, reps: int = 4):
 METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
 
 # DRAM bytes (read + write) per launch of the roofline kernel on each workload,
-# from one ncu capture (the summary under profiles/ named for the kernel and
-# workload gives the command); reported only while the kernel sources still
-# hash to `src`, i.e. the counters were taken on the code that runs.
+# from one ncu capture of that kernel on that workload; reported only while the
+# kernel sources still hash to `src`, i.e. the counters were taken on the code
+# that runs.
 NCU_TRAFFIC = {
     "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6>", "bytes": 22778368 + 66560, "src": "af22953946a39d50"},
 }

@@ -67,6 +67,8 @@ def _load():
                 "orc_nvfp4_block_scale": (u8, [d, f32]),
                 "orc_amax_bf16": (d, [P, i64, i64, i64]),
                 "orc_quantize": (i32, [i32, P, i64, i64, i64, P, P, P, i32]),
+                "orc_quantize_oas": (i32, [P, i64, i64, i64, P, P]),
+                "orc_qsnr_db": (d, [P, i64, i64, i64, P, P]),
                 "orc_dequantize_f64": (i32, [i32, P, P, f32, i64, i64, P]),
                 "orc_dequantize_bf16": (i32, [i32, P, P, f32, i64, i64, P, i64]),
                 "orc_gemm_f64": (i32, [P, P, P, i64, i64, i64, P, P]),
@@ -168,6 +170,30 @@ def quantize(fmt: int, src_bits: np.ndarray, gscale: float | None = None):
     if rc != 0:
         raise ValueError(f"oracle quantize failed with code {rc}")
     return codes, scales, float(g[0])
+
+
+def quantize_oas(src_bits: np.ndarray):
+    """MXFP4 with overflow-aware scaling (block max mapped into (3.5, 7]) ->
+    (codes, scales), in MXFP4 storage."""
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    M, K = src.shape
+    codes = np.zeros(codes_bytes(2, M, K), dtype=np.uint8)
+    scales = np.zeros(scales_bytes(2, M, K), dtype=np.uint8)
+    rc = _load().orc_quantize_oas(_ptr(src), M, K, K, _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise ValueError(f"oracle quantize_oas failed with code {rc}")
+    return codes, scales
+
+
+def qsnr_db(src_bits: np.ndarray, xhat: np.ndarray):
+    """(QSNR in dB, sum x^2, sum (x - xhat)^2) of bf16 bits [M, K] against fp64 xhat [M, K]."""
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    xh = np.ascontiguousarray(xhat, dtype=np.float64)
+    M, K = src.shape
+    assert xh.shape == (M, K)
+    sums = np.zeros(2, dtype=np.float64)
+    db = float(_load().orc_qsnr_db(_ptr(src), M, K, K, _ptr(xh), _ptr(sums)))
+    return db, float(sums[0]), float(sums[1])
 
 
 def dequantize_f64(fmt: int, codes: np.ndarray, scales: np.ndarray, gscale: float, M: int, K: int):

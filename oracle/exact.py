@@ -86,11 +86,13 @@ def round_to_grid(v: Fraction, grid, sign_bit: int, negative: bool) -> int:
     return best[1] | (sign_bit if negative else 0)
 
 
-def mx_scale_byte(block: list[Fraction], fmt: int) -> int:
-    """Smallest E8M0 byte in [0, 254] after which no element exceeds the
-    format's largest magnitude (254 if none does)."""
+def mx_scale_byte(block: list[Fraction], fmt: int, threshold: Fraction | None = None) -> int:
+    """Smallest E8M0 byte in [0, 254] after which no element exceeds
+    `threshold` (the format's largest magnitude by default; 7 for MXFP4 with
+    overflow-aware scaling), 254 if none does."""
+    lim = MAXELEM[fmt] if threshold is None else threshold
     for E in range(0, 255):
-        if all(abs(x) / Fraction(2) ** (E - 127) <= MAXELEM[fmt] for x in block):
+        if all(abs(x) / Fraction(2) ** (E - 127) <= lim for x in block):
             return E
     return 254
 
@@ -121,8 +123,9 @@ def nvfp4_block_scale(block: list[Fraction], g: Fraction) -> int:
     return 0x7E
 
 
-def quantize(fmt: int, bits: np.ndarray, g: Fraction | None = None):
-    """Exact quantization of a tiny bf16 matrix.
+def quantize(fmt: int, bits: np.ndarray, g: Fraction | None = None, mx_threshold: Fraction | None = None):
+    """Exact quantization of a tiny bf16 matrix (MX scales by the threshold
+    rule above; elements by RNE onto the format's grid, saturating).
 
     Returns (codes[M][K] unpacked ints, scales[M][K/bs] ints, g)."""
     M, K = bits.shape
@@ -141,7 +144,7 @@ def quantize(fmt: int, bits: np.ndarray, g: Fraction | None = None):
                 sc = nvfp4_block_scale(blk, g)
                 denom = g * e4m3(sc)
             else:
-                sc = mx_scale_byte(blk, fmt)
+                sc = mx_scale_byte(blk, fmt, mx_threshold)
                 denom = Fraction(2) ** (sc - 127)
             scales[r][j] = sc
             for i, x in enumerate(blk):

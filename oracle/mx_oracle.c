@@ -25,7 +25,7 @@
  *                 section "Metodologia e Propostas" A: the standard MX mapping
  *                 puts the block maximum into (3, 6] of the E2M1 range.
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *   R1  rounding of elements is round-to-nearest, ties to the even code, and
  *       saturating ("satfinite") at the format's largest finite magnitude;
  *   R2  the sign of a value that rounds to zero is kept (-0 -> 0x8 / 0x80);
@@ -334,9 +334,10 @@ double orc_amax_bf16(const uint16_t *src, int64_t M, int64_t K, int64_t ld) {
  * codes: orc_codes_bytes bytes; scales: orc_scales_bytes bytes (fully written,
  * padding 0).  NVFP4: if gscale_given, *gscale is used as g, else g is computed
  * and stored to *gscale.  Non-finite input is outside the contract: returns
- * ORC_ENONFINITE. */
-int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
-                 uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
+ * ORC_ENONFINITE.  mx_threshold: the value a block's max |x| is mapped at or
+ * below by the MX scale (the format's largest element for the OCP rule). */
+static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
+                         uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
     build_tables();
     int bs = fmt_block(fmt);
     if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
@@ -346,7 +347,7 @@ int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
     int64_t sf_cols = K / bs;
     memset(scales, 0, orc_scales_bytes(fmt, M, K));
     memset(codes, 0, orc_codes_bytes(fmt, M, K));
-    double maxelem = fmt_maxelem(fmt);
+    double maxelem = mx_threshold;
     float g = 1.0f;
     if (fmt == ORC_NVFP4) {
         if (gscale_given) g = *gscale;
@@ -389,6 +390,39 @@ int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
         }
     }
     return ORC_OK;
+}
+
+int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
+                 uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
+    return quantize_impl(fmt, fmt_maxelem(fmt), src, M, K, ld, codes, scales, gscale, gscale_given);
+}
+
+/* MXFP4 with overflow-aware scaling [OAS page, section 2.A]: the block scale
+ * maps the block's max |x| into (3.5, 7] instead of (3, 6], i.e.
+ * E = ceil(log2(max_val / 7)) + 127; elements above 6 after scaling saturate
+ * to 6 as any E2M1 value does.  Same storage as MXFP4. */
+int orc_quantize_oas(const uint16_t *src, int64_t M, int64_t K, int64_t ld, uint8_t *codes, uint8_t *scales) {
+    return quantize_impl(ORC_MXFP4, 7.0, src, M, K, ld, codes, scales, NULL, 0);
+}
+
+/* Quantization SNR in dB [OAS page, section 3: "QSNR"]: 10 log10(sum x^2 /
+ * sum (x - xhat)^2) over the tensor, in fp64 (xhat from orc_dequantize_f64).
+ * sums[0] = sum x^2, sums[1] = sum (x - xhat)^2.  Returns +inf for zero error. */
+double orc_qsnr_db(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const double *xhat, double *sums) {
+    double sx = 0.0, se = 0.0;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double x = orc_bf16_to_double(src[r * ld + k]);
+            double e = x - xhat[r * K + k];
+            sx += x * x;
+            se += e * e;
+        }
+    if (sums) {
+        sums[0] = sx;
+        sums[1] = se;
+    }
+    if (se == 0.0) return INFINITY;
+    return 10.0 * log10(sx / se);
 }
 
 /* Dequantize to fp64: x = g * s * q (g = 1 for MX) [MXFP4-page, Fundamentos:
