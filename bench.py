@@ -241,6 +241,28 @@ def run_gpu(args, wl, rank, world, device):
                 h2d=M * K * 2, d2h=M * N * 2)
 
 
+def qsnr_table(device):
+    """Quantization SNR (dB) of each format on the synthetic configs' tensors,
+    computed on the device by mx_qsnr (fp64 sums)."""
+    import torch
+    from fp8_quantization_block_b200 import mx, synth
+    tensors = {
+        "dit_activations_4096x3072": synth.dit_activations(1, 4096, 3072),
+        "mlp_activations_student_t_4608x3072": synth.student_t(3, 4608, 3072),
+        "weights_gaussian_3072x3072": synth.gaussian_weights(2, 3072, 3072),
+    }
+    table = {}
+    for name, bits in tensors.items():
+        x = synth.bits_to_tensor(bits).to(device)
+        row = {}
+        for label, quant in (("mxfp8_e4m3", lambda: mx.quantize(x, 0)), ("mxfp4", lambda: mx.quantize(x, 2)),
+                             ("mxfp4_oas", lambda: mx.quantize_oas(x)), ("nvfp4", lambda: mx.quantize(x, 3))):
+            s = mx.qsnr_sums(quant(), x).cpu().numpy()
+            row[label] = round(float(10.0 * np.log10(s[0] / s[1])), 3)
+        table[name] = row
+    return table
+
+
 def quant_bytes_per_elem(fmt):
     return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625}[fmt]
 
@@ -293,7 +315,16 @@ def extras_gpu(device):
                                                           "frac_hbm": round(gbs2 / peaks["hbm_gbs"], 3)}
             del qs
         del xs
+    # MXFP4 with overflow-aware scaling: same bytes as MXFP4
+    M, K = 65536, 4096
+    xs = [torch.randn((M, K), generator=g, device=device).to(torch.bfloat16) for _ in range(3)]
+    qs = [mx.empty(2, M, K) for _ in xs]
+    ms = timed(lambda i: mx.quantize_oas(xs[i % len(xs)], out=qs[i % len(xs)]), len(xs))
+    gbs = M * K * quant_bytes_per_elem(2) / (ms * 1e-3) / 1e9
+    sweep[f"mxfp4_oas_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    del xs, qs
     out["quantize_sweep"] = sweep
+    out["qsnr_db"] = qsnr_table(device)
     # GEMMs
     for name, (fmt, M, N, K) in {"mlp_nvfp4_gemm1": (3, 4608, 12288, 3072), "mlp_nvfp4_gemm2": (3, 4608, 3072, 12288),
                                  "skinny_nvfp4_M16": (3, 16, 28672, 8192), "skinny_mxfp4_M16": (2, 16, 28672, 8192),

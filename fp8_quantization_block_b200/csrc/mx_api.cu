@@ -84,7 +84,7 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, int64_t rows, int64_t row_by
 }
 
 // --- quantize ------------------------------------------------------------
-template <int FMT>
+template <int FMT, int RULE = RULE_OCP>
 void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
                      const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
@@ -96,7 +96,7 @@ void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, cons
     cudaLaunchAttribute attr[1];
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
-    cudaLaunchKernelEx(&cfg, quantize_kernel<FMT>, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
+    cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
                        sf_tiles_k, g_in, g_out, g_from_amax);
 }
 
@@ -426,6 +426,46 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
                                st);
         }
     }
+    }
+    return last_launch();
+}
+
+mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst, void *stream) {
+    if (!dst || dst->fmt != MX_MXFP4 || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    if (dst->rows != M || dst->cols != K) return MX_ERR_INVALID_ARG;
+    if (K % 32 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || K == 0) return MX_OK;
+    if (!src_bf16 || !dst->codes || !dst->scales) return MX_ERR_INVALID_ARG;
+    if (ld_src < K || (ld_src & 7) != 0) return MX_ERR_MISALIGNED;
+    if (!aligned16(src_bf16) || !aligned16(dst->codes) || !aligned16(dst->scales)) return MX_ERR_MISALIGNED;
+    if (cdiv(M, kQTileRows) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
+    launch_quantize<2, RULE_OAS>(static_cast<const uint16_t *>(src_bf16), M, K, ld_src, dst, nullptr, nullptr,
+                                 static_cast<cudaStream_t>(stream));
+    return last_launch();
+}
+
+mx_status mx_qsnr(const mx_tensor *q, const void *src_bf16, int64_t ld_src, double *sums, void *stream) {
+    mx_status s = check_tensor(q, true);
+    if (s != MX_OK) return s;
+    if (!sums) return MX_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sums) & 7u) != 0) return MX_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(sums, 0, 2 * sizeof(double), st) != cudaSuccess) return MX_ERR_CUDA;
+    if (q->rows == 0 || q->cols == 0) return MX_OK;
+    if (!src_bf16) return MX_ERR_INVALID_ARG;
+    if (ld_src < q->cols || (ld_src & 7) != 0 || !aligned16(src_bf16)) return MX_ERR_MISALIGNED;
+    const int64_t n = q->rows * (q->cols / 8);
+    int64_t blocks = cdiv(n, 256);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    const uint16_t *x = static_cast<const uint16_t *>(src_bf16);
+    const uint8_t *c = static_cast<const uint8_t *>(q->codes);
+    const unsigned b = (unsigned)blocks;
+    switch (q->fmt) {
+    case MX_MXFP8_E4M3: qsnr_kernel<0><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP8_E5M2: qsnr_kernel<1><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP4: qsnr_kernel<2><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
+    default: qsnr_kernel<3><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, q->gscale, q->rows, q->cols, sums);
     }
     return last_launch();
 }

@@ -54,10 +54,19 @@ struct FmtTraits<FMT_NVFP4> {
 // finite).  amax = 1.m * 2^(f-127) with max_elem = M * 2^k: the smallest e with
 // amax <= max_elem * 2^e is f - 127 - k, plus one when 1.m > M.  Zero and bf16
 // subnormals land below 0 and clamp to 0; finite inputs never exceed 253.
-template <int FMT>
+//
+// RULE_OAS (MXFP4 only; page "Unveiling the Potential of Quantization with
+// MXFP4", section 2.A, overflow-aware scaling): the block max is mapped into
+// (3.5, 7] instead of (3, 6], i.e. the threshold is 7 = 1.75 * 2^2; elements
+// above 6 then saturate to 6 as usual.
+enum { RULE_OCP = 0, RULE_OAS = 1 };
+
+template <int FMT, int RULE = RULE_OCP>
 MX_DEVICE_INLINE int mx_scale_byte(uint32_t amax_bits) {
     using T = FmtTraits<FMT>;
-    int e = (int)(amax_bits >> 7) - T::kExpOff + (((amax_bits & 0x7Fu) > (uint32_t)T::kMantThr) ? 1 : 0);
+    static_assert(RULE == RULE_OCP || FMT == FMT_MXFP4, "overflow-aware scaling is defined for MXFP4");
+    constexpr uint32_t thr = RULE == RULE_OAS ? 0x60u : (uint32_t)T::kMantThr;
+    int e = (int)(amax_bits >> 7) - T::kExpOff + (((amax_bits & 0x7Fu) > thr) ? 1 : 0);
     return e < 0 ? 0 : e;
 }
 
@@ -243,7 +252,7 @@ MX_DEVICE_INLINE uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
 // ceil((K / block) / 4) 512-byte tiles per 128-row band.  NVFP4: *gscale_in
 // is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
 // if gscale_out != nullptr, CTA 0 also stores g there.
-template <int FMT>
+template <int FMT, int RULE = RULE_OCP>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
                                                              int64_t ld, uint8_t *__restrict__ codes,
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
@@ -329,7 +338,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
                 *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
             }
         } else {
-            const int E = mx_scale_byte<FMT>(m);
+            const int E = mx_scale_byte<FMT, RULE>(m);
             sbyte = (uint32_t)E;
             if (ok) {
                 const float inv = mx_inv_scale(E);
@@ -411,24 +420,17 @@ __global__ void gscale_from_amax_kernel(float *__restrict__ slot) {
     *slot = amax > 0.0f ? __fdiv_ru(amax, 2688.0f) : 1.0f;
 }
 
-// Dequantize: 8 elements of one row per thread.  The exact value g*s*q is
-// formed in fp64 (at most 30 significant bits) and rounded once to bf16.
+// Decode 8 consecutive elements (row r, columns c..c+7) of a quantized matrix:
+// the block's scale s (g*s for NVFP4, exact in fp64) and the 8 element values.
 template <int FMT>
-__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restrict__ codes,
-                                                         const uint8_t *__restrict__ scales,
-                                                         const float *__restrict__ gscale, int64_t M, int64_t K,
-                                                         uint16_t *__restrict__ dst, int64_t ld) {
+MX_DEVICE_INLINE void load_dequant8(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                    const float *__restrict__ gscale, int64_t K, int64_t r, int64_t c, double &s,
+                                    float (&q)[8]) {
     using T = FmtTraits<FMT>;
-    const int64_t vec_per_row = K / 8;
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= M * vec_per_row) return;
-    const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
     const int64_t sf_cols = K / T::kBlock, tiles_k = (sf_cols + 3) / 4, j = c / T::kBlock;
     const uint8_t sb = scales[((r >> 7) * tiles_k + (j >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3)];
-    double s;
     if (FMT == FMT_NVFP4) s = (double)(*gscale) * (double)(sb == 0 ? 0.0f : e4m3_pos_value(sb));
     else s = sb == 0xFF ? (double)NAN : ldexp(1.0, (int)sb - 127);
-    float q[8];
     if (T::kBits == 8) {
         const uint2 w = *reinterpret_cast<const uint2 *>(codes + r * K + c);
         const uint32_t ww[2] = {w.x, w.y};
@@ -456,6 +458,22 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
             q[e] = (code & 8u) ? -mag : mag;
         }
     }
+}
+
+// Dequantize: 8 elements of one row per thread.  The exact value g*s*q is
+// formed in fp64 (at most 30 significant bits) and rounded once to bf16.
+template <int FMT>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restrict__ codes,
+                                                         const uint8_t *__restrict__ scales,
+                                                         const float *__restrict__ gscale, int64_t M, int64_t K,
+                                                         uint16_t *__restrict__ dst, int64_t ld) {
+    const int64_t vec_per_row = K / 8;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= M * vec_per_row) return;
+    const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
+    double s;
+    float q[8];
+    load_dequant8<FMT>(codes, scales, gscale, K, r, c, s, q);
     uint32_t out[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -464,6 +482,57 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
         out[e] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
     }
     *reinterpret_cast<uint4 *>(dst + r * ld + c) = make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// QSNR sums (page "Unveiling the Potential of Quantization with MXFP4",
+// sections 3-4: fidelity as quantization SNR): sums[0] += sum x^2 and
+// sums[1] += sum (x - xhat)^2 over a bf16 source [M x K] (pitch ld) and its
+// quantized form, in fp64 (x and xhat are exact there, the squares nearly so).
+// Grid-stride over 8-element vectors; one atomic add per block and sum.
+template <int FMT>
+__global__ void __launch_bounds__(256) qsnr_kernel(const uint16_t *__restrict__ src, int64_t ld,
+                                                   const uint8_t *__restrict__ codes,
+                                                   const uint8_t *__restrict__ scales,
+                                                   const float *__restrict__ gscale, int64_t M, int64_t K,
+                                                   double *__restrict__ sums) {
+    const int64_t vec_per_row = K / 8, nvec = M * vec_per_row;
+    double sx = 0.0, se = 0.0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
+        double s;
+        float q[8];
+        load_dequant8<FMT>(codes, scales, gscale, K, r, c, s, q);
+        const uint4 v = *reinterpret_cast<const uint4 *>(src + r * ld + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double x = (double)((e & 1) ? bf16hi(w[e >> 1]) : bf16lo(w[e >> 1]));
+            const double d = x - s * (double)q[e];
+            sx += x * x;
+            se += d * d;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sx += __shfl_xor_sync(0xffffffffu, sx, o);
+        se += __shfl_xor_sync(0xffffffffu, se, o);
+    }
+    __shared__ double red[2][8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[0][warp] = sx;
+        red[1][warp] = se;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double a = 0.0, b = 0.0;
+        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+            a += red[0][k];
+            b += red[1][k];
+        }
+        atomicAdd(&sums[0], a);
+        atomicAdd(&sums[1], b);
+    }
 }
 
 }  // namespace mx

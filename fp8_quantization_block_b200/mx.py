@@ -31,7 +31,7 @@ MX_DEBUG_WAIT_LIMIT_NS, MX_DEBUG_SKIP_PRODUCER, MX_DEBUG_PAIR_GEMM, MX_DEBUG_OVE
 EXPORTED = [
     "mx_codes_bytes", "mx_scales_bytes", "mx_block_size", "mx_quantize", "mx_dequantize", "mx_gemm",
     "mx_gemm_fused_act", "mx_fused_workspace_bytes", "mx_check_device_error", "mx_status_string",
-    "mx_version", "mx_debug_set", "mx_gemm_fused_act_noalloc",
+    "mx_version", "mx_debug_set", "mx_gemm_fused_act_noalloc", "mx_quantize_oas", "mx_qsnr",
 ]
 MX_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
                 "mx_block_size": (i32, [i32]),
                 "mx_quantize": (i32, [i32, P, i64, i64, i64, T, P, P]),
                 "mx_dequantize": (i32, [T, P, i64, P]),
+                "mx_quantize_oas": (i32, [P, i64, i64, i64, T, P]),
+                "mx_qsnr": (i32, [T, P, i64, P, P]),
                 "mx_gemm": (i32, [T, T, P, i64, P]),
                 "mx_gemm_fused_act": (i32, [i32, P, i64, i64, i64, T, P, i64, i32, P, P, P, P, sz, P]),
                 "mx_fused_workspace_bytes": (sz, [i32, i64, i64]),
@@ -99,6 +101,14 @@ def mx_block_size(fmt: int) -> int:
 
 def mx_quantize(fmt, src_ptr, M, K, ld, dst: MxTensorC, gscale_in_ptr, stream) -> int:
     return int(lib().mx_quantize(fmt, src_ptr, M, K, ld, ctypes.byref(dst), gscale_in_ptr, stream))
+
+
+def mx_quantize_oas(src_ptr, M, K, ld, dst: MxTensorC, stream) -> int:
+    return int(lib().mx_quantize_oas(src_ptr, M, K, ld, ctypes.byref(dst), stream))
+
+
+def mx_qsnr(q: MxTensorC, src_ptr, ld, sums_ptr, stream) -> int:
+    return int(lib().mx_qsnr(ctypes.byref(q), src_ptr, ld, sums_ptr, stream))
 
 
 def mx_dequantize(src: MxTensorC, dst_ptr, ld, stream) -> int:
@@ -194,6 +204,23 @@ def quantize(x: torch.Tensor, fmt: int, gscale: torch.Tensor | None = None, out:
     M, K = x.shape
     out = out if out is not None else empty(fmt, M, K, x.device)
     check(mx_quantize(fmt, x.data_ptr(), M, K, x.stride(0), out.c(), _ptr(gscale), _stream(stream)), "mx_quantize")
+    return out
+
+
+def quantize_oas(x: torch.Tensor, out: MxTensor | None = None, stream=None) -> MxTensor:
+    """bf16 [M, K] CUDA tensor -> MXFP4 MxTensor with overflow-aware block scales."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    out = out if out is not None else empty(MX_MXFP4, M, K, x.device)
+    check(mx_quantize_oas(x.data_ptr(), M, K, x.stride(0), out.c(), _stream(stream)), "mx_quantize_oas")
+    return out
+
+
+def qsnr_sums(t: MxTensor, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """float64 CUDA tensor [sum x^2, sum (x - dequant(t))^2]; QSNR dB = 10 log10(s[0] / s[1])."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    out = out if out is not None else torch.empty(2, dtype=torch.float64, device=x.device)
+    check(mx_qsnr(t.c(), x.data_ptr(), x.stride(0), out.data_ptr(), _stream(stream)), "mx_qsnr")
     return out
 
 

@@ -16,6 +16,10 @@
  *   [IMPL]  "Implementação da quantização NVFP4 e MXFP8" (matsubara.tec.br):
  *           Linear layers with both operands quantized, the quantize kernel as a
  *           bottleneck for small tensors, CUDA Graphs for batch-1 launches.
+ *   [OAS]   "Unveiling the Potential of Quantization with MXFP4: Strategies for
+ *           Quantization Error Reduction" (gist.science), section 2.A
+ *           (overflow-aware scaling) and sections 3-4 (QSNR as the fidelity
+ *           measure).
  *
  * Conventions for every call:
  *   - Device pointers are plain CUDA device addresses; the caller allocates and
@@ -108,6 +112,26 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
  * before the single rounding ([MX] "Fundamentos": x_real = S * x_elem).
  * ld_dst >= cols, ld_dst % 8 == 0. */
 mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, void *stream);
+
+/* MXFP4 with overflow-aware scaling ([OAS] section 2.A): as mx_quantize(MX_MXFP4, ...) except that each block's scale
+ * maps its max |x| into (3.5, 7] instead of (3, 6]:
+ *   E = ceil(log2(max|x| / 7)) + 127 clamped to [0, 254],
+ * elements = RNE(x / 2^(E-127)) saturating at 6 (so the block maximum may
+ * clip to 6 while the rest of the block gets a step half as large).  dst is an
+ * ordinary MXFP4 tensor (dst->fmt == MX_MXFP4): mx_dequantize and mx_gemm
+ * consume it unchanged.  Same requirements as mx_quantize. */
+mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
+                          void *stream);
+
+/* Quantization SNR inputs ([OAS] sections 3-4 report fidelity as QSNR):
+ * sums[0] = sum x^2 and sums[1] = sum (x - xhat)^2 over the bf16 source
+ * src [rows x cols] (pitch ld_src, ld_src % 8 == 0) and xhat = the
+ * dequantized value of q, accumulated in fp64 on the device; QSNR in dB is
+ * 10 log10(sums[0] / sums[1]).  sums: device pointer to 2 doubles (8-byte
+ * aligned), zeroed and then written by the call on `stream`; the summation
+ * order is unspecified (results agree with an fp64 reference to ~1e-12
+ * relative). */
+mx_status mx_qsnr(const mx_tensor *q, const void *src_bf16, int64_t ld_src, double *sums, void *stream);
 
 /* Block-scaled GEMM on the tensor cores ([MX] "Arquitetura Blackwell SM100"):
  *   C[i][j] = RNE_bf16( sum_k A_dq[i][k] * B_dq[j][k] ),  A [M x K], B [N x K],

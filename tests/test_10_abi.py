@@ -81,3 +81,15 @@ def test_host_checks_reject_bad_arguments(L):
     assert mx.mx_gemm(_t(0, 8, 256, codes=0x1001), B, 0x4000, 8, None) == mx.MX_ERR_MISALIGNED
     assert mx.mx_dequantize(_t(3, 4, 64, g=None), 0x4000, 64, None) == mx.MX_ERR_INVALID_ARG
     assert mx.mx_dequantize(_t(0, 4, 64), 0x4000, 60, None) == mx.MX_ERR_MISALIGNED
+
+
+def test_host_checks_oas_and_qsnr(L):
+    # fail before any CUDA call
+    assert mx.mx_quantize_oas(0x1000, 4, 64, 64, _t(0, 4, 64), None) == mx.MX_ERR_INVALID_ARG      # not MXFP4
+    assert mx.mx_quantize_oas(0x1000, 4, 48, 48, _t(2, 4, 48), None) == mx.MX_ERR_UNSUPPORTED_SHAPE
+    assert mx.mx_quantize_oas(0x1000, 4, 64, 64, _t(2, 4, 32), None) == mx.MX_ERR_INVALID_ARG      # shape mismatch
+    assert mx.mx_quantize_oas(0x1008, 4, 64, 64, _t(2, 4, 64), None) == mx.MX_ERR_MISALIGNED
+    assert mx.mx_quantize_oas(None, 0, 64, 64, _t(2, 0, 64), None) == mx.MX_OK                    # empty: no-op
+    assert mx.mx_qsnr(_t(2, 4, 64), 0x1000, 64, None, None) == mx.MX_ERR_INVALID_ARG               # no sums
+    assert mx.mx_qsnr(_t(2, 4, 64), 0x1000, 64, 0x5004, None) == mx.MX_ERR_MISALIGNED
+    assert mx.mx_qsnr(_t(9, 4, 64), 0x1000, 64, 0x5000, None) == mx.MX_ERR_INVALID_ARG
