@@ -263,6 +263,34 @@ def qsnr_table(device):
     return table
 
 
+def kv_cache_extras(device, peaks, timed):
+    """K/V-cache quantize of an 80-layer, 8-KV-head, 128-dim model: one row
+    per (token, layer, K or V) of 1024 values.  Prefill writes 4096 tokens at
+    once; a decode step writes one token for each of 54 concurrent sessions.
+    Synthetic N(0, 1) entries (drawn on the device)."""
+    import torch
+    from fp8_quantization_block_b200 import mx
+    rows_per_token, K = 160, 1024
+    g = torch.Generator(device=device).manual_seed(300)
+    res = {"bytes_per_token": {
+        "mxfp4": mx.mx_codes_bytes(2, rows_per_token, K) + rows_per_token * K // 32,
+        "mxfp8_e5m2": mx.mx_codes_bytes(1, rows_per_token, K) + rows_per_token * K // 32,
+        "bf16": rows_per_token * K * 2}}
+    for label, tokens in (("prefill_4096_tokens", 4096), ("decode_54_sessions", 54)):
+        M = tokens * rows_per_token
+        nsets = 2 if M * K * 2 > L2_BYTES else 8
+        xs = [torch.randn((M, K), generator=g, device=device).to(torch.bfloat16) for _ in range(nsets)]
+        for fmt, name in ((2, "mxfp4"), (1, "mxfp8_e5m2")):
+            qs = [mx.empty(fmt, M, K) for _ in xs]
+            ms = timed(lambda i: mx.quantize(xs[i % len(xs)], fmt, out=qs[i % len(xs)]), len(xs))
+            gbs = M * K * quant_bytes_per_elem(fmt) / (ms * 1e-3) / 1e9
+            res[f"{label}_{name}"] = {"rows": M, "us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                      "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+            del qs
+        del xs
+    return res
+
+
 def quant_bytes_per_elem(fmt):
     return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625}[fmt]
 
@@ -325,6 +353,7 @@ def extras_gpu(device):
     del xs, qs
     out["quantize_sweep"] = sweep
     out["qsnr_db"] = qsnr_table(device)
+    out["kv_cache"] = kv_cache_extras(device, peaks, timed)
     # GEMMs
     for name, (fmt, M, N, K) in {"mlp_nvfp4_gemm1": (3, 4608, 12288, 3072), "mlp_nvfp4_gemm2": (3, 4608, 3072, 12288),
                                  "skinny_nvfp4_M16": (3, 16, 28672, 8192), "skinny_mxfp4_M16": (2, 16, 28672, 8192),

@@ -75,6 +75,22 @@ def student_t(seed: int, M: int, K: int, nu: int = 3) -> np.ndarray:
     return to_bf16_bits(z / np.sqrt(chi2 / nu))
 
 
+def kv_cache(seed: int, tokens: int, layers: int = 80, kv_heads: int = 8, head_dim: int = 128,
+             outlier_dims: int = 2, factor: float = 15.0) -> np.ndarray:
+    """K/V cache entries of a grouped-query-attention model: one row per
+    (token, layer, K or V), row = kv_heads * head_dim values (heads
+    contiguous, each head_dim contiguous).  N(0, 1); in the K rows, a seeded
+    set of `outlier_dims` dimensions per head and layer is scaled by `factor`
+    (keys carry fixed outlier channels, values do not)."""
+    rng = _rng(seed)
+    x = rng.standard_normal((tokens, layers, 2, kv_heads, head_dim))
+    for layer in range(layers):
+        for h in range(kv_heads):
+            dims = rng.permutation(head_dim)[:outlier_dims]
+            x[:, layer, 0, h, dims] *= factor
+    return to_bf16_bits(x.reshape(tokens * layers * 2, kv_heads * head_dim))
+
+
 def sweep_tensor(seed: int, M: int, K: int = 4096) -> np.ndarray:
     rng = _rng(seed)
     return to_bf16_bits(normal_with_outliers(rng, (M, K), 0.005, 100.0))
