@@ -68,6 +68,8 @@ def _load():
                 "orc_amax_bf16": (d, [P, i64, i64, i64]),
                 "orc_quantize": (i32, [i32, P, i64, i64, i64, P, P, P, i32]),
                 "orc_quantize_oas": (i32, [P, i64, i64, i64, P, P]),
+                "orc_quantize_f32": (i32, [i32, P, i64, i64, i64, P, P, P, i32]),
+                "orc_rht32_f32": (i32, [P, i64, i64, i64, P]),
                 "orc_qsnr_db": (d, [P, i64, i64, i64, P, P]),
                 "orc_dequantize_f64": (i32, [i32, P, P, f32, i64, i64, P]),
                 "orc_dequantize_bf16": (i32, [i32, P, P, f32, i64, i64, P, i64]),
@@ -183,6 +185,37 @@ def quantize_oas(src_bits: np.ndarray):
     if rc != 0:
         raise ValueError(f"oracle quantize_oas failed with code {rc}")
     return codes, scales
+
+
+def rht32(src_bits: np.ndarray) -> np.ndarray:
+    """32-point Walsh-Hadamard rotation of every block along K, fp32 [M, K]
+    (butterflies of half-width 1, 2, 4, 8, 16 in fp32, then x RN_fp32(1/sqrt(32)))."""
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    M, K = src.shape
+    out = np.empty((M, K), dtype=np.float32)
+    rc = _load().orc_rht32_f32(_ptr(src), M, K, K, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle rht32 failed with code {rc}")
+    return out
+
+
+def quantize_f32(fmt: int, src: np.ndarray, gscale: float | None = None):
+    """fp32 [M, K] -> (codes, scales, g), the same rules as quantize()."""
+    x = np.ascontiguousarray(src, dtype=np.float32)
+    M, K = x.shape
+    codes = np.zeros(codes_bytes(fmt, M, K), dtype=np.uint8)
+    scales = np.zeros(scales_bytes(fmt, M, K), dtype=np.uint8)
+    g = np.array([1.0 if gscale is None else gscale], dtype=np.float32)
+    rc = _load().orc_quantize_f32(fmt, _ptr(x), M, K, K, _ptr(codes), _ptr(scales), _ptr(g),
+                                  0 if gscale is None else 1)
+    if rc != 0:
+        raise ValueError(f"oracle quantize_f32 failed with code {rc}")
+    return codes, scales, float(g[0])
+
+
+def quantize_rht(fmt: int, src_bits: np.ndarray, gscale: float | None = None):
+    """Rotate every 32-element block (rht32), then quantize the fp32 result."""
+    return quantize_f32(fmt, rht32(src_bits), gscale)
 
 
 def qsnr_db(src_bits: np.ndarray, xhat: np.ndarray):

@@ -129,10 +129,16 @@ def quantize(fmt: int, bits: np.ndarray, g: Fraction | None = None, mx_threshold
 
     Returns (codes[M][K] unpacked ints, scales[M][K/bs] ints, g)."""
     M, K = bits.shape
-    bs = BLOCK[fmt]
-    grid, sbit = GRIDS[fmt]
     X = [[bf16(int(bits[r, k])) for k in range(K)] for r in range(M)]
     neg = [[bool(int(bits[r, k]) & 0x8000) for k in range(K)] for r in range(M)]
+    return quantize_values(fmt, X, neg, g, mx_threshold)
+
+
+def quantize_values(fmt: int, X, neg, g: Fraction | None = None, mx_threshold: Fraction | None = None):
+    """quantize() on exact values X[M][K] (Fractions) with sign flags neg[M][K]."""
+    M, K = len(X), len(X[0])
+    bs = BLOCK[fmt]
+    grid, sbit = GRIDS[fmt]
     if fmt == 3 and g is None:
         g = nvfp4_global_scale(max(abs(x) for row in X for x in row))
     codes = [[0] * K for _ in range(M)]

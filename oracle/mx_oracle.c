@@ -330,20 +330,36 @@ double orc_amax_bf16(const uint16_t *src, int64_t M, int64_t K, int64_t ld) {
     return amax;
 }
 
-/* Quantize a row-major bf16 [M x K] matrix (row pitch ld elements).
+/* NVFP4 element: RNE of the real quotient |x| / denom onto E2M1 (ties to the
+ * even code), saturating at 6, decided by comparing |x| with each midpoint m
+ * times denom.  m has at most 3 significant bits and denom = g * s at most
+ * 28, so m * denom is exact in fp64 and every comparison is exact, whatever
+ * the precision of x (bf16 or fp32). */
+static uint8_t e2m1_encode_quotient(double x, double denom) {
+    static const double mids[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+    double a = fabs(x);
+    int c = 0;
+    for (int k = 0; k < 7; ++k) {
+        double t = mids[k] * denom;
+        if (a > t) c = k + 1;
+        else {
+            if (a == t) c = (k % 2 == 0) ? k : k + 1;   /* tie: the even code */
+            break;
+        }
+    }
+    return (uint8_t)(c | (signbit(x) ? 0x8 : 0));
+}
+
+/* Quantize a dense row-major [M x K] matrix of exactly-held values xv (fp64).
  * codes: orc_codes_bytes bytes; scales: orc_scales_bytes bytes (fully written,
  * padding 0).  NVFP4: if gscale_given, *gscale is used as g, else g is computed
- * and stored to *gscale.  Non-finite input is outside the contract: returns
- * ORC_ENONFINITE.  mx_threshold: the value a block's max |x| is mapped at or
- * below by the MX scale (the format's largest element for the OCP rule). */
-static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
-                         uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
+ * from max |xv| and stored to *gscale.  mx_threshold: the value a block's max
+ * |x| is mapped at or below by the MX scale (the format's largest element for
+ * the OCP rule). */
+static int quantize_core(int fmt, double mx_threshold, const double *xv, int64_t M, int64_t K, uint8_t *codes,
+                         uint8_t *scales, float *gscale, int gscale_given) {
     build_tables();
     int bs = fmt_block(fmt);
-    if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
-    for (int64_t r = 0; r < M; ++r)
-        for (int64_t k = 0; k < K; ++k)
-            if (!isfinite(orc_bf16_to_double(src[r * ld + k]))) return ORC_ENONFINITE;
     int64_t sf_cols = K / bs;
     memset(scales, 0, orc_scales_bytes(fmt, M, K));
     memset(codes, 0, orc_codes_bytes(fmt, M, K));
@@ -351,16 +367,21 @@ static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int6
     float g = 1.0f;
     if (fmt == ORC_NVFP4) {
         if (gscale_given) g = *gscale;
-        else { g = orc_nvfp4_global_scale(orc_amax_bf16(src, M, K, ld)); *gscale = g; }
+        else {
+            double amax_t = 0.0;
+            for (int64_t i = 0; i < M * K; ++i)
+                if (fabs(xv[i]) > amax_t) amax_t = fabs(xv[i]);
+            g = orc_nvfp4_global_scale(amax_t);
+            *gscale = g;
+        }
     }
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t j = 0; j < sf_cols; ++j) {
+            const double *blk = xv + r * K + j * bs;
             double amax = 0.0;
-            for (int i = 0; i < bs; ++i) {
-                double a = fabs(orc_bf16_to_double(src[r * ld + j * bs + i]));
-                if (a > amax) amax = a;
-            }
+            for (int i = 0; i < bs; ++i)
+                if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
             uint8_t sbyte;
             double denom;            /* the real number each element is divided by */
             if (fmt == ORC_NVFP4) {
@@ -372,23 +393,89 @@ static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int6
             }
             scales[orc_sf_offset(r, j, sf_cols)] = sbyte;
             for (int i = 0; i < bs; ++i) {
-                double x = orc_bf16_to_double(src[r * ld + j * bs + i]);
+                double x = blk[i];
                 uint8_t q;
-                if (denom == 0.0) {
+                if (denom == 0.0)
                     q = fmt_encode(fmt, signbit(x) ? -0.0 : 0.0);  /* all-zero NVFP4 block */
-                } else {
-                    /* MX: division by a power of two is exact.  NVFP4: if x/denom
-                     * is not a midpoint of the E2M1 grid it is at least 2^-31
-                     * (relative) away from every midpoint (x has 8 significant
-                     * bits, denom 28), far above the fp64 rounding error, and an
-                     * exact midpoint is returned exactly; so the fp64 quotient
-                     * rounds exactly as the real one does. */
-                    q = fmt_encode(fmt, x / denom);
-                }
+                else if (fmt == ORC_NVFP4)
+                    q = e2m1_encode_quotient(x, denom);
+                else
+                    q = fmt_encode(fmt, x / denom);                /* exact: a power of two */
                 put_code(fmt, codes, K, r, j * bs + i, q);
             }
         }
     }
+    return ORC_OK;
+}
+
+/* bf16 source with row pitch ld: checks, widening to fp64 (exact), quantize. */
+static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
+                         uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
+    int bs = fmt_block(fmt);
+    if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    double *xv = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
+    if (!xv) return ORC_EINVAL;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double x = orc_bf16_to_double(src[r * ld + k]);
+            if (!isfinite(x)) {
+                free(xv);
+                return ORC_ENONFINITE;
+            }
+            xv[r * K + k] = x;
+        }
+    int rc = quantize_core(fmt, mx_threshold, xv, M, K, codes, scales, gscale, gscale_given);
+    free(xv);
+    return rc;
+}
+
+/* Quantize an fp32 source [M x K] (row pitch ld), e.g. a rotated tensor. */
+int orc_quantize_f32(int fmt, const float *src, int64_t M, int64_t K, int64_t ld, uint8_t *codes, uint8_t *scales,
+                     float *gscale, int gscale_given) {
+    int bs = fmt_block(fmt);
+    if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    double *xv = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
+    if (!xv) return ORC_EINVAL;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double x = (double)src[r * ld + k];
+            if (!isfinite(x)) {
+                free(xv);
+                return ORC_ENONFINITE;
+            }
+            xv[r * K + k] = x;
+        }
+    int rc = quantize_core(fmt, fmt_maxelem(fmt), xv, M, K, codes, scales, gscale, gscale_given);
+    free(xv);
+    return rc;
+}
+
+/* Walsh-Hadamard rotation of every 32-element block along K [MX page, section
+ * "Técnicas de preservação de acurácia": Hadamard / Walsh-Hadamard rotations
+ * spread a block's outlier energy over its 32 elements]:
+ *   y_b = c * (H32 x_b),  H32 the Sylvester-ordered Hadamard matrix
+ *   (H1 = [1], H2n = [[Hn, Hn], [Hn, -Hn]]),  c = RN_fp32(1 / sqrt(32)),
+ * evaluated in fp32 exactly this way: butterflies with half-widths 1, 2, 4, 8,
+ * 16 in that order, each (a, b) -> (a + b, a - b) rounded to fp32, then one
+ * fp32 multiplication by c.  (The rounding of the intermediate sums is part of
+ * the definition, so that a device computing the same steps matches bit for
+ * bit.)  K % 32 == 0. */
+int orc_rht32_f32(const uint16_t *src, int64_t M, int64_t K, int64_t ld, float *dst) {
+    if (M < 0 || K < 0 || K % 32 != 0 || ld < K) return ORC_EINVAL;
+    const float c = (float)(1.0 / sqrt(32.0));
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t j = 0; j < K / 32; ++j) {
+            float v[32];
+            for (int i = 0; i < 32; ++i) v[i] = (float)orc_bf16_to_double(src[r * ld + j * 32 + i]);
+            for (int h = 1; h < 32; h <<= 1)
+                for (int i0 = 0; i0 < 32; i0 += 2 * h)
+                    for (int i = i0; i < i0 + h; ++i) {
+                        float a = v[i], b = v[i + h];
+                        v[i] = a + b;
+                        v[i + h] = a - b;
+                    }
+            for (int i = 0; i < 32; ++i) dst[r * K + j * 32 + i] = v[i] * c;
+        }
     return ORC_OK;
 }
 
