@@ -13,6 +13,7 @@
 #include "mx.h"
 #include "mx_common.cuh"
 #include "quantize.cuh"
+#include "rotate.cuh"
 #include "gemm_sm100.cuh"
 #include "gemm_pair_sm100.cuh"
 
@@ -97,6 +98,22 @@ void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, cons
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
     cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
+                       sf_tiles_k, g_in, g_out, g_from_amax);
+}
+
+template <int FMT>
+void launch_quantize_rht(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
+                         const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
+    const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows), 1);
+    cfg.blockDim = dim3(kQThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    cudaLaunchKernelEx(&cfg, quantize_rht_kernel<FMT>, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
                        sf_tiles_k, g_in, g_out, g_from_amax);
 }
 
@@ -441,6 +458,45 @@ mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld
     if (cdiv(M, kQTileRows) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
     launch_quantize<2, RULE_OAS>(static_cast<const uint16_t *>(src_bf16), M, K, ld_src, dst, nullptr, nullptr,
                                  static_cast<cudaStream_t>(stream));
+    return last_launch();
+}
+
+mx_status mx_quantize_rht(int fmt, const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
+                          const float *gscale_in, void *stream) {
+    if (!valid_fmt(fmt) || !dst || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    if (dst->fmt != fmt || dst->rows != M || dst->cols != K) return MX_ERR_INVALID_ARG;
+    if (K % 32 != 0) return MX_ERR_UNSUPPORTED_SHAPE;   // rotation blocks of 32
+    if (M == 0 || K == 0) return MX_OK;
+    if (!src_bf16 || !dst->codes || !dst->scales) return MX_ERR_INVALID_ARG;
+    if (fmt == MX_NVFP4 && !dst->gscale) return MX_ERR_INVALID_ARG;
+    if (ld_src < K || (ld_src & 7) != 0) return MX_ERR_MISALIGNED;
+    if (!aligned16(src_bf16) || !aligned16(dst->codes) || !aligned16(dst->scales)) return MX_ERR_MISALIGNED;
+    if (cdiv(M, kQTileRows) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint16_t *src = static_cast<const uint16_t *>(src_bf16);
+    switch (fmt) {
+    case MX_MXFP8_E4M3: launch_quantize_rht<0>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP8_E5M2: launch_quantize_rht<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP4: launch_quantize_rht<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    default: {
+        if (gscale_in == nullptr) {
+            // g from max |y| of the rotated tensor: an extra read of src
+            if (cudaMemsetAsync(dst->gscale, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
+            const int64_t pairs = M * (K / 32);
+            int64_t blocks = cdiv(pairs * 2, 256);
+            const int64_t cap = (int64_t)num_sms() * 8;
+            if (blocks > cap) blocks = cap;
+            if (blocks < 1) blocks = 1;
+            amax_rht_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, M, K, ld_src,
+                                                              reinterpret_cast<unsigned int *>(dst->gscale));
+            gscale_from_amax_kernel<<<1, 1, 0, st>>>(dst->gscale);
+            launch_quantize_rht<3>(src, M, K, ld_src, dst, dst->gscale, nullptr, st);
+        } else {
+            launch_quantize_rht<3>(src, M, K, ld_src, dst, gscale_in,
+                                   gscale_in == dst->gscale ? nullptr : dst->gscale, st);
+        }
+    }
+    }
     return last_launch();
 }
 

@@ -1,0 +1,274 @@
+// rotate.cuh -- 32-point Walsh-Hadamard block rotation fused with quantization.
+//
+// Page "Microscaling MXFP4/NVFP4 on Blackwell for reasoning LLMs", section
+// "Técnicas de preservação de acurácia: QuaRot, SpinQuant e ReSET": Hadamard /
+// Walsh-Hadamard rotations spread a block's outlier energy over its 32
+// elements before 4-bit quantization.  Each 32-element block b of a row is
+// replaced by y_b = c * (H32 x_b), H32 the Sylvester-ordered Hadamard matrix
+// and c = RN_fp32(1/sqrt(32)) (0x3E3504F3), evaluated in fp32 as butterflies of
+// half-width 1, 2, 4, 8, 16 in that order, each (a, b) -> (a + b, a - b) with
+// one rounding, then one product with c; the fp32 y is quantized by the usual
+// rules (MX: E = ceil(log2(max|y| / max_elem)) + 127; NVFP4: s and RNE of
+// y / (g s)).  Applying the same rotation to both GEMM operands leaves
+// A * B^T unchanged up to rounding, since H32 H32^T = 32 I.
+//
+// Thread layout as in quantize_kernel: a 128 x 128 tile per CTA, 16
+// consecutive elements per thread, so a 32-element block spans lanes 2m and
+// 2m + 1; the last butterfly stage exchanges halves with __shfl_xor(., 1).
+#pragma once
+
+#include "quantize.cuh"
+
+namespace mx {
+
+constexpr uint32_t kRhtScaleBits = 0x3E3504F3u;  // RN_fp32(1 / sqrt(32))
+
+// Rotate the 32-element block whose half (16 values) this thread holds: lower
+// = even lane (elements 0..15 of the block), upper = odd lane.  All 32 lanes
+// of the warp must call this together.
+MX_DEVICE_INLINE void rht32_halves(float (&x)[16], int lane) {
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i0 = 0; i0 < 16; i0 += 2 * h) {
+#pragma unroll
+            for (int i = i0; i < i0 + h; ++i) {
+                const float a = x[i], b = x[i + h];
+                x[i] = __fadd_rn(a, b);
+                x[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+    const bool upper = (lane & 1) != 0;
+    const float c = __uint_as_float(kRhtScaleBits);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float other = __shfl_xor_sync(0xffffffffu, x[i], 1);
+        // pair (i, i + 16): lower = a + b, upper = a - b, with a the lower value
+        const float v = upper ? __fsub_rn(other, x[i]) : __fadd_rn(x[i], other);
+        x[i] = __fmul_rn(v, c);
+    }
+}
+
+MX_DEVICE_INLINE void unpack16(const uint4 &v0, const uint4 &v1, float (&x)[16]) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = bf16lo(w[i]);
+        x[2 * i + 1] = bf16hi(w[i]);
+    }
+}
+
+// MX exponent from the fp32 bits of a block's max |y| (non-negative, finite):
+// amax = 1.m * 2^(f-127), max_elem = M * 2^k: E = f - k + (m > (M - 1) 2^23),
+// clamped below at 0 (zero and tiny maxima).
+template <int FMT>
+MX_DEVICE_INLINE int mx_scale_byte_f32(float amax) {
+    using T = FmtTraits<FMT>;
+    const uint32_t bits = __float_as_uint(amax);
+    const uint32_t thr = (uint32_t)T::kMantThr << 16;   // the bf16 threshold, widened to 23 mantissa bits
+    int e = (int)(bits >> 23) - T::kExpOff + (((bits & 0x7FFFFFu) > thr) ? 1 : 0);
+    return e < 0 ? 0 : e;
+}
+
+// NVFP4 codes of 16 fp32 values: the bracket of nv_codes16 on fp32 inputs.
+MX_DEVICE_INLINE uint32_t nv_settle_f32(uint32_t code, uint32_t diff, const float *x8, float g, float s) {
+    while (diff != 0u) {
+        const int nib = (__ffs(diff) - 1) >> 2;
+        diff &= ~(0xFu << (4 * nib));
+        float ax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i == nib) ax = fabsf(x8[i]);
+        const uint32_t c = (code >> (4 * nib)) & 7u;
+        const float d = __fmaf_rn(-g, s * e2m1_mid(c), ax);
+        if (d > 0.0f || (d == 0.0f && (c & 1u))) code += 1u << (4 * nib);
+    }
+    return code;
+}
+
+MX_DEVICE_INLINE void nv_codes16_f32(const float (&x)[16], float g, float s, float r_lo, float r_hi,
+                                     uint32_t &out0, uint32_t &out1) {
+    float lo[16], hi[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        lo[i] = __fmul_rz(x[i], r_lo);
+        hi[i] = __fmul_ru(fabsf(x[i]), r_hi);
+    }
+    const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
+    const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
+    const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
+    const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
+    uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
+    const uint32_t d0 = (c0 & 0x77777777u) ^ cvt8_e2m1(hi0), d1 = (c1 & 0x77777777u) ^ cvt8_e2m1(hi1);
+    if ((d0 | d1) != 0u) {
+        c0 = nv_settle_f32(c0, d0, &x[0], g, s);
+        c1 = nv_settle_f32(c1, d1, &x[8], g, s);
+    }
+    out0 = c0;
+    out1 = c1;
+}
+
+// Rotate and quantize a bf16 [M x K] matrix (K % 32 == 0) into codes / scales
+// laid out as quantize_kernel's.  NVFP4: *gscale_in is g, or max|y| when
+// g_from_amax (then g = RU(max|y| / 2688), 1 for 0); gscale_out as there.
+template <int FMT>
+__global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t *__restrict__ src, int64_t M,
+                                                                 int64_t K, int64_t ld, uint8_t *__restrict__ codes,
+                                                                 uint8_t *__restrict__ scales, int64_t sf_tiles_k,
+                                                                 const float *__restrict__ gscale_in,
+                                                                 float *__restrict__ gscale_out, int g_from_amax) {
+    using T = FmtTraits<FMT>;
+    constexpr int kBlocksPerRow = kQTileCols / T::kBlock;
+    constexpr int kSfBytes = kQTileRows * kBlocksPerRow;
+    constexpr int kPasses = kQTileRows / 32;
+    __shared__ __align__(16) uint8_t sf_tile[kSfBytes];
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row0 = (int64_t)blockIdx.y * kQTileRows;
+    const int64_t col0 = (int64_t)blockIdx.x * kQTileCols;
+    const int cl = (lane & 7) * 16;
+    const int64_t col = col0 + cl;
+    const bool col_ok = col < K;   // K % 32 == 0: both halves of a block exist or neither
+    const int jb = cl / T::kBlock;
+
+    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f;
+    __shared__ NvTables nvt;
+    griddep_wait();
+    if (FMT == FMT_NVFP4) {
+        g = *gscale_in;
+        if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;
+        if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
+        rg_lo = __frcp_rd(g);
+        rg_hi = __frcp_ru(g);
+        inv6g = 1.0f / (6.0f * g);
+        if (threadIdx.x < 128) {
+            const uint32_t c = threadIdx.x;
+            const float v = (c == 0u || c == 127u) ? 0.0f : e4m3_pos_value(c);
+            nvt.val[c] = v;
+            nvt.inv_lo[c] = v > 0.0f ? __frcp_rd(v) : 0.0f;
+            nvt.inv_hi[c] = v > 0.0f ? __frcp_ru(v) : 0.0f;
+        }
+        __syncthreads();
+    }
+
+    uint4 v[kPasses][2];
+#pragma unroll
+    for (int i = 0; i < kPasses; ++i) {
+        const int rl = i * 32 + warp * 4 + (lane >> 3);
+        const int64_t row = row0 + rl;
+        if (row < M && col_ok) {
+            const uint16_t *p = src + row * ld + col;
+            v[i][0] = ldg_stream(p);
+            v[i][1] = ldg_stream(p + 8);
+        } else {
+            v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+
+#pragma unroll
+    for (int i = 0; i < kPasses; ++i) {
+        const int rl = i * 32 + warp * 4 + (lane >> 3);
+        const int64_t row = row0 + rl;
+        const bool ok = row < M && col_ok;
+        float y[16];
+        unpack16(v[i][0], v[i][1], y);
+        rht32_halves(y, lane);
+        float m = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(y[e]));
+        if (T::kBlock == 32) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        uint32_t sbyte;
+        if (FMT == FMT_NVFP4) {
+            sbyte = nv_block_scale(m, g, inv6g, nvt.val);
+            if (ok) {
+                uint32_t q0 = 0, q1 = 0;
+                if (sbyte == 0u) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint32_t sgn = (__float_as_uint(y[e]) >> 31) & 1u;
+                        if (e < 8) q0 |= sgn << (4 * e + 3);
+                        else q1 |= sgn << (4 * (e - 8) + 3);
+                    }
+                } else {
+                    const float r_lo = __fmul_rd(rg_lo, nvt.inv_lo[sbyte]);
+                    const float r_hi = __fmul_ru(rg_hi, nvt.inv_hi[sbyte]);
+                    nv_codes16_f32(y, g, nvt.val[sbyte], r_lo, r_hi, q0, q1);
+                }
+                *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
+            }
+        } else {
+            const int E = mx_scale_byte_f32<FMT>(m);
+            sbyte = (uint32_t)E;
+            if (ok) {
+                const float inv = mx_inv_scale(E);
+                float f[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) f[e] = y[e] * inv;
+                if (T::kBits == 8) {
+                    uint4 q;
+                    q.x = cvt4_fp8<FMT>(f[0], f[1], f[2], f[3]);
+                    q.y = cvt4_fp8<FMT>(f[4], f[5], f[6], f[7]);
+                    q.z = cvt4_fp8<FMT>(f[8], f[9], f[10], f[11]);
+                    q.w = cvt4_fp8<FMT>(f[12], f[13], f[14], f[15]);
+                    *reinterpret_cast<uint4 *>(codes + row * K + col) = q;
+                } else {
+                    const float(&f0)[8] = *reinterpret_cast<const float(*)[8]>(&f[0]);
+                    const float(&f1)[8] = *reinterpret_cast<const float(*)[8]>(&f[8]);
+                    *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(cvt8_e2m1(f0), cvt8_e2m1(f1));
+                }
+            }
+        }
+        const bool owner = T::kBlock == 16 || (lane & 1) == 0;
+        if (owner) {
+            const int64_t jglob = col0 / T::kBlock + jb;
+            if (!(row < M) || jglob >= K / T::kBlock) sbyte = 0u;
+            sf_tile[(jb >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (jb & 3)] = (uint8_t)sbyte;
+        }
+    }
+    __syncthreads();
+    constexpr int kChunks = kSfBytes / 512;
+    const int64_t chunk0 = (int64_t)blockIdx.y * sf_tiles_k + (int64_t)blockIdx.x * kChunks;
+    const int64_t max_chunk = (int64_t)blockIdx.y * sf_tiles_k + sf_tiles_k;
+    if (threadIdx.x < kSfBytes / 16) {
+        const int c = threadIdx.x / 32;
+        if (chunk0 + c < max_chunk) {
+            uint4 val = *reinterpret_cast<const uint4 *>(sf_tile + threadIdx.x * 16);
+            *reinterpret_cast<uint4 *>(scales + chunk0 * 512 + threadIdx.x * 16) = val;
+        }
+    }
+    // the next kernel in the stream may start its setup now
+    griddep_launch_dependents();
+}
+
+// max |y| over the rotated tensor (for the NVFP4 global scale): one 32-element
+// block per thread pair, grid-stride over pairs; atomicMax on float bits.
+__global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
+                                                       int64_t ld, unsigned int *__restrict__ amax_bits) {
+    const int lane = threadIdx.x & 31;
+    const int64_t halves_per_row = K / 16;   // even: a block's two halves are 2b, 2b + 1
+    const int64_t nhalves = M * halves_per_row;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    float m = 0.0f;
+    // every lane of a warp runs the same iterations, so each shuffle has both halves
+    for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w * 32 < nhalves; w += nwarps) {
+        const int64_t i = w * 32 + lane;
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (i < nhalves) {
+            const int64_t r = i / halves_per_row, c = (i % halves_per_row) * 16;
+            const uint16_t *p = src + r * ld + c;
+            v0 = ldg_stream(p);
+            v1 = ldg_stream(p + 8);
+        }
+        float y[16];
+        unpack16(v0, v1, y);
+        rht32_halves(y, lane);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(y[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0 && m > 0.0f) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+}  // namespace mx

@@ -123,6 +123,24 @@ mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, vo
 mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
                           void *stream);
 
+/* Walsh-Hadamard rotation fused with quantization ([MX] section "Técnicas de
+ * preservação de acurácia": Hadamard rotations spread a block's outlier
+ * energy over its 32 elements before 4-bit quantization).  Every 32-element
+ * block x_b along K is replaced by
+ *   y_b = c * (H32 x_b),  H32 the Sylvester-ordered Hadamard matrix
+ *   (H1 = [1], H2n = [[Hn, Hn], [Hn, -Hn]]),  c = RN_fp32(1 / sqrt(32)),
+ * computed in fp32 as butterflies of half-width 1, 2, 4, 8, 16 in that order
+ * (each (a, b) -> (a + b, a - b), rounded), then one product with c; y is then
+ * quantized exactly as mx_quantize quantizes its input (NVFP4: g from
+ * gscale_in, else RU(max|y| / 2688) from an extra pass over src).  Rotating
+ * both GEMM operands this way leaves A * B^T unchanged up to rounding
+ * (H32 H32^T = 32 I).  K % 32 == 0; otherwise as mx_quantize.  A block
+ * whose butterfly sums overflow fp32 (possible only when its inputs come
+ * within a factor 32 of the bf16 maximum) is outside the contract, like a
+ * non-finite input. */
+mx_status mx_quantize_rht(int fmt, const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
+                          const float *gscale_in, void *stream);
+
 /* Quantization SNR inputs ([OAS] sections 3-4 report fidelity as QSNR):
  * sums[0] = sum x^2 and sums[1] = sum (x - xhat)^2 over the bf16 source
  * src [rows x cols] (pitch ld_src, ld_src % 8 == 0) and xhat = the
