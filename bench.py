@@ -259,8 +259,28 @@ def qsnr_table(device):
                              ("mxfp4_oas", lambda: mx.quantize_oas(x)), ("nvfp4", lambda: mx.quantize(x, 3))):
             s = mx.qsnr_sums(quant(), x).cpu().numpy()
             row[label] = round(float(10.0 * np.log10(s[0] / s[1])), 3)
+        for label, fmt in (("mxfp4_rht32", 2), ("nvfp4_rht32", 3)):
+            row[label] = round(rotated_qsnr_db(x, mx.quantize_rht(x, fmt)), 3)
         table[name] = row
     return table
+
+
+def rotated_qsnr_db(x, q):
+    """QSNR of a tensor quantized after the 32-point Walsh-Hadamard rotation,
+    measured in the original domain: dequantize (bf16), rotate back (the
+    normalised Hadamard matrix is its own inverse), compare with x in fp64.
+    The bf16 rounding of the dequantized values adds ~1e-6 of relative error
+    energy, negligible next to the 4-bit error."""
+    import torch
+    from fp8_quantization_block_b200 import mx
+    M, K = x.shape
+    h = torch.ones((1, 1), dtype=torch.float64, device=x.device)
+    while h.shape[0] < 32:
+        h = torch.cat([torch.cat([h, h], 1), torch.cat([h, -h], 1)], 0)
+    y = mx.dequantize(q).double().reshape(M, K // 32, 32)
+    xr = (y @ h) / np.sqrt(32.0)
+    xd = x.double().reshape(M, K // 32, 32)
+    return float(10.0 * torch.log10((xd * xd).sum() / ((xd - xr) ** 2).sum()))
 
 
 def kv_cache_extras(device, peaks, timed):
@@ -350,7 +370,18 @@ def extras_gpu(device):
     ms = timed(lambda i: mx.quantize_oas(xs[i % len(xs)], out=qs[i % len(xs)]), len(xs))
     gbs = M * K * quant_bytes_per_elem(2) / (ms * 1e-3) / 1e9
     sweep[f"mxfp4_oas_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
-    del xs, qs
+    del qs
+    # Walsh-Hadamard rotation fused with quantization: the same HBM bytes as the plain quantize
+    for fmt, name in ((2, "mxfp4_rht32"), (3, "nvfp4_rht32")):
+        qs = [mx.empty(fmt, M, K) for _ in xs]
+        gss = [mx.quantize_rht(x, fmt, out=qs[i]).gscale.clone() if fmt == 3 else None for i, x in enumerate(xs)]
+        ms = timed(lambda i: mx.quantize_rht(xs[i % len(xs)], fmt, gscale=gss[i % len(xs)], out=qs[i % len(xs)]),
+                   len(xs))
+        gbs = M * K * quant_bytes_per_elem(fmt) / (ms * 1e-3) / 1e9
+        sweep[f"{name}_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                 "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        del qs
+    del xs
     out["quantize_sweep"] = sweep
     out["qsnr_db"] = qsnr_table(device)
     out["kv_cache"] = kv_cache_extras(device, peaks, timed)
