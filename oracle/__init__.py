@@ -22,8 +22,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mx_oracle.c")
 _LIB = os.path.join(_HERE, "libmxoracle.so")
 
-MXFP8_E4M3, MXFP8_E5M2, MXFP4, NVFP4 = 0, 1, 2, 3
-FORMAT_NAMES = {MXFP8_E4M3: "mxfp8_e4m3", MXFP8_E5M2: "mxfp8_e5m2", MXFP4: "mxfp4", NVFP4: "nvfp4"}
+MXFP8_E4M3, MXFP8_E5M2, MXFP4, NVFP4, MXFP6_E3M2 = 0, 1, 2, 3, 4
+FORMAT_NAMES = {MXFP8_E4M3: "mxfp8_e4m3", MXFP8_E5M2: "mxfp8_e5m2", MXFP4: "mxfp4", NVFP4: "nvfp4",
+                MXFP6_E3M2: "mxfp6_e3m2"}
 
 _lock = threading.Lock()
 _lib = None
@@ -53,10 +54,12 @@ def _load():
                 "orc_e2m1_decode": (d, [u8]),
                 "orc_e4m3_decode": (d, [u8]),
                 "orc_e5m2_decode": (d, [u8]),
+                "orc_e3m2_decode": (d, [u8]),
                 "orc_e8m0_decode": (d, [u8]),
                 "orc_e2m1_encode": (u8, [d]),
                 "orc_e4m3_encode": (u8, [d]),
                 "orc_e5m2_encode": (u8, [d]),
+                "orc_e3m2_encode": (u8, [d]),
                 "orc_block_size": (i32, [i32]),
                 "orc_max_element": (d, [i32]),
                 "orc_codes_bytes": (ctypes.c_size_t, [i32, i64, i64]),

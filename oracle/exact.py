@@ -21,7 +21,7 @@ from fractions import Fraction
 
 import numpy as np
 
-E2M1_BITS, E4M3_BITS, E5M2_BITS = (1, 2, 1), (1, 4, 3), (1, 5, 2)
+E2M1_BITS, E4M3_BITS, E5M2_BITS, E3M2_BITS = (1, 2, 1), (1, 4, 3), (1, 5, 2), (1, 3, 2)
 
 
 def _minifloat(code: int, ebits: int, mbits: int, bias: int) -> Fraction | None:
@@ -51,6 +51,11 @@ def e5m2(code: int) -> Fraction | None:
     return _minifloat(code, 5, 2, 15)
 
 
+def e3m2(code: int) -> Fraction:
+    """OCP 6-bit E3M2: bias 3, every code finite."""
+    return _minifloat(code & 0x3F, 3, 2, 3)
+
+
 def bf16(bits: int) -> Fraction:
     s = (bits >> 15) & 1
     e = (bits >> 7) & 0xFF
@@ -67,9 +72,12 @@ def bf16(bits: int) -> Fraction:
 E2M1_GRID = [(e2m1(c), c) for c in range(8)]
 E4M3_GRID = [(e4m3(c), c) for c in range(0x7F)]
 E5M2_GRID = [(e5m2(c), c) for c in range(0x7C)]
-GRIDS = {0: (E4M3_GRID, 0x80), 1: (E5M2_GRID, 0x80), 2: (E2M1_GRID, 0x8), 3: (E2M1_GRID, 0x8)}
-MAXELEM = {0: Fraction(448), 1: Fraction(57344), 2: Fraction(6), 3: Fraction(6)}
-BLOCK = {0: 32, 1: 32, 2: 32, 3: 16}
+E3M2_GRID = [(e3m2(c), c) for c in range(0x20)]
+GRIDS = {0: (E4M3_GRID, 0x80), 1: (E5M2_GRID, 0x80), 2: (E2M1_GRID, 0x8), 3: (E2M1_GRID, 0x8),
+         4: (E3M2_GRID, 0x20)}
+MAXELEM = {0: Fraction(448), 1: Fraction(57344), 2: Fraction(6), 3: Fraction(6), 4: Fraction(28)}
+BLOCK = {0: 32, 1: 32, 2: 32, 3: 16, 4: 32}
+DECODE = {0: e4m3, 1: e5m2, 2: e2m1, 3: e2m1, 4: e3m2}
 
 
 def round_to_grid(v: Fraction, grid, sign_bit: int, negative: bool) -> int:
@@ -174,7 +182,7 @@ def dequant(fmt: int, codes, scales, g: Fraction | None):
                 v = e2m1(c)
             else:
                 s = Fraction(2) ** (sc - 127)
-                v = e2m1(c) if fmt == 2 else (e4m3(c) if fmt == 0 else e5m2(c))
+                v = DECODE[fmt](c)
             orow.append(s * v)
         out.append(orow)
     return out

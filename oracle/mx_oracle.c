@@ -1,6 +1,7 @@
 /*
  * mx_oracle.c -- plain, slow, obviously-correct CPU oracle for microscaling
- * quantization (MXFP8 E4M3/E5M2, MXFP4, NVFP4) and the block-scaled GEMM.
+ * quantization (MXFP8 E4M3/E5M2, MXFP6 E3M2, MXFP4, NVFP4) and the
+ * block-scaled GEMM.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
  * call this file; only the tests, the package's smoke check and the benchmark's
@@ -16,7 +17,9 @@
  *                 formula, dequantization by multiplication, 4.25 bits/element,
  *                 format table with the E4M3 range [-448, 448]) and the FAQ entry
  *                 on how E8M0 computes the block's shared exponent (the ceil
- *                 scale rule).
+ *                 scale rule).  The same page's format table lists MXFP6 as
+ *                 E3M2 elements with an E8M0 scale per 32-element block,
+ *                 6.25 bits/element.
  *   [NVFP4-news]  "NVIDIA's FP4 format delivers 1.68x speedup" (zubnet.ai):
  *                 NVFP4 = E2M1 elements in 16-element blocks; MXFP8 = E4M3/E5M2
  *                 elements in 32-element blocks (OCP standard).
@@ -39,7 +42,11 @@
  *   R6  FP4 packing: byte j of a row = code[2j] | code[2j+1] << 4;
  *   R7  block-scale byte (r, c) of an [R x C] scale matrix lives at
  *       ((r/128) * ceil(C/4) + c/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4,
- *       padding bytes are 0.
+ *       padding bytes are 0;
+ *   R18 E3M2 is the OCP 6-bit layout (sign, 3 exponent bits with bias 3, 2
+ *       mantissa bits, no infinities or NaN, largest magnitude 28); MXFP6
+ *       packing: code k of a row occupies bits 6k .. 6k+5 of the row read as
+ *       one little-endian bit string (16 codes in 12 bytes).
  */
 #include <math.h>
 #include <stdint.h>
@@ -50,7 +57,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_MXFP8_E4M3 = 0, ORC_MXFP8_E5M2 = 1, ORC_MXFP4 = 2, ORC_NVFP4 = 3 };
+enum { ORC_MXFP8_E4M3 = 0, ORC_MXFP8_E5M2 = 1, ORC_MXFP4 = 2, ORC_NVFP4 = 3, ORC_MXFP6_E3M2 = 4 };
 enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_ENONFINITE = 2 };
 
 /* ------------------------------------------------------------------------- */
@@ -147,6 +154,15 @@ double orc_e5m2_decode(uint8_t code) {
     return s ? -mag : mag;
 }
 
+/* E3M2 [MXFP4-page format table, MXFP6 (E3M2); reading R18]: bit 5 sign,
+ * bits 4-2 exponent with bias 3, bits 1-0 mantissa; exponent field 0 is
+ * subnormal (m/4 * 2^-2); every code is finite, the largest 1.75 * 2^4 = 28. */
+double orc_e3m2_decode(uint8_t code) {
+    int s = (code >> 5) & 1, e = (code >> 2) & 7, m = code & 3;
+    double mag = (e == 0) ? ldexp((double)m, -4) : ldexp(1.0 + m / 4.0, e - 3);
+    return s ? -mag : mag;
+}
+
 /* E8M0 [MXFP4-page, Fundamentos]: Escala = 2^(E - 127); 0xFF is NaN. */
 double orc_e8m0_decode(uint8_t code) {
     if (code == 0xFF) return NAN;
@@ -158,6 +174,7 @@ double orc_e8m0_decode(uint8_t code) {
 static double g_e2m1_pos[8];
 static double g_e4m3_pos[127];   /* codes 0x00 .. 0x7E */
 static double g_e5m2_pos[124];   /* codes 0x00 .. 0x7B */
+static double g_e3m2_pos[32];    /* codes 0x00 .. 0x1F */
 static int g_tables_ready = 0;
 
 static void build_tables(void) {
@@ -165,6 +182,7 @@ static void build_tables(void) {
     for (int c = 0; c < 8; ++c) g_e2m1_pos[c] = orc_e2m1_decode((uint8_t)c);
     for (int c = 0; c < 127; ++c) g_e4m3_pos[c] = orc_e4m3_decode((uint8_t)c);
     for (int c = 0; c < 124; ++c) g_e5m2_pos[c] = orc_e5m2_decode((uint8_t)c);
+    for (int c = 0; c < 32; ++c) g_e3m2_pos[c] = orc_e3m2_decode((uint8_t)c);
     g_tables_ready = 1;
 }
 
@@ -205,15 +223,25 @@ uint8_t orc_e5m2_encode(double v) {
     return (uint8_t)(c | (signbit(v) ? 0x80 : 0));
 }
 
+uint8_t orc_e3m2_encode(double v) {
+    build_tables();
+    int c = rne_index(g_e3m2_pos, 32, fabs(v));
+    return (uint8_t)(c | (signbit(v) ? 0x20 : 0));
+}
+
 /* ------------------------------------------------------------------------- */
 /* format parameters                                                         */
 /* ------------------------------------------------------------------------- */
 static int fmt_block(int fmt) { return fmt == ORC_NVFP4 ? 16 : 32; }
-static int fmt_bits(int fmt) { return (fmt == ORC_MXFP4 || fmt == ORC_NVFP4) ? 4 : 8; }
+static int fmt_ok(int fmt) { return fmt >= 0 && fmt <= 4; }
+static int fmt_bits(int fmt) {
+    return (fmt == ORC_MXFP4 || fmt == ORC_NVFP4) ? 4 : (fmt == ORC_MXFP6_E3M2 ? 6 : 8);
+}
 static double fmt_maxelem(int fmt) {
     switch (fmt) {
     case ORC_MXFP8_E4M3: return 448.0;
     case ORC_MXFP8_E5M2: return 57344.0;
+    case ORC_MXFP6_E3M2: return 28.0;
     default: return 6.0;
     }
 }
@@ -221,6 +249,7 @@ static double fmt_decode(int fmt, uint8_t code) {
     switch (fmt) {
     case ORC_MXFP8_E4M3: return orc_e4m3_decode(code);
     case ORC_MXFP8_E5M2: return orc_e5m2_decode(code);
+    case ORC_MXFP6_E3M2: return orc_e3m2_decode(code & 0x3F);
     default: return orc_e2m1_decode(code & 0xF);
     }
 }
@@ -228,6 +257,7 @@ static uint8_t fmt_encode(int fmt, double v) {
     switch (fmt) {
     case ORC_MXFP8_E4M3: return orc_e4m3_encode(v);
     case ORC_MXFP8_E5M2: return orc_e5m2_encode(v);
+    case ORC_MXFP6_E3M2: return orc_e3m2_encode(v);
     default: return orc_e2m1_encode(v);
     }
 }
@@ -306,6 +336,13 @@ uint8_t orc_nvfp4_block_scale(double amax_b, float g) {
 static void put_code(int fmt, uint8_t *codes, int64_t K, int64_t r, int64_t k, uint8_t q) {
     if (fmt_bits(fmt) == 8) {
         codes[r * K + k] = q;
+    } else if (fmt_bits(fmt) == 6) {
+        uint8_t *row = &codes[r * (K / 4) * 3];        /* [reading R18] bit 6k + i of the row */
+        for (int i = 0; i < 6; ++i) {
+            int64_t bit = 6 * k + i;
+            uint8_t mask = (uint8_t)(1u << (bit % 8));
+            if ((q >> i) & 1) row[bit / 8] |= mask; else row[bit / 8] &= (uint8_t)~mask;
+        }
     } else {
         uint8_t *byte = &codes[r * (K / 2) + k / 2];
         if (k % 2 == 0) *byte = (uint8_t)((*byte & 0xF0) | (q & 0xF));      /* [reading R6] */
@@ -315,6 +352,15 @@ static void put_code(int fmt, uint8_t *codes, int64_t K, int64_t r, int64_t k, u
 
 static uint8_t get_code(int fmt, const uint8_t *codes, int64_t K, int64_t r, int64_t k) {
     if (fmt_bits(fmt) == 8) return codes[r * K + k];
+    if (fmt_bits(fmt) == 6) {
+        const uint8_t *row = &codes[r * (K / 4) * 3];
+        uint8_t q = 0;
+        for (int i = 0; i < 6; ++i) {
+            int64_t bit = 6 * k + i;
+            q |= (uint8_t)(((row[bit / 8] >> (bit % 8)) & 1) << i);
+        }
+        return q;
+    }
     uint8_t byte = codes[r * (K / 2) + k / 2];
     return (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
 }
@@ -412,7 +458,7 @@ static int quantize_core(int fmt, double mx_threshold, const double *xv, int64_t
 static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
                          uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
     int bs = fmt_block(fmt);
-    if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    if (!fmt_ok(fmt) || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
     double *xv = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
     if (!xv) return ORC_EINVAL;
     for (int64_t r = 0; r < M; ++r)
@@ -433,7 +479,7 @@ static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int6
 int orc_quantize_f32(int fmt, const float *src, int64_t M, int64_t K, int64_t ld, uint8_t *codes, uint8_t *scales,
                      float *gscale, int gscale_given) {
     int bs = fmt_block(fmt);
-    if (fmt < 0 || fmt > 3 || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    if (!fmt_ok(fmt) || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
     double *xv = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
     if (!xv) return ORC_EINVAL;
     for (int64_t r = 0; r < M; ++r)
@@ -517,7 +563,7 @@ double orc_qsnr_db(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const 
 int orc_dequantize_f64(int fmt, const uint8_t *codes, const uint8_t *scales, float gscale,
                        int64_t M, int64_t K, double *dst) {
     int bs = fmt_block(fmt);
-    if (fmt < 0 || fmt > 3 || K % bs != 0) return ORC_EINVAL;
+    if (!fmt_ok(fmt) || K % bs != 0) return ORC_EINVAL;
     int64_t sf_cols = K / bs;
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
@@ -535,7 +581,7 @@ int orc_dequantize_f64(int fmt, const uint8_t *codes, const uint8_t *scales, flo
 int orc_dequantize_bf16(int fmt, const uint8_t *codes, const uint8_t *scales, float gscale,
                         int64_t M, int64_t K, uint16_t *dst, int64_t ld) {
     int bs = fmt_block(fmt);
-    if (fmt < 0 || fmt > 3 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    if (!fmt_ok(fmt) || K % bs != 0 || ld < K) return ORC_EINVAL;
     int64_t sf_cols = K / bs;
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
