@@ -59,9 +59,10 @@ def measured_peaks():
 
 def tensor_peak(fmt: int, peaks: dict, sustained: bool):
     """Dense block-scaled peak for the element type: the measured bf16 GEMM peak
-    times the nominal ratio (fp8 = 2x bf16, fp4 = 4x bf16)."""
+    times the nominal ratio (fp8 = 2x bf16, fp4 = 4x bf16; MXFP6 and mixed MX
+    operands run on kind::mxf8f6f4 at the fp8 rate)."""
     base = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    return base * (2.0 if fmt in (0, 1) else 4.0)
+    return base * (4.0 if fmt in (2, 3) else 2.0)
 
 
 class ClockSampler:
@@ -256,7 +257,8 @@ def qsnr_table(device):
         x = synth.bits_to_tensor(bits).to(device)
         row = {}
         for label, quant in (("mxfp8_e4m3", lambda: mx.quantize(x, 0)), ("mxfp4", lambda: mx.quantize(x, 2)),
-                             ("mxfp4_oas", lambda: mx.quantize_oas(x)), ("nvfp4", lambda: mx.quantize(x, 3))):
+                             ("mxfp4_oas", lambda: mx.quantize_oas(x)), ("nvfp4", lambda: mx.quantize(x, 3)),
+                             ("mxfp6_e3m2", lambda: mx.quantize(x, 4))):
             s = mx.qsnr_sums(quant(), x).cpu().numpy()
             row[label] = round(float(10.0 * np.log10(s[0] / s[1])), 3)
         for label, fmt in (("mxfp4_rht32", 2), ("nvfp4_rht32", 3)):
@@ -312,7 +314,7 @@ def kv_cache_extras(device, peaks, timed):
 
 
 def quant_bytes_per_elem(fmt):
-    return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625}[fmt]
+    return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625, 4: 2.78125}[fmt]
 
 
 def extras_gpu(device):
@@ -371,6 +373,13 @@ def extras_gpu(device):
     gbs = M * K * quant_bytes_per_elem(2) / (ms * 1e-3) / 1e9
     sweep[f"mxfp4_oas_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
     del qs
+    # MXFP6 E3M2: 2 B read + 0.75 B of codes + 1/32 B of scale per element
+    qs = [mx.empty(4, M, K) for _ in xs]
+    ms = timed(lambda i: mx.quantize(xs[i % len(xs)], 4, out=qs[i % len(xs)]), len(xs))
+    gbs = M * K * quant_bytes_per_elem(4) / (ms * 1e-3) / 1e9
+    sweep[f"mxfp6_e3m2_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                 "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    del qs
     # Walsh-Hadamard rotation fused with quantization: the same HBM bytes as the plain quantize
     for fmt, name in ((2, "mxfp4_rht32"), (3, "nvfp4_rht32")):
         qs = [mx.empty(fmt, M, K) for _ in xs]
@@ -385,23 +394,26 @@ def extras_gpu(device):
     out["quantize_sweep"] = sweep
     out["qsnr_db"] = qsnr_table(device)
     out["kv_cache"] = kv_cache_extras(device, peaks, timed)
-    # GEMMs
-    for name, (fmt, M, N, K) in {"mlp_nvfp4_gemm1": (3, 4608, 12288, 3072), "mlp_nvfp4_gemm2": (3, 4608, 3072, 12288),
-                                 "skinny_nvfp4_M16": (3, 16, 28672, 8192), "skinny_mxfp4_M16": (2, 16, 28672, 8192),
-                                 "skinny_nvfp4_M128": (3, 128, 28672, 8192)}.items():
+    # GEMMs (A format, B format, M, N, K); MXFP6 and mixed pairs run on kind::mxf8f6f4
+    for name, (fmt, wfmt, M, N, K) in {
+            "mlp_nvfp4_gemm1": (3, 3, 4608, 12288, 3072), "mlp_nvfp4_gemm2": (3, 3, 4608, 3072, 12288),
+            "skinny_nvfp4_M16": (3, 3, 16, 28672, 8192), "skinny_mxfp4_M16": (2, 2, 16, 28672, 8192),
+            "skinny_nvfp4_M128": (3, 3, 128, 28672, 8192),
+            "dit_mxfp6_gemm": (4, 4, 4096, 3072, 3072), "dit_mxfp8_x_mxfp4w_gemm": (0, 2, 4096, 3072, 3072),
+            "dit_mxfp8_x_mxfp6w_gemm": (0, 4, 4096, 3072, 3072)}.items():
         a = torch.randn((M, K), generator=g, device=device).to(torch.bfloat16)
         w = (torch.randn((N, K), generator=g, device=device) * 0.02).to(torch.bfloat16)
         qa = mx.quantize(a, fmt)
-        wbytes = mx.mx_codes_bytes(fmt, N, K) + mx.mx_scales_bytes(fmt, N, K)
+        wbytes = mx.mx_codes_bytes(wfmt, N, K) + mx.mx_scales_bytes(wfmt, N, K)
         nw = max(2, int(np.ceil(2 * L2_BYTES / wbytes)))
-        qws = [mx.quantize(w, fmt) for _ in range(nw)]
+        qws = [mx.quantize(w, wfmt) for _ in range(nw)]
         C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
         ms = timed(lambda i: mx.gemm(qa, qws[i % nw], out=C), nw)
         tf = 2 * M * N * K / (ms * 1e-3) / 1e12
         bytes_ = wbytes + mx.mx_codes_bytes(fmt, M, K) + mx.mx_scales_bytes(fmt, M, K) + M * N * 2
         gbs = bytes_ / (ms * 1e-3) / 1e9
         out[name] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1),
-                     "frac_tensor": round(tf / tensor_peak(fmt, peaks, False), 3),
+                     "frac_tensor": round(tf / tensor_peak(fmt if fmt == wfmt else 0, peaks, False), 3),
                      "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
         del a, w, qa, qws, C
     torch.cuda.empty_cache()

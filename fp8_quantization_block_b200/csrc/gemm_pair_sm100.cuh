@@ -116,7 +116,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (lane == 0) {
                         const uint32_t full_leader = full_leader0 + 8u * (uint32_t)s;
-                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (L::kABytes + L::kBBytes));
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(&full[s], FMT == kGemmRuntimeTypes ? p.stage_tx
+                                                                                     : 2u * (L::kABytes + L::kBBytes));
                         tma_load_2d_pair(smem + L::kOffA + s * L::kABytes, &tmA, kt * kStageKBytes, my_m, full_leader);
                         tma_load_2d_pair(smem + L::kOffB + s * L::kBBytes, &tmB, kt * kStageKBytes, my_n, full_leader);
                     }
@@ -156,6 +158,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t ad0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffA) >> 4) & 0x3FFFu);
             const uint64_t bd0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffB) >> 4) & 0x3FFFu);
             const uint32_t leader = lane == 0 ? 1u : 0u;
+            const uint32_t ab = FMT == kGemmRuntimeTypes ? p.ab_types : 0u;
             int last_n_mma, last_n_chunk;
             stage_extent<FMT>(p.num_kt - 1, p.K, last_n_mma, last_n_chunk);
             int s = 0, slot = 0;  // stage and scale-slot ring positions
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 auto run_stage = [&](int k, uint32_t acc) {
                     const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
                     issue_stage<FMT, true, 256, 8>(k + 1 < p.num_kt ? 4 : last_n_mma, t_acc, ad0 + (uint64_t)(s * (L::kABytes >> 4)),
-                        bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader);
+                        bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader, ab);
                     tc_commit_pair_if(&empty[s], 0x3, leader);
                     s = (s + 1 == STAGES) ? 0 : s + 1;
                     slot = (slot + 1) & (kSfSlots - 1);

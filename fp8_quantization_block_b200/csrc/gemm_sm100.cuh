@@ -67,6 +67,19 @@ struct GemmFmt<3> {  // NVFP4: kind::mxf4nvf4, scale_vec 4X (16-element blocks),
     static constexpr int kElemPerByte = 2, kBlock = 16, kChunks = 4, kMmaPerChunk = 1, kSfPerMma = 4;
     static constexpr uint32_t kAFmt = 1, kScaleUE8M0 = 0;
 };
+// kind::mxf8f6f4 with each operand's element type chosen at run time
+// (GemmParams::ab_types): MXFP6 E3M2 and mixed MX operands (E4M3 / E5M2 /
+// E3M2 / E2M1 on either side).  FP6 and FP4 codes arrive in shared memory
+// unpacked by the tensor-map copy to one 16-byte group per 16 elements, so a
+// stage is 128 elements = 128 bytes per row for every type, as for FP8.
+constexpr int kGemmRuntimeTypes = 4;
+template <>
+struct GemmFmt<kGemmRuntimeTypes> {
+    static constexpr int kElemPerByte = 1, kBlock = 32, kChunks = 1, kMmaPerChunk = 4, kSfPerMma = 1;
+    static constexpr uint32_t kAFmt = 0, kScaleUE8M0 = 1;
+};
+// Element-type fields of the kind::mxf8f6f4 instruction descriptor.
+enum : uint32_t { kTypeE4M3 = 0, kTypeE5M2 = 1, kTypeE3M2 = 4, kTypeE2M1 = 5 };
 
 constexpr int kBM = 128;
 constexpr int kStageKBytes = 128;
@@ -92,6 +105,10 @@ struct GemmParams {
     int epilogue;         // 0 none, 1 GELU
     int use_tma_store;    // 1: C via TMA bulk-tensor stores (ldc % 8 == 0, C 16-B aligned)
     int skip_producer;    // test hook: never issue loads
+    uint32_t ab_types;    // kGemmRuntimeTypes: (A type << 7) | (B type << 10) of the descriptor
+    uint32_t stage_tx;    // kGemmRuntimeTypes: bytes one stage's code copies report to this CTA's
+                          // barrier (the packed global bytes of FP6 / FP4 boxes, not their
+                          // unpacked shared-memory footprint)
     uint64_t wait_limit_ns;
 };
 
@@ -153,7 +170,7 @@ MX_DEVICE_INLINE uint32_t gemm_idesc(uint32_t sf_id) {
 template <int FMT>
 MX_DEVICE_INLINE void gemm_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
                                uint32_t acc) {
-    if (FMT <= 1) tc_mma_mxf8f6f4(d, a, b, idesc, sfa, sfb, acc);
+    if (FMT <= 1 || FMT == kGemmRuntimeTypes) tc_mma_mxf8f6f4(d, a, b, idesc, sfa, sfb, acc);
     else if (FMT == 2) tc_mma_mxf4(d, a, b, idesc, sfa, sfb, acc);
     else tc_mma_nvf4(d, a, b, idesc, sfa, sfb, acc);
 }
@@ -161,7 +178,7 @@ MX_DEVICE_INLINE void gemm_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t ides
 template <int FMT>
 MX_DEVICE_INLINE void gemm_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
                                   uint32_t acc, uint32_t issue) {
-    if (FMT <= 1) tc_mma_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+    if (FMT <= 1 || FMT == kGemmRuntimeTypes) tc_mma_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
     else if (FMT == 2) tc_mma_mxf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
     else tc_mma_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
 }
@@ -177,7 +194,7 @@ MX_DEVICE_INLINE uint32_t pair_idesc(uint32_t sf_id) {
 template <int FMT>
 MX_DEVICE_INLINE void pair_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
                                   uint32_t acc, uint32_t issue) {
-    if (FMT <= 1) tc_mma_pair_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
+    if (FMT <= 1 || FMT == kGemmRuntimeTypes) tc_mma_pair_mxf8f6f4_if(d, a, b, idesc, sfa, sfb, acc, issue);
     else if (FMT == 2) tc_mma_pair_mxf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
     else tc_mma_pair_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
 }
@@ -188,30 +205,31 @@ MX_DEVICE_INLINE void pair_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t i
 // 128-byte swizzle atom.  SFB_STEP: TMEM columns per scale chunk of B (4 per
 // 128-row band).  With n_mma == 4 the loop unrolls and every operand but the
 // stage's bases folds to a constant, keeping the issuing thread's per-stage
-// instruction chain short.
+// instruction chain short.  ab: run-time element-type bits of the descriptor
+// (0 for the formats whose types are fixed at compile time).
 template <int FMT, bool PAIR, int BN, int SFB_STEP>
 MX_DEVICE_INLINE void issue_one(int j, uint32_t t_acc, uint64_t ad, uint64_t bd, uint32_t t_sfa, uint32_t t_sfb,
-                                uint32_t acc, uint32_t issue) {
+                                uint32_t acc, uint32_t issue, uint32_t ab) {
     using F = GemmFmt<FMT>;
     const int chunk = j / F::kMmaPerChunk;
     const uint32_t sf_id = (uint32_t)((j % F::kMmaPerChunk) * F::kSfPerMma);
     const uint32_t a = acc | (j > 0 ? 1u : 0u);
     if (PAIR)
-        pair_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, pair_idesc<FMT>(sf_id), t_sfa + 4 * chunk,
+        pair_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, pair_idesc<FMT>(sf_id) | ab, t_sfa + 4 * chunk,
                          t_sfb + SFB_STEP * chunk, a, issue);
     else
-        gemm_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, gemm_idesc<FMT, BN>(sf_id), t_sfa + 4 * chunk,
+        gemm_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, gemm_idesc<FMT, BN>(sf_id) | ab, t_sfa + 4 * chunk,
                          t_sfb + SFB_STEP * chunk, a, issue);
 }
 
 template <int FMT, bool PAIR, int BN, int SFB_STEP>
 MX_DEVICE_INLINE void issue_stage(int n_mma, uint32_t t_acc, uint64_t ad, uint64_t bd, uint32_t t_sfa, uint32_t t_sfb,
-                                  uint32_t acc, uint32_t issue) {
+                                  uint32_t acc, uint32_t issue, uint32_t ab) {
     if (n_mma == 4) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) issue_one<FMT, PAIR, BN, SFB_STEP>(j, t_acc, ad, bd, t_sfa, t_sfb, acc, issue);
+        for (int j = 0; j < 4; ++j) issue_one<FMT, PAIR, BN, SFB_STEP>(j, t_acc, ad, bd, t_sfa, t_sfb, acc, issue, ab);
     } else {
-        for (int j = 0; j < n_mma; ++j) issue_one<FMT, PAIR, BN, SFB_STEP>(j, t_acc, ad, bd, t_sfa, t_sfb, acc, issue);
+        for (int j = 0; j < n_mma; ++j) issue_one<FMT, PAIR, BN, SFB_STEP>(j, t_acc, ad, bd, t_sfa, t_sfb, acc, issue, ab);
     }
 }
 
@@ -619,7 +637,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&full[s], (uint32_t)(L::kABytes + L::kBBytes));
+                        mbar_arrive_expect_tx(&full[s], FMT == kGemmRuntimeTypes ? p.stage_tx
+                                                                                 : (uint32_t)(L::kABytes + L::kBBytes));
                         tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, kt * kStageKBytes, m0, &full[s]);
                         tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, kt * kStageKBytes, n0, &full[s]);
                     }
@@ -659,6 +678,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint64_t ad0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffA) >> 4) & 0x3FFFu);
         const uint64_t bd0 = desc_ab | (uint64_t)((smem_u32(smem + L::kOffB) >> 4) & 0x3FFFu);
         const uint32_t leader = lane == 0 ? 1u : 0u;
+        const uint32_t ab = FMT == kGemmRuntimeTypes ? p.ab_types : 0u;
         int last_n_mma, last_n_chunk;
         stage_extent<FMT>(p.num_kt - 1, p.K, last_n_mma, last_n_chunk);
         int s = 0, slot = 0;  // stage and scale-slot ring positions
@@ -673,7 +693,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             auto run_stage = [&](int k, uint32_t acc) {
                 const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
                 issue_stage<FMT, false, BN, 4 * L::kBBands>(k + 1 < p.num_kt ? 4 : last_n_mma, t_acc, ad0 + (uint64_t)(s * (L::kABytes >> 4)),
-                    bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader);
+                    bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader, ab);
                 tc_commit_if(&empty[s], leader);
                 s = (s + 1 == STAGES) ? 0 : s + 1;
                 slot = (slot + 1) & (kSfSlots - 1);

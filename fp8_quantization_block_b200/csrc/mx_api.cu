@@ -35,9 +35,9 @@ int pdl_attr(cudaLaunchAttribute *a) {
     return 1;
 }
 
-bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 3; }
+bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 4; }
 int fmt_block(int fmt) { return fmt == MX_NVFP4 ? 16 : 32; }
-int fmt_bits(int fmt) { return (fmt == MX_MXFP4 || fmt == MX_NVFP4) ? 4 : 8; }
+int fmt_bits(int fmt) { return (fmt == MX_MXFP4 || fmt == MX_NVFP4) ? 4 : (fmt == MX_MXFP6_E3M2 ? 6 : 8); }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -83,6 +83,48 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, int64_t rows, int64_t row_by
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+// Codes of a kind::mxf8f6f4 operand as a 2D tensor of K elements per row, box
+// 128 elements x box_rows, 128-byte swizzle.  Every type lands in shared memory
+// as 128 bytes per row: FP8 bytes as they are; FP6 (16 codes in 12 bytes) and
+// FP4 (16 codes in 8 bytes) unpacked by the copy to one 16-byte group per 16
+// codes, the layout the MMA reads for these types.  The sub-byte types need a
+// 32-byte aligned base, row pitches that are multiples of 32 bytes and K a
+// multiple of 128 (the caller checks).
+bool make_tmap_codes_f8f6f4(CUtensorMap *m, int fmt, const void *base, int64_t rows, int64_t K, int box_rows) {
+    if (fmt_bits(fmt) == 8) return make_tmap_u8(m, base, rows, K, box_rows);
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const CUtensorMapDataType dt =
+        fmt_bits(fmt) == 6 ? CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K * fmt_bits(fmt) / 8)};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) fprintf(stderr, "libmx: tensor map for format %d codes failed (%d)\n", fmt, (int)r);
+    return r == CUDA_SUCCESS;
+}
+
+// Formats that kind::mxf8f6f4 multiplies (E8M0 scales on 32-element blocks),
+// and their element-type codes in its instruction descriptor.
+bool f8f6f4_fmt(int fmt) {
+    return fmt == MX_MXFP8_E4M3 || fmt == MX_MXFP8_E5M2 || fmt == MX_MXFP4 || fmt == MX_MXFP6_E3M2;
+}
+uint32_t f8f6f4_type(int fmt) {
+    switch (fmt) {
+    case MX_MXFP8_E4M3: return kTypeE4M3;
+    case MX_MXFP8_E5M2: return kTypeE5M2;
+    case MX_MXFP6_E3M2: return kTypeE3M2;
+    default: return kTypeE2M1;
+    }
+}
+// Can A and B be multiplied, and on which kernel: the format's own (same
+// format, 0..3) or the run-time-typed kind::mxf8f6f4 one.
+bool gemm_pair_ok(int fa, int fb) { return (fa == fb && fa <= MX_NVFP4) || (f8f6f4_fmt(fa) && f8f6f4_fmt(fb)); }
+bool gemm_runtime_types(int fa, int fb) { return !(fa == fb && fa <= MX_NVFP4); }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // --- quantize ------------------------------------------------------------
 template <int FMT, int RULE = RULE_OCP>
@@ -190,11 +232,16 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     using L = GemmSmem<FMT, BN, STAGES>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
-    const int64_t kbytes = K * fmt_bits(FMT) / 8;
+    const int64_t kbytes = K / GemmFmt<FMT>::kElemPerByte;   // shared-memory bytes of a row's K
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     CUtensorMap ta, tb, tc, tsa, tsb;
-    if (!make_tmap_u8(&ta, a_codes, M, kbytes, kBM)) return MX_ERR_CUDA;
-    if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN)) return MX_ERR_CUDA;
+    if (FMT == kGemmRuntimeTypes) {
+        if (!make_tmap_codes_f8f6f4(&ta, A->fmt, a_codes, M, K, kBM)) return MX_ERR_CUDA;
+        if (!make_tmap_codes_f8f6f4(&tb, B->fmt, B->codes, N, K, BN)) return MX_ERR_CUDA;
+    } else {
+        if (!make_tmap_u8(&ta, a_codes, M, kbytes, kBM)) return MX_ERR_CUDA;
+        if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN)) return MX_ERR_CUDA;
+    }
     if (!make_tmap_sf(&tsa, a_scales, cdiv(M, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 1)) return MX_ERR_CUDA;
     if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, L::kBBands))
         return MX_ERR_CUDA;
@@ -224,6 +271,8 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.epilogue = epilogue;
     p.use_tma_store = tma_store ? 1 : 0;
     p.skip_producer = g_skip_producer.load();
+    p.ab_types = (f8f6f4_type(A->fmt) << 7) | (f8f6f4_type(B->fmt) << 10);
+    p.stage_tx = (uint32_t)(kStageKBytes * (kBM * fmt_bits(A->fmt) + BN * fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
@@ -249,11 +298,16 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     using L = PairSmem<FMT, STAGES>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
-    const int64_t kbytes = K * fmt_bits(FMT) / 8;
+    const int64_t kbytes = K / GemmFmt<FMT>::kElemPerByte;   // shared-memory bytes of a row's K
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     CUtensorMap ta, tb, tc, tsa, tsb;
-    if (!make_tmap_u8(&ta, a_codes, M, kbytes, 128)) return MX_ERR_CUDA;
-    if (!make_tmap_u8(&tb, B->codes, N, kbytes, 128)) return MX_ERR_CUDA;
+    if (FMT == kGemmRuntimeTypes) {
+        if (!make_tmap_codes_f8f6f4(&ta, A->fmt, a_codes, M, K, 128)) return MX_ERR_CUDA;
+        if (!make_tmap_codes_f8f6f4(&tb, B->fmt, B->codes, N, K, 128)) return MX_ERR_CUDA;
+    } else {
+        if (!make_tmap_u8(&ta, a_codes, M, kbytes, 128)) return MX_ERR_CUDA;
+        if (!make_tmap_u8(&tb, B->codes, N, kbytes, 128)) return MX_ERR_CUDA;
+    }
     if (!make_tmap_sf(&tsa, a_scales, cdiv(M, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 1)) return MX_ERR_CUDA;
     if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 2))
         return MX_ERR_CUDA;
@@ -283,6 +337,9 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     p.epilogue = epilogue;
     p.use_tma_store = tma_store ? 1 : 0;
     p.skip_producer = g_skip_producer.load();
+    p.ab_types = (f8f6f4_type(A->fmt) << 7) | (f8f6f4_type(B->fmt) << 10);
+    // both CTAs' copies (128 rows of A and 128 of B each) report to the leader's barrier
+    p.stage_tx = (uint32_t)(2 * kStageKBytes * 128 * (fmt_bits(A->fmt) + fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const int64_t max_pairs = num_sms() / 2;
@@ -316,6 +373,8 @@ mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_
 
 mx_status launch_gemm(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                       const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
+    if (gemm_runtime_types(A->fmt, B->fmt))
+        return launch_gemm_fmt<kGemmRuntimeTypes>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     switch (A->fmt) {
     case MX_MXFP8_E4M3: return launch_gemm_fmt<0>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     case MX_MXFP8_E5M2: return launch_gemm_fmt<1>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
@@ -352,6 +411,7 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
     case MX_MXFP8_E4M3: launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
     case MX_MXFP8_E5M2: launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
     case MX_MXFP4: launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP6_E3M2: launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
     default:
         if (x_gscale != nullptr) {
             launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st);
@@ -433,6 +493,7 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
     case MX_MXFP8_E4M3: launch_quantize<0>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP8_E5M2: launch_quantize<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP4: launch_quantize<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP6_E3M2: launch_quantize<4>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     default: {
         if (gscale_in == nullptr) {
             mx_status s = nvfp4_gscale_prepass(src, M, K, ld_src, dst->gscale, st);
@@ -478,6 +539,7 @@ mx_status mx_quantize_rht(int fmt, const void *src_bf16, int64_t M, int64_t K, i
     case MX_MXFP8_E4M3: launch_quantize_rht<0>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP8_E5M2: launch_quantize_rht<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP4: launch_quantize_rht<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP6_E3M2: launch_quantize_rht<4>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     default: {
         if (gscale_in == nullptr) {
             // g from max |y| of the rotated tensor: an extra read of src
@@ -521,6 +583,7 @@ mx_status mx_qsnr(const mx_tensor *q, const void *src_bf16, int64_t ld_src, doub
     case MX_MXFP8_E4M3: qsnr_kernel<0><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
     case MX_MXFP8_E5M2: qsnr_kernel<1><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
     case MX_MXFP4: qsnr_kernel<2><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP6_E3M2: qsnr_kernel<4><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
     default: qsnr_kernel<3><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, q->gscale, q->rows, q->cols, sums);
     }
     return last_launch();
@@ -541,6 +604,7 @@ mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, vo
     case MX_MXFP8_E4M3: dequantize_kernel<0><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
     case MX_MXFP8_E5M2: dequantize_kernel<1><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
     case MX_MXFP4: dequantize_kernel<2><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP6_E3M2: dequantize_kernel<4><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
     default: dequantize_kernel<3><<<blocks, 256, 0, st>>>(c, src->scales, src->gscale, src->rows, src->cols, d, ld_dst);
     }
     return last_launch();
@@ -551,7 +615,7 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
     if (s != MX_OK) return s;
     s = check_tensor(B, true);
     if (s != MX_OK) return s;
-    if (A->fmt != B->fmt || A->cols != B->cols) return MX_ERR_INVALID_ARG;
+    if (!gemm_pair_ok(A->fmt, B->fmt) || A->cols != B->cols) return MX_ERR_INVALID_ARG;
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     if (M == 0 || N == 0) return MX_OK;
     if (!C_bf16) return MX_ERR_INVALID_ARG;
@@ -561,6 +625,9 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
     if (K == 0) return cuda_status(cudaMemset2DAsync(C_bf16, ldc * 2, 0, N * 2, M, st));
     if (K % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || cdiv(M, kBM) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (gemm_runtime_types(A->fmt, B->fmt) && ((fmt_bits(A->fmt) < 8 && !aligned32(A->codes)) ||
+                                               (fmt_bits(B->fmt) < 8 && !aligned32(B->codes))))
+        return MX_ERR_MISALIGNED;
     return launch_gemm(A, B, A->codes, A->scales, A->gscale, static_cast<uint16_t *>(C_bf16), ldc, 0, nullptr, st);
 }
 
@@ -575,7 +642,7 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     if (!valid_fmt(fmt) || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
     mx_status s = check_tensor(W, true);
     if (s != MX_OK) return s;
-    if (W->fmt != fmt || W->cols != K) return MX_ERR_INVALID_ARG;
+    if (!gemm_pair_ok(fmt, W->fmt) || W->cols != K) return MX_ERR_INVALID_ARG;
     if (epilogue != MX_EPI_NONE && epilogue != MX_EPI_GELU) return MX_ERR_INVALID_ARG;
     const int64_t N = W->rows;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -593,6 +660,7 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     if (!workspace) return MX_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MX_ERR_MISALIGNED;
     if (workspace_bytes < fused_ws_bytes(fmt, M, K)) return MX_ERR_INVALID_ARG;
+    if (gemm_runtime_types(fmt, W->fmt) && fmt_bits(W->fmt) < 8 && !aligned32(W->codes)) return MX_ERR_MISALIGNED;
     mx_tensor xa;
     const float *ga = nullptr;
     s = fused_quantize_x(fmt, static_cast<const uint16_t *>(X_bf16), M, K, ldx, static_cast<uint8_t *>(workspace),

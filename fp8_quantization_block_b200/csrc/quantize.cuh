@@ -1,9 +1,10 @@
 // quantize.cuh -- HBM-bound microscaling quantize / dequantize kernels (sm_100a).
 //
 // What is computed (page "Microscaling MXFP4/NVFP4 on Blackwell for reasoning
-// LLMs", section "Fundamentos matemáticos do formato MXFP4 e E8M0" and the FAQ
-// entry on how E8M0 picks the block exponent; NVFP4/MXFP8 block sizes from
-// "NVIDIA's FP4 format delivers 1.68x speedup"):
+// LLMs", section "Fundamentos matemáticos do formato MXFP4 e E8M0", its format
+// table (MXFP6 = E3M2 elements, E8M0 scale per 32) and the FAQ entry on how
+// E8M0 picks the block exponent; NVFP4/MXFP8 block sizes from "NVIDIA's FP4
+// format delivers 1.68x speedup"):
 //   MX:    E = ceil(log2(max|x| / max_elem)) + 127, clamped to [0, 254];
 //          q = RNE_sat(x / 2^(E-127)).
 //   NVFP4: s = smallest positive finite E4M3 with max|x| <= 6 g s;
@@ -23,7 +24,7 @@
 
 namespace mx {
 
-enum { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_MXFP4 = 2, FMT_NVFP4 = 3 };
+enum { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_MXFP4 = 2, FMT_NVFP4 = 3, FMT_MXFP6 = 4 };
 
 template <int FMT>
 struct FmtTraits;
@@ -47,6 +48,11 @@ template <>
 struct FmtTraits<FMT_NVFP4> {
     static constexpr int kBlock = 16, kBits = 4;
     static constexpr int kExpOff = 0, kMantThr = 0;
+};
+template <>
+struct FmtTraits<FMT_MXFP6> {  // E3M2 elements
+    static constexpr int kBlock = 32, kBits = 6;
+    static constexpr int kExpOff = 4, kMantThr = 0x60;  // 28 = 1.75 * 2^4
 };
 
 // ------------------------------------------------------------------ scale rules
@@ -137,6 +143,57 @@ MX_DEVICE_INLINE uint32_t cvt8_e2m1(const float (&a)[8]) {
         : "=r"(out)
         : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
     return out;
+}
+
+// Four fp32 -> four E3M2 codes, one per byte in bits 0-5, RNE, saturating.
+MX_DEVICE_INLINE uint32_t cvt4_e3m2(float a0, float a1, float a2, float a3) {
+    uint32_t out;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e3m2x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e3m2x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(out)
+        : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+    return out & 0x3F3F3F3Fu;
+}
+
+// The four 6-bit codes of w's bytes as 24 contiguous bits (byte i at bit 6i).
+MX_DEVICE_INLINE uint32_t pack4x6(uint32_t w) {
+    const uint32_t x = (w & 0x003F003Fu) | ((w & 0x3F003F00u) >> 2);   // 12-bit pairs in each half
+    return (x & 0xFFFu) | ((x >> 4) & 0xFFF000u);
+}
+
+// Store the codes of 16 MX elements already divided by their block scale
+// (row `row`, columns col .. col+15, col % 16 == 0).  FP8: one byte each; FP6:
+// code k of a row at bits 6k .. 6k+5 of the row's little-endian bit string
+// (16 codes in 12 bytes, the packed form the tensor map's 16 x U6 type reads);
+// FP4: two per byte, the even element in the low nibble.
+template <int FMT>
+MX_DEVICE_INLINE void store_mx_codes16(uint8_t *__restrict__ codes, int64_t row, int64_t K, int64_t col,
+                                       const float (&f)[16]) {
+    using T = FmtTraits<FMT>;
+    if (T::kBits == 8) {
+        uint4 q;
+        q.x = cvt4_fp8<FMT>(f[0], f[1], f[2], f[3]);
+        q.y = cvt4_fp8<FMT>(f[4], f[5], f[6], f[7]);
+        q.z = cvt4_fp8<FMT>(f[8], f[9], f[10], f[11]);
+        q.w = cvt4_fp8<FMT>(f[12], f[13], f[14], f[15]);
+        *reinterpret_cast<uint4 *>(codes + row * K + col) = q;
+    } else if (T::kBits == 6) {
+        const uint32_t t0 = pack4x6(cvt4_e3m2(f[0], f[1], f[2], f[3]));
+        const uint32_t t1 = pack4x6(cvt4_e3m2(f[4], f[5], f[6], f[7]));
+        const uint32_t t2 = pack4x6(cvt4_e3m2(f[8], f[9], f[10], f[11]));
+        const uint32_t t3 = pack4x6(cvt4_e3m2(f[12], f[13], f[14], f[15]));
+        // 12 bytes at a 4-byte aligned offset (K % 32 == 0, col % 16 == 0)
+        uint32_t *p = reinterpret_cast<uint32_t *>(codes + row * (K / 4 * 3) + col / 4 * 3);
+        p[0] = t0 | (t1 << 24);
+        p[1] = (t1 >> 8) | (t2 << 16);
+        p[2] = (t2 >> 16) | (t3 << 8);
+    } else {
+        const float(&f0)[8] = *reinterpret_cast<const float(*)[8]>(&f[0]);
+        const float(&f1)[8] = *reinterpret_cast<const float(*)[8]>(&f[8]);
+        *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(cvt8_e2m1(f0), cvt8_e2m1(f1));
+    }
 }
 
 MX_DEVICE_INLINE float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -350,18 +407,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
                     f[2 * e] = bf16lo(w[e]) * inv;
                     f[2 * e + 1] = bf16hi(w[e]) * inv;
                 }
-                if (T::kBits == 8) {
-                    uint4 q;
-                    q.x = cvt4_fp8<FMT>(f[0], f[1], f[2], f[3]);
-                    q.y = cvt4_fp8<FMT>(f[4], f[5], f[6], f[7]);
-                    q.z = cvt4_fp8<FMT>(f[8], f[9], f[10], f[11]);
-                    q.w = cvt4_fp8<FMT>(f[12], f[13], f[14], f[15]);
-                    *reinterpret_cast<uint4 *>(codes + row * K + col) = q;
-                } else {
-                    const float(&f0)[8] = *reinterpret_cast<const float(*)[8]>(&f[0]);
-                    const float(&f1)[8] = *reinterpret_cast<const float(*)[8]>(&f[8]);
-                    *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(cvt8_e2m1(f0), cvt8_e2m1(f1));
-                }
+                store_mx_codes16<FMT>(codes, row, K, col, f);
             }
         }
         // Scale byte of (rl, jb) inside the tile's 512-byte tensor-core tiles.
@@ -448,6 +494,18 @@ MX_DEVICE_INLINE void load_dequant8(const uint8_t *__restrict__ codes, const uin
                 q[4 * h + 2 * p] = __low2float(hh);
                 q[4 * h + 2 * p + 1] = __high2float(hh);
             }
+        }
+    } else if (T::kBits == 6) {
+        // 8 codes = 6 bytes at a 2-byte aligned offset
+        const uint16_t *p = reinterpret_cast<const uint16_t *>(codes + r * (K / 4 * 3) + c / 4 * 3);
+        const uint64_t w = (uint64_t)p[0] | ((uint64_t)p[1] << 16) | ((uint64_t)p[2] << 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t code = (uint32_t)(w >> (6 * e)) & 0x3Fu;
+            const uint32_t ex = (code >> 2) & 7u, m = code & 3u;
+            // E3M2: subnormal m * 2^-4, else (1 + m/4) * 2^(ex - 3)
+            const float mag = ex == 0u ? 0.0625f * (float)m : __uint_as_float(((ex + 124u) << 23) | (m << 21));
+            q[e] = (code & 0x20u) ? -mag : mag;
         }
     } else {
         const uint32_t w = *reinterpret_cast<const uint32_t *>(codes + r * (K / 2) + c / 2);

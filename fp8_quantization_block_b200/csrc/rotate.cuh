@@ -205,18 +205,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t 
                 float f[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) f[e] = y[e] * inv;
-                if (T::kBits == 8) {
-                    uint4 q;
-                    q.x = cvt4_fp8<FMT>(f[0], f[1], f[2], f[3]);
-                    q.y = cvt4_fp8<FMT>(f[4], f[5], f[6], f[7]);
-                    q.z = cvt4_fp8<FMT>(f[8], f[9], f[10], f[11]);
-                    q.w = cvt4_fp8<FMT>(f[12], f[13], f[14], f[15]);
-                    *reinterpret_cast<uint4 *>(codes + row * K + col) = q;
-                } else {
-                    const float(&f0)[8] = *reinterpret_cast<const float(*)[8]>(&f[0]);
-                    const float(&f1)[8] = *reinterpret_cast<const float(*)[8]>(&f[8]);
-                    *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(cvt8_e2m1(f0), cvt8_e2m1(f1));
-                }
+                store_mx_codes16<FMT>(codes, row, K, col, f);
             }
         }
         const bool owner = T::kBlock == 16 || (lane & 1) == 0;

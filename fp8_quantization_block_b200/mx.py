@@ -21,8 +21,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmx.so")
 
-MX_MXFP8_E4M3, MX_MXFP8_E5M2, MX_MXFP4, MX_NVFP4 = 0, 1, 2, 3
-FORMATS = {"mxfp8_e4m3": 0, "mxfp8_e5m2": 1, "mxfp4": 2, "nvfp4": 3}
+MX_MXFP8_E4M3, MX_MXFP8_E5M2, MX_MXFP4, MX_NVFP4, MX_MXFP6_E3M2 = 0, 1, 2, 3, 4
+FORMATS = {"mxfp8_e4m3": 0, "mxfp8_e5m2": 1, "mxfp4": 2, "nvfp4": 3, "mxfp6_e3m2": 4}
 MX_OK, MX_ERR_INVALID_ARG, MX_ERR_UNSUPPORTED_SHAPE, MX_ERR_MISALIGNED = 0, 1, 2, 3
 MX_ERR_CUDA, MX_ERR_TIMEOUT, MX_ERR_DEVICE = 4, 5, 6
 MX_EPI_NONE, MX_EPI_GELU = 0, 1
@@ -256,14 +256,16 @@ def gemm(A: MxTensor, B: MxTensor, out: torch.Tensor | None = None, stream=None)
 def gemm_fused_act(x: torch.Tensor, W: MxTensor, out: torch.Tensor | None = None, epilogue: int = MX_EPI_NONE,
                    amax_out: torch.Tensor | None = None, x_gscale: torch.Tensor | None = None,
                    x_amax: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                   stream=None) -> torch.Tensor:
+                   stream=None, x_fmt: int | None = None) -> torch.Tensor:
+    """x_fmt: the format X is quantized to (default W's; any MX format pairs with an MX W)."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     M, K = x.shape
+    fmt = W.fmt if x_fmt is None else x_fmt
     out = out if out is not None else torch.empty((M, W.rows), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = fused_workspace(W.fmt, M, K, x.device)
+        workspace = fused_workspace(fmt, M, K, x.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    check(mx_gemm_fused_act(W.fmt, x.data_ptr(), M, K, x.stride(0), W.c(), out.data_ptr(), out.stride(0), epilogue,
+    check(mx_gemm_fused_act(fmt, x.data_ptr(), M, K, x.stride(0), W.c(), out.data_ptr(), out.stride(0), epilogue,
                             _ptr(amax_out), _ptr(x_gscale), _ptr(x_amax), _ptr(workspace), ws_bytes,
                             _stream(stream)), "mx_gemm_fused_act")
     return out

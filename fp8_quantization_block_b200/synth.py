@@ -117,13 +117,17 @@ def edge_rows(K: int) -> np.ndarray:
 
 def tie_rows(K: int, fmt: int) -> np.ndarray:
     """Rows whose block maximum pins the scale so that other elements land
-    exactly on E2M1 / E4M3 rounding midpoints (MX formats: scale = 1)."""
+    exactly on E2M1 / E4M3 / E5M2 / E3M2 rounding midpoints (MX formats:
+    scale = 1)."""
     if fmt in (2, 3):
         mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 5.5, 6.5, 0.125, 0.375]
         top = 6.0
     elif fmt == 0:
         mids = [1.0625, 1.1875, 17.0, 19.0, 240.0, 416.0, 432.0, 2.0 ** -10, 3 * 2.0 ** -10]
         top = 448.0
+    elif fmt == 4:   # E3M2
+        mids = [2.0 ** -5, 3 * 2.0 ** -5, 0.28125, 1.125, 1.375, 2.25, 3.75, 4.5, 6.5, 7.5, 9.0, 13.0, 15.0, 18.0, 26.0]
+        top = 28.0
     else:
         mids = [1.125, 1.375, 2.5, 3.5, 40960.0, 2.0 ** -17, 3 * 2.0 ** -17]
         top = 57344.0

@@ -1,13 +1,14 @@
 /*
- * mx.h -- C ABI of libmx.so: microscaling quantization (MXFP8 E4M3/E5M2, MXFP4,
- * NVFP4) and the block-scaled matrix multiply that consumes it, on one NVIDIA
- * B200 (sm_100a).
+ * mx.h -- C ABI of libmx.so: microscaling quantization (MXFP8 E4M3/E5M2, MXFP6
+ * E3M2, MXFP4, NVFP4) and the block-scaled matrix multiply that consumes it, on
+ * one NVIDIA B200 (sm_100a).
  *
  * Sources for what each call computes (page title, section):
  *   [MX]    "Microscaling MXFP4/NVFP4 on Blackwell for reasoning LLMs"
  *           (produtoramaxvision.com.br), sections "Fundamentos matemáticos do
  *           formato MXFP4 e E8M0" (E2M1 values, E8M0 = 2^(E-127), x = S * x_elem,
- *           4.25 bits/element, E4M3 range [-448, 448]), "Arquitetura Blackwell
+ *           4.25 bits/element, E4M3 range [-448, 448], the format table's
+ *           MXFP6 = E3M2 with an E8M0 scale per 32, 6.25 bits), "Arquitetura Blackwell
  *           SM100 e aceleração nativa de NVFP4" (the tensor core applies the
  *           block scales during FP32 accumulation) and the FAQ entry on how E8M0
  *           picks the block exponent (E = ceil(log2(max|x| / max_elem)) + 127).
@@ -43,13 +44,16 @@
 extern "C" {
 #endif
 
-/* Element formats.  Block size 32 with an E8M0 scale for the three MX formats;
- * block size 16 with an E4M3 scale plus one FP32 per-tensor scale for NVFP4. */
+/* Element formats.  Block size 32 with an E8M0 scale for the four MX formats;
+ * block size 16 with an E4M3 scale plus one FP32 per-tensor scale for NVFP4.
+ * E3M2 ([MX] format table, MXFP6): sign, 3 exponent bits with bias 3, 2
+ * mantissa bits, no infinities or NaN, largest magnitude 28. */
 typedef enum {
     MX_MXFP8_E4M3 = 0,
     MX_MXFP8_E5M2 = 1,
     MX_MXFP4 = 2,
-    MX_NVFP4 = 3
+    MX_NVFP4 = 3,
+    MX_MXFP6_E3M2 = 4
 } mx_format;
 
 typedef enum {
@@ -65,7 +69,10 @@ typedef enum {
 /* A quantized [rows x cols] matrix (cols = K, the blocked dimension).
  *   codes : device, mx_codes_bytes(fmt, rows, cols) bytes.  FP8: one code per
  *           byte, row-major.  FP4: two codes per byte, byte j of a row holds
- *           code 2j in its low nibble and code 2j+1 in its high nibble.
+ *           code 2j in its low nibble and code 2j+1 in its high nibble.  FP6:
+ *           code k of a row occupies bits 6k .. 6k+5 of the row read as a
+ *           little-endian bit string (16 codes in 12 bytes; a row is 3K/4
+ *           bytes).
  *   scales: device, mx_scales_bytes(fmt, rows, cols) bytes.  One scale byte per
  *           block (E8M0 for MX, E4M3 for NVFP4), laid out in 512-byte tiles of
  *           128 rows x 4 scale columns: scale (r, c) of a matrix with C scale
@@ -94,7 +101,8 @@ int mx_block_size(int fmt);
  * ld_src % 8 == 0) into dst ([MX] "Fundamentos" and FAQ; [NEWS]).
  *   MX formats: per block, E = ceil(log2(max|x| / max_elem)) + 127 clamped to
  *     [0, 254] (0 for an all-zero block), elements = RNE(x / 2^(E-127))
- *     saturating to the element format (max_elem = 448 / 57344 / 6).
+ *     saturating to the element format (max_elem = 448 / 57344 / 6 / 28 for
+ *     E4M3 / E5M2 / E2M1 / E3M2).
  *   NVFP4: g = the FP32 value *gscale_in if gscale_in != NULL, else
  *     amax(|src|) / 2688 rounded up to FP32 (1.0 for an all-zero tensor),
  *     computed on the device (an extra read of src).  g is written to
@@ -155,8 +163,12 @@ mx_status mx_qsnr(const mx_tensor *q, const void *src_bf16, int64_t ld_src, doub
  *   C[i][j] = RNE_bf16( sum_k A_dq[i][k] * B_dq[j][k] ),  A [M x K], B [N x K],
  * A_dq / B_dq the dequantized operands (the scales are applied inside the
  * tensor core during FP32 accumulation; NVFP4 also multiplies by gA * gB in
- * the epilogue).  A->fmt == B->fmt, A->cols == B->cols == K, K % 128 == 0.
- * C is bf16 [M x N] with row pitch ldc (ldc >= N).  Accuracy contract:
+ * the epilogue).  A->cols == B->cols == K, K % 128 == 0.  Formats: A->fmt ==
+ * B->fmt, or any two of the four MX formats (E4M3, E5M2, E3M2, MXFP4 E2M1;
+ * all with E8M0 scales on 32-element blocks), which run on kind::mxf8f6f4 at
+ * the FP8 rate (MXFP6 x MXFP6 included); such a call needs the codes of an
+ * FP6 or FP4 operand 32-byte aligned (else MX_ERR_MISALIGNED).  NVFP4 pairs
+ * only with NVFP4.  C is bf16 [M x N] with row pitch ldc (ldc >= N).  Accuracy contract:
  *   |C - C_ref| <= 2^-8 |C_ref| + 1e-4 (|A_dq| |B_dq|^T)  elementwise.       */
 mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t ldc, void *stream);
 
@@ -164,7 +176,9 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
 typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
 
 /* Fused activation-quantize + GEMM: X is bf16 [M x K] (row pitch ldx), W a
- * pre-quantized [N x K] mx_tensor of format fmt.  X is quantized exactly as
+ * pre-quantized [N x K] mx_tensor; X is quantized to format fmt, and W's format
+ * is fmt or, as in mx_gemm, any MX format that pairs with it (e.g. MXFP8
+ * activations with MXFP4 or MXFP6 weights).  X is quantized exactly as
  * mx_quantize would (same codes and scales, bit for bit) once, into the
  * caller's `workspace` (which stays resident in L2 at these sizes), and the
  * block-scaled GEMM consumes it in the same stream: C = X_dq * W_dq^T as in

@@ -108,7 +108,7 @@ def test_workspace_checks():
     s = mx.mx_gemm_fused_act(0, X.data_ptr(), 64, 256, 256, W.c(), C.data_ptr(), 64, 0, None, None, None,
                              ws.data_ptr() + 16, need, None)
     assert s == mx.MX_ERR_MISALIGNED
-    s = mx.mx_gemm_fused_act(2, X.data_ptr(), 64, 256, 256, W.c(), C.data_ptr(), 64, 0, None, None, None,
+    s = mx.mx_gemm_fused_act(3, X.data_ptr(), 64, 256, 256, W.c(), C.data_ptr(), 64, 0, None, None, None,
                              ws.data_ptr(), need, None)
-    assert s == mx.MX_ERR_INVALID_ARG                                      # W format differs
+    assert s == mx.MX_ERR_INVALID_ARG                                      # NVFP4 X with an MXFP8 W
     torch.cuda.synchronize()
