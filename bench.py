@@ -399,6 +399,7 @@ def extras_gpu(device):
             "mlp_nvfp4_gemm1": (3, 3, 4608, 12288, 3072), "mlp_nvfp4_gemm2": (3, 3, 4608, 3072, 12288),
             "skinny_nvfp4_M16": (3, 3, 16, 28672, 8192), "skinny_mxfp4_M16": (2, 2, 16, 28672, 8192),
             "skinny_nvfp4_M128": (3, 3, 128, 28672, 8192),
+            "dit_mxfp8_gemm_back_to_back": (0, 0, 4096, 3072, 3072),
             "dit_mxfp6_gemm": (4, 4, 4096, 3072, 3072), "dit_mxfp8_x_mxfp4w_gemm": (0, 2, 4096, 3072, 3072),
             "dit_mxfp8_x_mxfp6w_gemm": (0, 4, 4096, 3072, 3072)}.items():
         a = torch.randn((M, K), generator=g, device=device).to(torch.bfloat16)
@@ -483,8 +484,12 @@ def run_reference(args, wl):
 
 
 PROFILE_CASES = {
-    # name: (kind, fmt, M, N, K)
+    # name: (kind, fmt, M, N, K[, B's format when it differs])
     "gemm_dit_mxfp8": ("gemm", 0, 4096, 3072, 3072),
+    "gemm_dit_mxfp6": ("gemm", 4, 4096, 3072, 3072),
+    "gemm_dit_mxfp8_x_mxfp4w": ("gemm", 0, 4096, 3072, 3072, 2),
+    "quant_mxfp6_32768x4096": ("quant", 4, 32768, 0, 4096),
+    "rht_mxfp4_32768x4096": ("rht", 2, 32768, 0, 4096),
     "gemm_mlp1_nvfp4": ("gemm", 3, 4608, 12288, 3072),
     "gemm_mlp2_nvfp4": ("gemm", 3, 4608, 3072, 12288),
     "gemm_skinny_nvfp4": ("gemm", 3, 16, 28672, 8192),
@@ -500,7 +505,8 @@ def run_profile_case(name: str, reps: int = 4):
     from fp8_quantization_block_b200 import build as mxbuild
     from fp8_quantization_block_b200 import mx
     mxbuild.build()
-    kind, fmt, M, N, K = PROFILE_CASES[name]
+    kind, fmt, M, N, K = PROFILE_CASES[name][:5]
+    wfmt = PROFILE_CASES[name][5] if len(PROFILE_CASES[name]) > 5 else fmt
     g = torch.Generator(device="cuda").manual_seed(1)
     x = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
     if kind == "quant":
@@ -508,9 +514,14 @@ def run_profile_case(name: str, reps: int = 4):
         gs = mx.quantize(x, fmt, out=q).gscale.clone() if fmt == 3 else None   # NVFP4: g of this input
         for _ in range(reps):
             mx.quantize(x, fmt, out=q, gscale=gs)
+    elif kind == "rht":
+        q = mx.empty(fmt, M, K)
+        gs = mx.quantize_rht(x, fmt, out=q).gscale.clone() if fmt == 3 else None
+        for _ in range(reps):
+            mx.quantize_rht(x, fmt, out=q, gscale=gs)
     else:
         w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
-        qa, qw = mx.quantize(x, fmt), mx.quantize(w, fmt)
+        qa, qw = mx.quantize(x, fmt), mx.quantize(w, wfmt)
         C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         for _ in range(reps):
             mx.gemm(qa, qw, out=C)
@@ -526,7 +537,7 @@ METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
 # kernel sources still hash to `src`, i.e. the counters were taken on the code
 # that runs.
 NCU_TRAFFIC = {
-    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6>", "bytes": 22778368 + 66560, "src": "af22953946a39d50"},
+    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6>", "bytes": 22786048 + 78592, "src": "004058843ebbe0b1"},
 }
 
 
