@@ -40,8 +40,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                      const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = PairSmem<FMT, STAGES>;
-    static_assert(STAGES >= kSfSlots, "scale slots are recycled through the stage barriers");
-    static_assert((kSfSlots & (kSfSlots - 1)) == 0, "scale slots: a power of two");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);  // leader's count both CTAs' code tiles
@@ -51,7 +49,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *acc_full = sfree + L::kSfGroups;  // [2]
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *mma_done = acc_empty + 1;
-    uint64_t *sf_full = mma_done + 1;           // [kSfSlots], leader's count both CTAs' scale warps
+    uint64_t *sf_full = mma_done + 1;           // [L::kSlots], leader's count both CTAs' scale warps
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
     uint32_t *ready_count = reinterpret_cast<uint32_t *>(smem + L::kOffMisc + 8);  // gate -> MMA issuer
@@ -74,7 +72,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_init(&acc_full[1], 1);
         mbar_init(acc_empty, 2 * kEpiWarps);
         mbar_init(mma_done, 1);
-        for (int i = 0; i < kSfSlots; ++i) mbar_init(&sf_full[i], 8);
+        for (int i = 0; i < L::kSlots; ++i) mbar_init(&sf_full[i], 8);
         *abort_flag = 0;
         *ready_count = 0;
         fence_barrier_init();
@@ -176,7 +174,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader, ab);
                     tc_commit_pair_if(&empty[s], 0x3, leader);
                     s = (s + 1 == STAGES) ? 0 : s + 1;
-                    slot = (slot + 1) & (kSfSlots - 1);
+                    slot = (slot + 1 == L::kSlots) ? 0 : slot + 1;
                     ++kg;
                 };
                 // Two stages per iteration: the loop's own instructions then fall between
@@ -215,7 +213,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (rank == 0) {
             int my_tiles = 0;
             for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
-            gate_role<STAGES>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
+            gate_role<STAGES, L::kSlots>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
         }
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps

@@ -15,7 +15,7 @@
 //              operand brings kSfGroup stages' tiles (all of B's bands) into
 //              a ring of its own, ahead of the scale warps;
 //   warps 6-9  scale warps (one per TMEM lane quadrant): copy each stage's
-//              scale tiles from shared memory into one of kSfSlots TMEM slots
+//              scale tiles from shared memory into one of the TMEM scale slots
 //              with tcgen05.st, as soon as the MMAs that read the slot's
 //              previous contents have completed.  (Staging the scales with
 //              tcgen05.cp instead costs tensor-pipe cycles that do not overlap
@@ -86,7 +86,7 @@ constexpr int kStageKBytes = 128;
 constexpr int kGemmThreads = 384;  // 12 warps
 constexpr int kSfWarp = 10;        // the scale-tile producer
 constexpr int kGateWarp = 11;      // publishes how many stages the MMA issuer may consume
-constexpr int kSfSlots = 4;        // TMEM scale slots (a power of two)
+constexpr int kSfSlots = 4;        // TMEM scale slots (the layouts may use more, see kSlots)
 constexpr int kSfGroup = 2;        // stages per scale-tile copy
 constexpr int kEpiWarps = 4;
 constexpr int kEpiChunkBytes = 32 * 32 * 2;  // 32 rows x 32 bf16 columns per epilogue warp
@@ -125,10 +125,17 @@ struct GemmLayout {
     static constexpr int kSfaGroupBytes = kSfGroup * F::kChunks * 512;
     static constexpr int kSfbGroupBytes = kSfaGroupBytes * B_BANDS;
     static constexpr int kSfBandStride = kSfaGroupBytes;
+    // TMEM scale slots in the ring: a slot is rewritten once the MMAs of the
+    // stage kSlots earlier have completed, so more slots hide more of that
+    // round trip (commit -> scale warps -> gate -> MMA issuer).  FP8-type
+    // stages (one scale chunk) with 6 or more smem stages take 6 slots; the
+    // FP4 kinds, whose slots are 2-4x wider, keep 4 so that TMEM still holds
+    // the two accumulators.
+    static constexpr int kSlots = (F::kChunks == 1 && STAGES >= 6) ? 6 : kSfSlots;
     // full[S], empty[S], sfload[G], sfree[G], acc_full[2], acc_empty, mma_done, sf_full[slots]
     static constexpr int bytes_for(int groups, int bufs) {
         return STAGES * (kABytes + kBBytes) + groups * (kSfaGroupBytes + kSfbGroupBytes) +
-               kEpiWarps * bufs * kEpiChunkBytes + (2 * STAGES + 2 * groups + 4 + kSfSlots) * 8 + 16 + 1024;
+               kEpiWarps * bufs * kEpiChunkBytes + (2 * STAGES + 2 * groups + 4 + kSlots) * 8 + 16 + 1024;
     }
     // as many scale groups in flight, then epilogue staging buffers, as fit
     static constexpr int kSfGroups = bytes_for(4, 2) <= kSmemLimit ? 4 : (bytes_for(3, 1) <= kSmemLimit ? 3 : 2);
@@ -139,21 +146,22 @@ struct GemmLayout {
     static constexpr int kOffSfa = kOffEpi + kEpiWarps * kEpiBufs * kEpiChunkBytes;
     static constexpr int kOffSfb = kOffSfa + kSfGroups * kSfaGroupBytes;
     static constexpr int kOffBar = kOffSfb + kSfGroups * kSfbGroupBytes;
-    static constexpr int kNumBars = 2 * STAGES + 2 * kSfGroups + 4 + kSfSlots;
+    static constexpr int kNumBars = 2 * STAGES + 2 * kSfGroups + 4 + kSlots;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
     static_assert(kAlloc <= kSmemLimit, "shared memory budget");
     // TMEM: two accumulators at columns 0 and kAccStride (sharing BN - kAccStride
-    // columns), then kSfSlots scale slots of kSfSlotCols columns each.
+    // columns), then kSlots scale slots of kSfSlotCols columns each.
     static constexpr int kAccCols = 128 * B_BANDS;  // accumulator columns = N of the MMA
     static constexpr int kTmemCols = 512;
     static constexpr int kSfSlotCols = 4 * F::kChunks * (1 + B_BANDS);
-    static constexpr int kAccRoom = kTmemCols - kAccCols - kSfSlots * kSfSlotCols;
+    static constexpr int kAccRoom = kTmemCols - kAccCols - kSlots * kSfSlotCols;
     static constexpr int kAccStride = (kAccRoom >= kAccCols ? kAccCols : kAccRoom) / 32 * 32;
     static constexpr int kTmemSf = kAccStride + kAccCols;
     static_assert(kAccStride >= 32, "accumulator double buffering needs TMEM room");
-    static_assert(kTmemSf + kSfSlots * kSfSlotCols <= kTmemCols, "TMEM budget");
+    static_assert(kTmemSf + kSlots * kSfSlotCols <= kTmemCols, "TMEM budget");
+    static_assert(STAGES >= kSlots, "scale slots are recycled through the stage barriers");
 };
 
 template <int FMT, int BN, int STAGES>
@@ -332,9 +340,12 @@ MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *t
 
 // Scale warps (one per TMEM lane quadrant; lane r handles TMEM lane 32q + r):
 // for every stage of this CTA's tiles, wait for its scale group in smem and
-// for the MMAs that last read the TMEM slot (stage kg - kSfSlots, whose
+// for the MMAs that last read the TMEM slot (stage kg - L::kSlots, whose
 // commit completes empty[]), then write the slot and report it with
 // arrive_full(slot).  After a group's last stage the warp frees the group.
+// (Writing a group's two stages with one wait for the stores was measured
+// slower: the second slot's wait for older MMAs costs more than the store
+// latency it hides.)
 template <typename L, int STAGES, typename ArriveFull>
 MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *sfload, uint64_t *sfree, uint64_t *empty,
                                  uint32_t t_sf0, int my_tiles, int lane, volatile int *abort_flag,
@@ -352,7 +363,7 @@ MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *s
                 stop = true;
                 break;
             }
-            if (kg >= kSfSlots) {
+            if (kg >= L::kSlots) {
                 if (!mbar_wait_bounded(&empty[e], eph, p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
                     stop = true;
                     break;
@@ -370,7 +381,7 @@ MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *s
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_full(slot);
-            slot = (slot + 1) & (kSfSlots - 1);
+            slot = (slot + 1 == L::kSlots) ? 0 : slot + 1;
             if (gi == kSfGroup - 1 || kt == p.num_kt - 1) {
                 if (lane == 0) mbar_arrive(&sfree[g]);
                 if (++g == NG) {
@@ -390,7 +401,7 @@ MX_DEVICE_INLINE void tile_coords(int tile, int m_blocks, int &m0, int &n0, int 
 // Gate warp: for every stage of this CTA's tiles, in order, wait for its code
 // tiles (full) and its scale slot (sf_full), then publish the number of
 // stages ready so far.
-template <int STAGES>
+template <int STAGES, int SLOTS>
 MX_DEVICE_INLINE void gate_role(const GemmParams &p, uint64_t *full, uint64_t *sf_full, uint32_t *ready, int my_tiles,
                                 int lane, volatile int *abort_flag) {
     int s = 0, slot = 0;
@@ -407,8 +418,10 @@ MX_DEVICE_INLINE void gate_role(const GemmParams &p, uint64_t *full, uint64_t *s
                 s = 0;
                 fph ^= 1u;
             }
-            slot = (slot + 1) & (kSfSlots - 1);
-            sph ^= (slot == 0) ? 1u : 0u;
+            if (++slot == SLOTS) {
+                slot = 0;
+                sph ^= 1u;
+            }
         }
     }
 }
@@ -566,8 +579,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = GemmSmem<FMT, BN, STAGES>;
-    static_assert(STAGES >= kSfSlots, "scale slots are recycled through the stage barriers");
-    static_assert((kSfSlots & (kSfSlots - 1)) == 0, "scale slots: a power of two");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
@@ -577,7 +588,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *acc_full = sfree + L::kSfGroups;   // [2]
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *mma_done = acc_empty + 1;
-    uint64_t *sf_full = mma_done + 1;            // [kSfSlots]
+    uint64_t *sf_full = mma_done + 1;            // [L::kSlots]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
     uint32_t *ready_count = reinterpret_cast<uint32_t *>(smem + L::kOffMisc + 8);  // gate -> MMA issuer
@@ -598,7 +609,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_init(&acc_full[1], 1);
         mbar_init(acc_empty, kEpiWarps);
         mbar_init(mma_done, 1);
-        for (int i = 0; i < kSfSlots; ++i) mbar_init(&sf_full[i], 4);
+        for (int i = 0; i < L::kSlots; ++i) mbar_init(&sf_full[i], 4);
         *abort_flag = 0;
         *ready_count = 0;
         fence_barrier_init();
@@ -696,7 +707,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader, ab);
                 tc_commit_if(&empty[s], leader);
                 s = (s + 1 == STAGES) ? 0 : s + 1;
-                slot = (slot + 1) & (kSfSlots - 1);
+                slot = (slot + 1 == L::kSlots) ? 0 : slot + 1;
                 ++kg;
             };
             // Two stages per iteration: the loop's own instructions then fall between
@@ -733,7 +744,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ------------------------------------------------------------ gate
         int my_tiles = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
-        gate_role<STAGES>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
+        gate_role<STAGES, L::kSlots>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps
         const int q = warp & 3;
