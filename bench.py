@@ -133,6 +133,24 @@ def make_inputs(wl: dict):
     return X, W
 
 
+# ------------------------------------------------------------------ multi-rank host logic
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (a device time), so that a multi-rank
+    number is the slowest rank's; x itself with one process (dist is None)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step: float, steps: int, ms_max: float, world: int) -> float:
+    """Whole-job throughput of `world` replicas that each ran `steps` steps,
+    timed as the slowest rank's ms_max (weak scaling: the work grows with N)."""
+    return world * flops_per_step * steps / (ms_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, wl, rank, world, device):
     import torch
@@ -211,10 +229,7 @@ def run_gpu(args, wl, rank, world, device):
     ms = t0.elapsed_time(t1)
     q_ms = [e[0].elapsed_time(e[1]) for e in evs]
     g_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, device)
 
     # end-to-end through the C ABI with host buffers: H2D of X, quantize, GEMM, D2H of C
     X_host = synth.bits_to_tensor(X_bits).pin_memory()
@@ -239,11 +254,7 @@ def run_gpu(args, wl, rank, world, device):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     del sets
     torch.cuda.empty_cache()
     clocks["window"] = f"{n_load} untimed steps (~{args.load_window_s} s) then the {args.steps} timed steps"
@@ -573,7 +584,7 @@ def gemm_kernel_name(fmt: int, M: int, N: int) -> str:
     if M > 128 and N > 128:
         return f"gemm_pair_kernel<{fmt}, {6 if fmt < 2 else 5}>"
     return f"gemm_kernel<{fmt}, {128 if N <= 128 else 256}, 4>"
-FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4"}
+FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4", 4: "mxfp6_e3m2"}
 
 
 def main():
@@ -623,14 +634,14 @@ def main():
     fmt, M, N, K = wl["fmt"], wl["M"], wl["N"], wl["K"]
     flops = 2.0 * M * N * K
     ms_step = r["ms"] / args.steps
-    value = world * flops * args.steps / (r["ms"] * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, r["ms"], world)
     g_avg = sum(r["g_ms"]) / len(r["g_ms"])
     q_avg = sum(r["q_ms"]) / len(r["q_ms"])
     g_tf = flops / (g_avg * 1e-3) / 1e12
     tpeak = tensor_peak(fmt, peaks, sustained=False)
     q_bytes = M * K * quant_bytes_per_elem(fmt)
     q_gbs = q_bytes / (q_avg * 1e-3) / 1e9
-    e2e_value = world * flops * args.steps / (r["e2e_ms"] * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(flops, args.steps, r["e2e_ms"], world)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",

@@ -1,0 +1,69 @@
+"""The benchmark's multi-rank host logic on CPU: two gloo ranks on 127.0.0.1.
+
+bench.py at N > 1 runs N independent replicas (the path shards with no data
+collective); the only cross-rank steps are the barrier and the max over ranks
+of each device time, and only rank 0 prints.  These run here without a GPU.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, q):
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        # each rank's own device time: rank 1 is the slow one
+        mine = [2.5, 7.25][rank]
+        got = bench.max_over_ranks(mine, dist, torch.device("cpu"))
+        dist.barrier()
+        q.put((rank, got, bench.whole_job_tflops(1e12, 10, got, world)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [r[1] for r in res] == [7.25, 7.25]          # every rank sees the slowest rank's time
+    # 2 replicas x 10 steps x 1 TFLOP in 7.25 ms
+    assert res[0][2] == pytest.approx(2 * 10 * 1e12 / 7.25e-3 / 1e12)
+
+
+def test_single_process_is_its_own_max():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.0, None, None) == 3.0
+    assert bench.whole_job_tflops(2e12, 4, 8.0, 1) == pytest.approx(1000.0)
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    # under torchrun the reference arm runs on rank 0 only; rank 1 exits 0 and prints nothing
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1", MASTER_PORT="29511")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip() == ""
