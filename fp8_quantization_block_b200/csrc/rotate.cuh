@@ -23,31 +23,97 @@ namespace mx {
 
 constexpr uint32_t kRhtScaleBits = 0x3E3504F3u;  // RN_fp32(1 / sqrt(32))
 
-// Rotate the 32-element block whose half (16 values) this thread holds: lower
-// = even lane (elements 0..15 of the block), upper = odd lane.  All 32 lanes
-// of the warp must call this together.
-MX_DEVICE_INLINE void rht32_halves(float (&x)[16], int lane) {
+// Packed fp32 pairs (f32x2 arithmetic of sm_100: two IEEE operations per
+// instruction, each rounded to nearest-even exactly as its scalar form).
+MX_DEVICE_INLINE uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+MX_DEVICE_INLINE void upk2(uint64_t r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
+MX_DEVICE_INLINE uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// The unnormalised butterflies H32 x of the 32-element block whose half (16
+// values) this thread holds: lower = even lane (block elements 0..15), upper =
+// odd lane.  Stages of half-width 1, 2, 4 run on the pairs (x[j], x[j + 8]),
+// two sums per instruction; half-width 8 pairs x[j] with x[j + 8] inside this
+// thread; half-width 16 pairs this lane with lane ^ 1: lower keeps a + b,
+// upper b' - a' = fma(-1, own, other), one rounding as in the scalar form.
+// On return z[j] = (H32 x)[j] (this half), every sum rounded to fp32 in the
+// stage order of the definition; the caller applies c = RN_fp32(1/sqrt(32)).
+// All 32 lanes of the warp must call this together.
+MX_DEVICE_INLINE void rht32_butterflies(float (&z)[16], int lane) {
+    uint64_t P[8];
 #pragma unroll
-    for (int h = 1; h < 16; h <<= 1) {
+    for (int j = 0; j < 8; ++j) P[j] = pk2(z[j], z[j + 8]);
 #pragma unroll
-        for (int i0 = 0; i0 < 16; i0 += 2 * h) {
+    for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
-            for (int i = i0; i < i0 + h; ++i) {
-                const float a = x[i], b = x[i + h];
-                x[i] = __fadd_rn(a, b);
-                x[i + h] = __fsub_rn(a, b);
+        for (int j0 = 0; j0 < 8; j0 += 2 * h) {
+#pragma unroll
+            for (int j = j0; j < j0 + h; ++j) {
+                const uint64_t a = P[j], b = P[j + h];
+                P[j] = add2(a, b);
+                P[j + h] = sub2(a, b);
             }
         }
     }
-    const bool upper = (lane & 1) != 0;
-    const float c = __uint_as_float(kRhtScaleBits);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float other = __shfl_xor_sync(0xffffffffu, x[i], 1);
-        // pair (i, i + 16): lower = a + b, upper = a - b, with a the lower value
-        const float v = upper ? __fsub_rn(other, x[i]) : __fadd_rn(x[i], other);
-        x[i] = __fmul_rn(v, c);
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        upk2(P[j], a, b);
+        z[j] = __fadd_rn(a, b);
+        z[j + 8] = __fsub_rn(a, b);
     }
+    const float sg = (lane & 1) ? -1.0f : 1.0f;
+    const uint64_t S = pk2(sg, sg);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float o0 = __shfl_xor_sync(0xffffffffu, z[2 * j], 1);
+        const float o1 = __shfl_xor_sync(0xffffffffu, z[2 * j + 1], 1);
+        float r0, r1;
+        upk2(fma2(S, pk2(z[2 * j], z[2 * j + 1]), pk2(o0, o1)), r0, r1);
+        z[2 * j] = r0;
+        z[2 * j + 1] = r1;
+    }
+}
+
+// y = RN(c * z) for the 16 values (the normalised rotation).
+MX_DEVICE_INLINE void rht32_scale(float (&z)[16]) {
+    const float c = __uint_as_float(kRhtScaleBits);
+    const uint64_t C = pk2(c, c);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        upk2(mul2(C, pk2(z[2 * j], z[2 * j + 1])), a, b);
+        z[2 * j] = a;
+        z[2 * j + 1] = b;
+    }
+}
+
+// The rotated half-block: y = c * (H32 x) as defined above.
+MX_DEVICE_INLINE void rht32_halves(float (&x)[16], int lane) {
+    rht32_butterflies(x, lane);
+    rht32_scale(x);
 }
 
 MX_DEVICE_INLINE void unpack16(const uint4 &v0, const uint4 &v1, float (&x)[16]) {
@@ -171,15 +237,19 @@ __global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t 
         const int rl = i * 32 + warp * 4 + (lane >> 3);
         const int64_t row = row0 + rl;
         const bool ok = row < M && col_ok;
+        // z = H32 x (unnormalised); y = RN(c z).  max |y| = RN(c max |z|), since
+        // rounding is monotone and c > 0.
         float y[16];
         unpack16(v[i][0], v[i][1], y);
-        rht32_halves(y, lane);
-        float m = 0.0f;
+        rht32_butterflies(y, lane);
+        float mz = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(y[e]));
-        if (T::kBlock == 32) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        for (int e = 0; e < 16; ++e) mz = fmaxf(mz, fabsf(y[e]));
+        if (T::kBlock == 32) mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 1));
+        const float m = __fmul_rn(__uint_as_float(kRhtScaleBits), mz);
         uint32_t sbyte;
         if (FMT == FMT_NVFP4) {
+            rht32_scale(y);
             sbyte = nv_block_scale(m, g, inv6g, nvt.val);
             if (ok) {
                 uint32_t q0 = 0, q1 = 0;
@@ -201,10 +271,25 @@ __global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t 
             const int E = mx_scale_byte_f32<FMT>(m);
             sbyte = (uint32_t)E;
             if (ok) {
+                // RN(c z) * 2^(127-E) = RN(z * (c 2^(127-E))) whenever RN(c z) is a
+                // normal fp32 and c 2^(127-E) is too (E <= 250): scaling by a power
+                // of two commutes with rounding there.  With max |y| >= 2^-90, an
+                // element whose RN(c z) is subnormal scales to below 2^-17 of the
+                // element grid's top (448 x 2^-126 / 2^-90 at most): both forms
+                // give it a zero code of the same sign.  Other blocks take the
+                // two-step form.
                 const float inv = mx_inv_scale(E);
                 float f[16];
+                if (E <= 250 && m >= 0x1p-90f) {
+                    const float cs = __uint_as_float(kRhtScaleBits) * inv;   // exact
+                    const uint64_t CS = pk2(cs, cs);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) f[e] = y[e] * inv;
+                    for (int j = 0; j < 8; ++j) upk2(mul2(CS, pk2(y[2 * j], y[2 * j + 1])), f[2 * j], f[2 * j + 1]);
+                } else {
+                    rht32_scale(y);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) f[e] = y[e] * inv;
+                }
                 store_mx_codes16<FMT>(codes, row, K, col, f);
             }
         }
@@ -249,12 +334,13 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t *__restric
             v0 = ldg_stream(p);
             v1 = ldg_stream(p + 8);
         }
-        float y[16];
-        unpack16(v0, v1, y);
-        rht32_halves(y, lane);
+        float z[16];
+        unpack16(v0, v1, z);
+        rht32_butterflies(z, lane);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(y[e]));
+        for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(z[e]));
     }
+    m = __fmul_rn(__uint_as_float(kRhtScaleBits), m);   // max |RN(c z)| = RN(c max |z|)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0 && m > 0.0f) atomicMax(amax_bits, __float_as_uint(m));

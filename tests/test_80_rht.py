@@ -40,7 +40,10 @@ def edge_rows_in_range(K):
     big = synth.bits_to_tensor(rows).float().abs().amax(dim=1).numpy()
     keep = rows[big < 1e38]
     near = synth.to_bf16_bits(np.where(np.arange(K) % 5 == 0, -1e37, 1e37).astype(np.float32)[None, :])
-    return np.vstack([keep, near])
+    # all equal: the first rotated value is 32 c x ~ 5.6e37, near the largest a
+    # finite block reaches (MXFP4 scale byte 250)
+    flat = synth.to_bf16_bits(np.full((1, K), 1e37, dtype=np.float32))
+    return np.vstack([keep, near, flat])
 
 
 @pytest.mark.parametrize("fmt", FMTS)
