@@ -22,9 +22,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mx_oracle.c")
 _LIB = os.path.join(_HERE, "libmxoracle.so")
 
-MXFP8_E4M3, MXFP8_E5M2, MXFP4, NVFP4, MXFP6_E3M2 = 0, 1, 2, 3, 4
+MXFP8_E4M3, MXFP8_E5M2, MXFP4, NVFP4, MXFP6_E3M2, MXFP4_MBS = 0, 1, 2, 3, 4, 5
 FORMAT_NAMES = {MXFP8_E4M3: "mxfp8_e4m3", MXFP8_E5M2: "mxfp8_e5m2", MXFP4: "mxfp4", NVFP4: "nvfp4",
-                MXFP6_E3M2: "mxfp6_e3m2"}
+                MXFP6_E3M2: "mxfp6_e3m2", MXFP4_MBS: "mxfp4_mbs"}
 
 _lock = threading.Lock()
 _lib = None
@@ -65,6 +65,9 @@ def _load():
                 "orc_codes_bytes": (ctypes.c_size_t, [i32, i64, i64]),
                 "orc_scales_bytes": (ctypes.c_size_t, [i32, i64, i64]),
                 "orc_sf_offset": (ctypes.c_size_t, [i64, i64, i64]),
+                "orc_mbs_macro_offset": (ctypes.c_size_t, [i64, i64, i64, i64]),
+                "orc_mbs_static_mantissa": (i32, [d]),
+                "orc_mbs_block_exponent": (i32, [d, i32]),
                 "orc_mx_scale_byte": (i32, [d, d]),
                 "orc_nvfp4_global_scale": (f32, [d]),
                 "orc_nvfp4_block_scale": (u8, [d, f32]),
@@ -146,6 +149,24 @@ def sf_offset(r: int, c: int, sf_cols: int) -> int:
 
 def mx_scale_byte(amax: float, maxelem: float) -> int:
     return int(_load().orc_mx_scale_byte(float(amax), float(maxelem)))
+
+
+def mbs_macro_offset(rows: int, cols: int, r: int, mb: int) -> int:
+    return int(_load().orc_mbs_macro_offset(rows, cols, r, mb))
+
+
+def mbs_static_mantissa(alpha: float) -> int:
+    return int(_load().orc_mbs_static_mantissa(float(alpha)))
+
+
+def mbs_block_exponent(amax_b: float, m: int) -> int:
+    return int(_load().orc_mbs_block_exponent(float(amax_b), int(m)))
+
+
+def mbs_macro_bytes(scales: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """The [rows, cols/128] macro mantissas stored after an MXFP4-MBS scale buffer's tiles."""
+    off = mbs_macro_offset(rows, cols, 0, 0)
+    return np.asarray(scales[off:off + rows * (cols // 128)]).reshape(rows, cols // 128)
 
 
 def nvfp4_global_scale(amax_t: float) -> float:

@@ -170,6 +170,47 @@ def quantize_values(fmt: int, X, neg, g: Fraction | None = None, mx_threshold: F
     return codes, scales, g
 
 
+def mbs_static_mantissa(block: list[Fraction]) -> int:
+    """Macro mantissa by brute force: e = floor(log2(alpha / 6)) found by
+    scanning, then the smallest m in [0, 255] with alpha / (1 + m/256) <= 6 * 2^e
+    (0 for an all-zero block or when none suffices)."""
+    alpha = max(abs(x) for x in block)
+    if alpha == 0:
+        return 0
+    e = next(e for e in range(-200, 200) if 6 * Fraction(2) ** e <= alpha < 6 * Fraction(2) ** (e + 1))
+    for m in range(256):
+        if alpha / (1 + Fraction(m, 256)) <= 6 * Fraction(2) ** e:
+            return m
+    return 0
+
+
+def quantize_mbs(bits: np.ndarray):
+    """MXFP4 with static macro-block scaling, exhaustively: per 128 elements m
+    as above; per 16 the smallest E with every |x| / ((1 + m/256) 2^(E-127)) <= 6;
+    elements the nearest E2M1 value of that quotient, ties to the even code.
+    Returns (codes[M][K], scales[M][K/16], macro[M][K/128])."""
+    M, K = bits.shape
+    X = [[bf16(int(bits[r, k])) for k in range(K)] for r in range(M)]
+    codes = [[0] * K for _ in range(M)]
+    scales = [[0] * (K // 16) for _ in range(M)]
+    macro = [[0] * (K // 128) for _ in range(M)]
+    for r in range(M):
+        for mb in range(K // 128):
+            m = mbs_static_mantissa(X[r][mb * 128:(mb + 1) * 128])
+            macro[r][mb] = m
+            f = 1 + Fraction(m, 256)
+            for jb in range(8):
+                j = mb * 8 + jb
+                blk = X[r][j * 16:(j + 1) * 16]
+                E = next((E for E in range(255) if all(abs(x) / (f * Fraction(2) ** (E - 127)) <= 6 for x in blk)),
+                         254)
+                scales[r][j] = E
+                denom = f * Fraction(2) ** (E - 127)
+                for i, x in enumerate(blk):
+                    codes[r][j * 16 + i] = round_to_grid(x / denom, E2M1_GRID, 0x8, bool(int(bits[r, j * 16 + i]) & 0x8000))
+    return codes, scales, macro
+
+
 def dequant(fmt: int, codes, scales, g: Fraction | None):
     bs = BLOCK[fmt]
     out = []

@@ -47,6 +47,15 @@
  *       mantissa bits, no infinities or NaN, largest magnitude 28); MXFP6
  *       packing: code k of a row occupies bits 6k .. 6k+5 of the row read as
  *       one little-endian bit string (16 codes in 12 bytes).
+ *   R20 MXFP4 with static macro-block scaling [OAS/MBS page, section B]: E2M1
+ *       elements in 1x16 base blocks with E8M0 scales (tiled as NVFP4's), and
+ *       per 1x128 macro block a factor 1 + m/256 (m one byte, 8 mantissa
+ *       bits) chosen from the macro block's max alpha so that alpha / (1 +
+ *       m/256) lands at or just below 6 * 2^e, e = floor(log2(alpha / 6)):
+ *       m = the smallest integer in [0, 255] with alpha <= 6 (256 + m) 2^(e-8)
+ *       (0 if alpha == 0 or none suffices).  Each base block then takes the MX
+ *       rule on x / (1 + m/256) and RNE elements of that quotient.  The
+ *       macro bytes are stored after the scale tiles, row-major [rows][K/128].
  */
 #include <math.h>
 #include <stdint.h>
@@ -57,7 +66,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_MXFP8_E4M3 = 0, ORC_MXFP8_E5M2 = 1, ORC_MXFP4 = 2, ORC_NVFP4 = 3, ORC_MXFP6_E3M2 = 4 };
+enum { ORC_MXFP8_E4M3 = 0, ORC_MXFP8_E5M2 = 1, ORC_MXFP4 = 2, ORC_NVFP4 = 3, ORC_MXFP6_E3M2 = 4, ORC_MXFP4_MBS = 5 };
 enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_ENONFINITE = 2 };
 
 /* ------------------------------------------------------------------------- */
@@ -232,10 +241,10 @@ uint8_t orc_e3m2_encode(double v) {
 /* ------------------------------------------------------------------------- */
 /* format parameters                                                         */
 /* ------------------------------------------------------------------------- */
-static int fmt_block(int fmt) { return fmt == ORC_NVFP4 ? 16 : 32; }
-static int fmt_ok(int fmt) { return fmt >= 0 && fmt <= 4; }
+static int fmt_block(int fmt) { return (fmt == ORC_NVFP4 || fmt == ORC_MXFP4_MBS) ? 16 : 32; }
+static int fmt_ok(int fmt) { return fmt >= 0 && fmt <= 5; }
 static int fmt_bits(int fmt) {
-    return (fmt == ORC_MXFP4 || fmt == ORC_NVFP4) ? 4 : (fmt == ORC_MXFP6_E3M2 ? 6 : 8);
+    return (fmt == ORC_MXFP4 || fmt == ORC_NVFP4 || fmt == ORC_MXFP4_MBS) ? 4 : (fmt == ORC_MXFP6_E3M2 ? 6 : 8);
 }
 static double fmt_maxelem(int fmt) {
     switch (fmt) {
@@ -274,9 +283,21 @@ size_t orc_codes_bytes(int fmt, int64_t rows, int64_t cols) {
     return (size_t)(rows * cols * fmt_bits(fmt) / 8);
 }
 
-size_t orc_scales_bytes(int fmt, int64_t rows, int64_t cols) {
+/* Bytes of the 128x4 scale tiles; MXFP4-MBS appends its macro bytes. */
+static size_t tile_bytes(int fmt, int64_t rows, int64_t cols) {
     int64_t sc = cols / fmt_block(fmt);
     return (size_t)(ceil_div(rows, 128) * 128 * ceil_div(sc, 4) * 4);
+}
+
+size_t orc_scales_bytes(int fmt, int64_t rows, int64_t cols) {
+    size_t t = tile_bytes(fmt, rows, cols);
+    if (fmt == ORC_MXFP4_MBS) t += (size_t)(ceil_div(rows * (cols / 128), 16) * 16);
+    return t;
+}
+
+/* [reading R20] offset of macro byte (r, mb) in an MXFP4-MBS scale buffer */
+size_t orc_mbs_macro_offset(int64_t rows, int64_t cols, int64_t r, int64_t mb) {
+    return tile_bytes(ORC_MXFP4_MBS, rows, cols) + (size_t)(r * (cols / 128) + mb);
 }
 
 /* [reading R7] position of scale (r, c) in a scale matrix with sf_cols columns */
@@ -317,6 +338,29 @@ float orc_nvfp4_global_scale(double amax_t) {
         if (p > 0.0f && (double)p * 2688.0 >= amax_t) f = p; else break;
     }
     return f;
+}
+
+/* [reading R20] MBS-static macro mantissa of a macro block with max alpha:
+ * e with 6 * 2^e <= alpha < 6 * 2^(e+1), then the smallest m in [0, 255]
+ * with alpha <= 6 (256 + m) 2^(e - 8); 0 if alpha == 0 or no m suffices.
+ * Every product is an integer of at most 12 bits times a power of two: exact. */
+int orc_mbs_static_mantissa(double alpha) {
+    if (!(alpha > 0.0)) return 0;
+    int e = ilogb(alpha) - 2;
+    while (ldexp(6.0, e) > alpha) --e;
+    while (ldexp(6.0, e + 1) <= alpha) ++e;
+    for (int m = 0; m < 256; ++m)
+        if (alpha <= ldexp(6.0 * (256 + m), e - 8)) return m;
+    return 0;
+}
+
+/* [reading R20] base-block exponent under macro mantissa m: the smallest E in
+ * [0, 254] with amax_b <= 6 (256 + m) 2^(E - 135), i.e. amax_b / (1 + m/256)
+ * <= 6 * 2^(E - 127); 254 if none. */
+int orc_mbs_block_exponent(double amax_b, int m) {
+    for (int E = 0; E <= 254; ++E)
+        if (amax_b <= ldexp(6.0 * (256 + m), E - 135)) return E;
+    return 254;
 }
 
 /* [reading R5] smallest positive finite E4M3 s with amax_b <= 6 * g * s.
@@ -421,6 +465,35 @@ static int quantize_core(int fmt, double mx_threshold, const double *xv, int64_t
             *gscale = g;
         }
     }
+    if (fmt == ORC_MXFP4_MBS) {
+        /* [reading R20]: macro mantissa per 128 elements, then 16-element
+         * blocks on x / (1 + m/256), elements decided by exact comparisons
+         * with the quotient's E2M1 midpoints (denominator (256+m) 2^(E-135)). */
+        #pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < M; ++r) {
+            for (int64_t mb = 0; mb < K / 128; ++mb) {
+                const double *mac = xv + r * K + mb * 128;
+                double alpha = 0.0;
+                for (int i = 0; i < 128; ++i)
+                    if (fabs(mac[i]) > alpha) alpha = fabs(mac[i]);
+                int m = orc_mbs_static_mantissa(alpha);
+                scales[orc_mbs_macro_offset(M, K, r, mb)] = (uint8_t)m;
+                for (int jb = 0; jb < 8; ++jb) {
+                    const double *blk = mac + jb * 16;
+                    double amax = 0.0;
+                    for (int i = 0; i < 16; ++i)
+                        if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
+                    int E = orc_mbs_block_exponent(amax, m);
+                    int64_t j = mb * 8 + jb;
+                    scales[orc_sf_offset(r, j, sf_cols)] = (uint8_t)E;
+                    double denom = ldexp((double)(256 + m), E - 135);
+                    for (int i = 0; i < 16; ++i)
+                        put_code(fmt, codes, K, r, j * 16 + i, e2m1_encode_quotient(blk[i], denom));
+                }
+            }
+        }
+        return ORC_OK;
+    }
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t j = 0; j < sf_cols; ++j) {
@@ -459,6 +532,7 @@ static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int6
                          uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
     int bs = fmt_block(fmt);
     if (!fmt_ok(fmt) || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    if (fmt == ORC_MXFP4_MBS && K % 128 != 0) return ORC_EINVAL;
     double *xv = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
     if (!xv) return ORC_EINVAL;
     for (int64_t r = 0; r < M; ++r)
@@ -480,6 +554,7 @@ int orc_quantize_f32(int fmt, const float *src, int64_t M, int64_t K, int64_t ld
                      float *gscale, int gscale_given) {
     int bs = fmt_block(fmt);
     if (!fmt_ok(fmt) || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
+    if (fmt == ORC_MXFP4_MBS && K % 128 != 0) return ORC_EINVAL;
     double *xv = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
     if (!xv) return ORC_EINVAL;
     for (int64_t r = 0; r < M; ++r)
@@ -558,20 +633,29 @@ double orc_qsnr_db(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const 
     return 10.0 * log10(sx / se);
 }
 
+/* The real factor of element (r, k): g * s (NVFP4), 2^(E-127) (MX), or
+ * (1 + m/256) * 2^(E-127) (MXFP4-MBS, reading R20); exact in fp64. */
+static double block_scale(int fmt, const uint8_t *scales, int64_t M, int64_t K, int64_t r, int64_t k, float gscale) {
+    int bs = fmt_block(fmt);
+    uint8_t sb = scales[orc_sf_offset(r, k / bs, K / bs)];
+    if (fmt == ORC_NVFP4) return (double)gscale * orc_e4m3_decode(sb);
+    if (fmt == ORC_MXFP4_MBS) {
+        int m = scales[orc_mbs_macro_offset(M, K, r, k / 128)];
+        return ldexp((double)(256 + m), (int)sb - 135);
+    }
+    return orc_e8m0_decode(sb);
+}
+
 /* Dequantize to fp64: x = g * s * q (g = 1 for MX) [MXFP4-page, Fundamentos:
  * x_real = S_E8M0 * x_E2M1].  The products are exact in fp64. */
 int orc_dequantize_f64(int fmt, const uint8_t *codes, const uint8_t *scales, float gscale,
                        int64_t M, int64_t K, double *dst) {
     int bs = fmt_block(fmt);
-    if (!fmt_ok(fmt) || K % bs != 0) return ORC_EINVAL;
-    int64_t sf_cols = K / bs;
+    if (!fmt_ok(fmt) || K % bs != 0 || (fmt == ORC_MXFP4_MBS && K % 128 != 0)) return ORC_EINVAL;
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t k = 0; k < K; ++k) {
-            uint8_t sb = scales[orc_sf_offset(r, k / bs, sf_cols)];
-            double s = (fmt == ORC_NVFP4) ? (double)gscale * orc_e4m3_decode(sb)
-                                          : orc_e8m0_decode(sb);
-            dst[r * K + k] = s * fmt_decode(fmt, get_code(fmt, codes, K, r, k));
+            dst[r * K + k] = block_scale(fmt, scales, M, K, r, k, gscale) * fmt_decode(fmt, get_code(fmt, codes, K, r, k));
         }
     }
     return ORC_OK;
@@ -581,15 +665,12 @@ int orc_dequantize_f64(int fmt, const uint8_t *codes, const uint8_t *scales, flo
 int orc_dequantize_bf16(int fmt, const uint8_t *codes, const uint8_t *scales, float gscale,
                         int64_t M, int64_t K, uint16_t *dst, int64_t ld) {
     int bs = fmt_block(fmt);
-    if (!fmt_ok(fmt) || K % bs != 0 || ld < K) return ORC_EINVAL;
-    int64_t sf_cols = K / bs;
+    if (!fmt_ok(fmt) || K % bs != 0 || ld < K || (fmt == ORC_MXFP4_MBS && K % 128 != 0)) return ORC_EINVAL;
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t k = 0; k < K; ++k) {
-            uint8_t sb = scales[orc_sf_offset(r, k / bs, sf_cols)];
-            double s = (fmt == ORC_NVFP4) ? (double)gscale * orc_e4m3_decode(sb)
-                                          : orc_e8m0_decode(sb);
-            dst[r * ld + k] = orc_double_to_bf16_rne(s * fmt_decode(fmt, get_code(fmt, codes, K, r, k)));
+            dst[r * ld + k] =
+                orc_double_to_bf16_rne(block_scale(fmt, scales, M, K, r, k, gscale) * fmt_decode(fmt, get_code(fmt, codes, K, r, k)));
         }
     }
     return ORC_OK;
