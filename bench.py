@@ -278,7 +278,7 @@ def qsnr_table(device):
         row = {}
         for label, quant in (("mxfp8_e4m3", lambda: mx.quantize(x, 0)), ("mxfp4", lambda: mx.quantize(x, 2)),
                              ("mxfp4_oas", lambda: mx.quantize_oas(x)), ("nvfp4", lambda: mx.quantize(x, 3)),
-                             ("mxfp6_e3m2", lambda: mx.quantize(x, 4))):
+                             ("mxfp6_e3m2", lambda: mx.quantize(x, 4)), ("mxfp4_mbs", lambda: mx.quantize(x, 5))):
             s = mx.qsnr_sums(quant(), x).cpu().numpy()
             row[label] = round(float(10.0 * np.log10(s[0] / s[1])), 3)
         for label, fmt in (("mxfp4_rht32", 2), ("nvfp4_rht32", 3)):
@@ -334,7 +334,8 @@ def kv_cache_extras(device, peaks, timed):
 
 
 def quant_bytes_per_elem(fmt):
-    return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625, 4: 2.78125}[fmt]
+    # bf16 read + codes + scales (MXFP4-MBS: E8M0 per 16 and one macro byte per 128)
+    return {0: 3.03125, 1: 3.03125, 2: 2.53125, 3: 2.5625, 4: 2.78125, 5: 2.5703125}[fmt]
 
 
 def extras_gpu(device):
@@ -393,13 +394,15 @@ def extras_gpu(device):
     gbs = M * K * quant_bytes_per_elem(2) / (ms * 1e-3) / 1e9
     sweep[f"mxfp4_oas_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
     del qs
-    # MXFP6 E3M2: 2 B read + 0.75 B of codes + 1/32 B of scale per element
-    qs = [mx.empty(4, M, K) for _ in xs]
-    ms = timed(lambda i: mx.quantize(xs[i % len(xs)], 4, out=qs[i % len(xs)]), len(xs))
-    gbs = M * K * quant_bytes_per_elem(4) / (ms * 1e-3) / 1e9
-    sweep[f"mxfp6_e3m2_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+    # MXFP6 E3M2 (2 B read + 0.75 B of codes + 1/32 B of scale per element) and
+    # MXFP4 with static macro-block scaling
+    for fmt, name in ((4, "mxfp6_e3m2"), (5, "mxfp4_mbs")):
+        qs = [mx.empty(fmt, M, K) for _ in xs]
+        ms = timed(lambda i: mx.quantize(xs[i % len(xs)], fmt, out=qs[i % len(xs)]), len(xs))
+        gbs = M * K * quant_bytes_per_elem(fmt) / (ms * 1e-3) / 1e9
+        sweep[f"{name}_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
                                  "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
-    del qs
+        del qs
     # Walsh-Hadamard rotation fused with quantization: the same HBM bytes as the plain quantize
     for fmt, name in ((2, "mxfp4_rht32"), (3, "nvfp4_rht32")):
         qs = [mx.empty(fmt, M, K) for _ in xs]
@@ -509,6 +512,7 @@ PROFILE_CASES = {
     "gemm_dit_mxfp6": ("gemm", 4, 4096, 3072, 3072),
     "gemm_dit_mxfp8_x_mxfp4w": ("gemm", 0, 4096, 3072, 3072, 2),
     "quant_mxfp6_32768x4096": ("quant", 4, 32768, 0, 4096),
+    "quant_mbs_32768x4096": ("quant", 5, 32768, 0, 4096),
     "rht_mxfp4_32768x4096": ("rht", 2, 32768, 0, 4096),
     "gemm_mlp1_nvfp4": ("gemm", 3, 4608, 12288, 3072),
     "gemm_mlp2_nvfp4": ("gemm", 3, 4608, 3072, 12288),
@@ -584,7 +588,7 @@ def gemm_kernel_name(fmt: int, M: int, N: int) -> str:
     if M > 128 and N > 128:
         return f"gemm_pair_kernel<{fmt}, {6 if fmt < 2 else 5}>"
     return f"gemm_kernel<{fmt}, {128 if N <= 128 else 256}, 4>"
-FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4", 4: "mxfp6_e3m2"}
+FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4", 4: "mxfp6_e3m2", 5: "mxfp4_mbs"}
 
 
 def main():

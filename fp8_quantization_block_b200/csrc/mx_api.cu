@@ -35,10 +35,23 @@ int pdl_attr(cudaLaunchAttribute *a) {
     return 1;
 }
 
-bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 4; }
-int fmt_block(int fmt) { return fmt == MX_NVFP4 ? 16 : 32; }
-int fmt_bits(int fmt) { return (fmt == MX_MXFP4 || fmt == MX_NVFP4) ? 4 : (fmt == MX_MXFP6_E3M2 ? 6 : 8); }
+bool valid_fmt(int fmt) { return fmt >= 0 && fmt <= 5; }
+int fmt_block(int fmt) { return (fmt == MX_NVFP4 || fmt == MX_MXFP4_MBS) ? 16 : 32; }
+int fmt_bits(int fmt) {
+    return (fmt == MX_MXFP4 || fmt == MX_NVFP4 || fmt == MX_MXFP4_MBS) ? 4 : (fmt == MX_MXFP6_E3M2 ? 6 : 8);
+}
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+// Blocking granularity a format needs along K (MXFP4-MBS: its 128-element macro blocks).
+int fmt_k_multiple(int fmt) { return fmt == MX_MXFP4_MBS ? 128 : fmt_block(fmt); }
+// Scale tiles, and for MXFP4-MBS the macro mantissas after them ([rows][cols/128], padded to 16).
+size_t tile_bytes(int fmt, int64_t rows, int64_t cols) {
+    return (size_t)(cdiv(rows, 128) * 128 * cdiv(cols / fmt_block(fmt), 4) * 4);
+}
+size_t scales_bytes(int fmt, int64_t rows, int64_t cols) {
+    size_t t = tile_bytes(fmt, rows, cols);
+    if (fmt == MX_MXFP4_MBS) t += (size_t)(cdiv(rows * (cols / 128), 16) * 16);
+    return t;
+}
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 mx_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
@@ -159,6 +172,19 @@ void launch_quantize_rht(const uint16_t *src, int64_t M, int64_t K, int64_t ld, 
                        sf_tiles_k, g_in, g_out, g_from_amax);
 }
 
+void launch_quantize_mbs(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst, cudaStream_t st) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(K / kQTileCols), (unsigned)cdiv(M, kQTileRows), 1);
+    cfg.blockDim = dim3(kQThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    cudaLaunchKernelEx(&cfg, quantize_mbs_kernel, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
+                       cdiv(K / 16, 4), dst->scales + tile_bytes(MX_MXFP4_MBS, M, K));
+}
+
 int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -185,7 +211,7 @@ mx_status nvfp4_gscale_prepass(const uint16_t *src, int64_t M, int64_t K, int64_
 
 mx_status check_tensor(const mx_tensor *t, bool need_codes) {
     if (!t || !valid_fmt(t->fmt) || t->rows < 0 || t->cols < 0) return MX_ERR_INVALID_ARG;
-    if (t->cols % fmt_block(t->fmt) != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (t->cols % fmt_k_multiple(t->fmt) != 0) return MX_ERR_UNSUPPORTED_SHAPE;
     if (t->rows > 0 && t->cols > 0) {
         if (need_codes && (!t->codes || !t->scales)) return MX_ERR_INVALID_ARG;
         if (!aligned16(t->codes) || !aligned16(t->scales)) return MX_ERR_MISALIGNED;
@@ -446,7 +472,7 @@ size_t mx_codes_bytes(int fmt, int64_t rows, int64_t cols) {
 
 size_t mx_scales_bytes(int fmt, int64_t rows, int64_t cols) {
     if (!valid_fmt(fmt) || rows < 0 || cols < 0) return 0;
-    return (size_t)(cdiv(rows, 128) * 128 * cdiv(cols / fmt_block(fmt), 4) * 4);
+    return scales_bytes(fmt, rows, cols);
 }
 
 int mx_block_size(int fmt) { return valid_fmt(fmt) ? fmt_block(fmt) : 0; }
@@ -480,7 +506,7 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
                       const float *gscale_in, void *stream) {
     if (!valid_fmt(fmt) || !dst || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
     if (dst->fmt != fmt || dst->rows != M || dst->cols != K) return MX_ERR_INVALID_ARG;
-    if (K % fmt_block(fmt) != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (K % fmt_k_multiple(fmt) != 0) return MX_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 || K == 0) return MX_OK;
     if (!src_bf16 || !dst->codes || !dst->scales) return MX_ERR_INVALID_ARG;
     if (fmt == MX_NVFP4 && !dst->gscale) return MX_ERR_INVALID_ARG;
@@ -494,6 +520,7 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
     case MX_MXFP8_E5M2: launch_quantize<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP4: launch_quantize<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP6_E3M2: launch_quantize<4>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP4_MBS: launch_quantize_mbs(src, M, K, ld_src, dst, st); break;
     default: {
         if (gscale_in == nullptr) {
             mx_status s = nvfp4_gscale_prepass(src, M, K, ld_src, dst->gscale, st);
@@ -524,7 +551,7 @@ mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld
 
 mx_status mx_quantize_rht(int fmt, const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
                           const float *gscale_in, void *stream) {
-    if (!valid_fmt(fmt) || !dst || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt) || fmt == MX_MXFP4_MBS || !dst || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
     if (dst->fmt != fmt || dst->rows != M || dst->cols != K) return MX_ERR_INVALID_ARG;
     if (K % 32 != 0) return MX_ERR_UNSUPPORTED_SHAPE;   // rotation blocks of 32
     if (M == 0 || K == 0) return MX_OK;
@@ -579,12 +606,14 @@ mx_status mx_qsnr(const mx_tensor *q, const void *src_bf16, int64_t ld_src, doub
     const uint16_t *x = static_cast<const uint16_t *>(src_bf16);
     const uint8_t *c = static_cast<const uint8_t *>(q->codes);
     const unsigned b = (unsigned)blocks;
+    const uint8_t *mac = q->scales + tile_bytes(q->fmt, q->rows, q->cols);   // MXFP4-MBS only
     switch (q->fmt) {
-    case MX_MXFP8_E4M3: qsnr_kernel<0><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
-    case MX_MXFP8_E5M2: qsnr_kernel<1><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
-    case MX_MXFP4: qsnr_kernel<2><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
-    case MX_MXFP6_E3M2: qsnr_kernel<4><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, q->rows, q->cols, sums); break;
-    default: qsnr_kernel<3><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, q->gscale, q->rows, q->cols, sums);
+    case MX_MXFP8_E4M3: qsnr_kernel<0><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP8_E5M2: qsnr_kernel<1><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP4: qsnr_kernel<2><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP6_E3M2: qsnr_kernel<4><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, nullptr, q->rows, q->cols, sums); break;
+    case MX_MXFP4_MBS: qsnr_kernel<5><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, nullptr, mac, q->rows, q->cols, sums); break;
+    default: qsnr_kernel<3><<<b, 256, 0, st>>>(x, ld_src, c, q->scales, q->gscale, nullptr, q->rows, q->cols, sums);
     }
     return last_launch();
 }
@@ -600,12 +629,14 @@ mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, vo
     const unsigned blocks = (unsigned)cdiv(n, 256);
     const uint8_t *c = static_cast<const uint8_t *>(src->codes);
     uint16_t *d = static_cast<uint16_t *>(dst_bf16);
+    const uint8_t *mac = src->scales + tile_bytes(src->fmt, src->rows, src->cols);   // MXFP4-MBS only
     switch (src->fmt) {
-    case MX_MXFP8_E4M3: dequantize_kernel<0><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
-    case MX_MXFP8_E5M2: dequantize_kernel<1><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
-    case MX_MXFP4: dequantize_kernel<2><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
-    case MX_MXFP6_E3M2: dequantize_kernel<4><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, src->rows, src->cols, d, ld_dst); break;
-    default: dequantize_kernel<3><<<blocks, 256, 0, st>>>(c, src->scales, src->gscale, src->rows, src->cols, d, ld_dst);
+    case MX_MXFP8_E4M3: dequantize_kernel<0><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP8_E5M2: dequantize_kernel<1><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP4: dequantize_kernel<2><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP6_E3M2: dequantize_kernel<4><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, nullptr, src->rows, src->cols, d, ld_dst); break;
+    case MX_MXFP4_MBS: dequantize_kernel<5><<<blocks, 256, 0, st>>>(c, src->scales, nullptr, mac, src->rows, src->cols, d, ld_dst); break;
+    default: dequantize_kernel<3><<<blocks, 256, 0, st>>>(c, src->scales, src->gscale, nullptr, src->rows, src->cols, d, ld_dst);
     }
     return last_launch();
 }

@@ -24,7 +24,7 @@
 
 namespace mx {
 
-enum { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_MXFP4 = 2, FMT_NVFP4 = 3, FMT_MXFP6 = 4 };
+enum { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_MXFP4 = 2, FMT_NVFP4 = 3, FMT_MXFP6 = 4, FMT_MXFP4_MBS = 5 };
 
 template <int FMT>
 struct FmtTraits;
@@ -46,6 +46,11 @@ struct FmtTraits<FMT_MXFP4> {
 };
 template <>
 struct FmtTraits<FMT_NVFP4> {
+    static constexpr int kBlock = 16, kBits = 4;
+    static constexpr int kExpOff = 0, kMantThr = 0;
+};
+template <>
+struct FmtTraits<FMT_MXFP4_MBS> {  // E2M1 elements, E8M0 per 16, macro mantissa per 128
     static constexpr int kBlock = 16, kBits = 4;
     static constexpr int kExpOff = 0, kMantThr = 0;
 };
@@ -263,6 +268,45 @@ MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, floa
     out1 = c1;
 }
 
+// E2M1 codes of 16 fp32 values x / (g s): the bracket of nv_codes16 on fp32
+// inputs (r_lo <= 1/(g s) <= r_hi; g * s * mid must be exact for the settle).
+MX_DEVICE_INLINE uint32_t nv_settle_f32(uint32_t code, uint32_t diff, const float *x8, float g, float s) {
+    while (diff != 0u) {
+        const int nib = (__ffs(diff) - 1) >> 2;
+        diff &= ~(0xFu << (4 * nib));
+        float ax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i == nib) ax = fabsf(x8[i]);
+        const uint32_t c = (code >> (4 * nib)) & 7u;
+        const float d = __fmaf_rn(-g, s * e2m1_mid(c), ax);
+        if (d > 0.0f || (d == 0.0f && (c & 1u))) code += 1u << (4 * nib);
+    }
+    return code;
+}
+
+MX_DEVICE_INLINE void nv_codes16_f32(const float (&x)[16], float g, float s, float r_lo, float r_hi,
+                                     uint32_t &out0, uint32_t &out1) {
+    float lo[16], hi[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        lo[i] = __fmul_rz(x[i], r_lo);
+        hi[i] = __fmul_ru(fabsf(x[i]), r_hi);
+    }
+    const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
+    const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
+    const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
+    const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
+    uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
+    const uint32_t d0 = (c0 & 0x77777777u) ^ cvt8_e2m1(hi0), d1 = (c1 & 0x77777777u) ^ cvt8_e2m1(hi1);
+    if ((d0 | d1) != 0u) {
+        c0 = nv_settle_f32(c0, d0, &x[0], g, s);
+        c1 = nv_settle_f32(c1, d1, &x[8], g, s);
+    }
+    out0 = c0;
+    out1 = c1;
+}
+
 // Per-CTA tables for NVFP4, indexed by positive E4M3 code c (1..126):
 // the value s, and 1/s rounded down and up.
 struct NvTables {
@@ -435,6 +479,145 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
     griddep_launch_dependents();
 }
 
+// ------------------------------------------------------------------ MXFP4 with macro-block scaling
+// Page "Unveiling the Potential of Quantization with MXFP4", section B (Macro
+// Block Scaling), static variant: per 1x128 macro block a factor 1 + m/256
+// with m chosen from the block max alpha (e = floor(log2(alpha / 6)); m the
+// smallest byte with alpha <= 6 (256 + m) 2^(e-8), 0 if none), then E2M1
+// elements in 1x16 blocks with E8M0 scales applied to x / (1 + m/256).
+//
+// With alpha = M_a 2^(ea-7), M_a in [128, 255] (bf16 mantissa with its
+// leading one; subnormals normalised), alpha / 2^(e-8) is the integer
+// A = 16 M_a (M_a < 192) or 8 M_a, and m = ceil(A / 6) - 256.
+MX_DEVICE_INLINE void bf16_normalise(uint32_t bits, uint32_t &mant, int &ex) {
+    const uint32_t ef = (bits >> 7) & 0xFFu, fr = bits & 0x7Fu;
+    if (ef != 0u) {
+        mant = 128u + fr;
+        ex = (int)ef - 127;
+    } else {
+        // subnormal: fr != 0 (the caller handles zero); 8 - bit length of fr shifts
+        const int sh = __clz(fr) - 24;
+        mant = fr << sh;
+        ex = -126 - sh;
+    }
+}
+
+MX_DEVICE_INLINE uint32_t mbs_static_mantissa(uint32_t alpha_bits) {
+    if (alpha_bits == 0u) return 0u;
+    uint32_t ma;
+    int ea;
+    bf16_normalise(alpha_bits, ma, ea);
+    const uint32_t A = ma < 192u ? 16u * ma : 8u * ma;   // in [1536, 3072)
+    const uint32_t m = (A + 5u) / 6u - 256u;
+    return m > 255u ? 0u : m;
+}
+
+// Smallest E in [0, 254] with amax_b <= 6 (256 + m) 2^(E - 135): with
+// amax_b = M_b 2^(eb-7), M_b in [128, 255], the condition reads
+// M_b 2^(eb + 128 - E) <= 6 (256 + m), whose largest shift is 2, 3 or 4.
+MX_DEVICE_INLINE uint32_t mbs_block_exponent(uint32_t amax_bits, uint32_t m) {
+    if (amax_bits == 0u) return 0u;
+    uint32_t mb;
+    int eb;
+    bf16_normalise(amax_bits, mb, eb);
+    const uint32_t km = 6u * (256u + m);
+    const int d = (mb << 4) <= km ? 4 : ((mb << 3) <= km ? 3 : 2);
+    const int E = eb + 128 - d;
+    return (uint32_t)(E < 0 ? 0 : (E > 254 ? 254 : E));
+}
+
+// Per-CTA reciprocals of k = 256 + m (m = 0..255), rounded down and up.
+struct MbsTables {
+    float rcp_lo[256];
+    float rcp_hi[256];
+};
+
+// Same tile structure as quantize_kernel: a 128-column tile row is exactly one
+// macro block, spread over 8 lanes (16 elements each, one base block per lane).
+// Elements: v = x 2^(135-E) (two exact power-of-two products), code = RNE of
+// v / (256 + m) on E2M1 by the directed-rounding bracket, ties settled exactly.
+// macro_out: the [M][K/128] macro mantissa bytes (K % 128 == 0).
+__global__ void __launch_bounds__(kQThreads) quantize_mbs_kernel(const uint16_t *__restrict__ src, int64_t M,
+                                                                 int64_t K, int64_t ld, uint8_t *__restrict__ codes,
+                                                                 uint8_t *__restrict__ scales, int64_t sf_tiles_k,
+                                                                 uint8_t *__restrict__ macro_out) {
+    constexpr int kBlocksPerRow = kQTileCols / 16;
+    constexpr int kSfBytes = kQTileRows * kBlocksPerRow;   // 1024
+    constexpr int kPasses = kQTileRows / 32;
+    __shared__ __align__(16) uint8_t sf_tile[kSfBytes];
+    __shared__ MbsTables tab;
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row0 = (int64_t)blockIdx.y * kQTileRows;
+    const int64_t col0 = (int64_t)blockIdx.x * kQTileCols;
+    const int cl = (lane & 7) * 16;
+    const int64_t col = col0 + cl;
+    const int jb = cl / 16;
+    {
+        const float k = (float)(256 + threadIdx.x);   // kQThreads == 256
+        tab.rcp_lo[threadIdx.x] = __frcp_rd(k);
+        tab.rcp_hi[threadIdx.x] = __frcp_ru(k);
+    }
+    griddep_wait();
+    __syncthreads();
+
+    uint4 v[kPasses][2];
+#pragma unroll
+    for (int i = 0; i < kPasses; ++i) {
+        const int rl = i * 32 + warp * 4 + (lane >> 3);
+        const int64_t row = row0 + rl;
+        if (row < M) {
+            const uint16_t *p = src + row * ld + col;
+            v[i][0] = ldg_stream(p);
+            v[i][1] = ldg_stream(p + 8);
+        } else {
+            v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+
+#pragma unroll
+    for (int i = 0; i < kPasses; ++i) {
+        const int rl = i * 32 + warp * 4 + (lane >> 3);
+        const int64_t row = row0 + rl;
+        const bool ok = row < M;
+        const uint32_t amax = absmax16(v[i][0], v[i][1]);
+        uint32_t alpha = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        alpha = max(alpha, __shfl_xor_sync(0xffffffffu, alpha, 2));
+        alpha = max(alpha, __shfl_xor_sync(0xffffffffu, alpha, 4));
+        const uint32_t m = mbs_static_mantissa(alpha);
+        const uint32_t E = mbs_block_exponent(amax, m);
+        if (ok) {
+            // 2^(135 - E) as two fp32 powers of two (135 - E in [-119, 135])
+            const int t = 135 - (int)E, t1 = t / 2, t2 = t - t / 2;
+            const float p1 = __uint_as_float((uint32_t)(127 + t1) << 23), p2 = __uint_as_float((uint32_t)(127 + t2) << 23);
+            float x[16];
+            const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w, v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                x[2 * e] = (bf16lo(w[e]) * p1) * p2;
+                x[2 * e + 1] = (bf16hi(w[e]) * p1) * p2;
+            }
+            uint32_t q0, q1;
+            nv_codes16_f32(x, 1.0f, (float)(256u + m), tab.rcp_lo[m], tab.rcp_hi[m], q0, q1);
+            *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
+            if ((lane & 7) == 0) macro_out[row * (K / 128) + blockIdx.x] = (uint8_t)m;
+        }
+        sf_tile[(jb >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (jb & 3)] = ok ? (uint8_t)E : (uint8_t)0;
+    }
+    // the macro section's padding to 16 bytes is zero, as every padding byte
+    if (blockIdx.x == 0 && blockIdx.y == 0) {
+        const int64_t n = M * (K / 128), pad = ((n + 15) & ~(int64_t)15) - n;
+        if (threadIdx.x < pad) macro_out[n + threadIdx.x] = 0;
+    }
+    __syncthreads();
+    const int64_t chunk0 = (int64_t)blockIdx.y * sf_tiles_k + (int64_t)blockIdx.x * 2;
+    if (threadIdx.x < kSfBytes / 16) {
+        const uint4 val = *reinterpret_cast<const uint4 *>(sf_tile + threadIdx.x * 16);
+        *reinterpret_cast<uint4 *>(scales + chunk0 * 512 + threadIdx.x * 16) = val;
+    }
+    griddep_launch_dependents();
+}
+
 // max |x| over a bf16 tensor -> atomicMax on the float bits of *amax (init 0).
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
                                                    int64_t ld, unsigned int *__restrict__ amax_bits) {
@@ -468,14 +651,16 @@ __global__ void gscale_from_amax_kernel(float *__restrict__ slot) {
 
 // Decode 8 consecutive elements (row r, columns c..c+7) of a quantized matrix:
 // the block's scale s (g*s for NVFP4, exact in fp64) and the 8 element values.
+// macro: MXFP4-MBS only, the [rows][K/128] macro mantissas after the scale tiles.
 template <int FMT>
 MX_DEVICE_INLINE void load_dequant8(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
-                                    const float *__restrict__ gscale, int64_t K, int64_t r, int64_t c, double &s,
-                                    float (&q)[8]) {
+                                    const float *__restrict__ gscale, const uint8_t *__restrict__ macro, int64_t K,
+                                    int64_t r, int64_t c, double &s, float (&q)[8]) {
     using T = FmtTraits<FMT>;
     const int64_t sf_cols = K / T::kBlock, tiles_k = (sf_cols + 3) / 4, j = c / T::kBlock;
     const uint8_t sb = scales[((r >> 7) * tiles_k + (j >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3)];
     if (FMT == FMT_NVFP4) s = (double)(*gscale) * (double)(sb == 0 ? 0.0f : e4m3_pos_value(sb));
+    else if (FMT == FMT_MXFP4_MBS) s = ldexp((double)(256 + macro[r * (K / 128) + c / 128]), (int)sb - 135);
     else s = sb == 0xFF ? (double)NAN : ldexp(1.0, (int)sb - 127);
     if (T::kBits == 8) {
         const uint2 w = *reinterpret_cast<const uint2 *>(codes + r * K + c);
@@ -523,7 +708,8 @@ MX_DEVICE_INLINE void load_dequant8(const uint8_t *__restrict__ codes, const uin
 template <int FMT>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restrict__ codes,
                                                          const uint8_t *__restrict__ scales,
-                                                         const float *__restrict__ gscale, int64_t M, int64_t K,
+                                                         const float *__restrict__ gscale,
+                                                         const uint8_t *__restrict__ macro, int64_t M, int64_t K,
                                                          uint16_t *__restrict__ dst, int64_t ld) {
     const int64_t vec_per_row = K / 8;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -531,7 +717,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
     const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
     double s;
     float q[8];
-    load_dequant8<FMT>(codes, scales, gscale, K, r, c, s, q);
+    load_dequant8<FMT>(codes, scales, gscale, macro, K, r, c, s, q);
     uint32_t out[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -551,7 +737,8 @@ template <int FMT>
 __global__ void __launch_bounds__(256) qsnr_kernel(const uint16_t *__restrict__ src, int64_t ld,
                                                    const uint8_t *__restrict__ codes,
                                                    const uint8_t *__restrict__ scales,
-                                                   const float *__restrict__ gscale, int64_t M, int64_t K,
+                                                   const float *__restrict__ gscale,
+                                                   const uint8_t *__restrict__ macro, int64_t M, int64_t K,
                                                    double *__restrict__ sums) {
     const int64_t vec_per_row = K / 8, nvec = M * vec_per_row;
     double sx = 0.0, se = 0.0;
@@ -559,7 +746,7 @@ __global__ void __launch_bounds__(256) qsnr_kernel(const uint16_t *__restrict__ 
         const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
         double s;
         float q[8];
-        load_dequant8<FMT>(codes, scales, gscale, K, r, c, s, q);
+        load_dequant8<FMT>(codes, scales, gscale, macro, K, r, c, s, q);
         const uint4 v = *reinterpret_cast<const uint4 *>(src + r * ld + c);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll

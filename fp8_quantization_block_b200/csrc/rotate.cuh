@@ -137,44 +137,6 @@ MX_DEVICE_INLINE int mx_scale_byte_f32(float amax) {
     return e < 0 ? 0 : e;
 }
 
-// NVFP4 codes of 16 fp32 values: the bracket of nv_codes16 on fp32 inputs.
-MX_DEVICE_INLINE uint32_t nv_settle_f32(uint32_t code, uint32_t diff, const float *x8, float g, float s) {
-    while (diff != 0u) {
-        const int nib = (__ffs(diff) - 1) >> 2;
-        diff &= ~(0xFu << (4 * nib));
-        float ax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i == nib) ax = fabsf(x8[i]);
-        const uint32_t c = (code >> (4 * nib)) & 7u;
-        const float d = __fmaf_rn(-g, s * e2m1_mid(c), ax);
-        if (d > 0.0f || (d == 0.0f && (c & 1u))) code += 1u << (4 * nib);
-    }
-    return code;
-}
-
-MX_DEVICE_INLINE void nv_codes16_f32(const float (&x)[16], float g, float s, float r_lo, float r_hi,
-                                     uint32_t &out0, uint32_t &out1) {
-    float lo[16], hi[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        lo[i] = __fmul_rz(x[i], r_lo);
-        hi[i] = __fmul_ru(fabsf(x[i]), r_hi);
-    }
-    const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
-    const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
-    const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
-    const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
-    uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
-    const uint32_t d0 = (c0 & 0x77777777u) ^ cvt8_e2m1(hi0), d1 = (c1 & 0x77777777u) ^ cvt8_e2m1(hi1);
-    if ((d0 | d1) != 0u) {
-        c0 = nv_settle_f32(c0, d0, &x[0], g, s);
-        c1 = nv_settle_f32(c1, d1, &x[8], g, s);
-    }
-    out0 = c0;
-    out1 = c1;
-}
-
 // Rotate and quantize a bf16 [M x K] matrix (K % 32 == 0) into codes / scales
 // laid out as quantize_kernel's.  NVFP4: *gscale_in is g, or max|y| when
 // g_from_amax (then g = RU(max|y| / 2688), 1 for 0); gscale_out as there.

@@ -21,8 +21,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmx.so")
 
-MX_MXFP8_E4M3, MX_MXFP8_E5M2, MX_MXFP4, MX_NVFP4, MX_MXFP6_E3M2 = 0, 1, 2, 3, 4
-FORMATS = {"mxfp8_e4m3": 0, "mxfp8_e5m2": 1, "mxfp4": 2, "nvfp4": 3, "mxfp6_e3m2": 4}
+MX_MXFP8_E4M3, MX_MXFP8_E5M2, MX_MXFP4, MX_NVFP4, MX_MXFP6_E3M2, MX_MXFP4_MBS = 0, 1, 2, 3, 4, 5
+FORMATS = {"mxfp8_e4m3": 0, "mxfp8_e5m2": 1, "mxfp4": 2, "nvfp4": 3, "mxfp6_e3m2": 4, "mxfp4_mbs": 5}
 MX_OK, MX_ERR_INVALID_ARG, MX_ERR_UNSUPPORTED_SHAPE, MX_ERR_MISALIGNED = 0, 1, 2, 3
 MX_ERR_CUDA, MX_ERR_TIMEOUT, MX_ERR_DEVICE = 4, 5, 6
 MX_EPI_NONE, MX_EPI_GELU = 0, 1

@@ -45,7 +45,12 @@ extern "C" {
 #endif
 
 /* Element formats.  Block size 32 with an E8M0 scale for the four MX formats;
- * block size 16 with an E4M3 scale plus one FP32 per-tensor scale for NVFP4.
+ * block size 16 with an E4M3 scale plus one FP32 per-tensor scale for NVFP4;
+ * MXFP4_MBS ([OAS] section B, macro block scaling, static variant): E2M1 in
+ * blocks of 16 with E8M0 scales, plus one byte m per 128 elements (a factor
+ * 1 + m/256 on the whole macro block).  MXFP4_MBS is a storage and fidelity
+ * format: quantize, dequantize and QSNR take it; the GEMM does not (the tensor
+ * core applies only E8M0 / E4M3 block scales).
  * E3M2 ([MX] format table, MXFP6): sign, 3 exponent bits with bias 3, 2
  * mantissa bits, no infinities or NaN, largest magnitude 28. */
 typedef enum {
@@ -53,7 +58,8 @@ typedef enum {
     MX_MXFP8_E5M2 = 1,
     MX_MXFP4 = 2,
     MX_NVFP4 = 3,
-    MX_MXFP6_E3M2 = 4
+    MX_MXFP6_E3M2 = 4,
+    MX_MXFP4_MBS = 5
 } mx_format;
 
 typedef enum {
@@ -78,7 +84,9 @@ typedef enum {
  *           128 rows x 4 scale columns: scale (r, c) of a matrix with C scale
  *           columns is at ((r/128)*ceil(C/4) + c/4)*512 + (r%32)*16
  *           + ((r%128)/32)*4 + c%4 -- the layout the sm_100 tensor core reads.
- *           Padding bytes (rows >= rows, columns >= C) are 0.
+ *           Padding bytes (rows >= rows, columns >= C) are 0.  MXFP4_MBS
+ *           appends its macro bytes, [rows][cols/128] row-major, zero-padded to
+ *           a multiple of 16 bytes, after the tiles.
  *   gscale: device, one float (NVFP4 only; NULL otherwise): the per-tensor
  *           decode multiplier g.  Real value = g * scale * element.           */
 typedef struct {
@@ -98,7 +106,7 @@ size_t mx_scales_bytes(int fmt, int64_t rows, int64_t cols);
 int mx_block_size(int fmt);
 
 /* Quantize a bf16 matrix src [M x K] (row pitch ld_src elements, ld_src >= K,
- * ld_src % 8 == 0) into dst ([MX] "Fundamentos" and FAQ; [NEWS]).
+ * ld_src % 8 == 0) into dst ([MX] "Fundamentos" and FAQ; [NEWS]; [OAS] B).
  *   MX formats: per block, E = ceil(log2(max|x| / max_elem)) + 127 clamped to
  *     [0, 254] (0 for an all-zero block), elements = RNE(x / 2^(E-127))
  *     saturating to the element format (max_elem = 448 / 57344 / 6 / 28 for
@@ -109,6 +117,11 @@ int mx_block_size(int fmt);
  *     *dst->gscale.  Block scale s = smallest positive finite E4M3 with
  *     max|x| <= 6*g*s (0 for an all-zero block); element = RNE of the exact
  *     quotient x / (g*s) onto E2M1, saturating at 6.
+ *   MXFP4_MBS: per 128 elements, with alpha = max|x| and e = floor(log2(alpha
+ *     / 6)), m = the smallest byte with alpha <= 6 (256 + m) 2^(e-8) (0 for a
+ *     zero block); per 16 elements E = the smallest exponent with max|x| <=
+ *     6 (1 + m/256) 2^(E-127); elements = RNE of the exact quotient
+ *     x / ((1 + m/256) 2^(E-127)) onto E2M1, saturating at 6.  K % 128 == 0.
  * Rounding is to nearest, ties to even; a value that rounds to zero keeps its
  * sign.  K must be a multiple of the block size (32, or 16 for NVFP4).
  * dst->rows/cols must equal M/K and dst->fmt must equal fmt.  Non-finite

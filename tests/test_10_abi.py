@@ -40,13 +40,14 @@ def test_sizes_match_layout(L):
     assert mx.mx_scales_bytes(mx.MX_NVFP4, 129, 80) == 256 * 8
     assert mx.mx_block_size(mx.MX_NVFP4) == 16 and mx.mx_block_size(mx.MX_MXFP4) == 32
     assert mx.mx_codes_bytes(mx.MX_MXFP6_E3M2, 3, 64) == 144 and mx.mx_block_size(mx.MX_MXFP6_E3M2) == 32
+    assert mx.mx_scales_bytes(mx.MX_MXFP4_MBS, 3, 256) == 128 * 16 + 16 and mx.mx_block_size(mx.MX_MXFP4_MBS) == 16
     assert mx.mx_codes_bytes(7, 4, 4) == 0 and mx.mx_block_size(-1) == 0
 
 
 def test_sizes_agree_with_oracle(L):
     import oracle
-    for fmt in range(5):
-        for (r, c) in [(1, 64), (127, 128), (129, 4096), (4608, 3072)]:
+    for fmt in range(6):
+        for (r, c) in [(1, 128), (127, 128), (129, 4096), (4608, 3072)]:
             assert mx.mx_codes_bytes(fmt, r, c) == oracle.codes_bytes(fmt, r, c)
             assert mx.mx_scales_bytes(fmt, r, c) == oracle.scales_bytes(fmt, r, c)
 
@@ -80,6 +81,11 @@ def test_host_checks_reject_bad_arguments(L):
     assert mx.mx_gemm(A, _t(2, 8, 256, codes=0x1010), 0x4000, 8, None) == mx.MX_ERR_MISALIGNED
     assert mx.mx_gemm(_t(4, 8, 64), _t(4, 8, 64), 0x4000, 8, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
     assert mx.mx_quantize(4, 0x1000, 4, 48, 48, _t(4, 4, 48), None, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
+    # MXFP4 with macro-block scaling: K a multiple of 128; not a GEMM or rotation format
+    assert mx.mx_quantize(5, 0x1000, 4, 64, 64, _t(5, 4, 64), None, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
+    assert mx.mx_gemm(_t(5, 8, 256), _t(5, 8, 256), 0x4000, 8, None) == mx.MX_ERR_INVALID_ARG
+    assert mx.mx_quantize_rht(5, 0x1000, 4, 256, 256, _t(5, 4, 256), None, None) == mx.MX_ERR_INVALID_ARG
+    assert mx.mx_dequantize(_t(5, 4, 64), 0x4000, 64, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
     assert mx.mx_gemm(A, _t(0, 8, 128), 0x4000, 8, None) == mx.MX_ERR_INVALID_ARG               # K mismatch
     assert mx.mx_gemm(_t(0, 8, 96), _t(0, 8, 96), 0x4000, 8, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
     assert mx.mx_gemm(A, B, 0x4004, 8, None) == mx.MX_ERR_MISALIGNED
