@@ -268,6 +268,15 @@ MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, floa
     out1 = c1;
 }
 
+MX_DEVICE_INLINE void unpack16(const uint4 &v0, const uint4 &v1, float (&x)[16]) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = bf16lo(w[i]);
+        x[2 * i + 1] = bf16hi(w[i]);
+    }
+}
+
 // E2M1 codes of 16 fp32 values x / (g s): the bracket of nv_codes16 on fp32
 // inputs (r_lo <= 1/(g s) <= r_hi; g * s * mid must be exact for the settle).
 MX_DEVICE_INLINE uint32_t nv_settle_f32(uint32_t code, uint32_t diff, const float *x8, float g, float s) {
@@ -587,18 +596,22 @@ __global__ void __launch_bounds__(kQThreads) quantize_mbs_kernel(const uint16_t 
         const uint32_t m = mbs_static_mantissa(alpha);
         const uint32_t E = mbs_block_exponent(amax, m);
         if (ok) {
-            // 2^(135 - E) as two fp32 powers of two (135 - E in [-119, 135])
+            // The quotient is x / D, D = (256 + m) 2^(E - 135).  Its bracket
+            // reciprocals are 1/(256 + m) from the tables times 2^(135 - E),
+            // formed with outward rounding (two power-of-two factors, since
+            // 135 - E spans [-119, 135]); the settle compares |x| with
+            // 2^(E - 135) * ((256 + m) mid) inside one exact fma.
             const int t = 135 - (int)E, t1 = t / 2, t2 = t - t / 2;
             const float p1 = __uint_as_float((uint32_t)(127 + t1) << 23), p2 = __uint_as_float((uint32_t)(127 + t2) << 23);
+            const float r_lo = __fmul_rd(__fmul_rd(tab.rcp_lo[m], p1), p2);
+            const float r_hi = __fmul_ru(__fmul_ru(tab.rcp_hi[m], p1), p2);
+            // 2^(E - 135) as an fp32 (subnormal below E = 9, exact down to 2^-149)
+            const float d2 = E >= 9u ? __uint_as_float((uint32_t)(E - 8u) << 23)
+                                     : __uint_as_float(1u << (E + 14u));
             float x[16];
-            const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w, v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                x[2 * e] = (bf16lo(w[e]) * p1) * p2;
-                x[2 * e + 1] = (bf16hi(w[e]) * p1) * p2;
-            }
+            unpack16(v[i][0], v[i][1], x);
             uint32_t q0, q1;
-            nv_codes16_f32(x, 1.0f, (float)(256u + m), tab.rcp_lo[m], tab.rcp_hi[m], q0, q1);
+            nv_codes16_f32(x, d2, (float)(256u + m), r_lo, r_hi, q0, q1);
             *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
             if ((lane & 7) == 0) macro_out[row * (K / 128) + blockIdx.x] = (uint8_t)m;
         }

@@ -116,15 +116,6 @@ MX_DEVICE_INLINE void rht32_halves(float (&x)[16], int lane) {
     rht32_scale(x);
 }
 
-MX_DEVICE_INLINE void unpack16(const uint4 &v0, const uint4 &v1, float (&x)[16]) {
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        x[2 * i] = bf16lo(w[i]);
-        x[2 * i + 1] = bf16hi(w[i]);
-    }
-}
-
 // MX exponent from the fp32 bits of a block's max |y| (non-negative, finite):
 // amax = 1.m * 2^(f-127), max_elem = M * 2^k: E = f - k + (m > (M - 1) 2^23),
 // clamped below at 0 (zero and tiny maxima).
