@@ -211,13 +211,50 @@ MX_DEVICE_INLINE float e2m1_mag(uint32_t c) {
 
 // NVFP4 elements: codes of x / (g s) for 16 values, the exact RNE of the real
 // quotient q.  r_lo <= 1/(g s) <= r_hi.  lo = x * r_lo rounded toward zero
-// keeps the sign and bounds |q| from below; hi = |x| * r_hi rounded up bounds
-// it from above.  RNE is monotone, so the code lies between lo's and hi's;
-// the bracket is a few ulps wide, so they differ by at most one step, and
-// only when a midpoint m between the two codes lies inside it.  Such an
-// element (typically a tie: bf16 inputs divided by a short scale often land
-// exactly on a midpoint) is settled by the sign of |x| - g*s*m, which one fma
-// computes exactly (s*m is exact in fp32); a tie goes to the even code.
+// bounds |q| from below; hi = x * r_hi (1 + 2^-21) (the factor rounded up),
+// also rounded toward zero, bounds it from above: the product exceeds |q| by
+// a relative 2^-21, more than the 2^-23 that rounding toward zero can take
+// off.  Both are sign-symmetric, so each pair of elements takes one packed
+// f32x2 multiply per bound.  RNE is monotone, so the code lies between lo's
+// and hi's; the bracket is a few ulps wide, so they differ by at most one
+// step, and only when a midpoint m between the two codes lies inside it.
+// Such an element (typically a tie: bf16 inputs divided by a short scale often
+// land exactly on a midpoint) is settled by the sign of |x| - g*s*m, which one
+// fma computes exactly (s*m is exact in fp32); a tie goes to the even code.
+
+// Packed fp32 pairs (f32x2 arithmetic of sm_100: two IEEE operations per
+// instruction, each rounded to nearest-even exactly as its scalar form).
+MX_DEVICE_INLINE uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+MX_DEVICE_INLINE void upk2(uint64_t r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
+MX_DEVICE_INLINE uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t mul2_rz(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
 
 // Midpoint between E2M1 magnitudes c and c + 1 (c = 0..6).
 MX_DEVICE_INLINE float e2m1_mid(uint32_t c) {
@@ -242,24 +279,31 @@ MX_DEVICE_INLINE uint32_t nv_settle(uint32_t code, uint32_t diff, uint32_t w0, u
     return code;
 }
 
+// lo / hi brackets of 16 values held as 8 packed pairs (see above).
+MX_DEVICE_INLINE void bracket16(const uint64_t (&P)[8], float r_lo, float r_hi, float (&lo)[16], float (&hi)[16]) {
+    const float r_up = __fmul_ru(r_hi, 1.0f + 0x1p-21f);
+    const uint64_t RL = pk2(r_lo, r_lo), RU = pk2(r_up, r_up);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        upk2(mul2_rz(P[i], RL), lo[2 * i], lo[2 * i + 1]);
+        upk2(mul2_rz(P[i], RU), hi[2 * i], hi[2 * i + 1]);
+    }
+}
+
 MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, float s, float r_lo, float r_hi,
                                  uint32_t &out0, uint32_t &out1) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float lo[16], hi[16];
+    uint64_t P[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float a = bf16lo(w[i]), b = bf16hi(w[i]);
-        lo[2 * i] = __fmul_rz(a, r_lo);
-        lo[2 * i + 1] = __fmul_rz(b, r_lo);
-        hi[2 * i] = __fmul_ru(fabsf(a), r_hi);
-        hi[2 * i + 1] = __fmul_ru(fabsf(b), r_hi);
-    }
+    for (int i = 0; i < 8; ++i) P[i] = pk2(bf16lo(w[i]), bf16hi(w[i]));
+    float lo[16], hi[16];
+    bracket16(P, r_lo, r_hi, lo, hi);
     const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
     const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
     const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
     const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
     uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
-    const uint32_t d0 = (c0 & 0x77777777u) ^ cvt8_e2m1(hi0), d1 = (c1 & 0x77777777u) ^ cvt8_e2m1(hi1);
+    const uint32_t d0 = (c0 ^ cvt8_e2m1(hi0)) & 0x77777777u, d1 = (c1 ^ cvt8_e2m1(hi1)) & 0x77777777u;
     if ((d0 | d1) != 0u) {
         c0 = nv_settle(c0, d0, w[0], w[1], w[2], w[3], g, s);
         c1 = nv_settle(c1, d1, w[4], w[5], w[6], w[7], g, s);
@@ -296,18 +340,17 @@ MX_DEVICE_INLINE uint32_t nv_settle_f32(uint32_t code, uint32_t diff, const floa
 
 MX_DEVICE_INLINE void nv_codes16_f32(const float (&x)[16], float g, float s, float r_lo, float r_hi,
                                      uint32_t &out0, uint32_t &out1) {
-    float lo[16], hi[16];
+    uint64_t P[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        lo[i] = __fmul_rz(x[i], r_lo);
-        hi[i] = __fmul_ru(fabsf(x[i]), r_hi);
-    }
+    for (int i = 0; i < 8; ++i) P[i] = pk2(x[2 * i], x[2 * i + 1]);
+    float lo[16], hi[16];
+    bracket16(P, r_lo, r_hi, lo, hi);
     const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
     const float(&lo1)[8] = *reinterpret_cast<const float(*)[8]>(&lo[8]);
     const float(&hi0)[8] = *reinterpret_cast<const float(*)[8]>(&hi[0]);
     const float(&hi1)[8] = *reinterpret_cast<const float(*)[8]>(&hi[8]);
     uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
-    const uint32_t d0 = (c0 & 0x77777777u) ^ cvt8_e2m1(hi0), d1 = (c1 & 0x77777777u) ^ cvt8_e2m1(hi1);
+    const uint32_t d0 = (c0 ^ cvt8_e2m1(hi0)) & 0x77777777u, d1 = (c1 ^ cvt8_e2m1(hi1)) & 0x77777777u;
     if ((d0 | d1) != 0u) {
         c0 = nv_settle_f32(c0, d0, &x[0], g, s);
         c1 = nv_settle_f32(c1, d1, &x[8], g, s);

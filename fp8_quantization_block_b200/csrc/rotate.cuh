@@ -23,35 +23,6 @@ namespace mx {
 
 constexpr uint32_t kRhtScaleBits = 0x3E3504F3u;  // RN_fp32(1 / sqrt(32))
 
-// Packed fp32 pairs (f32x2 arithmetic of sm_100: two IEEE operations per
-// instruction, each rounded to nearest-even exactly as its scalar form).
-MX_DEVICE_INLINE uint64_t pk2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-MX_DEVICE_INLINE void upk2(uint64_t r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
-MX_DEVICE_INLINE uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t sub2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
 // The unnormalised butterflies H32 x of the 32-element block whose half (16
 // values) this thread holds: lower = even lane (block elements 0..15), upper =
 // odd lane.  Stages of half-width 1, 2, 4 run on the pairs (x[j], x[j + 8]),
