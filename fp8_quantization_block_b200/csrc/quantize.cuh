@@ -388,16 +388,18 @@ constexpr int kQTileCols = 128;
 constexpr int kQThreads = 256;
 
 // Largest bf16 magnitude (as its bit pattern) among the 16 values of v0, v1.
+// Per half: a value whose magnitude is max(|a|, |b|) (its sign is the XOR of
+// the inputs' signs, which the caller masks off once at the end).
+MX_DEVICE_INLINE uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 MX_DEVICE_INLINE uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    __nv_bfloat162 m[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t a = w[2 * i] & 0x7FFF7FFFu, b = w[2 * i + 1] & 0x7FFF7FFFu;
-        m[i] = __hmax2(*reinterpret_cast<const __nv_bfloat162 *>(&a), *reinterpret_cast<const __nv_bfloat162 *>(&b));
-    }
-    const __nv_bfloat162 r = __hmax2(__hmax2(m[0], m[1]), __hmax2(m[2], m[3]));
-    const uint32_t rb = *reinterpret_cast<const uint32_t *>(&r);
+    const uint32_t r = bf16x2_maxabs(bf16x2_maxabs(bf16x2_maxabs(v0.x, v0.y), bf16x2_maxabs(v0.z, v0.w)),
+                                     bf16x2_maxabs(bf16x2_maxabs(v1.x, v1.y), bf16x2_maxabs(v1.z, v1.w)));
+    const uint32_t rb = r & 0x7FFF7FFFu;
     return max(rb & 0xFFFFu, rb >> 16);
 }
 
