@@ -95,8 +95,13 @@ MX_DEVICE_INLINE float e4m3_pos_value(uint32_t c) {
 MX_DEVICE_INLINE bool nv_scale_ok(float s, float g, float amax) { return __fmaf_rn(6.0f * s, g, -amax) >= 0.0f; }
 
 // NVFP4 block scale: smallest positive finite E4M3 s with amax <= 6 g s,
-// 0 for an all-zero block, 0x7E (448) if none suffices.  inv6g ~ 1/(6g) only
-// seeds the search; the exact comparisons decide.
+// 0 for an all-zero block, 0x7E (448) if none suffices.  t = amax * inv6g is
+// within a few ulps of the exact quotient q = amax / (6 g), far less than the
+// E4M3 spacing (2^-3 relative, or 2^-9 below 2^-6), so its nearest E4M3 code
+// is either the answer c* (the smallest value >= q) or the code just below:
+// one exact test of 6 g s >= amax decides.  (For g below ~2^-102, where
+// 1/(6g) is no longer that accurate or overflows, the estimate only seeds an
+// exact walk up and down the codes.)
 MX_DEVICE_INLINE uint32_t nv_block_scale(float amax, float g, float inv6g, const float *val) {
     if (!(amax > 0.0f)) return 0u;
     const float approx = amax * inv6g;
@@ -105,11 +110,14 @@ MX_DEVICE_INLINE uint32_t nv_block_scale(float amax, float g, float inv6g, const
         : "=r"(c)
         : "f"(approx));
     c &= 0x7Fu;
-    if (c == 0x7Fu) c = 0x7Eu;  // NaN (g not positive): saturate
-    if (c == 0u) c = 1u;
-    // At most a step or two from the answer; the loops are bounded by the code range.
-    while (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ++c;
-    while (c > 1u && nv_scale_ok(val[c - 1u], g, amax)) --c;
+    c = c == 0x7Fu ? 0x7Eu : (c == 0u ? 1u : c);   // NaN (g not positive) saturates; 0 -> the smallest
+    if (inv6g <= 0x1p100f) {
+        if (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ++c;
+    } else {
+        // bounded by the code range
+        while (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ++c;
+        while (c > 1u && nv_scale_ok(val[c - 1u], g, amax)) --c;
+    }
     return c;
 }
 
@@ -265,13 +273,13 @@ MX_DEVICE_INLINE float e2m1_mid(uint32_t c) {
 // midpoint.  diff has a nonzero nibble where lo's and hi's magnitudes differ;
 // w0..w3 hold the word's 8 bf16 inputs (element 2j in the low half of wj).
 MX_DEVICE_INLINE uint32_t nv_settle(uint32_t code, uint32_t diff, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
-                                    float g, float s) {
+                                    float g, float s, float sc) {
     while (diff != 0u) {
         const int nib = (__ffs(diff) - 1) >> 2;
         diff &= ~(0xFu << (4 * nib));
         const int j = nib >> 1;
         const uint32_t wj = j == 0 ? w0 : (j == 1 ? w1 : (j == 2 ? w2 : w3));
-        const float ax = fabsf((nib & 1) ? __uint_as_float(wj & 0xFFFF0000u) : __uint_as_float(wj << 16));
+        const float ax = fabsf((nib & 1) ? __uint_as_float(wj & 0xFFFF0000u) : __uint_as_float(wj << 16)) * sc;
         const uint32_t c = (code >> (4 * nib)) & 7u;                  // lo's magnitude, < hi's <= 7
         const float d = __fmaf_rn(-g, s * e2m1_mid(c), ax);           // sign(|x| - g*s*mid)
         if (d > 0.0f || (d == 0.0f && (c & 1u))) code += 1u << (4 * nib);
@@ -290,12 +298,19 @@ MX_DEVICE_INLINE void bracket16(const uint64_t (&P)[8], float r_lo, float r_hi, 
     }
 }
 
+// sc: a power of two the values are multiplied by (exactly) before the
+// division, 1 unless g is so small that 1/g would overflow (see the kernel).
 MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, float s, float r_lo, float r_hi,
-                                 uint32_t &out0, uint32_t &out1) {
+                                 uint32_t &out0, uint32_t &out1, float sc) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     uint64_t P[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) P[i] = pk2(bf16lo(w[i]), bf16hi(w[i]));
+    if (sc != 1.0f) {
+        const uint64_t SC = pk2(sc, sc);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) P[i] = mul2(P[i], SC);
+    }
     float lo[16], hi[16];
     bracket16(P, r_lo, r_hi, lo, hi);
     const float(&lo0)[8] = *reinterpret_cast<const float(*)[8]>(&lo[0]);
@@ -305,8 +320,8 @@ MX_DEVICE_INLINE void nv_codes16(const uint4 &v0, const uint4 &v1, float g, floa
     uint32_t c0 = cvt8_e2m1(lo0), c1 = cvt8_e2m1(lo1);
     const uint32_t d0 = (c0 ^ cvt8_e2m1(hi0)) & 0x77777777u, d1 = (c1 ^ cvt8_e2m1(hi1)) & 0x77777777u;
     if ((d0 | d1) != 0u) {
-        c0 = nv_settle(c0, d0, w[0], w[1], w[2], w[3], g, s);
-        c1 = nv_settle(c1, d1, w[4], w[5], w[6], w[7], g, s);
+        c0 = nv_settle(c0, d0, w[0], w[1], w[2], w[3], g, s, sc);
+        c1 = nv_settle(c1, d1, w[4], w[5], w[6], w[7], g, s, sc);
     }
     out0 = c0;
     out1 = c1;
@@ -427,7 +442,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
     const bool col_ok = col < K;                    // K % 16 == 0: all 16 or none
     const int jb = cl / T::kBlock;                  // block index inside the tile row
 
-    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f;
+    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f, sc = 1.0f;
     __shared__ NvTables nvt;
     // src and g may come from the previous kernel in the stream
     griddep_wait();
@@ -435,6 +450,12 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
         g = *gscale_in;
         if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;   // g = RU(amax / (6 * 448))
         if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
+        // Below 2^-100, 1/g loses accuracy or overflows: divide x * 2^64 by
+        // g * 2^64 instead (both exact; every quotient is unchanged).
+        if (g < 0x1p-100f) {
+            sc = 0x1p64f;
+            g *= sc;
+        }
         rg_lo = __frcp_rd(g);
         rg_hi = __frcp_ru(g);
         inv6g = 1.0f / (6.0f * g);
@@ -471,7 +492,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
         if (T::kBlock == 32) m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         uint32_t sbyte;
         if (FMT == FMT_NVFP4) {
-            sbyte = nv_block_scale(__uint_as_float(m << 16), g, inv6g, nvt.val);
+            sbyte = nv_block_scale(__uint_as_float(m << 16) * sc, g, inv6g, nvt.val);
             if (ok) {
                 uint32_t q0 = 0, q1 = 0;
                 if (sbyte == 0u) {
@@ -488,7 +509,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
                     // r_lo <= 1/(g s) <= r_hi: products of one-sided bounds, rounded outward
                     const float r_lo = __fmul_rd(rg_lo, nvt.inv_lo[sbyte]);
                     const float r_hi = __fmul_ru(rg_hi, nvt.inv_hi[sbyte]);
-                    nv_codes16(v[i][0], v[i][1], g, nvt.val[sbyte], r_lo, r_hi, q0, q1);
+                    nv_codes16(v[i][0], v[i][1], g, nvt.val[sbyte], r_lo, r_hi, q0, q1, sc);
                 }
                 *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
             }

@@ -122,13 +122,18 @@ __global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t 
     const bool col_ok = col < K;   // K % 32 == 0: both halves of a block exist or neither
     const int jb = cl / T::kBlock;
 
-    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f;
+    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f, sc = 1.0f;
     __shared__ NvTables nvt;
     griddep_wait();
     if (FMT == FMT_NVFP4) {
         g = *gscale_in;
         if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;
         if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
+        // as in quantize_kernel: a tiny g is handled as (y 2^64) / (g 2^64)
+        if (g < 0x1p-100f) {
+            sc = 0x1p64f;
+            g *= sc;
+        }
         rg_lo = __frcp_rd(g);
         rg_hi = __frcp_ru(g);
         inv6g = 1.0f / (6.0f * g);
@@ -174,7 +179,11 @@ __global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t 
         uint32_t sbyte;
         if (FMT == FMT_NVFP4) {
             rht32_scale(y);
-            sbyte = nv_block_scale(m, g, inv6g, nvt.val);
+            if (sc != 1.0f) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) y[e] *= sc;   // exact: a power of two, scaling up
+            }
+            sbyte = nv_block_scale(m * sc, g, inv6g, nvt.val);
             if (ok) {
                 uint32_t q0 = 0, q1 = 0;
                 if (sbyte == 0u) {

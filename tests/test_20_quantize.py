@@ -47,6 +47,23 @@ def test_nvfp4_given_gscale(g):
     assert float(q.gscale.cpu()[0]) == g32
 
 
+@pytest.mark.parametrize("scale_exp", [-118, -125, 100])
+def test_nvfp4_extreme_global_scales(scale_exp):
+    # a whole tensor near the bottom of the bf16 range (g subnormal: the block
+    # scale search walks the codes exactly) or near the top, g computed
+    x = synth.bits_to_tensor(synth.student_t(14, 64, 512)).float().numpy() * np.float32(2.0 ** scale_exp)
+    bits = synth.to_bf16_bits(x)
+    assert_quant_equal(quantize_dev(bits, 3), bits, 3)
+
+
+@pytest.mark.parametrize("g", [1e-39, 3e-36])
+def test_nvfp4_given_tiny_gscale(g):
+    # subnormal and tiny given g on ordinary data: most blocks saturate at s = 448
+    bits = synth.student_t(15, 32, 256)
+    g32 = float(np.float32(g))
+    assert_quant_equal(quantize_dev(bits, 3, gscale=g32), bits, 3, gscale=g32)
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_row_pitch_larger_than_k(fmt):
     bits = synth.sweep_tensor(31, 70, 640)

@@ -67,6 +67,14 @@ def test_rht_nvfp4_given_gscale(g):
     assert_rht_equal(rht_dev(bits, 3, gscale=g32), bits, 3, gscale=g32)
 
 
+@pytest.mark.parametrize("scale_exp", [-122, 100])
+def test_rht_nvfp4_extreme_global_scales(scale_exp):
+    # the rotated tensor near the bottom of the range (g subnormal) or near the top
+    x = synth.bits_to_tensor(synth.student_t(56, 64, 512)).float().numpy() * np.float32(2.0 ** scale_exp)
+    bits = synth.to_bf16_bits(x)
+    assert_rht_equal(rht_dev(bits, 3), bits, 3)
+
+
 def test_rht_row_pitch_larger_than_k():
     bits = synth.sweep_tensor(52, 70, 640)
     padded = torch.zeros((70, 704), dtype=torch.bfloat16, device="cuda")
