@@ -199,12 +199,8 @@ int num_sms() {
 // amax(|src|) -> slot (float bits), then g = RU(amax / 2688) in place.
 mx_status nvfp4_gscale_prepass(const uint16_t *src, int64_t M, int64_t K, int64_t ld, float *slot, cudaStream_t st) {
     if (cudaMemsetAsync(slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
-    const int64_t vecs = M * (K / 8);
-    int64_t blocks = cdiv(vecs, 256 * 8);
-    const int64_t cap = (int64_t)num_sms() * 8;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    amax_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, M, K, ld, reinterpret_cast<unsigned int *>(slot));
+    amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(src, M, K, ld,
+                                                                           reinterpret_cast<unsigned int *>(slot));
     gscale_from_amax_kernel<<<1, 1, 0, st>>>(slot);
     return last_launch();
 }
@@ -446,12 +442,8 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
             const float *amax = x_amax;
             if (amax == nullptr) {
                 if (cudaMemsetAsync(amax_slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
-                const int64_t vecs = M * (K / 8);
-                int64_t blocks = cdiv(vecs, 256 * 8);
-                const int64_t cap = (int64_t)num_sms() * 8;
-                if (blocks > cap) blocks = cap;
-                if (blocks < 1) blocks = 1;
-                amax_kernel<<<(unsigned)blocks, 256, 0, st>>>(X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
+                amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(
+                    X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
                 amax = amax_slot;
             }
             launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1);

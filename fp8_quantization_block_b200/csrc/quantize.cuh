@@ -698,28 +698,52 @@ __global__ void __launch_bounds__(kQThreads) quantize_mbs_kernel(const uint16_t 
 }
 
 // max |x| over a bf16 tensor -> atomicMax on the float bits of *amax (init 0).
-__global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
-                                                   int64_t ld, unsigned int *__restrict__ amax_bits) {
+// Persistent: CTA b walks the 128 x 128 tiles n-1-b, n-1-b-G, ... (G CTAs), a
+// thread issuing its 8 16-byte loads of a tile (4 rows x 16 columns, as in
+// quantize_kernel) before reducing them.  Walking the tiles from the end of the
+// tensor towards its start leaves the first rows in L2 when the pass ends, and
+// the quantize kernel that follows reads those rows first.
+__global__ void __launch_bounds__(kQThreads) amax_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
+                                                         int64_t ld, unsigned int *__restrict__ amax_bits) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t tiles_x = (K + kQTileCols - 1) / kQTileCols;
+    const int64_t n_tiles = tiles_x * ((M + kQTileRows - 1) / kQTileRows);
+    const int cl = (lane & 7) * 16;
     uint32_t m = 0;
-    const int64_t vec_per_row = K / 8;
-    const int64_t total = M * vec_per_row;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
-        const uint4 v = ldg_stream(src + r * ld + c);
-        m = bf16x2_absmax(m, v.x);
-        m = bf16x2_absmax(m, v.y);
-        m = bf16x2_absmax(m, v.z);
-        m = bf16x2_absmax(m, v.w);
+    for (int64_t t = n_tiles - 1 - (int64_t)blockIdx.x; t >= 0; t -= gridDim.x) {
+        const int64_t row0 = (t / tiles_x) * kQTileRows, col = (t % tiles_x) * kQTileCols + cl;
+        uint4 v[4][2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t row = row0 + i * 32 + warp * 4 + (lane >> 3);
+            if (row < M && col < K) {
+                const uint16_t *p = src + row * ld + col;
+                v[i][0] = ldg_stream(p);
+                v[i][1] = ldg_stream(p + 8);
+            } else {
+                v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, absmax16(v[i][0], v[i][1]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __shared__ uint32_t red[8];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __shared__ uint32_t red[kQThreads / 32];
+    if (lane == 0) red[warp] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x / 32); ++w) m = max(m, red[w]);
+        for (int w = 1; w < kQThreads / 32; ++w) m = max(m, red[w]);
         if (m != 0u) atomicMax(amax_bits, m << 16);   // bf16 magnitude -> fp32 bits (order-preserving)
     }
+}
+
+// CTAs for amax_kernel: enough resident per SM to keep HBM busy, never more
+// than there are tiles.
+inline int64_t amax_grid(int64_t M, int64_t K, int num_sms) {
+    const int64_t tiles = ((K + kQTileCols - 1) / kQTileCols) * ((M + kQTileRows - 1) / kQTileRows);
+    const int64_t cap = (int64_t)num_sms * 4;
+    return tiles < 1 ? 1 : (tiles < cap ? tiles : cap);
 }
 
 // g = RU_fp32(amax / 2688), 1 for an all-zero tensor; in place (amax bits -> g).
