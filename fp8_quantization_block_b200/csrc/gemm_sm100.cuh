@@ -114,11 +114,19 @@ struct GemmParams {
 
 // Shared-memory and TMEM plan of a CTA whose MMAs read a 128-row A tile and
 // B_BANDS 128-row bands of B per stage (B_ROWS rows of B in this CTA's smem).
-template <int FMT, int B_BANDS, int B_ROWS, int STAGES>
+// A_ROWS < 128 (matrices with at most A_ROWS rows, e.g. decode-time
+// activations): only A_ROWS rows of A are loaded per stage, and the smem they
+// leave free holds more stages of B.  The M = 128 MMA still reads 128 rows
+// from the stage's base; the rows past A_ROWS are whatever the following
+// shared memory holds and only produce accumulator rows >= M, which the
+// epilogue neither stores nor counts.
+template <int FMT, int B_BANDS, int B_ROWS, int STAGES, int A_ROWS = kBM>
 struct GemmLayout {
     using F = GemmFmt<FMT>;
+    static_assert(A_ROWS % 8 == 0 && A_ROWS <= kBM, "A rows: whole 8-row swizzle atoms");
     static constexpr int kBBands = B_BANDS;
-    static constexpr int kABytes = kBM * kStageKBytes;
+    static constexpr int kARows = A_ROWS;
+    static constexpr int kABytes = A_ROWS * kStageKBytes;
     static constexpr int kBBytes = B_ROWS * kStageKBytes;
     // scale tiles of one group: kSfGroup stages x kChunks 512-byte tiles of A's
     // band, and the same for each of B's bands (band-major)
@@ -151,6 +159,8 @@ struct GemmLayout {
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
     static_assert(kAlloc <= kSmemLimit, "shared memory budget");
+    // the last stage's 128-row A read stays inside the allocation
+    static_assert(kOffA + (STAGES - 1) * kABytes + kBM * kStageKBytes <= kBytes, "A tile read past the smem plan");
     // TMEM: two accumulators at columns 0 and kAccStride (sharing BN - kAccStride
     // columns), then kSlots scale slots of kSfSlotCols columns each.
     static constexpr int kAccCols = 128 * B_BANDS;  // accumulator columns = N of the MMA
@@ -164,8 +174,8 @@ struct GemmLayout {
     static_assert(STAGES >= kSlots, "scale slots are recycled through the stage barriers");
 };
 
-template <int FMT, int BN, int STAGES>
-using GemmSmem = GemmLayout<FMT, BN / 128, BN, STAGES>;
+template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
+using GemmSmem = GemmLayout<FMT, BN / 128, BN, STAGES, A_ROWS>;
 
 // Instruction descriptor of the block-scaled MMA (M = 128, K-major A and B).
 template <int FMT, int BN>
@@ -572,13 +582,13 @@ MX_DEVICE_INLINE void epilogue_finish(const GemmParams &p, int lane, uint32_t am
     }
 }
 
-template <int FMT, int BN, int STAGES>
+template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSfa,
                 const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
-    using L = GemmSmem<FMT, BN, STAGES>;
+    using L = GemmSmem<FMT, BN, STAGES, A_ROWS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);

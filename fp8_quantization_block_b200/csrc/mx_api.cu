@@ -248,20 +248,20 @@ bool make_tmap_sf(CUtensorMap *m, const uint8_t *scales, int64_t bands, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int BN, int STAGES>
+template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                         const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
-    using L = GemmSmem<FMT, BN, STAGES>;
+    using L = GemmSmem<FMT, BN, STAGES, A_ROWS>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K / GemmFmt<FMT>::kElemPerByte;   // shared-memory bytes of a row's K
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     CUtensorMap ta, tb, tc, tsa, tsb;
     if (FMT == kGemmRuntimeTypes) {
-        if (!make_tmap_codes_f8f6f4(&ta, A->fmt, a_codes, M, K, kBM)) return MX_ERR_CUDA;
+        if (!make_tmap_codes_f8f6f4(&ta, A->fmt, a_codes, M, K, A_ROWS)) return MX_ERR_CUDA;
         if (!make_tmap_codes_f8f6f4(&tb, B->fmt, B->codes, N, K, BN)) return MX_ERR_CUDA;
     } else {
-        if (!make_tmap_u8(&ta, a_codes, M, kbytes, kBM)) return MX_ERR_CUDA;
+        if (!make_tmap_u8(&ta, a_codes, M, kbytes, A_ROWS)) return MX_ERR_CUDA;
         if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN)) return MX_ERR_CUDA;
     }
     if (!make_tmap_sf(&tsa, a_scales, cdiv(M, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 1)) return MX_ERR_CUDA;
@@ -273,8 +273,8 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_kernel<FMT, BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        L::kAlloc);
+        attr_err = cudaFuncSetAttribute(gemm_kernel<FMT, BN, STAGES, A_ROWS>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     });
     if (attr_err != cudaSuccess) return MX_ERR_CUDA;
     GemmParams p;
@@ -294,7 +294,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.use_tma_store = tma_store ? 1 : 0;
     p.skip_producer = g_skip_producer.load();
     p.ab_types = (f8f6f4_type(A->fmt) << 7) | (f8f6f4_type(B->fmt) << 10);
-    p.stage_tx = (uint32_t)(kStageKBytes * (kBM * fmt_bits(A->fmt) + BN * fmt_bits(B->fmt)) / 8);
+    p.stage_tx = (uint32_t)(kStageKBytes * (A_ROWS * fmt_bits(A->fmt) + BN * fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
@@ -307,7 +307,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     cudaLaunchAttribute attr[1];
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, BN, STAGES>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, BN, STAGES, A_ROWS>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
         return last_launch();
     return last_launch();
 }
@@ -390,6 +390,9 @@ mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_
     if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load())
         return launch_gemm_pair_t<FMT, (FMT == 2 || FMT == 3) ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    // at most 32 rows of A (decode-like activations): the weight stream gets a
+    // fifth stage from the shared memory a 128-row A tile would take
+    if (A->rows <= 32) return launch_gemm_t<FMT, 256, 5, 32>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
     return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
 }
 

@@ -422,8 +422,17 @@ MX_DEVICE_INLINE uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
 // ceil((K / block) / 4) 512-byte tiles per 128-row band.  NVFP4: *gscale_in
 // is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
 // if gscale_out != nullptr, CTA 0 also stores g there.
+// CTAs per SM that the register allocation of quantize_kernel<FMT> targets,
+// chosen by timing 2^28-element inputs: the FP8 and FP4 MX casts run fastest
+// with the registers left free (1), NVFP4 with four resident CTAs (the
+// bracket's working set), MXFP6 with five.
+template <int FMT>
+constexpr int quantize_min_blocks() {
+    return FMT == FMT_NVFP4 ? 4 : (FMT == FMT_MXFP6 ? 5 : 1);
+}
+
 template <int FMT, int RULE = RULE_OCP>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
+__global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantize_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
                                                              int64_t ld, uint8_t *__restrict__ codes,
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
                                                              const float *__restrict__ gscale_in,
@@ -494,23 +503,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const uint16_t *__r
         if (FMT == FMT_NVFP4) {
             sbyte = nv_block_scale(__uint_as_float(m << 16) * sc, g, inv6g, nvt.val);
             if (ok) {
-                uint32_t q0 = 0, q1 = 0;
-                if (sbyte == 0u) {
-                    // all-zero block: codes are the signs of the zeros
-                    const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w,
-                                           v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint32_t sgn = (w[e >> 1] >> (16 * (e & 1) + 15)) & 1u;
-                        if (e < 8) q0 |= sgn << (4 * e + 3);
-                        else q1 |= sgn << (4 * (e - 8) + 3);
-                    }
-                } else {
-                    // r_lo <= 1/(g s) <= r_hi: products of one-sided bounds, rounded outward
-                    const float r_lo = __fmul_rd(rg_lo, nvt.inv_lo[sbyte]);
-                    const float r_hi = __fmul_ru(rg_hi, nvt.inv_hi[sbyte]);
-                    nv_codes16(v[i][0], v[i][1], g, nvt.val[sbyte], r_lo, r_hi, q0, q1, sc);
-                }
+                uint32_t q0, q1;
+                // r_lo <= 1/(g s) <= r_hi: products of one-sided bounds, rounded outward.
+                // An all-zero block has s = 0 and both bounds 0, so its products are
+                // the zeros themselves and its codes their signs (0x0 / 0x8).
+                const float r_lo = __fmul_rd(rg_lo, nvt.inv_lo[sbyte]);
+                const float r_hi = __fmul_ru(rg_hi, nvt.inv_hi[sbyte]);
+                nv_codes16(v[i][0], v[i][1], g, nvt.val[sbyte], r_lo, r_hi, q0, q1, sc);
                 *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
             }
         } else {

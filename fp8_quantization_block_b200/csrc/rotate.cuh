@@ -103,7 +103,8 @@ MX_DEVICE_INLINE int mx_scale_byte_f32(float amax) {
 // laid out as quantize_kernel's.  NVFP4: *gscale_in is g, or max|y| when
 // g_from_amax (then g = RU(max|y| / 2688), 1 for 0); gscale_out as there.
 template <int FMT>
-__global__ void __launch_bounds__(kQThreads) quantize_rht_kernel(const uint16_t *__restrict__ src, int64_t M,
+// (four resident CTAs per SM for the register allocation: measured fastest)
+__global__ void __launch_bounds__(kQThreads, 4) quantize_rht_kernel(const uint16_t *__restrict__ src, int64_t M,
                                                                  int64_t K, int64_t ld, uint8_t *__restrict__ codes,
                                                                  uint8_t *__restrict__ scales, int64_t sf_tiles_k,
                                                                  const float *__restrict__ gscale_in,

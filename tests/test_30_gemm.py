@@ -101,6 +101,26 @@ def test_ragged_shapes(fmt, M, N, K):
     assert ok, worst
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,N,K", [(1, 300, 640), (17, 520, 384), (32, 257, 1152)])
+def test_small_m_kernel(fmt, M, N, K):
+    """At most 32 rows of A and more than 128 of B: the kernel loads 32-row A
+    tiles and keeps a fifth stage of B.  The tensor core's rows past 32 read
+    other shared memory; those accumulator rows must never reach C (ragged N,
+    a K tail inside a stage, M = 1 and M = 32)."""
+    A_bits = synth.sweep_tensor(5000 + M, M, K)
+    B_bits = synth.gaussian_weights(6000 + N, N, K)
+    qa, qb, Ad, Bd = quantized_pair(fmt, A_bits, B_bits)
+    big = torch.full((M + 3, N + 8), 5.0, dtype=torch.bfloat16, device="cuda")
+    C = big[:M, :N]
+    mx.gemm(qa, qb, out=C)
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    ok, worst = gemm_check(C, Ad, Bd)
+    assert ok, worst
+    assert torch.all(big[M:] == 5.0) and torch.all(big[:, N:] == 5.0)
+
+
 def test_output_row_pitch():
     fmt = 0
     A_bits, B_bits = synth.tiny_pair()

@@ -81,7 +81,7 @@ def test_mxfp6_qsnr_sums_and_ordering():
     assert s8[1] < got[1] < s4[1]
 
 
-GEMM_SHAPES = [(256, 384, 1024), (100, 96, 512), (128, 300, 256), (300, 520, 384)]
+GEMM_SHAPES = [(256, 384, 1024), (100, 96, 512), (128, 300, 256), (300, 520, 384), (24, 288, 640)]
 
 
 def _dq(bits, fmt):
@@ -104,7 +104,7 @@ MIXED = [(0, 2), (0, 4), (4, 2), (2, 0), (4, 0), (1, 0), (1, 4), (2, 4)]
 
 
 @pytest.mark.parametrize("fa,fb", MIXED)
-@pytest.mark.parametrize("M,N,K", [(256, 384, 1024), (100, 96, 512), (300, 520, 384)])
+@pytest.mark.parametrize("M,N,K", [(256, 384, 1024), (100, 96, 512), (300, 520, 384), (9, 272, 512)])
 def test_gemm_mixed_operands(fa, fb, M, N, K):
     xa = synth.dit_activations(97, M, K)
     wb = synth.gaussian_weights(98, N, K)
