@@ -141,8 +141,9 @@ bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) ==
 
 // --- quantize ------------------------------------------------------------
 template <int FMT, int RULE = RULE_OCP>
-void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
-                     const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
+mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
+                          const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
+    if (M == 0 || K == 0) return MX_OK;
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
@@ -152,8 +153,10 @@ void launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, cons
     cudaLaunchAttribute attr[1];
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
-    cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales,
-                       sf_tiles_k, g_in, g_out, g_from_amax);
+    if (cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes),
+                           dst->scales, sf_tiles_k, g_in, g_out, g_from_amax) != cudaSuccess)
+        return last_launch();
+    return MX_OK;
 }
 
 template <int FMT>
@@ -432,14 +435,15 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
     xa->scales = ws + kFusedWsHeader + align256((size_t)(M * K * fmt_bits(fmt) / 8));
     xa->gscale = g_slot;
     *ga = nullptr;
+    mx_status s = MX_OK;
     switch (fmt) {
-    case MX_MXFP8_E4M3: launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
-    case MX_MXFP8_E5M2: launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
-    case MX_MXFP4: launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
-    case MX_MXFP6_E3M2: launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP8_E4M3: s = launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP8_E5M2: s = launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP4: s = launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP6_E3M2: s = launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
     default:
         if (x_gscale != nullptr) {
-            launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st);
+            s = launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st);
             *ga = x_gscale;
         } else {
             const float *amax = x_amax;
@@ -449,10 +453,11 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
                     X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
                 amax = amax_slot;
             }
-            launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1);
+            s = launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1);
             *ga = g_slot;
         }
     }
+    if (s != MX_OK) return s;
     return last_launch();
 }
 
@@ -510,23 +515,25 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
     if (cdiv(M, kQTileRows) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *src = static_cast<const uint16_t *>(src_bf16);
+    mx_status s = MX_OK;
     switch (fmt) {
-    case MX_MXFP8_E4M3: launch_quantize<0>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
-    case MX_MXFP8_E5M2: launch_quantize<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
-    case MX_MXFP4: launch_quantize<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
-    case MX_MXFP6_E3M2: launch_quantize<4>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP8_E4M3: s = launch_quantize<0>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP8_E5M2: s = launch_quantize<1>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP4: s = launch_quantize<2>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
+    case MX_MXFP6_E3M2: s = launch_quantize<4>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP4_MBS: launch_quantize_mbs(src, M, K, ld_src, dst, st); break;
     default: {
         if (gscale_in == nullptr) {
-            mx_status s = nvfp4_gscale_prepass(src, M, K, ld_src, dst->gscale, st);
+            s = nvfp4_gscale_prepass(src, M, K, ld_src, dst->gscale, st);
             if (s != MX_OK) return s;
-            launch_quantize<3>(src, M, K, ld_src, dst, dst->gscale, nullptr, st);
+            s = launch_quantize<3>(src, M, K, ld_src, dst, dst->gscale, nullptr, st);
         } else {
-            launch_quantize<3>(src, M, K, ld_src, dst, gscale_in, gscale_in == dst->gscale ? nullptr : dst->gscale,
-                               st);
+            s = launch_quantize<3>(src, M, K, ld_src, dst, gscale_in, gscale_in == dst->gscale ? nullptr : dst->gscale,
+                                   st);
         }
     }
     }
+    if (s != MX_OK) return s;
     return last_launch();
 }
 
@@ -539,8 +546,9 @@ mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld
     if (ld_src < K || (ld_src & 7) != 0) return MX_ERR_MISALIGNED;
     if (!aligned16(src_bf16) || !aligned16(dst->codes) || !aligned16(dst->scales)) return MX_ERR_MISALIGNED;
     if (cdiv(M, kQTileRows) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
-    launch_quantize<2, RULE_OAS>(static_cast<const uint16_t *>(src_bf16), M, K, ld_src, dst, nullptr, nullptr,
-                                 static_cast<cudaStream_t>(stream));
+    const mx_status s = launch_quantize<2, RULE_OAS>(static_cast<const uint16_t *>(src_bf16), M, K, ld_src, dst,
+                                                     nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    if (s != MX_OK) return s;
     return last_launch();
 }
 
