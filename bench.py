@@ -409,7 +409,8 @@ def quant_bytes_per_elem(fmt):
 
 def extras_gpu(device):
     """Short measurements of the other hot-path rows (quantize sweep, NVFP4
-    MLP GEMM, skinny weight-stream GEMM), each on rotating buffers > L2."""
+    MLP GEMM, skinny weight-stream GEMM), each on rotating buffers > L2 and
+    timed as a CUDA-graph replay of 20 calls."""
     import torch
     from fp8_quantization_block_b200 import mx
 
@@ -417,15 +418,24 @@ def extras_gpu(device):
     out = {}
 
     def timed(fn, n, reps=20, warm=3):
+        """Device ms per call of fn(warm), ..., fn(warm + reps - 1), replayed
+        from a CUDA graph (so that small cases are not bound by the host's
+        per-call cost)."""
         for i in range(warm):
             fn(i)
         torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(reps):
+                fn(warm + i)
+        g.replay()
+        torch.cuda.synchronize()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        for i in range(reps):
-            fn(warm + i)
+        g.replay()
         e.record()
         torch.cuda.synchronize()
+        del g
         return s.elapsed_time(e) / reps
 
     g = torch.Generator(device=device).manual_seed(100)

@@ -224,6 +224,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
                               my_tiles, lane, abort_flag,
                               [&](int slot) { mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot); });
+        // then the upper half of the columns of this CTA's rows of the last tile
+        // (the pair's MMAs have completed, so the B stage ring is free for the
+        // staging buffers)
+        if (my_tiles > 0 && !*abort_flag) {
+            const int it = my_tiles - 1, b = it & 1;
+            const int tile = pair + it * npairs;
+            int m0, n0;
+            tile_coords(tile, p.m_blocks, m0, n0, 256);
+            m0 = (tile % p.m_blocks) * 256 + 128 * (int)rank;
+            if (mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) {
+                tc_fence_after();
+                float scale = 1.0f;
+                if (FMT == 3) scale = (*p.ga) * (*p.gb);
+                uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
+                uint32_t amax = 0, nstore = 0;
+                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
+                                                       m0 + 32 * q, n0, 4, 8, lane, bufs, nstore, amax, scale);
+                epilogue_finish(p, lane, amax);
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue (this CTA's 128 rows)
         const int q = warp & 3;
@@ -241,6 +261,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
+            if (tile + npairs >= num_tiles) {
+                // the last tile: the lower half of the columns (the scale warp of
+                // this quadrant drains the upper half); nothing waits for its release
+                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, 0, 4, lane, bufs, nstore, amax,
+                                                       scale);
+                break;
+            }
             epilogue_tile<256, L::kAccStride, L::kEpiBufs, FMT == 3>(
                 p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
                 [&] {

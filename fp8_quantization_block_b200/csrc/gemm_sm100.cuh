@@ -560,6 +560,33 @@ MX_DEVICE_INLINE void epilogue_tile_t(const GemmParams &p, const CUtensorMap *tm
     }
 }
 
+// Chunks [c_begin, c_end) of 32 columns of an accumulator in plain order (no
+// shared columns to release first): the last tile of a CTA, whose columns are
+// split between the epilogue warp and the scale warp of each TMEM lane
+// quadrant (the scale warps are idle once the tile's scales are in TMEM).
+template <int NBUF, bool SCALED, bool GELU>
+MX_DEVICE_INLINE void epilogue_chunks_t(const GemmParams &p, const CUtensorMap *tmC, uint32_t t_acc, int m0q, int n0,
+                                        int c_begin, int c_end, int lane, uint8_t *bufs, uint32_t &nstore,
+                                        uint32_t &amax, float scale) {
+    const int n_valid = p.N - n0;
+    for (int c = c_begin; c < c_end; ++c) {
+        const int col = 32 * c;
+        if (col >= n_valid) break;  // warp-uniform; columns ascend
+        uint32_t packed[16];
+        epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
+        epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+    }
+}
+template <int NBUF, bool SCALED>
+MX_DEVICE_INLINE void epilogue_chunks(const GemmParams &p, const CUtensorMap *tmC, uint32_t t_acc, int m0q, int n0,
+                                      int c_begin, int c_end, int lane, uint8_t *bufs, uint32_t &nstore,
+                                      uint32_t &amax, float scale) {
+    if (p.epilogue == 1)
+        epilogue_chunks_t<NBUF, SCALED, true>(p, tmC, t_acc, m0q, n0, c_begin, c_end, lane, bufs, nstore, amax, scale);
+    else
+        epilogue_chunks_t<NBUF, SCALED, false>(p, tmC, t_acc, m0q, n0, c_begin, c_end, lane, bufs, nstore, amax, scale);
+}
+
 template <int BN, int ACC_STRIDE, int NBUF, bool SCALED, typename Release>
 MX_DEVICE_INLINE void epilogue_tile(const GemmParams &p, const CUtensorMap *tmC, uint32_t t_acc, int b, int m0q,
                                     int n0, int lane, uint8_t *bufs, uint32_t &nstore, uint32_t &amax, float scale,
@@ -762,6 +789,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
         scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
                               my_tiles, lane, abort_flag, [&](int slot) { mbar_arrive(&sf_full[slot]); });
+        // then the upper half of the columns of this CTA's last tile (its MMAs have
+        // completed, so the B stage ring is free for the staging buffers)
+        if (my_tiles > 0 && !*abort_flag) {
+            const int it = my_tiles - 1, b = it & 1;
+            int m0, n0;
+            tile_coords(blockIdx.x + it * gridDim.x, p.m_blocks, m0, n0, BN);
+            if (mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) {
+                tc_fence_after();
+                float scale = 1.0f;
+                if (FMT == 3) scale = (*p.ga) * (*p.gb);
+                uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
+                uint32_t amax = 0, nstore = 0;
+                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
+                                                       m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs, nstore, amax, scale);
+                epilogue_finish(p, lane, amax);
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
@@ -777,6 +821,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
+            if (tile + (int)gridDim.x >= num_tiles) {
+                // the last tile: the lower half of the columns (the scale warp of
+                // this quadrant drains the upper half); nothing waits for its release
+                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, 0, BN / 64, lane, bufs, nstore,
+                                                       amax, scale);
+                break;
+            }
             epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs,
                                                                      nstore, amax, scale, [&] {
                                                                          if (lane == 0) mbar_arrive(acc_empty);

@@ -455,6 +455,10 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
     __shared__ NvTables nvt;
     // src and g may come from the previous kernel in the stream
     griddep_wait();
+    // Every CTA of this grid has started once all have passed here, so the next
+    // kernel in the stream may take SMs as this grid's CTAs leave them (it still
+    // waits for this grid's completion before reading anything).
+    griddep_launch_dependents();
     if (FMT == FMT_NVFP4) {
         g = *gscale_in;
         if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;   // g = RU(amax / (6 * 448))
@@ -548,9 +552,6 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
             *reinterpret_cast<uint4 *>(scales + chunk0 * 512 + threadIdx.x * 16) = val;
         }
     }
-    // the next kernel in the stream may start its setup now (it still waits
-    // for this grid's completion before reading anything)
-    griddep_launch_dependents();
 }
 
 // ------------------------------------------------------------------ MXFP4 with macro-block scaling
