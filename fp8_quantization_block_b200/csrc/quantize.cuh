@@ -101,19 +101,21 @@ MX_DEVICE_INLINE bool nv_scale_ok(float s, float g, float amax) { return __fmaf_
 // is either the answer c* (the smallest value >= q) or the code just below:
 // one exact test of 6 g s >= amax decides.  (For g below ~2^-102, where
 // 1/(6g) is no longer that accurate or overflows, the estimate only seeds an
-// exact walk up and down the codes.)
+// exact walk up and down the codes.)  The common path has no branch: the
+// clamp, the correction and the all-zero case are selects (3-4% of the NVFP4
+// quantize's time against early returns and compare-and-set).
 MX_DEVICE_INLINE uint32_t nv_block_scale(float amax, float g, float inv6g, const float *val) {
-    if (!(amax > 0.0f)) return 0u;
     const float approx = amax * inv6g;
     uint32_t c;
     asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %1;\n\tcvt.u32.u16 %0, h;\n\t}"
         : "=r"(c)
         : "f"(approx));
-    c &= 0x7Fu;
-    c = c == 0x7Fu ? 0x7Eu : (c == 0u ? 1u : c);   // NaN (g not positive) saturates; 0 -> the smallest
+    c = min(max(c & 0x7Fu, 1u), 0x7Eu);   // NaN (g not positive) saturates; 0 -> the smallest
     if (inv6g <= 0x1p100f) {
-        if (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ++c;
+        c += (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ? 1u : 0u;
+        return amax > 0.0f ? c : 0u;
     } else {
+        if (!(amax > 0.0f)) return 0u;
         // bounded by the code range
         while (c < 0x7Eu && !nv_scale_ok(val[c], g, amax)) ++c;
         while (c > 1u && nv_scale_ok(val[c - 1u], g, amax)) --c;
