@@ -113,3 +113,56 @@ def test_workspace_checks():
                              ws.data_ptr(), need, None)
     assert s == mx.MX_ERR_INVALID_ARG                                      # NVFP4 X with an MXFP8 W
     torch.cuda.synchronize()
+
+
+def test_nvfp4_mlp_pair_full_size_sampled_rows():
+    """The NVFP4 MLP pair at its full size (X [4608 x 3072] Student-t, W1
+    [12288 x 3072], W2 [3072 x 12288]): H = GELU(X W1^T) by the fused call
+    with |H| max, then Y = H W2^T with H quantized in the call from that max,
+    as one chain without a host sync.  Y equals the unfused chain bitwise; on
+    sampled rows, X's and H's codes equal the oracle's and H and Y are within
+    the tolerance of the fp64 oracle."""
+    M, D, F = 4608, 3072, 12288
+    X_bits = synth.student_t(3, M, D)
+    W1 = mx.quantize(to_dev(synth.gaussian_weights(4, F, D)), 3)
+    W2 = mx.quantize(to_dev(synth.gaussian_weights(5, D, F)), 3)
+    X = to_dev(X_bits)
+    aH = torch.empty(1, device="cuda")
+    H = mx.gemm_fused_act(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=aH)
+    Y = mx.gemm_fused_act(H, W2, x_amax=aH)
+    qX = mx.quantize(X, 3)
+    qH = mx.quantize(H, 3)
+    Y_u = mx.gemm(qH, W2)
+    torch.cuda.synchronize()
+    mx.check_device_error()
+    assert torch.equal(Y.view(torch.int16), Y_u.view(torch.int16))
+    assert float(aH.cpu()[0]) == float(H.abs().max().float().cpu())
+    rows = np.sort(np.random.default_rng(11).choice(M, 24, replace=False))
+    sel = torch.from_numpy(rows).cuda()
+
+    def rows_quantized(q, row_bits, amax):
+        """The oracle's codes of the sampled rows with the tensor's g, checked
+        against the GPU's, and their fp64 values."""
+        g = oracle.nvfp4_global_scale(amax)
+        assert np.float32(float(q.gscale.cpu()[0])) == np.float32(g)
+        c, s, _ = oracle.quantize(3, row_bits, gscale=g)
+        K = row_bits.shape[1]
+        gpu_codes = q.codes.view(-1, K // 2)[sel].cpu().numpy().reshape(-1)
+        assert np.array_equal(gpu_codes, c)
+        return oracle.dequantize_f64(3, c, s, g, len(rows), K)
+
+    Xd = rows_quantized(qX, X_bits[rows], float(X.abs().max().float().cpu()))
+    cw1, sw1, gw1 = host(W1)
+    W1d = oracle.dequantize_f64(3, cw1, sw1, gw1, F, D)
+    C1, C1abs = oracle.gemm_f64(Xd, W1d)
+    del W1d
+    Href = oracle.gelu(C1)
+    Hg = H[sel].float().cpu().double().numpy()
+    bound = 1.13 * (2.0 ** -8 * np.abs(C1) + 1e-4 * C1abs) + 2.0 ** -8 * np.abs(Href) + 1e-30
+    assert np.all(np.abs(Hg - Href) <= bound), float(np.max(np.abs(Hg - Href) / bound))
+    Hd = rows_quantized(qH, bits16(H[sel]), float(aH.cpu()[0]))
+    cw2, sw2, gw2 = host(W2)
+    W2d = oracle.dequantize_f64(3, cw2, sw2, gw2, D, F)
+    Yref, Yabs = oracle.gemm_f64(Hd, W2d)
+    ok, worst = oracle.gemm_tolerance_ok(Y[sel].float().cpu().double().numpy(), Yref, Yabs)
+    assert ok, worst
