@@ -519,6 +519,31 @@ def extras_gpu(device):
                      "frac_tensor": round(tf / tensor_peak(fmt if fmt == wfmt else 0, peaks, False), 3),
                      "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
         del a, w, qa, qws, C
+    # The NVFP4 MLP pair as the configuration states it: X [4608 x 3072]
+    # (Student-t) quantized inside the fused call for H = GELU(X W1^T) with
+    # |H| max, then H quantized inside the second fused call (g from that max)
+    # for Y = H W2^T; two launches of the library per call pair, no host sync.
+    from fp8_quantization_block_b200 import synth
+    M, D, F = 4608, 3072, 12288
+    X = synth.bits_to_tensor(synth.student_t(3, M, D)).to(device)
+    W1 = mx.quantize(synth.bits_to_tensor(synth.gaussian_weights(4, F, D)).to(device), 3)
+    W2 = mx.quantize(synth.bits_to_tensor(synth.gaussian_weights(5, D, F)).to(device), 3)
+    H = torch.empty((M, F), dtype=torch.bfloat16, device=device)
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device=device)
+    aH = torch.empty(1, device=device)
+    ws1, ws2 = mx.fused_workspace(3, M, D, device), mx.fused_workspace(3, M, F, device)
+
+    def mlp_pair(i):
+        mx.gemm_fused_act(X, W1, out=H, epilogue=mx.MX_EPI_GELU, amax_out=aH, workspace=ws1)
+        mx.gemm_fused_act(H, W2, out=Y, x_amax=aH, workspace=ws2)
+
+    ms = timed(mlp_pair, 1)
+    tf = 2 * 2 * M * D * F / (ms * 1e-3) / 1e12
+    out["mlp_nvfp4_pair_fused"] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1),
+                                   "frac_tensor": round(tf / tensor_peak(3, peaks, False), 3),
+                                   "steps": "X->H (amax pre-pass, quantize, GEMM1 + GELU + |H| max), "
+                                            "H->Y (quantize with g from |H| max, GEMM2)"}
+    del X, W1, W2, H, Y, ws1, ws2
     torch.cuda.empty_cache()
     mx.check_device_error()
     return out
