@@ -625,6 +625,7 @@ PROFILE_CASES = {
     "quant_mxfp4_32768x4096": ("quant", 2, 32768, 0, 4096),
     "quant_nvfp4_32768x4096": ("quant", 3, 32768, 0, 4096),
     "quant_mxfp8_dit_4096x3072": ("quant", 0, 4096, 0, 3072),
+    "fused_gelu_mlp1_nvfp4": ("fused_gelu", 3, 4608, 12288, 3072),
 }
 
 
@@ -648,6 +649,13 @@ def run_profile_case(name: str, reps: int = 4):
         gs = mx.quantize_rht(x, fmt, out=q).gscale.clone() if fmt == 3 else None
         for _ in range(reps):
             mx.quantize_rht(x, fmt, out=q, gscale=gs)
+    elif kind == "fused_gelu":
+        w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        qw = mx.quantize(w, wfmt)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        amax = torch.empty(1, device="cuda")
+        for _ in range(reps):
+            mx.gemm_fused_act(x, qw, out=C, epilogue=mx.MX_EPI_GELU, amax_out=amax)
     else:
         w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
         qa, qw = mx.quantize(x, fmt), mx.quantize(w, wfmt)
