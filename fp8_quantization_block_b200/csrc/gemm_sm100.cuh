@@ -251,28 +251,6 @@ MX_DEVICE_INLINE void issue_stage(int n_mma, uint32_t t_acc, uint64_t ad, uint64
     }
 }
 
-MX_DEVICE_INLINE uint64_t f2x(float v) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t fma2x(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t mul2x(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t pack2x(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-MX_DEVICE_INLINE void unpack2x(uint64_t r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
-
 // GELU of two values at once, the exact-erf form GELU(x) = x Phi(x) =
 // 0.5 x erfc(-x / sqrt(2)), with erfc from the Chebyshev fit of Numerical
 // Recipes (Press, Teukolsky, Vetterling and Flannery, 2nd ed., section 6.2,
@@ -288,30 +266,30 @@ MX_DEVICE_INLINE void unpack2x(uint64_t r, float &a, float &b) { asm("mov.b64 {%
 // GEMM1 with this epilogue runs 15% faster (the epilogue warps were the
 // bottleneck).
 MX_DEVICE_INLINE void gelu_erf2(float &x0, float &x1) {
-    const uint64_t X = pack2x(x0, x1);
+    const uint64_t X = pk2(x0, x1);
     const float z0 = fabsf(x0) * 0.70710678118654752440f, z1 = fabsf(x1) * 0.70710678118654752440f;
     float t0, t1;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t0) : "f"(fmaf(0.5f, z0, 1.0f)));
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t1) : "f"(fmaf(0.5f, z1, 1.0f)));
-    const uint64_t T = pack2x(t0, t1);
-    uint64_t P = fma2x(f2x(0.17087277f), T, f2x(-0.82215223f));
-    P = fma2x(P, T, f2x(1.48851587f));
-    P = fma2x(P, T, f2x(-1.13520398f));
-    P = fma2x(P, T, f2x(0.27886807f));
-    P = fma2x(P, T, f2x(-0.18628806f));
-    P = fma2x(P, T, f2x(0.09678418f));
-    P = fma2x(P, T, f2x(0.37409196f));
-    P = fma2x(P, T, f2x(1.00002368f));
-    P = fma2x(P, T, f2x(-1.26551223f));
-    P = fma2x(pack2x(-z0, -z1), pack2x(z0, z1), P);
+    const uint64_t T = pk2(t0, t1);
+    uint64_t P = fma2(pk2(0.17087277f, 0.17087277f), T, pk2(-0.82215223f, -0.82215223f));
+    P = fma2(P, T, pk2(1.48851587f, 1.48851587f));
+    P = fma2(P, T, pk2(-1.13520398f, -1.13520398f));
+    P = fma2(P, T, pk2(0.27886807f, 0.27886807f));
+    P = fma2(P, T, pk2(-0.18628806f, -0.18628806f));
+    P = fma2(P, T, pk2(0.09678418f, 0.09678418f));
+    P = fma2(P, T, pk2(0.37409196f, 0.37409196f));
+    P = fma2(P, T, pk2(1.00002368f, 1.00002368f));
+    P = fma2(P, T, pk2(-1.26551223f, -1.26551223f));
+    P = fma2(pk2(-z0, -z1), pk2(z0, z1), P);
     float a0, a1;
-    unpack2x(P, a0, a1);
-    const uint64_t E = mul2x(T, pack2x(__expf(a0), __expf(a1)));
+    upk2(P, a0, a1);
+    const uint64_t E = mul2(T, pk2(__expf(a0), __expf(a1)));
     float e0, e1;
-    unpack2x(E, e0, e1);
+    upk2(E, e0, e1);
     // erfc(-x / sqrt(2)): e for x <= 0, 2 - e for x > 0
     const float c0 = x0 > 0.0f ? 2.0f - e0 : e0, c1 = x1 > 0.0f ? 2.0f - e1 : e1;
-    unpack2x(mul2x(mul2x(X, f2x(0.5f)), pack2x(c0, c1)), x0, x1);
+    upk2(mul2(mul2(X, pk2(0.5f, 0.5f)), pk2(c0, c1)), x0, x1);
 }
 
 // Number of valid 32-byte MMA steps and 512-byte scale chunks in stage kt.

@@ -95,18 +95,6 @@ MX_DEVICE_INLINE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 
-// Non-blocking test of an mbarrier phase (no suspension).
-MX_DEVICE_INLINE bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 
 // Wait for the phase with the given parity to complete, for at most limit_ns.
 // Returns false (and records a timeout) if it did not, or if *abort is set by
@@ -171,6 +159,41 @@ MX_DEVICE_INLINE uint32_t wait_counter_above(const uint32_t *counter, uint32_t n
     }
 }
 
+// ---------------------------------------------------------------- packed fp32 pairs
+// f32x2 arithmetic of sm_100: two IEEE operations per instruction, each
+// rounded exactly as its scalar form (nearest-even, or toward zero for mul2_rz).
+MX_DEVICE_INLINE uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+MX_DEVICE_INLINE void upk2(uint64_t r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
+MX_DEVICE_INLINE uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t mul2_rz(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+MX_DEVICE_INLINE uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 // ---------------------------------------------------------------- TMA / bulk copies
 MX_DEVICE_INLINE void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -194,14 +217,6 @@ MX_DEVICE_INLINE void tma_load_3d(void *smem_dst, const void *tmap, int32_t x, i
         : "memory");
 }
 
-// Untiled bulk copy global -> shared (no multicast); 16-B aligned, size % 16 == 0.
-MX_DEVICE_INLINE void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
 
 
 // 2D tiled TMA store (bulk-group completion) from this CTA's shared memory.
@@ -235,18 +250,7 @@ MX_DEVICE_INLINE void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 MX_DEVICE_INLINE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 MX_DEVICE_INLINE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Arrive on an mbarrier once all prior tcgen05 async operations of this thread complete.
-MX_DEVICE_INLINE void tc_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
 
-// Copy one 32-row x 16-byte scale tile from shared memory into 4 TMEM columns,
-// replicated into all four 32-lane sub-partitions (the layout the block-scaled
-// MMA reads its scale factors from).
-MX_DEVICE_INLINE void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 
 // Block-scaled MMAs: D(tmem) (+)= (A * sfA) x (B * sfB)^T, A/B described in smem.
 MX_DEVICE_INLINE void tc_mma_mxf8f6f4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
@@ -439,11 +443,5 @@ MX_DEVICE_INLINE uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t
     return d;
 }
 
-MX_DEVICE_INLINE bool elect_one() {
-    uint32_t pred;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred)::"memory");
-    return pred != 0;
-}
 
 }  // namespace mx

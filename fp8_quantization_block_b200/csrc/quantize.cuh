@@ -232,40 +232,6 @@ MX_DEVICE_INLINE float e2m1_mag(uint32_t c) {
 // land exactly on a midpoint) is settled by the sign of |x| - g*s*m, which one
 // fma computes exactly (s*m is exact in fp32); a tie goes to the even code.
 
-// Packed fp32 pairs (f32x2 arithmetic of sm_100: two IEEE operations per
-// instruction, each rounded to nearest-even exactly as its scalar form).
-MX_DEVICE_INLINE uint64_t pk2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-MX_DEVICE_INLINE void upk2(uint64_t r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
-MX_DEVICE_INLINE uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t sub2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t mul2_rz(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-MX_DEVICE_INLINE uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
 // Midpoint between E2M1 magnitudes c and c + 1 (c = 0..6).
 MX_DEVICE_INLINE float e2m1_mid(uint32_t c) {
     return c < 4u ? 0.25f + 0.5f * (float)c : (c < 6u ? (float)c - 1.5f : 5.0f);
@@ -391,12 +357,6 @@ MX_DEVICE_INLINE uint4 ldg_stream(const void *p) {
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                  : "l"(p));
     return r;
-}
-
-MX_DEVICE_INLINE uint32_t bf16x2_absmax(uint32_t m, uint32_t w) {
-    uint32_t a = w & 0x7FFF7FFFu;
-    uint32_t lo = a & 0xFFFFu, hi = a >> 16;
-    return max(m, max(lo, hi));
 }
 
 // ------------------------------------------------------------------ kernels
