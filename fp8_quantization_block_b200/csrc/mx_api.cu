@@ -9,6 +9,8 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "mx.h"
 #include "mx_common.cuh"
@@ -188,13 +190,17 @@ void launch_quantize_mbs(const uint16_t *src, int64_t M, int64_t K, int64_t ld, 
                        cdiv(K / 16, 4), dst->scales + tile_bytes(MX_MXFP4_MBS, M, K));
 }
 
+// SM count of the current device, read once per device.
 int num_sms() {
-    static int n = 0;
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cache[kMaxDev];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool cached = dev >= 0 && dev < kMaxDev;
+    int n = cached ? cache[dev].load(std::memory_order_relaxed) : 0;
     if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        if (cached) cache[dev].store(n, std::memory_order_relaxed);
     }
     return n;
 }
@@ -251,6 +257,21 @@ bool make_tmap_sf(CUtensorMap *m, const uint8_t *scales, int64_t bands, int64_t 
     return r == CUDA_SUCCESS;
 }
 
+// Raise the dynamic shared memory limit of kernel fn to `bytes` on the current
+// device, once per (kernel, device): the attribute belongs to the device's
+// context, so a process that drives several GPUs sets it on each.
+cudaError_t smem_limit_once(const void *fn, int bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({fn, dev}) != 0) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert({fn, dev});
+    return e;
+}
+
 template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                         const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
@@ -273,13 +294,9 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_kernel<FMT, BN, STAGES, A_ROWS>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    });
-    if (attr_err != cudaSuccess) return MX_ERR_CUDA;
+    if (smem_limit_once(reinterpret_cast<const void *>(gemm_kernel<FMT, BN, STAGES, A_ROWS>), L::kAlloc) !=
+        cudaSuccess)
+        return MX_ERR_CUDA;
     GemmParams p;
     p.sf_tiles_k = sf_tiles_k;
     p.C = C;
@@ -339,13 +356,8 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_pair_kernel<FMT, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        L::kAlloc);
-    });
-    if (attr_err != cudaSuccess) return MX_ERR_CUDA;
+    if (smem_limit_once(reinterpret_cast<const void *>(gemm_pair_kernel<FMT, STAGES>), L::kAlloc) != cudaSuccess)
+        return MX_ERR_CUDA;
     GemmParams p;
     p.sf_tiles_k = sf_tiles_k;
     p.C = C;
