@@ -198,8 +198,12 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  * mx_gemm.  X's quantized form is not an output of this call.
  *   workspace: device buffer of at least mx_fused_workspace_bytes(fmt, M, K)
  *              bytes, 256-byte aligned; its contents are scratch.
- *   epilogue : MX_EPI_NONE, or MX_EPI_GELU (exact erf form, applied in FP32
- *              before the bf16 rounding).
+ *   epilogue : MX_EPI_NONE, or MX_EPI_GELU: the exact-erf form x Phi(x) =
+ *              0.5 x erfc(-x / sqrt 2), applied in FP32 before the bf16
+ *              rounding, with erfc from the Chebyshev fit of Numerical Recipes
+ *              (relative error < 1.2e-7) and the hardware's approximate
+ *              reciprocal and exponential: within one bf16 ulp of the form
+ *              evaluated with erff.
  *   amax_out : NULL, or a device float that receives max |C| over the bf16
  *              outputs (it is zeroed by this call first).  Feeding it to the
  *              next call's x_amax chains two NVFP4 GEMMs without a host sync.
