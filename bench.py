@@ -793,7 +793,9 @@ def main():
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_gemm_fused_act -> D2H C, upload / compute / download on three "
                         "streams with double buffers (consecutive steps overlap)"},
-        "gpu_launches": 2 * args.steps,
+        # per step: the quantize and the GEMM; NVFP4 without a given g adds the
+        # amax pre-pass and the kernel that turns the amax into g
+        "gpu_launches": (4 if fmt == 3 else 2) * args.steps,
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_extras:
