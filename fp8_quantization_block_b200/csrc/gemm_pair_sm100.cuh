@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
-        mbar_init(acc_empty, 2 * kEpiWarps);
+        // both CTAs' epilogue warps (with GELU, their scale warps too)
+        mbar_init(acc_empty, (p.epilogue == 1 ? 4 : 2) * kEpiWarps);
         mbar_init(mma_done, 1);
         for (int i = 0; i < L::kSlots; ++i) mbar_init(&sf_full[i], 8);
         *abort_flag = 0;
@@ -219,31 +220,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ------------------------------------------------------------ scale warps
         const int q = warp & 3;
         const uint32_t sf_full_leader0 = mapa_shared(smem_u32(&sf_full[0]), 0);
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
         int my_tiles = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
+        float scale = 1.0f;
+        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        uint32_t amax = 0;
+        auto rows_of = [&](int t, int &m0, int &n0) {
+            tile_coords(pair + t * npairs, p.m_blocks, m0, n0, 256);
+            m0 = ((pair + t * npairs) % p.m_blocks) * 256 + 128 * (int)rank;
+        };
+        // GELU: this warp's share of the shared columns of tile t (all but the
+        // last tile), drained before the first wait on a stage of tile t + 1 or
+        // later, whose MMAs cannot start until both CTAs have released tile t's
+        // columns
+        int help_next = 0;
+        auto help = [&](int t) -> bool {
+            int m0, n0;
+            rows_of(t, m0, n0);
+            const int b = t & 1;
+            if (!mbar_wait_bounded(&acc_full[b], (t >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag))
+                return false;
+            tc_fence_after();
+            help_drain_t<256, L::kAccStride, FMT == 3>(
+                p, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride), b, m0 + 32 * q, n0, lane, amax,
+                scale);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+            return true;
+        };
         scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
                               my_tiles, lane, abort_flag,
-                              [&](int slot) { mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot); });
+                              [&](int slot) { mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot); },
+                              [&](int kg) -> bool {
+                                  if (p.epilogue != 1) return true;
+                                  for (; help_next < my_tiles - 1 && kg - L::kSlots >= (help_next + 1) * p.num_kt;
+                                       ++help_next)
+                                      if (!help(help_next)) return false;
+                                  return true;
+                              });
+        if (p.epilogue == 1 && !*abort_flag)
+            for (; help_next < my_tiles - 1; ++help_next)
+                if (!help(help_next)) break;
         // then the upper half of the columns of this CTA's rows of the last tile
         // (the pair's MMAs have completed, so the B stage ring is free for the
         // staging buffers)
         if (my_tiles > 0 && !*abort_flag) {
             const int it = my_tiles - 1, b = it & 1;
-            const int tile = pair + it * npairs;
             int m0, n0;
-            tile_coords(tile, p.m_blocks, m0, n0, 256);
-            m0 = (tile % p.m_blocks) * 256 + 128 * (int)rank;
-            if (mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) {
+            rows_of(it, m0, n0);
+            // mma_done (one phase) rather than acc_full[b]: without GELU this warp
+            // may finish its slots several tiles ahead of the MMAs, and a parity
+            // wait on acc_full[b], whose phases alternate every second tile,
+            // could then be satisfied by an older tile's phase
+            if (mbar_wait_bounded(mma_done, 0, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) {
                 tc_fence_after();
-                float scale = 1.0f;
-                if (FMT == 3) scale = (*p.ga) * (*p.gb);
                 uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
-                uint32_t amax = 0, nstore = 0;
+                uint32_t nstore = 0;
                 epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
                                                        m0 + 32 * q, n0, 4, 8, lane, bufs, nstore, amax, scale);
-                epilogue_finish(p, lane, amax);
             }
         }
+        epilogue_finish(p, lane, amax);
     } else {
         // ------------------------------------------------------------ epilogue (this CTA's 128 rows)
         const int q = warp & 3;

@@ -394,11 +394,13 @@ MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *t
 // arrive_full(slot).  After a group's last stage the warp frees the group.
 // (Writing a group's two stages with one wait for the stores was measured
 // slower: the second slot's wait for older MMAs costs more than the store
-// latency it hides.)
-template <typename L, int STAGES, typename ArriveFull>
+// latency it hides.)  before_wait(kg) runs just before the wait for stage
+// kg - L::kSlots; the kernels use it to drain accumulator columns whose
+// release that stage's MMAs may be waiting for.
+template <typename L, int STAGES, typename ArriveFull, typename BeforeWait>
 MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *sfload, uint64_t *sfree, uint64_t *empty,
                                  uint32_t t_sf0, int my_tiles, int lane, volatile int *abort_flag,
-                                 ArriveFull arrive_full) {
+                                 ArriveFull arrive_full, BeforeWait before_wait) {
     constexpr int NG = L::kSfGroups;
     constexpr int kChunks = L::F::kChunks;
     int g = 0, slot = 0, e = 0;
@@ -413,7 +415,10 @@ MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *s
                 break;
             }
             if (kg >= L::kSlots) {
-                if (!mbar_wait_bounded(&empty[e], eph, p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
+                // stage kg reuses the slot of stage kg - kSlots: hand the wait's idle
+                // time to before_wait first (false: give up, as on a timeout)
+                if (!before_wait(kg) ||
+                    !mbar_wait_bounded(&empty[e], eph, p.wait_limit_ns, SITE_GEMM_SF_EMPTY, abort_flag)) {
                     stop = true;
                     break;
                 }
@@ -504,7 +509,8 @@ MX_DEVICE_INLINE void epi_load_convert(uint32_t t_addr, float scale, uint32_t (&
 // chunks earlier to have finished reading shared memory.
 template <int NBUF>
 MX_DEVICE_INLINE void epi_emit(const GemmParams &p, const CUtensorMap *tmC, const uint32_t (&packed)[16], int m0q,
-                               int n0, int col, int lane, uint8_t *bufs, uint32_t &nstore, uint32_t &amax) {
+                               int n0, int col, int lane, uint8_t *bufs, uint32_t &nstore, uint32_t &amax,
+                               bool via_tma) {
     const int row = m0q + lane;
     const int n_valid = p.N - n0;
     if (p.amax_out != nullptr && row < p.M) {
@@ -523,7 +529,7 @@ MX_DEVICE_INLINE void epi_emit(const GemmParams &p, const CUtensorMap *tmC, cons
         }
     }
     if (m0q >= p.M) return;  // warp-uniform: no rows of this quadrant exist
-    if (p.use_tma_store) {
+    if (via_tma) {
         uint8_t *buf = bufs + (nstore % NBUF) * kEpiChunkBytes;
         if (lane == 0) bulk_wait_group_read<NBUF - 1>();  // this buffer's previous store has read it
         __syncwarp();
@@ -540,10 +546,30 @@ MX_DEVICE_INLINE void epi_emit(const GemmParams &p, const CUtensorMap *tmC, cons
         ++nstore;
     } else if (row < p.M) {
         uint16_t *dst = p.C + (int64_t)row * p.ldc + n0 + col;
+        if (p.use_tma_store && col + 32 <= n_valid) {
+            // C 16-byte aligned and ldc % 8 == 0 (the TMA store's conditions):
+            // this row's 64 bytes as four 16-byte stores
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (col + i < n_valid) dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
+            for (int v = 0; v < 4; ++v)
+                d4[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (col + i < n_valid) dst[i] = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
+        }
     }
+}
+
+// With GELU, the chunks of an accumulator whose columns the next tile shares
+// are drained by two warps per TMEM lane quadrant: the epilogue warp and the
+// scale warp, which would otherwise sit waiting for the MMAs that this release
+// holds back.  The scale warp takes this many of them (the last ones in
+// drain order), through direct global stores (shared memory has no room for
+// its own staging buffers).
+template <int BN, int ACC_STRIDE>
+__host__ __device__ constexpr int gelu_help_chunks() {
+    return ((BN - ACC_STRIDE) / 32) / 2;
 }
 
 // Drain one accumulator tile (BN columns) for this warp's TMEM quadrant.  The
@@ -562,24 +588,21 @@ MX_DEVICE_INLINE void epilogue_tile_t(const GemmParams &p, const CUtensorMap *tm
     const int n_valid = p.N - n0;
     if constexpr (GELU) {
         // GELU needs more live registers per chunk: drain in order, releasing
-        // after the shared chunks have been written out.
-        for (int idx = 0; idx < kChunks; ++idx) {
-            if (idx == kOv) {
-                tc_fence_before();
-                __syncwarp();
-                release();
-            }
+        // after the shared chunks have been written out.  The last
+        // gelu_help_chunks() shared chunks are the scale warp's (help_drain_t).
+        constexpr int kMine = kOv - gelu_help_chunks<BN, ACC_STRIDE>();
+        auto drain = [&](int idx) {
             const int col = 32 * ((b == 0) ? (idx + (kChunks - kOv)) % kChunks : idx);
-            if (col >= n_valid) continue;  // warp-uniform
+            if (col >= n_valid) return;  // warp-uniform
             uint32_t packed[16];
             epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
-            epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
-        }
-        if (kOv == kChunks) {
-            tc_fence_before();
-            __syncwarp();
-            release();
-        }
+            epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax, p.use_tma_store);
+        };
+        for (int idx = 0; idx < kMine; ++idx) drain(idx);
+        tc_fence_before();
+        __syncwarp();
+        release();
+        for (int idx = kOv; idx < kChunks; ++idx) drain(idx);
     } else {
         uint32_t ov[kOv > 0 ? kOv : 1][16];
 #pragma unroll
@@ -593,14 +616,14 @@ MX_DEVICE_INLINE void epilogue_tile_t(const GemmParams &p, const CUtensorMap *tm
 #pragma unroll
         for (int i = 0; i < kOv; ++i) {
             const int col = 32 * ((b == 0) ? (kChunks - kOv + i) : i);
-            if (col < n_valid) epi_emit<NBUF>(p, tmC, ov[i], m0q, n0, col, lane, bufs, nstore, amax);
+            if (col < n_valid) epi_emit<NBUF>(p, tmC, ov[i], m0q, n0, col, lane, bufs, nstore, amax, p.use_tma_store);
         }
         for (int i = 0; i < kChunks - kOv; ++i) {
             const int col = 32 * ((b == 0) ? i : (kOv + i));
             if (col >= n_valid) break;  // warp-uniform; columns ascend
             uint32_t packed[16];
             epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
-            epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+            epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax, p.use_tma_store);
         }
     }
 }
@@ -619,7 +642,7 @@ MX_DEVICE_INLINE void epilogue_chunks_t(const GemmParams &p, const CUtensorMap *
         if (col >= n_valid) break;  // warp-uniform; columns ascend
         uint32_t packed[16];
         epi_load_convert<SCALED, GELU>(t_acc + (uint32_t)col, scale, packed);
-        epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax);
+        epi_emit<NBUF>(p, tmC, packed, m0q, n0, col, lane, bufs, nstore, amax, p.use_tma_store);
     }
 }
 template <int NBUF, bool SCALED>
@@ -642,6 +665,25 @@ MX_DEVICE_INLINE void epilogue_tile(const GemmParams &p, const CUtensorMap *tmC,
     else
         epilogue_tile_t<BN, ACC_STRIDE, NBUF, SCALED, false>(p, tmC, t_acc, b, m0q, n0, lane, bufs, nstore, amax, scale,
                                                              release);
+}
+
+// The scale warp's share of a GELU tile's shared chunks (the last
+// gelu_help_chunks() of them in epilogue_tile_t's drain order), written to C
+// with direct stores; the caller releases the columns afterwards.
+template <int BN, int ACC_STRIDE, bool SCALED>
+MX_DEVICE_INLINE void help_drain_t(const GemmParams &p, uint32_t t_acc, int b, int m0q, int n0, int lane,
+                                   uint32_t &amax, float scale) {
+    constexpr int kChunks = BN / 32;
+    constexpr int kOv = (BN - ACC_STRIDE) / 32;
+    const int n_valid = p.N - n0;
+    uint32_t unused = 0;
+    for (int idx = kOv - gelu_help_chunks<BN, ACC_STRIDE>(); idx < kOv; ++idx) {
+        const int col = 32 * ((b == 0) ? (idx + (kChunks - kOv)) % kChunks : idx);
+        if (col >= n_valid) continue;  // warp-uniform
+        uint32_t packed[16];
+        epi_load_convert<SCALED, true>(t_acc + (uint32_t)col, scale, packed);
+        epi_emit<1>(p, nullptr, packed, m0q, n0, col, lane, nullptr, unused, amax, false);
+    }
 }
 
 // Flush this warp's stores and publish its |C| maximum.
@@ -689,7 +731,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
-        mbar_init(acc_empty, kEpiWarps);
+        // with GELU the scale warps also release shared accumulator columns
+        mbar_init(acc_empty, (p.epilogue == 1 ? 2 : 1) * kEpiWarps);
         mbar_init(mma_done, 1);
         for (int i = 0; i < L::kSlots; ++i) mbar_init(&sf_full[i], 4);
         *abort_flag = 0;
@@ -832,25 +875,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int q = warp & 3;
         int my_tiles = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
+        float scale = 1.0f;
+        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        uint32_t amax = 0;
+        // GELU: this warp's share of the shared columns of tile t (all but the
+        // last tile), drained before the first wait on a stage of tile t + 1 or
+        // later, whose MMAs cannot start until tile t's columns are released
+        int help_next = 0;
+        auto help = [&](int t) -> bool {
+            int m0, n0;
+            tile_coords(blockIdx.x + t * gridDim.x, p.m_blocks, m0, n0, BN);
+            const int b = t & 1;
+            if (!mbar_wait_bounded(&acc_full[b], (t >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag))
+                return false;
+            tc_fence_after();
+            help_drain_t<BN, L::kAccStride, FMT == 3>(
+                p, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride), b, m0 + 32 * q, n0, lane, amax,
+                scale);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            return true;
+        };
         scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
-                              my_tiles, lane, abort_flag, [&](int slot) { mbar_arrive(&sf_full[slot]); });
+                              my_tiles, lane, abort_flag, [&](int slot) { mbar_arrive(&sf_full[slot]); },
+                              [&](int kg) -> bool {
+                                  if (p.epilogue != 1) return true;
+                                  for (; help_next < my_tiles - 1 && kg - L::kSlots >= (help_next + 1) * p.num_kt;
+                                       ++help_next)
+                                      if (!help(help_next)) return false;
+                                  return true;
+                              });
+        if (p.epilogue == 1 && !*abort_flag)
+            for (; help_next < my_tiles - 1; ++help_next)
+                if (!help(help_next)) break;
         // then the upper half of the columns of this CTA's last tile (its MMAs have
         // completed, so the B stage ring is free for the staging buffers)
         if (my_tiles > 0 && !*abort_flag) {
             const int it = my_tiles - 1, b = it & 1;
             int m0, n0;
             tile_coords(blockIdx.x + it * gridDim.x, p.m_blocks, m0, n0, BN);
-            if (mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) {
+            // mma_done (one phase) rather than acc_full[b]: without GELU this warp
+            // may finish its slots several tiles ahead of the MMAs, and a parity
+            // wait on acc_full[b], whose phases alternate every second tile,
+            // could then be satisfied by an older tile's phase
+            if (mbar_wait_bounded(mma_done, 0, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) {
                 tc_fence_after();
-                float scale = 1.0f;
-                if (FMT == 3) scale = (*p.ga) * (*p.gb);
                 uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
-                uint32_t amax = 0, nstore = 0;
+                uint32_t nstore = 0;
                 epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
                                                        m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs, nstore, amax, scale);
-                epilogue_finish(p, lane, amax);
             }
         }
+        epilogue_finish(p, lane, amax);
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quadrant this warp may access

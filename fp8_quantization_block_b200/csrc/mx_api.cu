@@ -27,6 +27,7 @@ std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<int> g_skip_producer{0};
 std::atomic<int> g_pair_enabled{1};
 std::atomic<int> g_pdl_enabled{1};
+std::atomic<int> g_max_gemm_ctas{0};  // 0: one CTA (or CTA pair) per SM pair of the device
 
 // Launch attributes shared by the kernels that may overlap the previous kernel
 // in the stream (they call griddep_wait() before reading any input).
@@ -317,7 +318,9 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.stage_tx = (uint32_t)(kStageKBytes * (A_ROWS * fmt_bits(A->fmt) + BN * fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
-    const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
+    const int cap = g_max_gemm_ctas.load();
+    const int64_t max_ctas = cap > 0 && cap < num_sms() ? cap : num_sms();
+    const unsigned grid = (unsigned)(tiles < max_ctas ? tiles : max_ctas);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(grid, 1, 1);
@@ -379,7 +382,8 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     p.stage_tx = (uint32_t)(2 * kStageKBytes * 128 * (fmt_bits(A->fmt) + fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
-    const int64_t max_pairs = num_sms() / 2;
+    const int cap = g_max_gemm_ctas.load();
+    const int64_t max_pairs = cap > 0 && cap < num_sms() ? (cap + 1) / 2 : num_sms() / 2;
     const unsigned pairs = (unsigned)(tiles < max_pairs ? tiles : max_pairs);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
@@ -510,6 +514,7 @@ mx_status mx_debug_set(int key, uint64_t value) {
     case MX_DEBUG_SKIP_PRODUCER: g_skip_producer.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_PAIR_GEMM: g_pair_enabled.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_OVERLAP_LAUNCH: g_pdl_enabled.store(value ? 1 : 0); return MX_OK;
+    case MX_DEBUG_MAX_GEMM_CTAS: g_max_gemm_ctas.store(value > 65535 ? 0 : (int)value); return MX_OK;
     default: return MX_ERR_INVALID_ARG;
     }
 }

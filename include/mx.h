@@ -271,12 +271,19 @@ int mx_version(void);
  *                            the tail of the previous kernel in the stream, and
  *                            they read no input before that kernel completes.
  *                            0 = ordinary stream order.
+ *   MX_DEBUG_MAX_GEMM_CTAS : n > 0 = GEMM grids of at most n CTAs (CTA-pair
+ *                            grids: at most ceil(n / 2) pairs), so that each
+ *                            CTA walks several tiles even on small shapes;
+ *                            0 (default) = one CTA per SM.  The result does
+ *                            not depend on it (each tile is summed in the
+ *                            same order wherever it runs).
  * Returns MX_ERR_INVALID_ARG for an unknown key. */
 typedef enum {
     MX_DEBUG_WAIT_LIMIT_NS = 1,
     MX_DEBUG_SKIP_PRODUCER = 2,
     MX_DEBUG_PAIR_GEMM = 3,
-    MX_DEBUG_OVERLAP_LAUNCH = 4
+    MX_DEBUG_OVERLAP_LAUNCH = 4,
+    MX_DEBUG_MAX_GEMM_CTAS = 5
 } mx_debug_key;
 mx_status mx_debug_set(int key, uint64_t value);
 

@@ -71,6 +71,49 @@ def test_gelu_and_amax_epilogue(fmt, M):
     assert float(amax.cpu()[0]) == float(H.abs().max().float().cpu())     # zeroed, then max |H|
 
 
+@pytest.mark.parametrize("fmt", [0, 2, 3])
+@pytest.mark.parametrize("M,N,K", [(300, 1000, 256), (300, 1000, 2048), (100, 1000, 256), (100, 1000, 2048),
+                                   (20, 1000, 2048), (300, 100, 512)])
+def test_several_tiles_per_cta(fmt, M, N, K):
+    """A grid of one CTA (or one CTA pair) walks every tile, so consecutive
+    tiles alternate between the two accumulators whose TMEM columns overlap.
+    With GELU those shared columns are drained by the epilogue and the scale
+    warps together, before (K > 4 stages) or after (K within the scale slots)
+    the scale warps' last wait.  Shapes: the CTA-pair kernel (M = 300: a ragged
+    second row block whose upper CTA has no rows), the single-CTA 128 x 256 and
+    32-row variants, 128-wide N tiles; N = 1000 ends in a partial chunk.  The
+    result must equal the one-tile-per-CTA launch bitwise, and GELU the fp64
+    oracle within the GEMM bound."""
+    X_bits = synth.student_t(90 + M, M, K)
+    W_bits = synth.gaussian_weights(91 + N, N, K)
+    X = to_dev(X_bits)
+    W = mx.quantize(to_dev(W_bits), fmt)
+    qX = mx.quantize(X, fmt)
+    a_ref = torch.empty(1, device="cuda")
+    H_ref = mx.gemm_fused_act(X, W, epilogue=mx.MX_EPI_GELU, amax_out=a_ref)
+    C_ref = mx.gemm(qX, W)
+    a = torch.empty(1, device="cuda")
+    try:
+        assert mx.mx_debug_set(mx.MX_DEBUG_MAX_GEMM_CTAS, 1) == mx.MX_OK
+        H = mx.gemm_fused_act(X, W, epilogue=mx.MX_EPI_GELU, amax_out=a)
+        C = mx.gemm(qX, W)
+        torch.cuda.synchronize()
+        mx.check_device_error()
+    finally:
+        mx.mx_debug_set(mx.MX_DEBUG_MAX_GEMM_CTAS, 0)
+    assert torch.equal(C.view(torch.int16), C_ref.view(torch.int16))
+    assert torch.equal(H.view(torch.int16), H_ref.view(torch.int16))
+    assert float(a.cpu()[0]) == float(a_ref.cpu()[0]) == float(H.abs().max().float().cpu())
+    cx, sx, gx = oracle.quantize(fmt, X_bits)
+    cw, sw, gw = host(W)
+    Cref, Cabs = oracle.gemm_f64(oracle.dequantize_f64(fmt, cx, sx, gx, M, K),
+                                 oracle.dequantize_f64(fmt, cw, sw, gw, N, K))
+    Href = oracle.gelu(Cref)
+    Hg = H.float().cpu().double().numpy()
+    bound = 1.13 * (2.0 ** -8 * np.abs(Cref) + 1e-4 * Cabs) + 2.0 ** -8 * np.abs(Href) + 1e-30
+    assert np.all(np.abs(Hg - Href) <= bound), float(np.max(np.abs(Hg - Href) / bound))
+
+
 def test_nvfp4_mlp_chain_without_host_sync():
     M, D, F = 256, 512, 1024
     X = to_dev(synth.student_t(70, M, D))
