@@ -146,3 +146,34 @@ def test_fused_act_with_mixed_weights(xf, wf):
     mx.check_device_error()
     ok, worst = gemm_check(C, _dq(xa, xf), _dq(wb, wf))
     assert ok, worst
+
+
+@pytest.mark.parametrize("xf,wf", [(0, 2), (4, 4), (1, 0)])
+@pytest.mark.parametrize("M,N,K", [(300, 1000, 256), (100, 1000, 2048)])
+def test_several_tiles_per_cta_mixed(xf, wf, M, N, K):
+    """The runtime-typed kernel (mixed operands, MXFP6) with a grid of one CTA
+    (or one CTA pair), so that every CTA walks several tiles through both
+    accumulators: plain and GELU results equal the one-tile-per-CTA launch
+    bitwise, and GELU the fp64 oracle within the GEMM bound."""
+    xa = synth.dit_activations(102, M, K)
+    wb = synth.gaussian_weights(103, N, K)
+    X = to_dev(xa)
+    W = quantize_dev(wb, wf)
+    qX = quantize_dev(xa, xf)
+    H_ref = mx.gemm_fused_act(X, W, x_fmt=xf, epilogue=mx.MX_EPI_GELU)
+    C_ref = mx.gemm(qX, W)
+    try:
+        assert mx.mx_debug_set(mx.MX_DEBUG_MAX_GEMM_CTAS, 1) == mx.MX_OK
+        H = mx.gemm_fused_act(X, W, x_fmt=xf, epilogue=mx.MX_EPI_GELU)
+        C = mx.gemm(qX, W)
+        torch.cuda.synchronize()
+        mx.check_device_error()
+    finally:
+        mx.mx_debug_set(mx.MX_DEBUG_MAX_GEMM_CTAS, 0)
+    assert torch.equal(C.view(torch.int16), C_ref.view(torch.int16))
+    assert torch.equal(H.view(torch.int16), H_ref.view(torch.int16))
+    Cref, Cabs = oracle.gemm_f64(_dq(xa, xf), _dq(wb, wf))
+    Href = oracle.gelu(Cref)
+    Hg = H.float().cpu().double().numpy()
+    bound = 1.13 * (2.0 ** -8 * np.abs(Cref) + 1e-4 * Cabs) + 2.0 ** -8 * np.abs(Href) + 1e-30
+    assert np.all(np.abs(Hg - Href) <= bound), float(np.max(np.abs(Hg - Href) / bound))
