@@ -56,6 +56,9 @@ def test_status_strings_and_version(L):
     assert mx.mx_status_string(mx.MX_ERR_TIMEOUT) == "MX_ERR_TIMEOUT"
     assert mx.mx_version() >= 100
     assert mx.mx_debug_set(99, 0) == mx.MX_ERR_INVALID_ARG
+    # the grid cap is host state only: set and restored without a GPU
+    assert mx.mx_debug_set(mx.MX_DEBUG_MAX_GEMM_CTAS, 2) == mx.MX_OK
+    assert mx.mx_debug_set(mx.MX_DEBUG_MAX_GEMM_CTAS, 0) == mx.MX_OK
 
 
 def _t(fmt, rows, cols, codes=0x1000, scales=0x2000, g=0x3000):
