@@ -1,0 +1,199 @@
+"""Model check of the GEMM kernels' barrier protocol (gemm_sm100.cuh,
+gemm_pair_sm100.cuh), on the CPU.
+
+Every warp role of one CTA is played as a coroutine against mbarriers with the
+hardware's phase semantics: a barrier completes a phase when its arrival count
+is reached, and a parity wait passes while the current (incomplete) phase's
+parity differs from the one asked for, so it only tells the latest two phases
+apart.  Random schedules (including a tensor pipe that completes MMAs, in
+order, at arbitrary times) check that
+
+* no schedule deadlocks, and
+* every wait passes on exactly the phase its role means (not an older phase
+  still showing the right parity, nor a newer one that reused the buffer).
+
+The roles: code-tile producer (empty -> full), gate (full + sf_full -> ready
+count), MMA issuer (ready, acc_empty -> commits to empty / acc_full /
+mma_done), scale warps (empty of stage kg - slots -> sf_full; with GELU they
+drain a share of each tile's shared accumulator columns and arrive on
+acc_empty; the last tile after mma_done), epilogue warps (acc_full ->
+acc_empty).  A CTA pair runs the same protocol with both CTAs' arrivals
+counted on the leader's barriers, which only scales the counts.
+
+The planted variants re-create three mistakes this protocol rules out and
+must be caught: the scale warps' last-tile wait as a parity wait on acc_full
+(an older tile's phase can satisfy it when K spans few stages), waiting on
+every tile's acc_full in order after the slots are written (a warp that far
+behind no longer tells the phases apart), and the GELU share drained after,
+instead of before, the wait on a stage of the next tile (that stage's MMAs
+wait for the release the share is part of: a deadlock)."""
+import itertools
+import random
+
+import pytest
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.completed = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        assert self.pending >= 0, "more arrivals than the barrier's count"
+        if self.pending == 0:
+            self.completed += 1
+            self.pending = self.count
+
+    def passes(self, phase):
+        # the hardware parity test for "phase `phase` has completed"
+        return (self.completed & 1) != (phase & 1)
+
+
+class Violation(AssertionError):
+    pass
+
+
+def wait(bar, phase, what):
+    return ("wait", bar, phase, what)
+
+
+def until(cond):
+    return ("until", cond)
+
+
+def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_wait="mma_done",
+                 in_order_waits=False, help_before_wait=True):
+    rng = random.Random(seed)
+    G = T * num_kt  # stages this CTA walks
+    full = [Bar(1) for _ in range(stages)]
+    empty = [Bar(1) for _ in range(stages)]
+    sf_full = [Bar(n_scale) for _ in range(slots)]
+    acc_full = [Bar(1), Bar(1)]
+    acc_empty = Bar(n_epi + (n_scale if gelu else 0))
+    mma_done = Bar(1)
+    st = {"ready": 0}
+    pipe = []  # commits, completed in issue order by the tensor pipe
+
+    def producer():
+        for g in range(G):
+            yield wait(empty[g % stages], g // stages - 1, "producer empty")
+            full[g % stages].arrive()  # the TMA fill completing
+
+    def gate():
+        for g in range(G):
+            yield wait(full[g % stages], g // stages, "gate full")
+            yield wait(sf_full[g % slots], g // slots, "gate sf_full")
+            st["ready"] = g + 1
+
+    def mma():
+        g = 0
+        for t in range(T):
+            for kt in range(num_kt):
+                yield until(lambda g=g: st["ready"] > g)
+                if kt == 0 and t > 0:
+                    yield wait(acc_empty, t - 1, "mma acc_empty")
+                pipe.append(empty[g % stages])
+                g += 1
+            pipe.append(acc_full[t & 1])
+        pipe.append(mma_done)
+
+    def epilogue():
+        for t in range(T):
+            yield wait(acc_full[t & 1], t // 2, "epilogue acc_full")
+            if t == T - 1:
+                break  # the last tile: nothing waits for its release
+            acc_empty.arrive()
+
+    def scale_warp():
+        help_next = 0
+        for g in range(G):
+            if g >= slots:
+                # before_wait(kg): drain shared columns of every tile whose
+                # release the awaited stage's MMAs may need
+                if not help_before_wait:
+                    yield wait(empty[(g - slots) % stages], (g - slots) // stages, "scale empty")
+                while gelu and help_next < T - 1 and g - slots >= (help_next + 1) * num_kt:
+                    yield wait(acc_full[help_next & 1], help_next // 2, "help acc_full")
+                    acc_empty.arrive()
+                    help_next += 1
+                if help_before_wait:
+                    yield wait(empty[(g - slots) % stages], (g - slots) // stages, "scale empty")
+            sf_full[g % slots].arrive()
+        while gelu and help_next < T - 1:
+            yield wait(acc_full[help_next & 1], help_next // 2, "help acc_full")
+            acc_empty.arrive()
+            help_next += 1
+        if in_order_waits:
+            for t in range(help_next, T - 1):
+                yield wait(acc_full[t & 1], t // 2, "in-order acc_full")
+        if T > 0:
+            if last_wait == "mma_done":
+                yield wait(mma_done, 0, "last-tile mma_done")
+            else:
+                yield wait(acc_full[(T - 1) & 1], (T - 1) // 2, "last-tile acc_full")
+
+    actors = [producer(), gate(), mma()] + [epilogue() for _ in range(n_epi)] + \
+             [scale_warp() for _ in range(n_scale)]
+    pending = {}
+    for a in actors:
+        try:
+            pending[a] = next(a)
+        except StopIteration:
+            pass
+    while pending or pipe:
+        runnable = [a for a, c in pending.items() if
+                    (c[0] == "wait" and c[1].passes(c[2])) or (c[0] == "until" and c[1]())]
+        choices = runnable + (["pipe"] if pipe else [])
+        if not choices:
+            raise Violation("deadlock: " + ", ".join(c[3] for c in pending.values() if c[0] == "wait"))
+        a = rng.choice(choices)
+        if a == "pipe":
+            pipe.pop(0).arrive()
+            continue
+        c = pending[a]
+        if c[0] == "wait" and c[1].completed != c[2] + 1:
+            kind = "an older" if c[1].completed < c[2] + 1 else "a newer"
+            raise Violation(f"{c[3]} for phase {c[2]} passed on {kind} phase "
+                            f"({c[1].completed} completed)")
+        try:
+            pending[a] = next(a)
+        except StopIteration:
+            del pending[a]
+    return True
+
+
+# STAGES >= slots, as the kernels assert; num_kt from one stage up to past the
+# slot count; 1 to 5 tiles per CTA (both accumulators, the last-tile split)
+CASES = [(T, kt, s, sl, gelu) for T, kt, (s, sl), gelu in
+         itertools.product([1, 2, 3, 5], [1, 2, 3, 7], [(4, 4), (5, 4), (6, 6)], [False, True])]
+
+
+@pytest.mark.parametrize("T,num_kt,stages,slots,gelu", CASES)
+def test_protocol_has_no_deadlock_or_phase_alias(T, num_kt, stages, slots, gelu):
+    for seed in range(12):
+        run_protocol(T, num_kt, stages, slots, gelu, seed)
+
+
+def _caught(gelu=False, **kw):
+    for T, num_kt in [(3, 1), (5, 1), (4, 2), (5, 3), (3, 7)]:
+        for seed in range(40):
+            try:
+                run_protocol(T, num_kt, 6, 6, gelu, seed, **kw)
+            except Violation as e:
+                return str(e)
+    return None
+
+
+def test_planted_last_tile_parity_wait_is_caught():
+    msg = _caught(last_wait="acc_full")
+    assert msg is not None and "older phase" in msg, msg
+
+
+def test_planted_in_order_waits_are_caught():
+    msg = _caught(in_order_waits=True)
+    assert msg is not None, msg
+
+
+def test_planted_help_after_the_wait_is_caught():
+    msg = _caught(gelu=True, help_before_wait=False)
+    assert msg is not None and msg.startswith("deadlock"), msg
