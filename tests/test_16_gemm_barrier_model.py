@@ -12,13 +12,16 @@ order, at arbitrary times) check that
 * every wait passes on exactly the phase its role means (not an older phase
   still showing the right parity, nor a newer one that reused the buffer).
 
-The roles: code-tile producer (empty -> full), gate (full + sf_full -> ready
-count), MMA issuer (ready, acc_empty -> commits to empty / acc_full /
-mma_done), scale warps (empty of stage kg - slots -> sf_full; with GELU they
-drain a share of each tile's shared accumulator columns and arrive on
-acc_empty; the last tile after mma_done), epilogue warps (acc_full ->
-acc_empty).  A CTA pair runs the same protocol with both CTAs' arrivals
-counted on the leader's barriers, which only scales the counts.
+The roles: code-tile producer (empty -> full), scale-tile producer (sfree
+-> sfload, groups of two stages that never span two tiles), gate (full +
+sf_full -> ready count), MMA issuer (ready, acc_empty -> commits to empty /
+acc_full / mma_done), scale warps (sfload and empty of stage kg - slots ->
+sf_full, sfree after a group's last stage; with GELU they drain a share of
+each tile's shared accumulator columns and arrive on acc_empty; the last tile
+after mma_done), epilogue warps (acc_full -> acc_empty), and the producers'
+tail waits before exit.  A CTA pair runs the same protocol with both CTAs'
+arrivals counted on the leader's barriers, which only scales the counts.
+The abort paths (a bounded wait running out) are not modelled.
 
 The planted variants re-create three mistakes this protocol rules out and
 must be caught: the scale warps' last-tile wait as a parity wait on acc_full
@@ -61,10 +64,16 @@ def until(cond):
     return ("until", cond)
 
 
-def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_wait="mma_done",
+SF_GROUP = 2  # stages per scale-tile copy
+
+
+def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, groups=3, last_wait="mma_done",
                  in_order_waits=False, help_before_wait=True):
     rng = random.Random(seed)
     G = T * num_kt  # stages this CTA walks
+    U = T * -(-num_kt // SF_GROUP)  # scale-tile groups (a group never spans two tiles)
+    sfload = [Bar(1) for _ in range(groups)]
+    sfree = [Bar(n_scale) for _ in range(groups)]
     full = [Bar(1) for _ in range(stages)]
     empty = [Bar(1) for _ in range(stages)]
     sf_full = [Bar(n_scale) for _ in range(slots)]
@@ -78,6 +87,15 @@ def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_
         for g in range(G):
             yield wait(empty[g % stages], g // stages - 1, "producer empty")
             full[g % stages].arrive()  # the TMA fill completing
+        for u in range(max(0, G - stages), G):  # no exit with copies in flight
+            yield wait(full[u % stages], u // stages, "producer tail full")
+
+    def sf_producer():
+        for u in range(U):
+            yield wait(sfree[u % groups], u // groups - 1, "sf producer sfree")
+            sfload[u % groups].arrive()
+        for u in range(max(0, U - groups), U):
+            yield wait(sfload[u % groups], u // groups, "sf producer tail sfload")
 
     def gate():
         for g in range(G):
@@ -106,7 +124,11 @@ def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_
 
     def scale_warp():
         help_next = 0
+        u = 0  # scale-tile groups consumed
         for g in range(G):
+            kt = g % num_kt
+            if kt % SF_GROUP == 0:
+                yield wait(sfload[u % groups], u // groups, "scale sfload")
             if g >= slots:
                 # before_wait(kg): drain shared columns of every tile whose
                 # release the awaited stage's MMAs may need
@@ -119,6 +141,9 @@ def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_
                 if help_before_wait:
                     yield wait(empty[(g - slots) % stages], (g - slots) // stages, "scale empty")
             sf_full[g % slots].arrive()
+            if kt % SF_GROUP == SF_GROUP - 1 or kt == num_kt - 1:
+                sfree[u % groups].arrive()
+                u += 1
         while gelu and help_next < T - 1:
             yield wait(acc_full[help_next & 1], help_next // 2, "help acc_full")
             acc_empty.arrive()
@@ -132,7 +157,7 @@ def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_
             else:
                 yield wait(acc_full[(T - 1) & 1], (T - 1) // 2, "last-tile acc_full")
 
-    actors = [producer(), gate(), mma()] + [epilogue() for _ in range(n_epi)] + \
+    actors = [producer(), sf_producer(), gate(), mma()] + [epilogue() for _ in range(n_epi)] + \
              [scale_warp() for _ in range(n_scale)]
     pending = {}
     for a in actors:
@@ -164,6 +189,7 @@ def run_protocol(T, num_kt, stages, slots, gelu, seed, n_epi=2, n_scale=2, last_
 
 # STAGES >= slots, as the kernels assert; num_kt from one stage up to past the
 # slot count; 1 to 5 tiles per CTA (both accumulators, the last-tile split)
+# and 2 to 4 scale-tile groups in flight
 CASES = [(T, kt, s, sl, gelu) for T, kt, (s, sl), gelu in
          itertools.product([1, 2, 3, 5], [1, 2, 3, 7], [(4, 4), (5, 4), (6, 6)], [False, True])]
 
@@ -171,7 +197,7 @@ CASES = [(T, kt, s, sl, gelu) for T, kt, (s, sl), gelu in
 @pytest.mark.parametrize("T,num_kt,stages,slots,gelu", CASES)
 def test_protocol_has_no_deadlock_or_phase_alias(T, num_kt, stages, slots, gelu):
     for seed in range(12):
-        run_protocol(T, num_kt, stages, slots, gelu, seed)
+        run_protocol(T, num_kt, stages, slots, gelu, seed, groups=2 + seed % 3)
 
 
 def _caught(gelu=False, **kw):
