@@ -697,11 +697,102 @@ def traffic_bytes(workload_key: str, kernel: str):
 
 
 def gemm_kernel_name(fmt: int, M: int, N: int) -> str:
-    """The GEMM kernel mx_gemm dispatches to for this shape."""
+    """The GEMM kernel mx_gemm dispatches to for this shape (both operands in
+    format fmt), named as ncu shows it: CTA pairs for M > 128 and N > 128 (5
+    stages for the FP4 kinds, 6 otherwise; MXFP6 runs on the run-time-typed
+    kernel, template format 4), else one CTA with 128-wide N tiles for
+    N <= 128, 32-row A tiles and 5 stages for M <= 32, 128 x 256 tiles
+    otherwise."""
     if M > 128 and N > 128:
-        return f"gemm_pair_kernel<{fmt}, {6 if fmt < 2 else 5}>"
-    return f"gemm_kernel<{fmt}, {128 if N <= 128 else 256}, 4>"
+        return f"gemm_pair_kernel<{fmt}, {5 if fmt in (2, 3) else 6}>"
+    if N <= 128:
+        return f"gemm_kernel<{fmt}, 128, 4, 128>"
+    if M <= 32:
+        return f"gemm_kernel<{fmt}, 256, 5, 32>"
+    return f"gemm_kernel<{fmt}, 256, 4, 128>"
+
+
+def gemm_bytes(fmt: int, M: int, N: int, K: int) -> int:
+    """Algorithmic bytes of one GEMM launch: A and B codes and scales read
+    once, C (bf16) written once."""
+    from fp8_quantization_block_b200 import mx
+    return (mx.mx_codes_bytes(fmt, M, K) + mx.mx_scales_bytes(fmt, M, K) + mx.mx_codes_bytes(fmt, N, K)
+            + mx.mx_scales_bytes(fmt, N, K) + 2 * M * N)
+
+
+def gemm_roofline(fmt: int, M: int, N: int, K: int, gemm_ms: float, peaks: dict, tpeak: float,
+                  tpeak_burst: float) -> dict:
+    """The roofline object of the GEMM: tensor-bound when its arithmetic
+    intensity (FLOPs per algorithmic byte) is above the ridge of the tensor
+    peak over the measured HBM bandwidth, HBM-bound below it (the skinny
+    weight-streaming shapes), each against its own measured peak."""
+    flops = 2.0 * M * N * K
+    nbytes = gemm_bytes(fmt, M, N, K)
+    tf = flops / (gemm_ms * 1e-3) / 1e12
+    gbs = nbytes / (gemm_ms * 1e-3) / 1e9
+    ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / nbytes >= ridge:
+        return {"bound": "tensor", "achieved": round(tf, 1), "peak": round(tpeak, 1), "unit": "TFLOP/s",
+                "frac": round(tf / tpeak, 4), "frac_of_burst_peak": round(tf / tpeak_burst, 4),
+                "frac_of_page_spec": round(tf / SPEC["fp8_tflops" if fmt < 2 else "fp4_tflops"], 4)}
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes,
+            "tensor_TFLOP/s": round(tf, 1), "frac_of_tensor_peak": round(tf / tpeak, 4)}
 FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4", 4: "mxfp6_e3m2", 5: "mxfp4_mbs"}
+
+
+def result_line(args, wl: dict, r: dict, world: int) -> dict:
+    """The JSON line of the GPU arm from run_gpu's measurements r (device
+    times in ms, already the maximum over ranks)."""
+    peaks, peak_src = measured_peaks()
+    fmt, M, N, K = wl["fmt"], wl["M"], wl["N"], wl["K"]
+    flops = 2.0 * M * N * K
+    ms_step = r["ms"] / args.steps
+    value = whole_job_tflops(flops, args.steps, r["ms"], world)
+    g_avg = sum(r["g_ms"]) / len(r["g_ms"])
+    q_avg = sum(r["q_ms"]) / len(r["q_ms"])
+    g_iso = sum(r["g_ms_iso"]) / len(r["g_ms_iso"])
+    q_iso = sum(r["q_ms_iso"]) / len(r["q_ms_iso"])
+    # the GEMM is timed inside a long run (a ~1.5 s load window of the same
+    # steps, then the timed replay) under the 1 kW power cap: its peak is the
+    # sustained figure; the burst one is reported beside it
+    tpeak = tensor_peak(fmt, peaks, sustained=True)
+    tpeak_burst = tensor_peak(fmt, peaks, sustained=False)
+    q_bytes = M * K * quant_bytes_per_elem(fmt)
+    q_gbs = q_bytes / (q_avg * 1e-3) / 1e9
+    e2e_value = whole_job_tflops(flops, args.steps, r["e2e_ms"], world)
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": FMT_NAMES[fmt], "data": "synthetic",
+        "config": {"workload": wl["name"], "format": FMT_NAMES[fmt], "M": M, "N": N, "K": K,
+                   "step": "mx_quantize(X) + mx_gemm(Xq, Wq pre-quantized)",
+                   "timed_as": "one replay of a CUDA graph holding the K steps' launches",
+                   "ms_per_step_eager": round(r["eager_ms"] / args.steps, 4),
+                   "l2": f"inputs larger than L2: {r['n_sets']} rotating input sets x {r['per_set'] / 2**20:.1f} MB",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": gemm_kernel_name(fmt, M, N),
+                     **gemm_roofline(fmt, M, N, K, g_avg, peaks, tpeak, tpeak_burst),
+                     "traffic": traffic_bytes(args.workload, gemm_kernel_name(fmt, M, N)),
+                     "peak_source": f"{peak_src} sustained bf16 x {2 if fmt < 2 else 4} (nominal dtype ratio) "
+                                    f"for the tensor bound; {peak_src} copy bandwidth for the HBM bound",
+                     "kernel_us": round(g_avg * 1e3, 2),
+                     "kernel_us_isolated": round(g_iso * 1e3, 2),
+                     "timing": "CUDA events on the launching stream around one graph replay of the K launches of "
+                               "this kernel alone (the timed steps' inputs, back to back), right after the timed "
+                               "replay; kernel_us_isolated: events around each launch of a further eager pass"},
+        "quantize": {"kernel": f"quantize_kernel<{FMT_NAMES[fmt]}>", "us": round(q_avg * 1e3, 2),
+                     "us_isolated": round(q_iso * 1e3, 2),
+                     "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
+                     "bytes_per_elem": quant_bytes_per_elem(fmt)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_gemm_fused_act -> D2H C, upload / compute / download on three "
+                        "streams with double buffers (consecutive steps overlap)"},
+        # per step: the quantize and the GEMM; NVFP4 without a given g adds the
+        # amax pre-pass and the kernel that turns the amax into g
+        "gpu_launches": (4 if fmt == 3 else 2) * args.steps,
+        "clocks": r["clocks"],
+    }
 
 
 def main():
@@ -747,57 +838,7 @@ def main():
         torch.distributed.barrier()
 
     r = run_gpu(args, wl, rank, world, device)
-    peaks, peak_src = measured_peaks()
-    fmt, M, N, K = wl["fmt"], wl["M"], wl["N"], wl["K"]
-    flops = 2.0 * M * N * K
-    ms_step = r["ms"] / args.steps
-    value = whole_job_tflops(flops, args.steps, r["ms"], world)
-    g_avg = sum(r["g_ms"]) / len(r["g_ms"])
-    q_avg = sum(r["q_ms"]) / len(r["q_ms"])
-    g_iso = sum(r["g_ms_iso"]) / len(r["g_ms_iso"])
-    q_iso = sum(r["q_ms_iso"]) / len(r["q_ms_iso"])
-    g_tf = flops / (g_avg * 1e-3) / 1e12
-    # the GEMM is timed inside a long run (a ~1.5 s load window of the same
-    # steps, then the timed replay) under the 1 kW power cap: its peak is the
-    # sustained figure; the burst one is reported beside it
-    tpeak = tensor_peak(fmt, peaks, sustained=True)
-    tpeak_burst = tensor_peak(fmt, peaks, sustained=False)
-    q_bytes = M * K * quant_bytes_per_elem(fmt)
-    q_gbs = q_bytes / (q_avg * 1e-3) / 1e9
-    e2e_value = whole_job_tflops(flops, args.steps, r["e2e_ms"], world)
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": FMT_NAMES[fmt], "data": "synthetic",
-        "config": {"workload": wl["name"], "format": FMT_NAMES[fmt], "M": M, "N": N, "K": K,
-                   "step": "mx_quantize(X) + mx_gemm(Xq, Wq pre-quantized)",
-                   "timed_as": "one replay of a CUDA graph holding the K steps' launches",
-                   "ms_per_step_eager": round(r["eager_ms"] / args.steps, 4),
-                   "l2": f"inputs larger than L2: {r['n_sets']} rotating input sets x {r['per_set'] / 2**20:.1f} MB",
-                   "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": gemm_kernel_name(fmt, M, N), "achieved": round(g_tf, 1),
-                     "peak": round(tpeak, 1), "unit": "TFLOP/s", "frac": round(g_tf / tpeak, 4),
-                     "traffic": traffic_bytes(args.workload, gemm_kernel_name(fmt, M, N)),
-                     "peak_source": f"{peak_src} sustained bf16 x {2 if fmt < 2 else 4} (nominal dtype ratio)",
-                     "frac_of_burst_peak": round(g_tf / tpeak_burst, 4),
-                     "frac_of_page_spec": round(g_tf / SPEC["fp8_tflops" if fmt < 2 else "fp4_tflops"], 4),
-                     "kernel_us": round(g_avg * 1e3, 2),
-                     "kernel_us_isolated": round(g_iso * 1e3, 2),
-                     "timing": "CUDA events on the launching stream around one graph replay of the K launches of "
-                               "this kernel alone (the timed steps' inputs, back to back), right after the timed "
-                               "replay; kernel_us_isolated: events around each launch of a further eager pass"},
-        "quantize": {"kernel": f"quantize_kernel<{FMT_NAMES[fmt]}>", "us": round(q_avg * 1e3, 2),
-                     "us_isolated": round(q_iso * 1e3, 2),
-                     "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
-                     "bytes_per_elem": quant_bytes_per_elem(fmt)},
-        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
-                "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_gemm_fused_act -> D2H C, upload / compute / download on three "
-                        "streams with double buffers (consecutive steps overlap)"},
-        # per step: the quantize and the GEMM; NVFP4 without a given g adds the
-        # amax pre-pass and the kernel that turns the amax into g
-        "gpu_launches": (4 if fmt == 3 else 2) * args.steps,
-        "clocks": r["clocks"],
-    }
+    line = result_line(args, wl, r, world)
     if rank == 0 and world == 1 and not args.no_extras:
         line["extras"] = extras_gpu(device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -1,0 +1,112 @@
+"""Host-side helpers of bench.py, on the CPU: the kernel each GEMM shape runs
+(named as the built library's kernel symbols), and the roofline object that
+picks the tensor or the HBM bound by arithmetic intensity."""
+import importlib.util
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PEAKS = {"hbm_gbs": 6537.3, "bf16_tflops": 1647.8, "bf16_tflops_sustained": 1379.4}
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.fixture(scope="module")
+def kernel_symbols():
+    from fp8_quantization_block_b200 import build
+    lib = build.build()
+    if shutil.which("nm") is None:
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-C", lib], capture_output=True, text=True, check=True).stdout
+    names = set()
+    for line in out.splitlines():
+        for kind in ("gemm_pair_kernel<", "gemm_kernel<"):
+            i = line.find("mx::" + kind)
+            if i >= 0:
+                j = line.index(">", i)
+                names.add(line[i + 4:j + 1])
+    return names
+
+
+SHAPES = [(4096, 3072), (4608, 12288), (16, 28672), (1, 300), (32, 257), (33, 4096), (128, 28672),
+          (300, 100), (129, 129), (128, 129)]
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3, 4])
+def test_kernel_names_are_built_kernels(bench, kernel_symbols, fmt):
+    for M, N in SHAPES:
+        assert bench.gemm_kernel_name(fmt, M, N) in kernel_symbols, (fmt, M, N, sorted(kernel_symbols))
+
+
+def test_kernel_choice_by_shape(bench):
+    assert bench.gemm_kernel_name(0, 4096, 3072) == "gemm_pair_kernel<0, 6>"
+    assert bench.gemm_kernel_name(3, 4608, 12288) == "gemm_pair_kernel<3, 5>"
+    assert bench.gemm_kernel_name(4, 4096, 3072) == "gemm_pair_kernel<4, 6>"
+    assert bench.gemm_kernel_name(3, 16, 28672) == "gemm_kernel<3, 256, 5, 32>"
+    assert bench.gemm_kernel_name(3, 128, 28672) == "gemm_kernel<3, 256, 4, 128>"
+    assert bench.gemm_kernel_name(2, 300, 100) == "gemm_kernel<2, 128, 4, 128>"
+
+
+def test_roofline_bound_follows_arithmetic_intensity(bench):
+    # DiT MXFP8 GEMM: ~1600 FLOP per algorithmic byte, far above the ridge
+    tp, tb = bench.tensor_peak(0, PEAKS, True), bench.tensor_peak(0, PEAKS, False)
+    r = bench.gemm_roofline(0, 4096, 3072, 3072, 0.04, PEAKS, tp, tb)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(2 * 4096 * 3072 * 3072 / 0.04e-3 / 1e12, rel=1e-3)
+    assert r["frac"] == pytest.approx(r["achieved"] / tp, rel=1e-3)
+    # skinny NVFP4 weight stream: ~32 FLOP per byte, below the ridge
+    tp, tb = bench.tensor_peak(3, PEAKS, True), bench.tensor_peak(3, PEAKS, False)
+    r = bench.gemm_roofline(3, 16, 28672, 8192, 0.025, PEAKS, tp, tb)
+    nbytes = bench.gemm_bytes(3, 16, 28672, 8192)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["algorithmic_bytes"] == nbytes
+    # W: 28672 x 8192 codes at 4 bits plus one E4M3 scale per 16 (padded tiles), X and C small
+    assert nbytes == 28672 * 8192 // 2 + 28672 * 8192 // 16 + 128 * 8192 // 16 + 16 * 8192 // 2 + 2 * 16 * 28672
+    assert r["achieved"] == pytest.approx(nbytes / 0.025e-3 / 1e9, rel=1e-3)
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["hbm_gbs"], rel=1e-3)
+
+
+def test_result_line_keeps_the_contract(bench):
+    """The GPU arm's JSON line built from fake device times: every key of the
+    contract, whole-job value = world x per-replica work / slowest time, the
+    roofline object of the dominant kernel, e2e with the copy bytes."""
+    import argparse
+    args = argparse.Namespace(steps=50, warmup=5, workload="dit_mxfp8")
+    wl = bench.WORKLOADS["dit_mxfp8"]
+    r = {"ms": 50 * 0.049, "g_ms": [0.0405] * 50, "q_ms": [0.0085] * 50, "g_ms_iso": [0.044] * 50,
+         "q_ms_iso": [0.009] * 50, "e2e_ms": 50 * 0.55, "eager_ms": 50 * 0.048, "n_sets": 6,
+         "per_set": 73_000_000, "h2d": 4096 * 3072 * 2, "d2h": 4096 * 3072 * 2,
+         "clocks": {"sm_mhz": 1762.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}}
+    for world in (1, 2):
+        line = bench.result_line(args, wl, r, world)
+        for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                  "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+            assert k in line, k
+        flops = 2.0 * 4096 * 3072 * 3072
+        assert line["n_gpus"] == world and line["steps"] == 50 and line["scaling"] == "weak"
+        assert line["value"] == pytest.approx(world * flops * 50 / (r["ms"] * 1e-3) / 1e12, rel=1e-3)
+        assert line["higher_is_better"] is True and line["vs_baseline"] is None
+        assert line["config"]["workload"] == wl["name"]
+        roof = line["roofline"]
+        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6>"
+        assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"], rel=1e-3)
+        assert "traffic" in roof
+        assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
+        assert line["e2e"]["h2d_bytes_per_step"] == r["h2d"]
+        assert line["gpu_launches"] == 2 * 50
+    # the skinny workload's GEMM is reported against HBM
+    args.workload = "skinny_nvfp4"
+    line = bench.result_line(args, bench.WORKLOADS["skinny_nvfp4"], dict(r, g_ms=[0.025] * 50), 1)
+    assert line["roofline"]["bound"] == "hbm" and line["roofline"]["unit"] == "GB/s"
+    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32>"
+    assert line["gpu_launches"] == 4 * 50
+    json_line = __import__("json").dumps(line)
+    assert "\n" not in json_line
