@@ -33,6 +33,21 @@ def test_every_declared_symbol_is_exported(L):
     assert set(names) == set(mx.EXPORTED)
 
 
+def test_header_constants_match_the_binding():
+    """Every enumerator (and the scratch-size macro) that include/mx.h
+    declares has the same value in the Python binding."""
+    src = open(os.path.join(ROOT, "include", "mx.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    consts = {}
+    for body in re.findall(r"typedef\s+enum\s*\{(.*?)\}", src, flags=re.S):
+        for name, value in re.findall(r"\b(MX_[A-Z0-9_]+)\s*=\s*(\d+)", body):
+            consts[name] = int(value)
+    assert len(consts) >= 20
+    for name, value in consts.items():
+        assert getattr(mx, name) == value, name
+    assert mx.MX_NOALLOC_SCRATCH_BYTES == 4 << 20 and "((size_t)4 << 20)" in src
+
+
 def test_sizes_match_layout(L):
     assert mx.mx_codes_bytes(mx.MX_MXFP8_E4M3, 3, 64) == 192
     assert mx.mx_codes_bytes(mx.MX_NVFP4, 3, 64) == 96
