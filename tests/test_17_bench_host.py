@@ -58,14 +58,27 @@ def test_kernel_choice_by_shape(bench):
 
 def test_roofline_bound_follows_arithmetic_intensity(bench):
     # DiT MXFP8 GEMM: ~1600 FLOP per algorithmic byte, far above the ridge
-    tp, tb = bench.tensor_peak(0, PEAKS, True), bench.tensor_peak(0, PEAKS, False)
-    r = bench.gemm_roofline(0, 4096, 3072, 3072, 0.04, PEAKS, tp, tb)
+    ts, tb = bench.tensor_peak(0, PEAKS, True), bench.tensor_peak(0, PEAKS, False)
+    assert tb == pytest.approx(2 * 1647.8) and ts == pytest.approx(2 * 1379.4)
+    clocks = {"sm_mhz": 1710.0, "sm_max_mhz": 1965.0}
+    r = bench.gemm_roofline(0, 4096, 3072, 3072, 0.0397, PEAKS, tb, ts, clocks)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
-    assert r["achieved"] == pytest.approx(2 * 4096 * 3072 * 3072 / 0.04e-3 / 1e12, rel=1e-3)
-    assert r["frac"] == pytest.approx(r["achieved"] / tp, rel=1e-3)
+    flops = 2 * 4096 * 3072 * 3072
+    assert r["achieved"] == pytest.approx(flops / 0.0397e-3 / 1e12, rel=1e-3)
+    # the headline fraction is against the burst peak (the kernel is timed as a
+    # short graph replay): 77.31 GFLOP / 39.7 us / (2 x 1647.8) = 0.59
+    assert r["peak"] == pytest.approx(tb, rel=1e-3)
+    assert r["frac"] == pytest.approx(flops / 0.0397e-3 / 1e12 / (2 * 1647.8), rel=1e-3)
+    assert r["frac"] == pytest.approx(0.591, abs=2e-3)
+    assert r["frac_of_sustained_peak"] == pytest.approx(r["achieved"] / ts, rel=1e-3)
+    # clock-normalised: 39.7 us x 1710 / 1965 = 34.55 us
+    assert r["clock_normalised_kernel_us"] == pytest.approx(39.7 * 1710 / 1965, abs=0.01)
+    assert r["clock_normalised_frac"] == pytest.approx(flops / (39.7e-6 * 1710 / 1965) / 1e12 / tb, rel=1e-3)
+    # without clock samples there is no clock-normalised figure
+    assert "clock_normalised_frac" not in bench.gemm_roofline(0, 4096, 3072, 3072, 0.0397, PEAKS, tb, ts, None)
     # skinny NVFP4 weight stream: ~32 FLOP per byte, below the ridge
-    tp, tb = bench.tensor_peak(3, PEAKS, True), bench.tensor_peak(3, PEAKS, False)
-    r = bench.gemm_roofline(3, 16, 28672, 8192, 0.025, PEAKS, tp, tb)
+    ts, tb = bench.tensor_peak(3, PEAKS, True), bench.tensor_peak(3, PEAKS, False)
+    r = bench.gemm_roofline(3, 16, 28672, 8192, 0.025, PEAKS, tb, ts, clocks)
     nbytes = bench.gemm_bytes(3, 16, 28672, 8192)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["algorithmic_bytes"] == nbytes
     # W: 28672 x 8192 codes at 4 bits plus one E4M3 scale per 16 (padded tiles), X and C small
@@ -98,6 +111,8 @@ def test_result_line_keeps_the_contract(bench):
         roof = line["roofline"]
         assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6>"
         assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"], rel=1e-3)
+        assert roof["peak"] == pytest.approx(bench.tensor_peak(0, bench.measured_peaks()[0], False), rel=1e-3)
+        assert roof["clock_normalised_kernel_us"] == pytest.approx(40.5 * 1762 / 1965, abs=0.01)
         assert "traffic" in roof
         assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
         assert line["e2e"]["h2d_bytes_per_step"] == r["h2d"]
@@ -110,3 +125,13 @@ def test_result_line_keeps_the_contract(bench):
     assert line["gpu_launches"] == 4 * 50
     json_line = __import__("json").dumps(line)
     assert "\n" not in json_line
+
+
+def test_extras_get_clock_normalised_fractions(bench):
+    ex = {"mlp_nvfp4_gemm1": {"us": 81.5, "frac_tensor": 0.647}, "quantize_sweep": {"x": {"frac_hbm": 0.8}}}
+    bench.add_clock_normalised(ex, {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0})
+    assert ex["mlp_nvfp4_gemm1"]["clock_normalised_frac_tensor"] == pytest.approx(0.647 * 1965 / 1700, abs=1e-3)
+    assert "clock_normalised_frac_tensor" not in ex["quantize_sweep"]
+    ex2 = {"g": {"frac_tensor": 0.5}}
+    bench.add_clock_normalised(ex2, {"sm_mhz": None, "sm_max_mhz": None})
+    assert "clock_normalised_frac_tensor" not in ex2["g"]
