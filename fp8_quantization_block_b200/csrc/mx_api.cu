@@ -755,6 +755,9 @@ mx_status mx_gemm_fused_act_noalloc(int fmt, const void *X_bf16, int64_t M, int6
                                     const mx_tensor *W, void *C_bf16, int64_t ldc, int epilogue, float *amax_out,
                                     const float *x_gscale, const float *x_amax, void *stream) {
     if (!valid_fmt(fmt) || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    // sizes the fused call rejects anyway, checked first so that the byte
+    // count below cannot overflow
+    if (M > INT32_MAX || K > INT32_MAX || cdiv(M, kBM) > 65535) return MX_ERR_UNSUPPORTED_SHAPE;
     if (fused_ws_bytes(fmt, M, K) > MX_NOALLOC_SCRATCH_BYTES) return MX_ERR_UNSUPPORTED_SHAPE;
     void *scratch = nullptr;
     const mx_status s = noalloc_scratch(&scratch);

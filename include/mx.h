@@ -188,7 +188,12 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
 /* Epilogues of the fused call. */
 typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
 
-/* Fused activation-quantize + GEMM: X is bf16 [M x K] (row pitch ldx), W a
+/* Fused activation-quantize + GEMM ([IMPL] section "Implementação da
+ * quantização NVFP4 e MXFP8": a Linear layer with both its activations and its
+ * weights quantized, and section "Desafios e soluções na implementação": the
+ * activation quantize as the bottleneck on small tensors; [MX] FAQ entry on
+ * applying microscaling to activations as well as weights).
+ * X is bf16 [M x K] (row pitch ldx), W a
  * pre-quantized [N x K] mx_tensor; X is quantized to format fmt, and W's format
  * is fmt or, as in mx_gemm, any MX format that pairs with it (e.g. MXFP8
  * activations with MXFP4 or MXFP6 weights).  X is quantized exactly as
@@ -221,11 +226,11 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
 size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K);
 
 /* mx_gemm_fused_act without a workspace argument, for callers that cannot
- * allocate device memory: code running while a stream is being captured or
- * inside an engine's enqueue/plugin callback where allocation is forbidden,
+ * allocate device memory: code inside an inference engine's enqueue or plugin
+ * callback, where the engine owns all memory and forbids allocation;
  * latency-critical paths that must not pay for cudaMalloc's implicit device
- * synchronization, and runtimes with a fixed memory budget.  The pages have no
- * counterpart to this call; it exists for those callers only.
+ * synchronization; and runtimes that run under a fixed memory budget.  The
+ * pages have no counterpart to this call; it exists for those callers only.
  *   Scratch: a fixed array of MX_NOALLOC_SCRATCH_BYTES inside libmx.so itself,
  *   one per GPU that loads the library, kept until the process exits.  The
  *   call allocates nothing (no cudaMalloc, cudaFree or allocating library

@@ -374,6 +374,21 @@ def test_gelu_against_normal_cdf():
     assert np.allclose(y - oracle.gelu(-x), x, rtol=0, atol=1e-14)      # GELU(x) - GELU(-x) = x
 
 
+def test_gelu_lipschitz_constant_of_the_fused_tolerance():
+    """The fused GEMM tests bound GELU's error by 1.13 x the GEMM bound: the
+    largest |GELU'| is Phi(sqrt 2) + sqrt 2 phi(sqrt 2) = 1.128904, below 1.13.
+    Checked on the oracle's GELU by central differences on a fine grid."""
+    from scipy.special import ndtr
+    x = np.linspace(-10, 10, 400001)
+    h = 1e-6
+    d = (oracle.gelu(x + h) - oracle.gelu(x - h)) / (2 * h)
+    s2 = np.sqrt(2.0)
+    closed = ndtr(s2) + s2 * np.exp(-1.0) / np.sqrt(2 * np.pi)
+    assert closed == pytest.approx(1.128904, abs=1e-6)
+    assert np.max(np.abs(d)) == pytest.approx(closed, abs=1e-6)
+    assert np.max(np.abs(d)) < 1.13
+
+
 def test_ridge_point_arithmetic(facts):
     r = facts["roofline_ridge"]
     assert r["fp4_dense_tflops"] * 1e12 / (r["hbm_gbs"] * 1e9) == r["ridge_flop_per_byte"]

@@ -1,12 +1,18 @@
 """mx_gemm_fused_act_noalloc: the fused quantize + GEMM for callers that cannot
-allocate device memory (for example while a stream is being captured, inside an
-inference engine's plugin callback, or under a fixed memory budget).  It uses a
-fixed scratch array inside the library instead of a caller workspace.
+allocate device memory (for example code inside an inference engine's plugin
+callback, where the engine owns all memory, or a runtime under a fixed memory
+budget).  It uses a fixed scratch array inside the library instead of a caller
+workspace.
 
 Checked through the C ABI against the workspace-taking mx_gemm_fused_act on the
 same inputs, on two calls in a row (the second call reuses the scratch the
 first one left behind), and against the fp64 oracle's tolerance.  This file is
-collected last and also runs on its own in a fresh process."""
+collected last; one test also makes the call first thing in a fresh process
+(where the first call looks up the scratch array's device address)."""
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -74,18 +80,68 @@ def test_noalloc_epilogue_and_amax_chain():
     assert float(a1.cpu()[0]) == float(a2.cpu()[0])
 
 
-def test_noalloc_rejects_shapes_beyond_its_scratch():
-    fmt, K = 0, 4096
-    M = mx.MX_NOALLOC_SCRATCH_BYTES // K + 128       # codes alone exceed the scratch
-    assert mx.mx_fused_workspace_bytes(fmt, M, K) > mx.MX_NOALLOC_SCRATCH_BYTES
-    W = mx.quantize(torch.zeros((64, K), dtype=torch.bfloat16, device="cuda"), fmt)
-    s = mx.mx_gemm_fused_act_noalloc(fmt, 0x1000, M, K, K, W.c(), 0x2000, 64, 0, None, None, None, None)
+def _largest_accepted_rows(fmt: int, K: int) -> int:
+    """The largest M whose fused workspace fits the scratch array (the size is
+    non-decreasing in M, so M + 1 is the smallest rejected shape)."""
+    lo, hi = 0, mx.MX_NOALLOC_SCRATCH_BYTES    # fits at lo, not at hi
+    assert mx.mx_fused_workspace_bytes(fmt, hi, K) > mx.MX_NOALLOC_SCRATCH_BYTES
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if mx.mx_fused_workspace_bytes(fmt, mid, K) <= mx.MX_NOALLOC_SCRATCH_BYTES:
+            lo = mid
+        else:
+            hi = mid
+    return lo
+
+
+@pytest.mark.parametrize("fmt", [0, 2, 3])
+def test_noalloc_largest_shape_runs_and_the_next_is_rejected(fmt):
+    K, N = 4096, 256
+    M = _largest_accepted_rows(fmt, K)
+    assert M > 128
+    W = mx.quantize(synth.bits_to_tensor(synth.gaussian_weights(914 + fmt, N, K)).cuda(), fmt)
+    # one row more: rejected on the host before any launch (the pointers are never used)
+    s = mx.mx_gemm_fused_act_noalloc(fmt, 0x1000, M + 1, K, K, W.c(), 0x2000, N, 0, None, None, None, None)
     assert s == mx.MX_ERR_UNSUPPORTED_SHAPE
-    # the largest accepted shape runs
-    M_ok = 256
-    assert mx.mx_fused_workspace_bytes(fmt, M_ok, K) <= mx.MX_NOALLOC_SCRATCH_BYTES
-    X = synth.bits_to_tensor(synth.sweep_tensor(913, M_ok, K)).cuda()
+    # sizes whose byte count would overflow are rejected too
+    for big_m, big_k in ((1 << 40, K), (256, 1 << 40), ((1 << 62) // 4096, 4096)):
+        s = mx.mx_gemm_fused_act_noalloc(fmt, 0x1000, big_m, big_k, big_k, W.c(), 0x2000, N, 0, None, None, None,
+                                         None)
+        assert s in (mx.MX_ERR_UNSUPPORTED_SHAPE, mx.MX_ERR_INVALID_ARG)
+    # the largest accepted shape fills the array to its end: bit for bit the workspace entry
+    X = synth.bits_to_tensor(synth.sweep_tensor(913 + fmt, M, K)).cuda()
     got = _noalloc(X, W)
     want = mx.gemm_fused_act(X, W)
     torch.cuda.synchronize()
+    mx.check_device_error()
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+_FRESH = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from fp8_quantization_block_b200 import mx, synth
+fmt, M, N, K = 0, 200, 384, 512
+W = mx.quantize(synth.bits_to_tensor(synth.gaussian_weights(920, N, K)).cuda(), fmt)
+X = synth.bits_to_tensor(synth.student_t(921, M, K)).cuda()
+outs = []
+for _ in range(2):
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    s = mx.mx_gemm_fused_act_noalloc(fmt, X.data_ptr(), M, K, K, W.c(), out.data_ptr(), N, 0, None, None, None,
+                                     torch.cuda.current_stream().cuda_stream)
+    mx.check(s, "mx_gemm_fused_act_noalloc")
+    outs.append(out)
+want = mx.gemm_fused_act(X, W)
+torch.cuda.synchronize()
+mx.check_device_error()
+for o in outs:
+    assert torch.equal(o.view(torch.int16), want.view(torch.int16))
+print("fresh-process noalloc ok")
+"""
+
+
+def test_noalloc_first_call_in_a_fresh_process():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FRESH, root], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "fresh-process noalloc ok" in r.stdout
