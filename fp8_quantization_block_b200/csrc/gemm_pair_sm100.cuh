@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                      const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = PairSmem<FMT, STAGES>;
+    static_assert(sizeof(FusedQuantSmem) <= L::kEpiAreaBytes, "fused quantize scratch in the staging buffers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);  // leader's count both CTAs' code tiles
@@ -103,11 +104,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int used = 0, s = 0;
             uint32_t ph = 0;
             bool stop = false;
+            int ready_band = -1;   // fused quantize: the last A band known to be written
             for (int tile = pair; tile < num_tiles && !stop; tile += npairs) {
                 int m0, n0;
-                tile_coords(tile, p.m_blocks, m0, n0, 256);
-                m0 = (tile % p.m_blocks) * 256;
+                tile_coords(p, tile, m0, n0, 256, 256);
                 const int my_m = m0 + 128 * (int)rank, my_n = n0 + 128 * (int)rank;
+                if (p.fused && my_m / 128 != ready_band) {
+                    if (!wait_band_ready(p, my_m / 128, lane, abort_flag)) break;
+                    ready_band = my_m / 128;
+                }
                 for (int kt = 0; kt < p.num_kt; ++kt) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY, abort_flag)) {
                         stop = true;
@@ -144,8 +149,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, pair, npairs, num_tiles,
                                 [&](int tile, int &a_band, int &b_band) {
                                     int m0, n0;
-                                    tile_coords(tile, p.m_blocks, m0, n0, 256);
-                                    a_band = (tile % p.m_blocks) * 2 + (int)rank;
+                                    tile_coords(p, tile, m0, n0, 256, 256);
+                                    a_band = m0 / 128 + (int)rank;
                                     b_band = n0 / 128;
                                 },
                                 lane, abort_flag);
@@ -224,11 +229,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int my_tiles = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
         float scale = 1.0f;
-        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         uint32_t amax = 0;
         auto rows_of = [&](int t, int &m0, int &n0) {
-            tile_coords(pair + t * npairs, p.m_blocks, m0, n0, 256);
-            m0 = ((pair + t * npairs) % p.m_blocks) * 256 + 128 * (int)rank;
+            tile_coords(p, pair + t * npairs, m0, n0, 256, 256);
+            m0 += 128 * (int)rank;
         };
         // GELU: this warp's share of the shared columns of tile t (all but the
         // last tile), drained before the first wait on a stage of tile t + 1 or
@@ -285,17 +290,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         epilogue_finish(p, lane, amax);
     } else {
         // ------------------------------------------------------------ epilogue (this CTA's 128 rows)
+        // (fused: first the activation quantize, in the staging buffers' space)
+        if (p.fused) fused_quantize_role<FMT>(p, reinterpret_cast<FusedQuantSmem *>(smem + L::kOffEpi), threadIdx.x - 64);
         const int q = warp & 3;
         uint8_t *bufs = smem + L::kOffEpi + (warp - 2) * L::kEpiBufs * kEpiChunkBytes;
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
         uint32_t amax = 0, nstore = 0;
         float scale = 1.0f;
-        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         int it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             int m0, n0;
-            tile_coords(tile, p.m_blocks, m0, n0, 256);
-            m0 = (tile % p.m_blocks) * 256 + 128 * (int)rank;
+            tile_coords(p, tile, m0, n0, 256, 256);
+            m0 += 128 * (int)rank;
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();

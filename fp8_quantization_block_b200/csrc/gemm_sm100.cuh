@@ -40,6 +40,7 @@
 #pragma once
 
 #include "mx_common.cuh"
+#include "quantize.cuh"
 
 namespace mx {
 
@@ -110,7 +111,41 @@ struct GemmParams {
                           // barrier (the packed global bytes of FP6 / FP4 boxes, not their
                           // unpacked shared-memory footprint)
     uint64_t wait_limit_ns;
+    int ga_from_amax;     // NVFP4: *ga holds amax(|A|) and gA = RU(amax / 2688) (1 for 0)
+    int band_major;       // tile order: 1 = N fastest (consecutive tiles share A's band), 0 = M fastest
+    // Fused activation quantize (fused != 0): A is the bf16 matrix x [M x K]
+    // (row pitch ldx), quantized to format x_fmt by the epilogue warps of every
+    // CTA before their first tile (fused_quantize_role) into xq_codes /
+    // xq_scales, which the TMA producers then read as A.  Work unit: a 128 x 128
+    // tile of x; next_item hands them out in band-major order, band_ready[b]
+    // counts those of 128-row band b that are written.
+    int fused;
+    int x_fmt;
+    int x_items_k;        // 128-column tiles per band = ceil(K / 128)
+    int x_bands;          // ceil(M / 128)
+    int64_t ldx;
+    int64_t x_sf_tiles_k; // 512-byte scale chunks per band of x's format
+    const uint16_t *x;
+    uint8_t *xq_codes;
+    uint8_t *xq_scales;
+    uint32_t *band_ready;
+    uint32_t *next_item;
 };
+
+// gA of an NVFP4 A operand (the epilogue multiplies by gA * gB).
+MX_DEVICE_INLINE float gemm_ga(const GemmParams &p) { return nv_g_from(p.ga, p.ga_from_amax); }
+
+// Fused quantize: wait until every 128 x 128 tile of A's 128-row band `band`
+// is written (lane 0 polls, the warp learns the outcome); bands past x's end
+// (the second half of a ragged CTA pair's rows) have nothing to wait for.
+MX_DEVICE_INLINE bool wait_band_ready(const GemmParams &p, int band, int lane, volatile int *abort_flag) {
+    bool ok = true;
+    if (band < p.x_bands && lane == 0)
+        ok = wait_global_at_least(p.band_ready + band, (uint32_t)p.x_items_k, p.wait_limit_ns, SITE_FUSED_BAND_READY,
+                                  abort_flag);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 
 // Shared-memory and TMEM plan of a CTA whose MMAs read a 128-row A tile and
 // B_BANDS 128-row bands of B per stage (B_ROWS rows of B in this CTA's smem).
@@ -172,6 +207,7 @@ struct GemmLayout {
     static_assert(kAccStride >= 32, "accumulator double buffering needs TMEM room");
     static_assert(kTmemSf + kSlots * kSfSlotCols <= kTmemCols, "TMEM budget");
     static_assert(STAGES >= kSlots, "scale slots are recycled through the stage barriers");
+    static constexpr int kEpiAreaBytes = kEpiWarps * kEpiBufs * kEpiChunkBytes;
 };
 
 template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
@@ -361,9 +397,17 @@ MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *t
     int used = 0, g = 0;
     uint32_t ph = 0;
     bool stop = false;
+    int ready_band = -1;   // fused quantize: the last A band known to be written
     for (int tile = tile0; tile < num_tiles && !stop; tile += tile_step) {
         int a_band, b_band;
         bands_of(tile, a_band, b_band);
+        if (p.fused && a_band != ready_band) {
+            if (!wait_band_ready(p, a_band, lane, abort_flag)) {
+                stop = true;
+                break;
+            }
+            ready_band = a_band;
+        }
         for (int kt0 = 0; kt0 < p.num_kt; kt0 += kSfGroup) {
             if (!mbar_wait_bounded(&sfree[g], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_SF_FREE, abort_flag)) {
                 stop = true;
@@ -447,9 +491,75 @@ MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *s
     }
 }
 
-MX_DEVICE_INLINE void tile_coords(int tile, int m_blocks, int &m0, int &n0, int bn) {
-    m0 = (tile % m_blocks) * kBM;
-    n0 = (tile / m_blocks) * bn;
+// Origin of output tile `tile` (bm x bn tiles): M-fastest order, or N-fastest
+// (band-major) when the fused quantize produces A band by band.
+MX_DEVICE_INLINE void tile_coords(const GemmParams &p, int tile, int &m0, int &n0, int bm, int bn) {
+    int mb, nb;
+    if (p.band_major) {
+        mb = tile / p.n_blocks;
+        nb = tile - mb * p.n_blocks;
+    } else {
+        mb = tile % p.m_blocks;
+        nb = tile / p.m_blocks;
+    }
+    m0 = mb * bm;
+    n0 = nb * bn;
+}
+
+// Shared memory of the fused quantize, inside the epilogue warps' staging
+// buffers (idle until their first tile): the scale chunks of the tile being
+// quantized, the NVFP4 tables and the claimed work item.
+struct FusedQuantSmem {
+    uint8_t sf[1024];
+    NvTables nvt;
+    uint32_t claim;
+};
+
+// The epilogue warps (t = 0..127) of a CTA: claim 128 x 128 tiles of x from the
+// global counter until none is left, quantize each (quantize_tile: the
+// arithmetic of quantize_kernel, so codes and scales are those of mx_quantize)
+// and count it in its band once written.  Nothing here waits on another CTA,
+// so the tiles get done as long as any CTA of the grid runs.
+template <int XFMT>
+MX_DEVICE_INLINE void fused_quantize_role_t(const GemmParams &p, FusedQuantSmem *fq, int t) {
+    NvScale ns{1.0f, 1.0f, 1.0f, 1.0f, 1.0f};
+    if (XFMT == FMT_NVFP4) {
+        ns = nv_scale_setup(nv_g_from(p.ga, p.ga_from_amax));
+        nv_tables_fill(&fq->nvt, (uint32_t)t);
+    }
+    const uint32_t n_items = (uint32_t)p.x_bands * (uint32_t)p.x_items_k;
+    if (t == 0) fq->claim = atomicAdd(p.next_item, 1u);
+    sync_epilogue_warps();
+    uint32_t cur = fq->claim;
+    while (cur < n_items) {
+        uint32_t nxt = 0;
+        if (t == 0) nxt = atomicAdd(p.next_item, 1u);   // the next claim overlaps this tile
+        const int band = (int)(cur / (uint32_t)p.x_items_k), tx = (int)(cur % (uint32_t)p.x_items_k);
+        quantize_tile<XFMT, 128>(p.x, p.M, p.K, p.ldx, p.xq_codes, p.xq_scales, p.x_sf_tiles_k, band, tx, ns,
+                                 &fq->nvt, fq->sf, t, sync_epilogue_warps);
+        fence_proxy_async_global();   // this thread's stores, before the band count (TMA reads them)
+        if (t == 0) fq->claim = nxt;
+        sync_epilogue_warps();
+        if (t == 0) {
+            __threadfence();
+            red_release_gpu_add(p.band_ready + band, 1u);
+        }
+        cur = fq->claim;
+    }
+}
+
+template <int FMT>
+MX_DEVICE_INLINE void fused_quantize_role(const GemmParams &p, FusedQuantSmem *fq, int t) {
+    if constexpr (FMT == kGemmRuntimeTypes) {
+        switch (p.x_fmt) {
+        case FMT_E4M3: fused_quantize_role_t<FMT_E4M3>(p, fq, t); break;
+        case FMT_E5M2: fused_quantize_role_t<FMT_E5M2>(p, fq, t); break;
+        case FMT_MXFP4: fused_quantize_role_t<FMT_MXFP4>(p, fq, t); break;
+        default: fused_quantize_role_t<FMT_MXFP6>(p, fq, t); break;
+        }
+    } else {
+        fused_quantize_role_t<FMT>(p, fq, t);
+    }
 }
 
 // Gate warp: for every stage of this CTA's tiles, in order, wait for its code
@@ -703,6 +813,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
     using L = GemmSmem<FMT, BN, STAGES, A_ROWS>;
+    static_assert(sizeof(FusedQuantSmem) <= L::kEpiAreaBytes, "fused quantize scratch in the staging buffers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
@@ -764,9 +875,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int used = 0, s = 0;
             uint32_t ph = 0;
             bool stop = false;
+            int ready_band = -1;   // fused quantize: the last A band known to be written
             for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
                 int m0, n0;
-                tile_coords(tile, p.m_blocks, m0, n0, BN);
+                tile_coords(p, tile, m0, n0, kBM, BN);
+                if (p.fused && m0 / kBM != ready_band) {
+                    if (!wait_band_ready(p, m0 / kBM, lane, abort_flag)) break;
+                    ready_band = m0 / kBM;
+                }
                 for (int kt = 0; kt < p.num_kt; ++kt) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY, abort_flag)) {
                         stop = true;
@@ -798,7 +914,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, blockIdx.x, gridDim.x, num_tiles,
                                 [&](int tile, int &a_band, int &b_band) {
                                     int m0, n0;
-                                    tile_coords(tile, p.m_blocks, m0, n0, BN);
+                                    tile_coords(p, tile, m0, n0, kBM, BN);
                                     a_band = m0 / 128;
                                     b_band = n0 / 128;
                                 },
@@ -876,7 +992,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int my_tiles = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
         float scale = 1.0f;
-        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         uint32_t amax = 0;
         // GELU: this warp's share of the shared columns of tile t (all but the
         // last tile), drained before the first wait on a stage of tile t + 1 or
@@ -884,7 +1000,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int help_next = 0;
         auto help = [&](int t) -> bool {
             int m0, n0;
-            tile_coords(blockIdx.x + t * gridDim.x, p.m_blocks, m0, n0, BN);
+            tile_coords(p, blockIdx.x + t * gridDim.x, m0, n0, kBM, BN);
             const int b = t & 1;
             if (!mbar_wait_bounded(&acc_full[b], (t >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag))
                 return false;
@@ -914,7 +1030,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (my_tiles > 0 && !*abort_flag) {
             const int it = my_tiles - 1, b = it & 1;
             int m0, n0;
-            tile_coords(blockIdx.x + it * gridDim.x, p.m_blocks, m0, n0, BN);
+            tile_coords(p, blockIdx.x + it * gridDim.x, m0, n0, kBM, BN);
             // mma_done (one phase) rather than acc_full[b]: without GELU this warp
             // may finish its slots several tiles ahead of the MMAs, and a parity
             // wait on acc_full[b], whose phases alternate every second tile,
@@ -930,15 +1046,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         epilogue_finish(p, lane, amax);
     } else {
         // ------------------------------------------------------------ epilogue
+        // (fused: first the activation quantize, in the staging buffers' space)
+        if (p.fused) fused_quantize_role<FMT>(p, reinterpret_cast<FusedQuantSmem *>(smem + L::kOffEpi), threadIdx.x - 64);
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         uint8_t *bufs = smem + L::kOffEpi + (warp - 2) * L::kEpiBufs * kEpiChunkBytes;
         uint32_t amax = 0, nstore = 0;
         float scale = 1.0f;
-        if (FMT == 3) scale = (*p.ga) * (*p.gb);
+        if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             int m0, n0;
-            tile_coords(tile, p.m_blocks, m0, n0, BN);
+            tile_coords(p, tile, m0, n0, kBM, BN);
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();

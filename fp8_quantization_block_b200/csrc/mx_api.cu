@@ -28,6 +28,7 @@ std::atomic<int> g_skip_producer{0};
 std::atomic<int> g_pair_enabled{1};
 std::atomic<int> g_pdl_enabled{1};
 std::atomic<int> g_max_gemm_ctas{0};  // 0: one CTA (or CTA pair) per SM pair of the device
+std::atomic<int> g_fused_two_kernels{0};  // 1: the fused call runs quantize_kernel, then the GEMM
 
 // Launch attributes shared by the kernels that may overlap the previous kernel
 // in the stream (they call griddep_wait() before reading any input).
@@ -273,9 +274,38 @@ cudaError_t smem_limit_once(const void *fn, int bytes) {
     return e;
 }
 
+// The activation of a fused call: bf16 x quantized inside the GEMM kernel (see
+// GemmParams::fused); A's codes and scales are its destination.
+struct FusedX {
+    const uint16_t *x;
+    int64_t ldx;
+    int x_fmt;
+    int ga_from_amax;
+    uint32_t *band_ready;
+    uint32_t *next_item;
+};
+
+void set_fused(GemmParams &p, const FusedX *fx, const void *a_codes, const uint8_t *a_scales, int64_t M, int64_t K) {
+    if (fx == nullptr) return;
+    p.fused = 1;
+    p.band_major = 1;
+    p.x = fx->x;
+    p.ldx = fx->ldx;
+    p.x_fmt = fx->x_fmt;
+    p.x_items_k = (int)cdiv(K, kQTileCols);
+    p.x_bands = (int)cdiv(M, kQTileRows);
+    p.x_sf_tiles_k = cdiv(K / fmt_block(fx->x_fmt), 4);
+    p.xq_codes = static_cast<uint8_t *>(const_cast<void *>(a_codes));
+    p.xq_scales = const_cast<uint8_t *>(a_scales);
+    p.band_ready = fx->band_ready;
+    p.next_item = fx->next_item;
+    p.ga_from_amax = fx->ga_from_amax;
+}
+
 template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
-                        const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st) {
+                        const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st,
+                        const FusedX *fx) {
     using L = GemmSmem<FMT, BN, STAGES, A_ROWS>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
@@ -298,7 +328,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     if (smem_limit_once(reinterpret_cast<const void *>(gemm_kernel<FMT, BN, STAGES, A_ROWS>), L::kAlloc) !=
         cudaSuccess)
         return MX_ERR_CUDA;
-    GemmParams p;
+    GemmParams p{};
     p.sf_tiles_k = sf_tiles_k;
     p.C = C;
     p.ldc = ldc;
@@ -317,6 +347,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.ab_types = (f8f6f4_type(A->fmt) << 7) | (f8f6f4_type(B->fmt) << 10);
     p.stage_tx = (uint32_t)(kStageKBytes * (A_ROWS * fmt_bits(A->fmt) + BN * fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
+    set_fused(p, fx, a_codes, a_scales, M, K);
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const int cap = g_max_gemm_ctas.load();
     const int64_t max_ctas = cap > 0 && cap < num_sms() ? cap : num_sms();
@@ -339,7 +370,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
 template <int FMT, int STAGES>
 mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                              const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out,
-                             cudaStream_t st) {
+                             cudaStream_t st, const FusedX *fx) {
     using L = PairSmem<FMT, STAGES>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
@@ -361,7 +392,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
     if (smem_limit_once(reinterpret_cast<const void *>(gemm_pair_kernel<FMT, STAGES>), L::kAlloc) != cudaSuccess)
         return MX_ERR_CUDA;
-    GemmParams p;
+    GemmParams p{};
     p.sf_tiles_k = sf_tiles_k;
     p.C = C;
     p.ldc = ldc;
@@ -381,6 +412,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     // both CTAs' copies (128 rows of A and 128 of B each) report to the leader's barrier
     p.stage_tx = (uint32_t)(2 * kStageKBytes * 128 * (fmt_bits(A->fmt) + fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
+    set_fused(p, fx, a_codes, a_scales, M, K);
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
     const int cap = g_max_gemm_ctas.load();
     const int64_t max_pairs = cap > 0 && cap < num_sms() ? (cap + 1) / 2 : num_sms() / 2;
@@ -405,35 +437,66 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
 
 template <int FMT>
 mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
-                          const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
+                          const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st,
+                          const FusedX *fx) {
     if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load())
-        return launch_gemm_pair_t<FMT, (FMT == 2 || FMT == 3) ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
-    if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+        return launch_gemm_pair_t<FMT, (FMT == 2 || FMT == 3) ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi,
+                                                                       amax_out, st, fx);
+    if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
     // at most 32 rows of A (decode-like activations): the weight stream gets a
     // fifth stage from the shared memory a 128-row A tile would take
-    if (A->rows <= 32) return launch_gemm_t<FMT, 256, 5, 32>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
-    return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    if (A->rows <= 32)
+        return launch_gemm_t<FMT, 256, 5, 32>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+    return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
 }
 
 mx_status launch_gemm(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
-                      const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st) {
+                      const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st,
+                      const FusedX *fx = nullptr) {
     if (gemm_runtime_types(A->fmt, B->fmt))
-        return launch_gemm_fmt<kGemmRuntimeTypes>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+        return launch_gemm_fmt<kGemmRuntimeTypes>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
     switch (A->fmt) {
-    case MX_MXFP8_E4M3: return launch_gemm_fmt<0>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
-    case MX_MXFP8_E5M2: return launch_gemm_fmt<1>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
-    case MX_MXFP4: return launch_gemm_fmt<2>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
-    default: return launch_gemm_fmt<3>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st);
+    case MX_MXFP8_E4M3: return launch_gemm_fmt<0>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+    case MX_MXFP8_E5M2: return launch_gemm_fmt<1>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+    case MX_MXFP4: return launch_gemm_fmt<2>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+    default: return launch_gemm_fmt<3>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
     }
 }
 
-// The fused call's workspace: a 256-byte header (g, amax of X), then X's codes
-// and scales, each starting on a 256-byte boundary.
-constexpr size_t kFusedWsHeader = 256;
+// The fused call's workspace: a header, then X's codes and scales, each
+// starting on a 256-byte boundary.  Header words: [0] g of X (NVFP4), [1]
+// amax(|X|) of the pre-pass, [2] the fused kernel's work counter, [3] unused,
+// [16 ..] one ready counter per 128-row band of X.
+constexpr size_t kWsBandOffset = 64;
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t fused_ws_header(int64_t M) { return align256(kWsBandOffset + 4 * (size_t)cdiv(M, 128)); }
 size_t fused_ws_bytes(int fmt, int64_t M, int64_t K) {
-    return kFusedWsHeader + align256((size_t)(M * K * fmt_bits(fmt) / 8)) +
+    return fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8)) +
            align256((size_t)(cdiv(M, 128) * 128 * cdiv(K / fmt_block(fmt), 4) * 4));
+}
+
+// Zero the fused kernel's counters (the work counter and the band counters).
+// Launched with programmatic stream serialization: it lets the GEMM that follows
+// start its setup at once, and clears the counters only after the previous
+// kernel in the stream (which may be a fused GEMM on the same workspace) has
+// completed; the GEMM reads them only after this kernel has completed.
+__global__ void fused_reset_kernel(uint32_t *__restrict__ words, int n) {
+    griddep_launch_dependents();
+    griddep_wait();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) words[i] = 0u;
+}
+
+mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    if (cudaLaunchKernelEx(&cfg, fused_reset_kernel, words, n) != cudaSuccess) return last_launch();
+    return MX_OK;
 }
 
 // Quantize X into the workspace as the A operand of the GEMM.  Returns the
@@ -447,8 +510,8 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
     xa->reserved = 0;
     xa->rows = M;
     xa->cols = K;
-    xa->codes = ws + kFusedWsHeader;
-    xa->scales = ws + kFusedWsHeader + align256((size_t)(M * K * fmt_bits(fmt) / 8));
+    xa->codes = ws + fused_ws_header(M);
+    xa->scales = ws + fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8));
     xa->gscale = g_slot;
     *ga = nullptr;
     mx_status s = MX_OK;
@@ -515,6 +578,7 @@ mx_status mx_debug_set(int key, uint64_t value) {
     case MX_DEBUG_PAIR_GEMM: g_pair_enabled.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_OVERLAP_LAUNCH: g_pdl_enabled.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_MAX_GEMM_CTAS: g_max_gemm_ctas.store(value > 65535 ? 0 : (int)value); return MX_OK;
+    case MX_DEBUG_FUSED_TWO_KERNELS: g_fused_two_kernels.store(value ? 1 : 0); return MX_OK;
     default: return MX_ERR_INVALID_ARG;
     }
 }
@@ -679,7 +743,8 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
     if (gemm_runtime_types(A->fmt, B->fmt) && ((fmt_bits(A->fmt) < 8 && !aligned32(A->codes)) ||
                                                (fmt_bits(B->fmt) < 8 && !aligned32(B->codes))))
         return MX_ERR_MISALIGNED;
-    return launch_gemm(A, B, A->codes, A->scales, A->gscale, static_cast<uint16_t *>(C_bf16), ldc, 0, nullptr, st);
+    return launch_gemm(A, B, A->codes, A->scales, A->gscale, static_cast<uint16_t *>(C_bf16), ldc, 0, nullptr, st,
+                       nullptr);
 }
 
 size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K) {
@@ -714,10 +779,52 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     if (gemm_runtime_types(fmt, W->fmt) && fmt_bits(W->fmt) < 8 && !aligned32(W->codes)) return MX_ERR_MISALIGNED;
     mx_tensor xa;
     const float *ga = nullptr;
-    s = fused_quantize_x(fmt, static_cast<const uint16_t *>(X_bf16), M, K, ldx, static_cast<uint8_t *>(workspace),
-                         x_gscale, x_amax, &xa, &ga, st);
+    const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (g_fused_two_kernels.load()) {
+        // quantize_kernel into the workspace, then the plain GEMM
+        s = fused_quantize_x(fmt, X, M, K, ldx, ws, x_gscale, x_amax, &xa, &ga, st);
+        if (s != MX_OK) return s;
+        return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out,
+                           st);
+    }
+    // One GEMM kernel whose epilogue warps quantize X into the workspace first
+    // (GemmParams::fused); NVFP4 without a given g or amax first runs the amax
+    // pre-pass into the header.
+    xa.fmt = fmt;
+    xa.reserved = 0;
+    xa.rows = M;
+    xa.cols = K;
+    xa.codes = ws + fused_ws_header(M);
+    xa.scales = ws + fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8));
+    xa.gscale = reinterpret_cast<float *>(ws);
+    FusedX fx;
+    fx.x = X;
+    fx.ldx = ldx;
+    fx.x_fmt = fmt;
+    fx.ga_from_amax = 0;
+    fx.band_ready = reinterpret_cast<uint32_t *>(ws + kWsBandOffset);
+    fx.next_item = reinterpret_cast<uint32_t *>(ws + 8);
+    if (fmt == MX_NVFP4) {
+        if (x_gscale != nullptr) {
+            ga = x_gscale;
+        } else {
+            ga = x_amax;
+            fx.ga_from_amax = 1;
+            if (x_amax == nullptr) {
+                float *amax_slot = reinterpret_cast<float *>(ws + 4);
+                if (cudaMemsetAsync(amax_slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
+                amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(
+                    X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
+                ga = amax_slot;
+            }
+        }
+    }
+    // words 2 .. 15 and the band counters
+    s = launch_fused_reset(reinterpret_cast<uint32_t *>(ws + 8), (int)((fused_ws_header(M) - 8) / 4), st);
     if (s != MX_OK) return s;
-    return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out, st);
+    return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out, st,
+                       &fx);
 }
 
 }  // extern "C"

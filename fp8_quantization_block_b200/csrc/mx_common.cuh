@@ -36,6 +36,7 @@ enum : unsigned {
     SITE_GEMM_SF_LOAD = 11,
     SITE_GEMM_SF_FREE = 12,
     SITE_GEMM_MMA_READY = 13,
+    SITE_FUSED_BAND_READY = 14,   // a TMA producer waiting for a band of the fused quantize
 };
 
 // {flags, first site, first block, count}
@@ -158,6 +159,49 @@ MX_DEVICE_INLINE uint32_t wait_counter_above(const uint32_t *counter, uint32_t n
         }
     }
 }
+
+// ---------------------------------------------------------------- cross-CTA counters
+// A global counter advanced by the CTAs that produce data (release at gpu scope)
+// and polled by the CTAs that consume it (acquire at gpu scope).  The consumers
+// read the data with TMA, i.e. through the async proxy: the producer orders its
+// ordinary stores before the release with fence.proxy.async.global, and the
+// consumer orders its TMA loads after the acquire with another one.
+MX_DEVICE_INLINE void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+MX_DEVICE_INLINE uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+MX_DEVICE_INLINE void red_release_gpu_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Poll *counter until it reaches target (bounded like the mbarrier waits), then
+// order the caller's later async-proxy (TMA) reads after what it observed.
+MX_DEVICE_INLINE bool wait_global_at_least(const uint32_t *counter, uint32_t target, uint64_t limit_ns, unsigned site,
+                                           volatile int *abort) {
+    if (ld_acquire_gpu(counter) < target) {
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t i = 1;; ++i) {
+            __nanosleep(64);
+            if (ld_acquire_gpu(counter) >= target) break;
+            if ((i & 7u) == 0u) {
+                if (abort != nullptr && *abort) return false;
+                if (globaltimer_ns() - t0 > limit_ns) {
+                    record_error(DEVERR_TIMEOUT, site);
+                    if (abort != nullptr) *abort = 1;
+                    return false;
+                }
+            }
+        }
+    }
+    fence_proxy_async_global();
+    return true;
+}
+
+// Barrier over the 128 threads of warps 2-5 of a GEMM CTA (hardware barrier 1;
+// barrier 0 is __syncthreads).
+MX_DEVICE_INLINE void sync_epilogue_warps() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // ---------------------------------------------------------------- packed fp32 pairs
 // f32x2 arithmetic of sm_100: two IEEE operations per instruction, each

@@ -380,6 +380,163 @@ MX_DEVICE_INLINE uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
     return max(rb & 0xFFFFu, rb >> 16);
 }
 
+// NVFP4 per-tensor constants of the quantize, formed once per CTA from g: the
+// bracket reciprocals of 1/g rounded down and up and 1/(6g).  Below 2^-100,
+// 1/g loses accuracy or overflows: the values are then divided as x * 2^64 by
+// g * 2^64 instead (both exact; every quotient is unchanged), sc = 2^64.
+struct NvScale {
+    float g, rg_lo, rg_hi, inv6g, sc;
+};
+MX_DEVICE_INLINE NvScale nv_scale_setup(float g) {
+    NvScale n;
+    n.sc = 1.0f;
+    if (g < 0x1p-100f) {
+        n.sc = 0x1p64f;
+        g *= n.sc;
+    }
+    n.g = g;
+    n.rg_lo = __frcp_rd(g);
+    n.rg_hi = __frcp_ru(g);
+    n.inv6g = 1.0f / (6.0f * g);
+    return n;
+}
+// g of an NVFP4 tensor from *src: g itself, or (from_amax) amax(|x|) with
+// g = RU(amax / (6 * 448)), 1 for an all-zero tensor.
+MX_DEVICE_INLINE float nv_g_from(const float *src, int from_amax) {
+    float g = *src;
+    if (from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;
+    return g;
+}
+// Entry c (0..127) of the per-CTA NVFP4 tables.
+MX_DEVICE_INLINE void nv_tables_fill(NvTables *nvt, uint32_t c) {
+    const float v = (c == 0u || c == 127u) ? 0.0f : e4m3_pos_value(c);
+    nvt->val[c] = v;
+    nvt->inv_lo[c] = v > 0.0f ? __frcp_rd(v) : 0.0f;
+    nvt->inv_hi[c] = v > 0.0f ? __frcp_ru(v) : 0.0f;
+}
+
+// One 16-element segment of a 128 x 128 quantize tile: values (v0, v1) of
+// global row `row` (tile row rl), columns col .. col + 15 (tile columns cl ..
+// cl + 15).  Stores the segment's codes when row and columns exist, and the
+// block's scale byte into the tile's 512-byte tensor-core chunks in sf_tile
+// (0 for padding).  A 32-element MX block spans lanes lane and lane ^ 1, which
+// must call together (one shuffle).
+template <int FMT, int RULE>
+MX_DEVICE_INLINE void quantize_seg16(const uint4 &v0, const uint4 &v1, int64_t row, int64_t M, int64_t col, int64_t K,
+                                     int64_t col0, int rl, int cl, int lane, const NvScale &ns,
+                                     const NvTables *__restrict__ nvt, uint8_t *__restrict__ codes,
+                                     uint8_t *__restrict__ sf_tile) {
+    using T = FmtTraits<FMT>;
+    const bool col_ok = col < K;   // K % 16 == 0: all 16 or none
+    const bool ok = row < M && col_ok;
+    const int jb = cl / T::kBlock;  // block index inside the tile row
+    uint32_t m = absmax16(v0, v1);
+    if (T::kBlock == 32) m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    uint32_t sbyte;
+    if (FMT == FMT_NVFP4) {
+        sbyte = nv_block_scale(__uint_as_float(m << 16) * ns.sc, ns.g, ns.inv6g, nvt->val);
+        if (ok) {
+            uint32_t q0, q1;
+            // r_lo <= 1/(g s) <= r_hi: products of one-sided bounds, rounded outward.
+            // An all-zero block has s = 0 and both bounds 0, so its products are
+            // the zeros themselves and its codes their signs (0x0 / 0x8).
+            const float r_lo = __fmul_rd(ns.rg_lo, nvt->inv_lo[sbyte]);
+            const float r_hi = __fmul_ru(ns.rg_hi, nvt->inv_hi[sbyte]);
+            nv_codes16(v0, v1, ns.g, nvt->val[sbyte], r_lo, r_hi, q0, q1, ns.sc);
+            *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
+        }
+    } else {
+        const int E = mx_scale_byte<FMT, RULE>(m);
+        sbyte = (uint32_t)E;
+        if (ok) {
+            const float inv = mx_inv_scale(E);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float f[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                f[2 * e] = bf16lo(w[e]) * inv;
+                f[2 * e + 1] = bf16hi(w[e]) * inv;
+            }
+            store_mx_codes16<FMT>(codes, row, K, col, f);
+        }
+    }
+    // Scale byte of (rl, jb) inside the tile's 512-byte tensor-core tiles.
+    const bool owner = T::kBlock == 16 || (lane & 1) == 0;
+    if (owner) {
+        const int64_t jglob = col0 / T::kBlock + jb;
+        if (!(row < M) || jglob >= K / T::kBlock) sbyte = 0u;   // padding bytes are 0
+        sf_tile[(jb >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (jb & 3)] = (uint8_t)sbyte;
+    }
+}
+
+// Bytes of a 128 x 128 tile's scale chunks (one or two 512-byte tensor-core tiles).
+template <int FMT>
+__host__ __device__ constexpr int quantize_sf_bytes() {
+    return kQTileRows * (kQTileCols / FmtTraits<FMT>::kBlock);
+}
+
+// Write a tile's scale chunks from shared memory (16 bytes per thread t <
+// bytes / 16): tile (band, tile_x) owns the consecutive chunks from
+// band * sf_tiles_k + tile_x * chunks, cut at the band's last chunk.
+template <int FMT>
+MX_DEVICE_INLINE void store_sf_chunks(const uint8_t *sf_tile, uint8_t *__restrict__ scales, int64_t band,
+                                      int64_t tile_x, int64_t sf_tiles_k, int t) {
+    constexpr int kChunks = quantize_sf_bytes<FMT>() / 512;
+    const int64_t chunk0 = band * sf_tiles_k + tile_x * kChunks;
+    const int64_t max_chunk = band * sf_tiles_k + sf_tiles_k;   // past this band's last tile
+    if (t < quantize_sf_bytes<FMT>() / 16) {
+        const int c = t / 32;
+        if (chunk0 + c < max_chunk) {
+            const uint4 val = *reinterpret_cast<const uint4 *>(sf_tile + t * 16);
+            *reinterpret_cast<uint4 *>(scales + chunk0 * 512 + t * 16) = val;
+        }
+    }
+}
+
+// The 128 x 128 tile (band, tile_x) of src quantized by NT threads (t = 0 ..
+// NT - 1, NT = 128 or 256, whole warps): 8 threads per row, 16 elements per
+// thread per pass, the loads of four passes issued together; the scale chunks
+// assembled in sf_tile (shared memory, quantize_sf_bytes<FMT>() bytes) and
+// written out after sync(), a barrier over the NT threads.
+template <int FMT, int NT, typename Sync>
+MX_DEVICE_INLINE void quantize_tile(const uint16_t *__restrict__ src, int64_t M, int64_t K, int64_t ld,
+                                    uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t sf_tiles_k,
+                                    int64_t band, int64_t tile_x, const NvScale &ns, const NvTables *nvt,
+                                    uint8_t *sf_tile, int t, Sync sync) {
+    static_assert(NT % 32 == 0 && NT >= 32 && kQTileRows % (NT / 8) == 0, "whole warps, whole passes");
+    constexpr int kRowsPerPass = NT / 8;
+    constexpr int kPasses = kQTileRows / kRowsPerPass;
+    constexpr int kGroup = kPasses < 4 ? kPasses : 4;
+    const int lane = t & 31, warp = t >> 5;
+    const int64_t row0 = band * kQTileRows, col0 = tile_x * kQTileCols;
+    const int cl = (lane & 7) * 16;
+    const int64_t col = col0 + cl;
+#pragma unroll 1
+    for (int i0 = 0; i0 < kPasses; i0 += kGroup) {
+        uint4 v[kGroup][2];
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int rl = (i0 + i) * kRowsPerPass + warp * 4 + (lane >> 3);
+            const int64_t row = row0 + rl;
+            if (row < M && col < K) {
+                const uint16_t *p = src + row * ld + col;
+                v[i][0] = ldg_stream(p);
+                v[i][1] = ldg_stream(p + 8);
+            } else {
+                v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int rl = (i0 + i) * kRowsPerPass + warp * 4 + (lane >> 3);
+            quantize_seg16<FMT, RULE_OCP>(v[i][0], v[i][1], row0 + rl, M, col, K, col0, rl, cl, lane, ns, nvt, codes,
+                                          sf_tile);
+        }
+    }
+    sync();
+    store_sf_chunks<FMT>(sf_tile, scales, band, tile_x, sf_tiles_k, t);
+}
+
 // src bf16 [M x K] (row pitch ld).  codes / scales as in mx.h.  sf_tiles_k =
 // ceil((K / block) / 4) 512-byte tiles per 128-row band.  NVFP4: *gscale_in
 // is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
@@ -399,21 +556,16 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
                                                              const float *__restrict__ gscale_in,
                                                              float *__restrict__ gscale_out, int g_from_amax) {
-    using T = FmtTraits<FMT>;
-    constexpr int kBlocksPerRow = kQTileCols / T::kBlock;  // 4 (MX) or 8 (NVFP4)
-    constexpr int kSfBytes = kQTileRows * kBlocksPerRow;   // 512 or 1024
     constexpr int kPasses = kQTileRows / 32;               // 32 rows per pass (8 warps x 4 rows)
-    __shared__ __align__(16) uint8_t sf_tile[kSfBytes];
+    __shared__ __align__(16) uint8_t sf_tile[quantize_sf_bytes<FMT>()];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row0 = (int64_t)blockIdx.y * kQTileRows;
     const int64_t col0 = (int64_t)blockIdx.x * kQTileCols;
     const int cl = (lane & 7) * 16;                 // first of this lane's 16 columns inside the tile
     const int64_t col = col0 + cl;
-    const bool col_ok = col < K;                    // K % 16 == 0: all 16 or none
-    const int jb = cl / T::kBlock;                  // block index inside the tile row
 
-    float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f, sc = 1.0f;
+    NvScale ns{1.0f, 1.0f, 1.0f, 1.0f, 1.0f};
     __shared__ NvTables nvt;
     // src and g may come from the previous kernel in the stream
     griddep_wait();
@@ -422,25 +574,10 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
     // waits for this grid's completion before reading anything).
     griddep_launch_dependents();
     if (FMT == FMT_NVFP4) {
-        g = *gscale_in;
-        if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;   // g = RU(amax / (6 * 448))
+        const float g = nv_g_from(gscale_in, g_from_amax);
         if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
-        // Below 2^-100, 1/g loses accuracy or overflows: divide x * 2^64 by
-        // g * 2^64 instead (both exact; every quotient is unchanged).
-        if (g < 0x1p-100f) {
-            sc = 0x1p64f;
-            g *= sc;
-        }
-        rg_lo = __frcp_rd(g);
-        rg_hi = __frcp_ru(g);
-        inv6g = 1.0f / (6.0f * g);
-        if (threadIdx.x < 128) {
-            const uint32_t c = threadIdx.x;
-            const float v = (c == 0u || c == 127u) ? 0.0f : e4m3_pos_value(c);
-            nvt.val[c] = v;
-            nvt.inv_lo[c] = v > 0.0f ? __frcp_rd(v) : 0.0f;
-            nvt.inv_hi[c] = v > 0.0f ? __frcp_ru(v) : 0.0f;
-        }
+        ns = nv_scale_setup(g);
+        if (threadIdx.x < 128) nv_tables_fill(&nvt, threadIdx.x);
         __syncthreads();
     }
 
@@ -449,7 +586,7 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
     for (int i = 0; i < kPasses; ++i) {
         const int rl = i * 32 + warp * 4 + (lane >> 3);
         const int64_t row = row0 + rl;
-        if (row < M && col_ok) {
+        if (row < M && col < K) {
             const uint16_t *p = src + row * ld + col;
             v[i][0] = ldg_stream(p);
             v[i][1] = ldg_stream(p + 8);
@@ -461,59 +598,11 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
 #pragma unroll
     for (int i = 0; i < kPasses; ++i) {
         const int rl = i * 32 + warp * 4 + (lane >> 3);
-        const int64_t row = row0 + rl;
-        const bool ok = row < M && col_ok;
-        uint32_t m = absmax16(v[i][0], v[i][1]);
-        if (T::kBlock == 32) m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        uint32_t sbyte;
-        if (FMT == FMT_NVFP4) {
-            sbyte = nv_block_scale(__uint_as_float(m << 16) * sc, g, inv6g, nvt.val);
-            if (ok) {
-                uint32_t q0, q1;
-                // r_lo <= 1/(g s) <= r_hi: products of one-sided bounds, rounded outward.
-                // An all-zero block has s = 0 and both bounds 0, so its products are
-                // the zeros themselves and its codes their signs (0x0 / 0x8).
-                const float r_lo = __fmul_rd(rg_lo, nvt.inv_lo[sbyte]);
-                const float r_hi = __fmul_ru(rg_hi, nvt.inv_hi[sbyte]);
-                nv_codes16(v[i][0], v[i][1], g, nvt.val[sbyte], r_lo, r_hi, q0, q1, sc);
-                *reinterpret_cast<uint2 *>(codes + row * (K / 2) + col / 2) = make_uint2(q0, q1);
-            }
-        } else {
-            const int E = mx_scale_byte<FMT, RULE>(m);
-            sbyte = (uint32_t)E;
-            if (ok) {
-                const float inv = mx_inv_scale(E);
-                const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w,
-                                       v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
-                float f[16];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    f[2 * e] = bf16lo(w[e]) * inv;
-                    f[2 * e + 1] = bf16hi(w[e]) * inv;
-                }
-                store_mx_codes16<FMT>(codes, row, K, col, f);
-            }
-        }
-        // Scale byte of (rl, jb) inside the tile's 512-byte tensor-core tiles.
-        const bool owner = T::kBlock == 16 || (lane & 1) == 0;
-        if (owner) {
-            const int64_t jglob = col0 / T::kBlock + jb;
-            if (!(row < M) || jglob >= K / T::kBlock) sbyte = 0u;   // padding bytes are 0
-            sf_tile[(jb >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (jb & 3)] = (uint8_t)sbyte;
-        }
+        quantize_seg16<FMT, RULE>(v[i][0], v[i][1], row0 + rl, M, col, K, col0, rl, cl, lane, ns, &nvt, codes,
+                                  sf_tile);
     }
     __syncthreads();
-    // The tile's chunks are consecutive 512-byte tiles in the scale buffer.
-    constexpr int kChunks = kSfBytes / 512;
-    const int64_t chunk0 = (int64_t)blockIdx.y * sf_tiles_k + (int64_t)blockIdx.x * kChunks;
-    const int64_t max_chunk = (int64_t)blockIdx.y * sf_tiles_k + sf_tiles_k;   // past this band's last tile
-    if (threadIdx.x < kSfBytes / 16) {
-        const int c = threadIdx.x / 32;
-        if (chunk0 + c < max_chunk) {
-            uint4 val = *reinterpret_cast<const uint4 *>(sf_tile + threadIdx.x * 16);
-            *reinterpret_cast<uint4 *>(scales + chunk0 * 512 + threadIdx.x * 16) = val;
-        }
-    }
+    store_sf_chunks<FMT>(sf_tile, scales, blockIdx.y, blockIdx.x, sf_tiles_k, threadIdx.x);
 }
 
 // ------------------------------------------------------------------ MXFP4 with macro-block scaling

@@ -198,11 +198,17 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  * is fmt or, as in mx_gemm, any MX format that pairs with it (e.g. MXFP8
  * activations with MXFP4 or MXFP6 weights).  X is quantized exactly as
  * mx_quantize would (same codes and scales, bit for bit) once, into the
- * caller's `workspace` (which stays resident in L2 at these sizes), and the
- * block-scaled GEMM consumes it in the same stream: C = X_dq * W_dq^T as in
- * mx_gemm.  X's quantized form is not an output of this call.
+ * caller's `workspace`, by the GEMM kernel itself: the epilogue warps of every
+ * CTA (idle until the first accumulator is ready) share X's 128 x 128 tiles,
+ * band by band, and the TMA producers load A from a 128-row band as soon as
+ * its tiles are written (per-band counters in the workspace).  The result is
+ * C = X_dq * W_dq^T as in mx_gemm.  X's quantized form is not an output of
+ * this call.  Launches: the GEMM kernel and a one-thread-block kernel that
+ * clears the workspace's counters (NVFP4 without x_gscale or x_amax: also the
+ * amax pre-pass).
  *   workspace: device buffer of at least mx_fused_workspace_bytes(fmt, M, K)
- *              bytes, 256-byte aligned; its contents are scratch.
+ *              bytes, 256-byte aligned; its contents are scratch, and calls
+ *              that overlap on the GPU must not share one.
  *   epilogue : MX_EPI_NONE, or MX_EPI_GELU: the exact-erf form x Phi(x) =
  *              0.5 x erfc(-x / sqrt 2), applied in FP32 before the bf16
  *              rounding, with erfc from the Chebyshev fit of Numerical Recipes
@@ -222,7 +228,8 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
                             float *amax_out, const float *x_gscale, const float *x_amax,
                             void *workspace, size_t workspace_bytes, void *stream);
 /* Workspace bytes mx_gemm_fused_act needs for an [M x K] activation of format
- * fmt (a 256-byte header, then X's codes and scales); 0 for a bad format. */
+ * fmt (a header of 64 bytes plus 4 per 128-row band, rounded up to 256, then
+ * X's codes and scales); 0 for a bad format. */
 size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K);
 
 /* mx_gemm_fused_act without a workspace argument, for callers that cannot
@@ -282,13 +289,18 @@ int mx_version(void);
  *                            0 (default) = one CTA per SM.  The result does
  *                            not depend on it (each tile is summed in the
  *                            same order wherever it runs).
+ *   MX_DEBUG_FUSED_TWO_KERNELS: 1 = mx_gemm_fused_act runs the quantize kernel
+ *                            and then the GEMM kernel (two launches) instead of
+ *                            quantizing X inside the GEMM kernel; 0 (default)
+ *                            = one GEMM kernel.  Same results bit for bit.
  * Returns MX_ERR_INVALID_ARG for an unknown key. */
 typedef enum {
     MX_DEBUG_WAIT_LIMIT_NS = 1,
     MX_DEBUG_SKIP_PRODUCER = 2,
     MX_DEBUG_PAIR_GEMM = 3,
     MX_DEBUG_OVERLAP_LAUNCH = 4,
-    MX_DEBUG_MAX_GEMM_CTAS = 5
+    MX_DEBUG_MAX_GEMM_CTAS = 5,
+    MX_DEBUG_FUSED_TWO_KERNELS = 6
 } mx_debug_key;
 mx_status mx_debug_set(int key, uint64_t value);
 
