@@ -95,7 +95,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
     // The setup above overlaps the previous kernel in the stream; its outputs
     // (our operands, NVFP4 scales, C's prior contents) are read only after this.
-    griddep_wait();
+    // (fused == 2: that kernel is the quantize of A, whose CTAs started only
+    // after everything before it had completed; A is read band by band as its
+    // counters say.)
+    if (p.fused != 2) griddep_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ code-tile producer
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue (this CTA's 128 rows)
         // (fused: first the activation quantize, in the staging buffers' space)
-        if (p.fused) fused_quantize_role<FMT>(p, reinterpret_cast<FusedQuantSmem *>(smem + L::kOffEpi), threadIdx.x - 64);
+        if (p.fused == 1) fused_quantize_role<FMT>(p, reinterpret_cast<FusedQuantSmem *>(smem + L::kOffEpi), threadIdx.x - 64);
         const int q = warp & 3;
         uint8_t *bufs = smem + L::kOffEpi + (warp - 2) * L::kEpiBufs * kEpiChunkBytes;
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);

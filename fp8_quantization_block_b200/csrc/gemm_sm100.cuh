@@ -113,13 +113,19 @@ struct GemmParams {
     uint64_t wait_limit_ns;
     int ga_from_amax;     // NVFP4: *ga holds amax(|A|) and gA = RU(amax / 2688) (1 for 0)
     int band_major;       // tile order: 1 = N fastest (consecutive tiles share A's band), 0 = M fastest
-    // Fused activation quantize (fused != 0): A is the bf16 matrix x [M x K]
-    // (row pitch ldx), quantized to format x_fmt by the epilogue warps of every
-    // CTA before their first tile (fused_quantize_role) into xq_codes /
-    // xq_scales, which the TMA producers then read as A.  Work unit: a 128 x 128
-    // tile of x; next_item hands them out in band-major order, band_ready[b]
-    // counts those of 128-row band b that are written.
+    // Fused activation quantize.  A is the bf16 matrix x [M x K] (row pitch
+    // ldx) quantized to format x_fmt into xq_codes / xq_scales, which the TMA
+    // producers read once band_ready[b] of A's 128-row band b has reached
+    // x_band_target:
+    //   fused == 1: by the epilogue warps of every CTA before their first tile
+    //     (fused_quantize_role); work unit 32 rows x 128 columns of x (one
+    //     warp's), handed out by next_item in band-major order;
+    //   fused == 2: by the quantize kernel just before this one in the stream,
+    //     one count per 128 x 128 CTA of it; this kernel then starts without
+    //     waiting for that grid to complete (griddepcontrol.wait), so its CTAs
+    //     work on the bands already written while the quantize still runs.
     int fused;
+    uint32_t x_band_target;
     int x_fmt;
     int x_items_k;        // 128-column tiles per band = ceil(K / 128)
     int x_bands;          // ceil(M / 128)
@@ -141,7 +147,7 @@ MX_DEVICE_INLINE float gemm_ga(const GemmParams &p) { return nv_g_from(p.ga, p.g
 MX_DEVICE_INLINE bool wait_band_ready(const GemmParams &p, int band, int lane, volatile int *abort_flag) {
     bool ok = true;
     if (band < p.x_bands && lane == 0)
-        ok = wait_global_at_least(p.band_ready + band, (uint32_t)p.x_items_k, p.wait_limit_ns, SITE_FUSED_BAND_READY,
+        ok = wait_global_at_least(p.band_ready + band, p.x_band_target, p.wait_limit_ns, SITE_FUSED_BAND_READY,
                                   abort_flag);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
@@ -507,45 +513,85 @@ MX_DEVICE_INLINE void tile_coords(const GemmParams &p, int tile, int &m0, int &n
 }
 
 // Shared memory of the fused quantize, inside the epilogue warps' staging
-// buffers (idle until their first tile): the scale chunks of the tile being
-// quantized, the NVFP4 tables and the claimed work item.
+// buffers (idle until their first tile): each warp's scale chunks of the rows
+// it is quantizing, and the NVFP4 tables.
 struct FusedQuantSmem {
-    uint8_t sf[1024];
+    uint8_t sf[kEpiWarps][1024];
     NvTables nvt;
-    uint32_t claim;
 };
 
-// The epilogue warps (t = 0..127) of a CTA: claim 128 x 128 tiles of x from the
-// global counter until none is left, quantize each (quantize_tile: the
-// arithmetic of quantize_kernel, so codes and scales are those of mx_quantize)
-// and count it in its band once written.  Nothing here waits on another CTA,
-// so the tiles get done as long as any CTA of the grid runs.
+// Work items of the fused quantize: 32 rows x 128 columns of x, one warp's
+// (quadrant q of the 128 x 128 tile (band, tile_x)); item
+// ((band * x_items_k) + tile_x) * 4 + q, handed out in that order, so bands
+// complete in order.  A band is written once x_items_k * 4 items are counted.
+constexpr int kFusedQuads = kQTileRows / 32;
+
+// Each epilogue warp (w = 0..3) of a CTA: claim items from the global counter
+// until none is left, quantize each (tile_load / tile_quantize: the arithmetic
+// of quantize_kernel, so codes and scales are those of mx_quantize), write its
+// rows' scale bytes and count it in its band.  The four warps run independent
+// pipelines (no barrier between them until the end), and each issues its next
+// item's loads as soon as this item's values are consumed, so they fly while
+// this item is published.  Nothing here waits on another CTA, so the items get done as long
+// as any CTA of the grid runs.
 template <int XFMT>
 MX_DEVICE_INLINE void fused_quantize_role_t(const GemmParams &p, FusedQuantSmem *fq, int t) {
+    const int w = t >> 5, lane = t & 31;
     NvScale ns{1.0f, 1.0f, 1.0f, 1.0f, 1.0f};
     if (XFMT == FMT_NVFP4) {
         ns = nv_scale_setup(nv_g_from(p.ga, p.ga_from_amax));
         nv_tables_fill(&fq->nvt, (uint32_t)t);
-    }
-    const uint32_t n_items = (uint32_t)p.x_bands * (uint32_t)p.x_items_k;
-    if (t == 0) fq->claim = atomicAdd(p.next_item, 1u);
-    sync_epilogue_warps();
-    uint32_t cur = fq->claim;
-    while (cur < n_items) {
-        uint32_t nxt = 0;
-        if (t == 0) nxt = atomicAdd(p.next_item, 1u);   // the next claim overlaps this tile
-        const int band = (int)(cur / (uint32_t)p.x_items_k), tx = (int)(cur % (uint32_t)p.x_items_k);
-        quantize_tile<XFMT, 128>(p.x, p.M, p.K, p.ldx, p.xq_codes, p.xq_scales, p.x_sf_tiles_k, band, tx, ns,
-                                 &fq->nvt, fq->sf, t, sync_epilogue_warps);
-        fence_proxy_async_global();   // this thread's stores, before the band count (TMA reads them)
-        if (t == 0) fq->claim = nxt;
         sync_epilogue_warps();
-        if (t == 0) {
-            __threadfence();
-            red_release_gpu_add(p.band_ready + band, 1u);
-        }
-        cur = fq->claim;
     }
+    constexpr int kChunks = quantize_sf_bytes<XFMT>() / 512;
+    uint8_t *sf = fq->sf[w];
+    const uint32_t items_k = (uint32_t)p.x_items_k;
+    const uint32_t n_items = (uint32_t)p.x_bands * items_k * kFusedQuads;
+    uint32_t cur = 0;
+    if (lane == 0) cur = atomicAdd(p.next_item, 1u);
+    cur = __shfl_sync(0xffffffffu, cur, 0);
+    TileRegs<32, 32> r;
+    auto rows_of = [&](uint32_t item, int64_t &band, int64_t &tx, int &q) {
+        q = (int)(item % kFusedQuads);
+        const uint32_t tile = item / kFusedQuads;
+        band = tile / items_k;
+        tx = tile % items_k;
+    };
+    int64_t band, tx;
+    int q;
+    if (cur < n_items) {
+        rows_of(cur, band, tx, q);
+        tile_load<32, 32>(r, p.x, p.M, p.K, p.ldx, band * kQTileRows + q * 32, tx * kQTileCols, lane);
+    }
+    while (cur < n_items) {
+        rows_of(cur, band, tx, q);
+        uint32_t nxt = 0;
+        if (lane == 0) nxt = atomicAdd(p.next_item, 1u);   // its latency hides behind this item's arithmetic
+        tile_quantize<XFMT, 32, 32>(r, p.M, p.K, band * kQTileRows, q * 32, tx * kQTileCols, ns, &fq->nvt,
+                                    p.xq_codes, sf, lane);
+        __syncwarp();
+        // this warp's rows of the tile's scale chunks: row lane's 4 bytes of each chunk
+        const int64_t chunk0 = band * p.x_sf_tiles_k + tx * kChunks, chunk_end = (band + 1) * p.x_sf_tiles_k;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+            if (chunk0 + c < chunk_end)
+                *reinterpret_cast<uint32_t *>(p.xq_scales + (chunk0 + c) * 512 + lane * 16 + q * 4) =
+                    *reinterpret_cast<const uint32_t *>(sf + c * 512 + lane * 16 + q * 4);
+        nxt = __shfl_sync(0xffffffffu, nxt, 0);
+        if (nxt < n_items) {
+            int64_t nb, ntx;
+            int nq;
+            rows_of(nxt, nb, ntx, nq);
+            tile_load<32, 32>(r, p.x, p.M, p.K, p.ldx, nb * kQTileRows + nq * 32, ntx * kQTileCols, lane);
+        }
+        fence_proxy_async_global();   // this lane's stores, before the band count (TMA reads them)
+        __syncwarp();
+        if (lane == 0) red_release_gpu_add(p.band_ready + band, 1u);
+        cur = nxt;
+    }
+    // the epilogue reuses this shared memory as staging buffers: no warp starts
+    // its epilogue while another still quantizes
+    sync_epilogue_warps();
 }
 
 template <int FMT>
@@ -865,7 +911,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
     // The setup above overlaps the previous kernel in the stream; its outputs
     // (our operands, NVFP4 scales, C's prior contents) are read only after this.
-    griddep_wait();
+    // (fused == 2: that kernel is the quantize of A, whose CTAs started only
+    // after everything before it had completed; A is read band by band as its
+    // counters say.)
+    if (p.fused != 2) griddep_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ code-tile producer
@@ -1047,7 +1096,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         // (fused: first the activation quantize, in the staging buffers' space)
-        if (p.fused) fused_quantize_role<FMT>(p, reinterpret_cast<FusedQuantSmem *>(smem + L::kOffEpi), threadIdx.x - 64);
+        if (p.fused == 1) fused_quantize_role<FMT>(p, reinterpret_cast<FusedQuantSmem *>(smem + L::kOffEpi), threadIdx.x - 64);
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         uint8_t *bufs = smem + L::kOffEpi + (warp - 2) * L::kEpiBufs * kEpiChunkBytes;
         uint32_t amax = 0, nstore = 0;

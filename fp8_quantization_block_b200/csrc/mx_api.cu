@@ -28,7 +28,7 @@ std::atomic<int> g_skip_producer{0};
 std::atomic<int> g_pair_enabled{1};
 std::atomic<int> g_pdl_enabled{1};
 std::atomic<int> g_max_gemm_ctas{0};  // 0: one CTA (or CTA pair) per SM pair of the device
-std::atomic<int> g_fused_two_kernels{0};  // 1: the fused call runs quantize_kernel, then the GEMM
+std::atomic<int> g_fused_mode{MX_FUSED_PIPELINED};  // how mx_gemm_fused_act runs (MX_DEBUG_FUSED_MODE)
 
 // Launch attributes shared by the kernels that may overlap the previous kernel
 // in the stream (they call griddep_wait() before reading any input).
@@ -146,7 +146,8 @@ bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) ==
 // --- quantize ------------------------------------------------------------
 template <int FMT, int RULE = RULE_OCP>
 mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
-                          const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
+                          const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0,
+                          uint32_t *band_ready = nullptr) {
     if (M == 0 || K == 0) return MX_OK;
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     cudaLaunchConfig_t cfg;
@@ -158,7 +159,7 @@ mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld,
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
     if (cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes),
-                           dst->scales, sf_tiles_k, g_in, g_out, g_from_amax) != cudaSuccess)
+                           dst->scales, sf_tiles_k, g_in, g_out, g_from_amax, band_ready) != cudaSuccess)
         return last_launch();
     return MX_OK;
 }
@@ -277,6 +278,7 @@ cudaError_t smem_limit_once(const void *fn, int bytes) {
 // The activation of a fused call: bf16 x quantized inside the GEMM kernel (see
 // GemmParams::fused); A's codes and scales are its destination.
 struct FusedX {
+    int mode;            // GemmParams::fused: 1 in-kernel quantize, 2 quantize kernel feeding bands
     const uint16_t *x;
     int64_t ldx;
     int x_fmt;
@@ -287,13 +289,16 @@ struct FusedX {
 
 void set_fused(GemmParams &p, const FusedX *fx, const void *a_codes, const uint8_t *a_scales, int64_t M, int64_t K) {
     if (fx == nullptr) return;
-    p.fused = 1;
+    p.fused = fx->mode;
     p.band_major = 1;
     p.x = fx->x;
     p.ldx = fx->ldx;
     p.x_fmt = fx->x_fmt;
     p.x_items_k = (int)cdiv(K, kQTileCols);
     p.x_bands = (int)cdiv(M, kQTileRows);
+    // items per band: four 32-row items per 128 x 128 tile in the kernel's own
+    // quantize, one quantize-kernel CTA per tile otherwise
+    p.x_band_target = (uint32_t)p.x_items_k * (fx->mode == 1 ? (uint32_t)kFusedQuads : 1u);
     p.x_sf_tiles_k = cdiv(K / fmt_block(fx->x_fmt), 4);
     p.xq_codes = static_cast<uint8_t *>(const_cast<void *>(a_codes));
     p.xq_scales = const_cast<uint8_t *>(a_scales);
@@ -503,7 +508,7 @@ mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st) {
 // device pointer of X's g (NVFP4) through *ga.
 mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int64_t ldx, uint8_t *ws,
                            const float *x_gscale, const float *x_amax, mx_tensor *xa, const float **ga,
-                           cudaStream_t st) {
+                           cudaStream_t st, uint32_t *band_ready = nullptr) {
     float *g_slot = reinterpret_cast<float *>(ws);
     float *amax_slot = reinterpret_cast<float *>(ws + 4);
     xa->fmt = fmt;
@@ -516,13 +521,13 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
     *ga = nullptr;
     mx_status s = MX_OK;
     switch (fmt) {
-    case MX_MXFP8_E4M3: s = launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
-    case MX_MXFP8_E5M2: s = launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
-    case MX_MXFP4: s = launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
-    case MX_MXFP6_E3M2: s = launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st); break;
+    case MX_MXFP8_E4M3: s = launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
+    case MX_MXFP8_E5M2: s = launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
+    case MX_MXFP4: s = launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
+    case MX_MXFP6_E3M2: s = launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
     default:
         if (x_gscale != nullptr) {
-            s = launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st);
+            s = launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st, 0, band_ready);
             *ga = x_gscale;
         } else {
             const float *amax = x_amax;
@@ -532,7 +537,7 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
                     X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
                 amax = amax_slot;
             }
-            s = launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1);
+            s = launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1, band_ready);
             *ga = g_slot;
         }
     }
@@ -578,7 +583,10 @@ mx_status mx_debug_set(int key, uint64_t value) {
     case MX_DEBUG_PAIR_GEMM: g_pair_enabled.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_OVERLAP_LAUNCH: g_pdl_enabled.store(value ? 1 : 0); return MX_OK;
     case MX_DEBUG_MAX_GEMM_CTAS: g_max_gemm_ctas.store(value > 65535 ? 0 : (int)value); return MX_OK;
-    case MX_DEBUG_FUSED_TWO_KERNELS: g_fused_two_kernels.store(value ? 1 : 0); return MX_OK;
+    case MX_DEBUG_FUSED_MODE:
+        if (value > MX_FUSED_TWO_KERNELS) return MX_ERR_INVALID_ARG;
+        g_fused_mode.store((int)value);
+        return MX_OK;
     default: return MX_ERR_INVALID_ARG;
     }
 }
@@ -781,15 +789,22 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     const float *ga = nullptr;
     const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    if (g_fused_two_kernels.load()) {
-        // quantize_kernel into the workspace, then the plain GEMM
+    int mode = g_fused_mode.load();
+    // a single 128-row band is written only when the whole quantize is: no band
+    // of it to start early on, so the pipelined mode would only add its counter
+    // reset
+    if (mode == MX_FUSED_PIPELINED && M <= kQTileRows) mode = MX_FUSED_TWO_KERNELS;
+    if (mode == MX_FUSED_TWO_KERNELS) {
+        // quantize_kernel into the workspace, then the plain GEMM in stream order
         s = fused_quantize_x(fmt, X, M, K, ldx, ws, x_gscale, x_amax, &xa, &ga, st);
         if (s != MX_OK) return s;
         return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out,
                            st);
     }
-    // One GEMM kernel whose epilogue warps quantize X into the workspace first
-    // (GemmParams::fused); NVFP4 without a given g or amax first runs the amax
+    // X quantized by the GEMM kernel itself (MX_FUSED_IN_KERNEL) or by the
+    // quantize kernel, band by band, with the GEMM starting on the bands already
+    // written (MX_FUSED_PIPELINED); either way the workspace's counters are
+    // cleared first, and NVFP4 without a given g or amax first runs the amax
     // pre-pass into the header.
     xa.fmt = fmt;
     xa.reserved = 0;
@@ -799,33 +814,42 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     xa.scales = ws + fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8));
     xa.gscale = reinterpret_cast<float *>(ws);
     FusedX fx;
+    fx.mode = mode == MX_FUSED_IN_KERNEL ? 1 : 2;
     fx.x = X;
     fx.ldx = ldx;
     fx.x_fmt = fmt;
     fx.ga_from_amax = 0;
     fx.band_ready = reinterpret_cast<uint32_t *>(ws + kWsBandOffset);
     fx.next_item = reinterpret_cast<uint32_t *>(ws + 8);
+    // gA for the GEMM's epilogue: never the g the quantize kernel writes (the
+    // pipelined GEMM may run before that store is visible), always its source
+    float *amax_slot = reinterpret_cast<float *>(ws + 4);
+    const float *x_amax_src = x_amax;
     if (fmt == MX_NVFP4) {
         if (x_gscale != nullptr) {
             ga = x_gscale;
         } else {
-            ga = x_amax;
             fx.ga_from_amax = 1;
             if (x_amax == nullptr) {
-                float *amax_slot = reinterpret_cast<float *>(ws + 4);
                 if (cudaMemsetAsync(amax_slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
                 amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(
                     X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
-                ga = amax_slot;
+                x_amax_src = amax_slot;
             }
+            ga = x_amax_src;
         }
     }
     // words 2 .. 15 and the band counters
     s = launch_fused_reset(reinterpret_cast<uint32_t *>(ws + 8), (int)((fused_ws_header(M) - 8) / 4), st);
     if (s != MX_OK) return s;
+    if (fx.mode == 2) {
+        mx_tensor xq;
+        const float *unused = nullptr;
+        s = fused_quantize_x(fmt, X, M, K, ldx, ws, x_gscale, x_amax_src, &xq, &unused, st, fx.band_ready);
+        if (s != MX_OK) return s;
+    }
     return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out, st,
-                       &fx);
-}
+                       &fx);}
 
 }  // extern "C"
 

@@ -493,54 +493,61 @@ MX_DEVICE_INLINE void store_sf_chunks(const uint8_t *sf_tile, uint8_t *__restric
     }
 }
 
-// The 128 x 128 tile (band, tile_x) of src quantized by NT threads (t = 0 ..
-// NT - 1, NT = 128 or 256, whole warps): 8 threads per row, 16 elements per
-// thread per pass, the loads of four passes issued together; the scale chunks
-// assembled in sf_tile (shared memory, quantize_sf_bytes<FMT>() bytes) and
-// written out after sync(), a barrier over the NT threads.
-template <int FMT, int NT, typename Sync>
-MX_DEVICE_INLINE void quantize_tile(const uint16_t *__restrict__ src, int64_t M, int64_t K, int64_t ld,
-                                    uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t sf_tiles_k,
-                                    int64_t band, int64_t tile_x, const NvScale &ns, const NvTables *nvt,
-                                    uint8_t *sf_tile, int t, Sync sync) {
-    static_assert(NT % 32 == 0 && NT >= 32 && kQTileRows % (NT / 8) == 0, "whole warps, whole passes");
-    constexpr int kRowsPerPass = NT / 8;
-    constexpr int kPasses = kQTileRows / kRowsPerPass;
-    constexpr int kGroup = kPasses < 4 ? kPasses : 4;
+// ROWS rows x 128 columns of src quantized by NT threads (t = 0 .. NT - 1,
+// whole warps): 8 threads per row, 16 elements per thread per pass, ROWS /
+// (NT / 8) passes.  tile_load issues every load of the rows (two 16-byte loads
+// per pass) into registers; tile_quantize then stores the codes and writes each
+// block's scale byte into the 128-row tile's scale chunks in sf_tile (shared
+// memory, quantize_sf_bytes<FMT>() bytes; rows are placed by their row index
+// inside the 128-row band, rl0 being that of the first).
+template <int NT, int ROWS = kQTileRows>
+struct TileRegs {
+    static_assert(NT % 32 == 0 && NT >= 32 && ROWS % (NT / 8) == 0 && ROWS <= kQTileRows, "whole warps and passes");
+    static constexpr int kRowsPerPass = NT / 8;
+    static constexpr int kPasses = ROWS / kRowsPerPass;
+    uint4 v[kPasses][2];
+};
+
+template <int NT, int ROWS>
+MX_DEVICE_INLINE void tile_load(TileRegs<NT, ROWS> &r, const uint16_t *__restrict__ src, int64_t M, int64_t K,
+                                int64_t ld, int64_t row0, int64_t col0, int t) {
+    using R = TileRegs<NT, ROWS>;
     const int lane = t & 31, warp = t >> 5;
-    const int64_t row0 = band * kQTileRows, col0 = tile_x * kQTileCols;
-    const int cl = (lane & 7) * 16;
-    const int64_t col = col0 + cl;
-#pragma unroll 1
-    for (int i0 = 0; i0 < kPasses; i0 += kGroup) {
-        uint4 v[kGroup][2];
+    const int64_t col = col0 + (lane & 7) * 16;
 #pragma unroll
-        for (int i = 0; i < kGroup; ++i) {
-            const int rl = (i0 + i) * kRowsPerPass + warp * 4 + (lane >> 3);
-            const int64_t row = row0 + rl;
-            if (row < M && col < K) {
-                const uint16_t *p = src + row * ld + col;
-                v[i][0] = ldg_stream(p);
-                v[i][1] = ldg_stream(p + 8);
-            } else {
-                v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i) {
-            const int rl = (i0 + i) * kRowsPerPass + warp * 4 + (lane >> 3);
-            quantize_seg16<FMT, RULE_OCP>(v[i][0], v[i][1], row0 + rl, M, col, K, col0, rl, cl, lane, ns, nvt, codes,
-                                          sf_tile);
+    for (int i = 0; i < R::kPasses; ++i) {
+        const int64_t row = row0 + i * R::kRowsPerPass + warp * 4 + (lane >> 3);
+        if (row < M && col < K) {
+            const uint16_t *p = src + row * ld + col;
+            r.v[i][0] = ldg_stream(p);
+            r.v[i][1] = ldg_stream(p + 8);
+        } else {
+            r.v[i][0] = r.v[i][1] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
-    sync();
-    store_sf_chunks<FMT>(sf_tile, scales, band, tile_x, sf_tiles_k, t);
+}
+
+template <int FMT, int NT, int ROWS>
+MX_DEVICE_INLINE void tile_quantize(const TileRegs<NT, ROWS> &r, int64_t M, int64_t K, int64_t band_row0, int rl0,
+                                    int64_t col0, const NvScale &ns, const NvTables *nvt,
+                                    uint8_t *__restrict__ codes, uint8_t *sf_tile, int t) {
+    using R = TileRegs<NT, ROWS>;
+    const int lane = t & 31, warp = t >> 5;
+    const int cl = (lane & 7) * 16;
+#pragma unroll
+    for (int i = 0; i < R::kPasses; ++i) {
+        const int rl = rl0 + i * R::kRowsPerPass + warp * 4 + (lane >> 3);
+        quantize_seg16<FMT, RULE_OCP>(r.v[i][0], r.v[i][1], band_row0 + rl, M, col0 + cl, K, col0, rl, cl, lane, ns,
+                                      nvt, codes, sf_tile);
+    }
 }
 
 // src bf16 [M x K] (row pitch ld).  codes / scales as in mx.h.  sf_tiles_k =
 // ceil((K / block) / 4) 512-byte tiles per 128-row band.  NVFP4: *gscale_in
 // is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
-// if gscale_out != nullptr, CTA 0 also stores g there.
+// if gscale_out != nullptr, CTA 0 also stores g there.  band_ready (nullable):
+// each CTA adds one to its 128-row band's counter once its codes and scales
+// are written (release, gpu scope).
 // CTAs per SM that the register allocation of quantize_kernel<FMT> targets,
 // chosen by timing 2^28-element inputs: the FP8 and FP4 MX casts run fastest
 // with the registers left free (1), NVFP4 with four resident CTAs (the
@@ -555,7 +562,8 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
                                                              int64_t ld, uint8_t *__restrict__ codes,
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
                                                              const float *__restrict__ gscale_in,
-                                                             float *__restrict__ gscale_out, int g_from_amax) {
+                                                             float *__restrict__ gscale_out, int g_from_amax,
+                                                             uint32_t *__restrict__ band_ready) {
     constexpr int kPasses = kQTileRows / 32;               // 32 rows per pass (8 warps x 4 rows)
     __shared__ __align__(16) uint8_t sf_tile[quantize_sf_bytes<FMT>()];
 
@@ -603,6 +611,13 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
     }
     __syncthreads();
     store_sf_chunks<FMT>(sf_tile, scales, blockIdx.y, blockIdx.x, sf_tiles_k, threadIdx.x);
+    if (band_ready != nullptr) {
+        // a GEMM of the same fused call reads this tile with TMA as soon as its
+        // band's count is complete (one count per CTA of the band)
+        fence_proxy_async_global();
+        __syncthreads();
+        if (threadIdx.x == 0) red_release_gpu_add(band_ready + blockIdx.y, 1u);
+    }
 }
 
 // ------------------------------------------------------------------ MXFP4 with macro-block scaling

@@ -28,7 +28,8 @@ MX_ERR_CUDA, MX_ERR_TIMEOUT, MX_ERR_DEVICE = 4, 5, 6
 MX_EPI_NONE, MX_EPI_GELU = 0, 1
 MX_DEBUG_WAIT_LIMIT_NS, MX_DEBUG_SKIP_PRODUCER, MX_DEBUG_PAIR_GEMM, MX_DEBUG_OVERLAP_LAUNCH = 1, 2, 3, 4
 MX_DEBUG_MAX_GEMM_CTAS = 5
-MX_DEBUG_FUSED_TWO_KERNELS = 6
+MX_DEBUG_FUSED_MODE = 6
+MX_FUSED_PIPELINED, MX_FUSED_IN_KERNEL, MX_FUSED_TWO_KERNELS = 0, 1, 2
 
 EXPORTED = [
     "mx_codes_bytes", "mx_scales_bytes", "mx_block_size", "mx_quantize", "mx_dequantize", "mx_gemm",

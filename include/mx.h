@@ -198,14 +198,15 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  * is fmt or, as in mx_gemm, any MX format that pairs with it (e.g. MXFP8
  * activations with MXFP4 or MXFP6 weights).  X is quantized exactly as
  * mx_quantize would (same codes and scales, bit for bit) once, into the
- * caller's `workspace`, by the GEMM kernel itself: the epilogue warps of every
- * CTA (idle until the first accumulator is ready) share X's 128 x 128 tiles,
- * band by band, and the TMA producers load A from a 128-row band as soon as
- * its tiles are written (per-band counters in the workspace).  The result is
- * C = X_dq * W_dq^T as in mx_gemm.  X's quantized form is not an output of
- * this call.  Launches: the GEMM kernel and a one-thread-block kernel that
- * clears the workspace's counters (NVFP4 without x_gscale or x_amax: also the
- * amax pre-pass).
+ * caller's `workspace`, 128-row band by band, and the GEMM's TMA producers
+ * load A from a band as soon as its count in the workspace says it is written
+ * (by default the quantize kernel writes X while the GEMM kernel, launched to
+ * overlap it, starts on the bands already done; MX_DEBUG_FUSED_MODE selects
+ * the quantize inside the GEMM kernel instead).  The result is C = X_dq *
+ * W_dq^T as in mx_gemm.  X's quantized form is not an output of this call.
+ * Launches: a one-thread-block kernel that clears the workspace's counters,
+ * the quantize kernel and the GEMM kernel (NVFP4 without x_gscale or x_amax:
+ * also the amax pre-pass).
  *   workspace: device buffer of at least mx_fused_workspace_bytes(fmt, M, K)
  *              bytes, 256-byte aligned; its contents are scratch, and calls
  *              that overlap on the GPU must not share one.
@@ -289,10 +290,19 @@ int mx_version(void);
  *                            0 (default) = one CTA per SM.  The result does
  *                            not depend on it (each tile is summed in the
  *                            same order wherever it runs).
- *   MX_DEBUG_FUSED_TWO_KERNELS: 1 = mx_gemm_fused_act runs the quantize kernel
- *                            and then the GEMM kernel (two launches) instead of
- *                            quantizing X inside the GEMM kernel; 0 (default)
- *                            = one GEMM kernel.  Same results bit for bit.
+ *   MX_DEBUG_FUSED_MODE    : how mx_gemm_fused_act runs (same results bit for
+ *                            bit in every mode):
+ *                            MX_FUSED_PIPELINED (default): the quantize kernel
+ *                            counts each 128-row band of X as written, and the
+ *                            GEMM kernel, launched to overlap it, loads a band
+ *                            of A as soon as its count is complete (an X of at
+ *                            most 128 rows, one band, runs as
+ *                            MX_FUSED_TWO_KERNELS);
+ *                            MX_FUSED_IN_KERNEL: one GEMM kernel whose epilogue
+ *                            warps (idle until the first accumulator) quantize
+ *                            X band by band before their first tile;
+ *                            MX_FUSED_TWO_KERNELS: the quantize kernel, then the
+ *                            GEMM kernel after it has completed.
  * Returns MX_ERR_INVALID_ARG for an unknown key. */
 typedef enum {
     MX_DEBUG_WAIT_LIMIT_NS = 1,
@@ -300,8 +310,14 @@ typedef enum {
     MX_DEBUG_PAIR_GEMM = 3,
     MX_DEBUG_OVERLAP_LAUNCH = 4,
     MX_DEBUG_MAX_GEMM_CTAS = 5,
-    MX_DEBUG_FUSED_TWO_KERNELS = 6
+    MX_DEBUG_FUSED_MODE = 6
 } mx_debug_key;
+/* Values of MX_DEBUG_FUSED_MODE. */
+typedef enum {
+    MX_FUSED_PIPELINED = 0,
+    MX_FUSED_IN_KERNEL = 1,
+    MX_FUSED_TWO_KERNELS = 2
+} mx_fused_mode;
 mx_status mx_debug_set(int key, uint64_t value);
 
 #ifdef __cplusplus

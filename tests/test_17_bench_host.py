@@ -94,8 +94,8 @@ def test_result_line_keeps_the_contract(bench):
     import argparse
     args = argparse.Namespace(steps=50, warmup=5, workload="dit_mxfp8")
     wl = bench.WORKLOADS["dit_mxfp8"]
-    r = {"ms": 50 * 0.049, "g_ms": [0.0405] * 50, "q_ms": [0.0085] * 50, "g_ms_iso": [0.044] * 50,
-         "q_ms_iso": [0.009] * 50, "e2e_ms": 50 * 0.55, "eager_ms": 50 * 0.048, "n_sets": 6,
+    r = {"ms": 50 * 0.049, "f_ms": [0.0405] * 50, "f_ms_iso": [0.044] * 50, "two_ms": 0.052, "q_ms": 0.0099,
+         "g_ms": 0.042, "e2e_ms": 50 * 0.55, "eager_ms": 50 * 0.048, "n_sets": 6,
          "per_set": 73_000_000, "h2d": 4096 * 3072 * 2, "d2h": 4096 * 3072 * 2,
          "clocks": {"sm_mhz": 1762.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}}
     for world in (1, 2):
@@ -109,7 +109,7 @@ def test_result_line_keeps_the_contract(bench):
         assert line["higher_is_better"] is True and line["vs_baseline"] is None
         assert line["config"]["workload"] == wl["name"]
         roof = line["roofline"]
-        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6>"
+        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6> (fused quantize)"
         assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"], rel=1e-3)
         assert roof["peak"] == pytest.approx(bench.tensor_peak(0, bench.measured_peaks()[0], False), rel=1e-3)
         assert roof["clock_normalised_kernel_us"] == pytest.approx(40.5 * 1762 / 1965, abs=0.01)
@@ -117,12 +117,15 @@ def test_result_line_keeps_the_contract(bench):
         assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
         assert line["e2e"]["h2d_bytes_per_step"] == r["h2d"]
         assert line["gpu_launches"] == 2 * 50
+        split = line["two_kernel_split"]
+        assert split["step_us"] == pytest.approx(52.0) and split["gemm_us"] == pytest.approx(42.0)
+        assert split["quantize_GB/s"] == pytest.approx(4096 * 3072 * 3.03125 / 9.9e-6 / 1e9, rel=1e-3)
     # the skinny workload's GEMM is reported against HBM
     args.workload = "skinny_nvfp4"
-    line = bench.result_line(args, bench.WORKLOADS["skinny_nvfp4"], dict(r, g_ms=[0.025] * 50), 1)
+    line = bench.result_line(args, bench.WORKLOADS["skinny_nvfp4"], dict(r, f_ms=[0.025] * 50), 1)
     assert line["roofline"]["bound"] == "hbm" and line["roofline"]["unit"] == "GB/s"
-    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32>"
-    assert line["gpu_launches"] == 4 * 50
+    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32> (fused quantize)"
+    assert line["gpu_launches"] == 3 * 50
     json_line = __import__("json").dumps(line)
     assert "\n" not in json_line
 
