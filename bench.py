@@ -64,7 +64,7 @@ def tensor_peak(fmt: int, peaks: dict, sustained: bool):
     times the nominal ratio (fp8 = 2x bf16, fp4 = 4x bf16; MXFP6 and mixed MX
     operands run on kind::mxf8f6f4 at the fp8 rate)."""
     base = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    return base * (4.0 if fmt in (2, 3) else 2.0)
+    return base * (4.0 if fmt in (2, 3, 5) else 2.0)
 
 
 class ClockSampler:
@@ -532,7 +532,8 @@ def extras_gpu(device):
             "skinny_nvfp4_M128": (3, 3, 128, 28672, 8192),
             "dit_mxfp8_gemm_back_to_back": (0, 0, 4096, 3072, 3072),
             "dit_mxfp6_gemm": (4, 4, 4096, 3072, 3072), "dit_mxfp8_x_mxfp4w_gemm": (0, 2, 4096, 3072, 3072),
-            "dit_mxfp8_x_mxfp6w_gemm": (0, 4, 4096, 3072, 3072)}.items():
+            "dit_mxfp8_x_mxfp6w_gemm": (0, 4, 4096, 3072, 3072),
+            "dit_mxfp4_gemm": (2, 2, 4096, 3072, 3072), "dit_mxfp4_mbs_gemm": (5, 5, 4096, 3072, 3072)}.items():
         a = torch.randn((M, K), generator=g, device=device).to(torch.bfloat16)
         w = (torch.randn((N, K), generator=g, device=device) * 0.02).to(torch.bfloat16)
         qa = mx.quantize(a, fmt)
@@ -548,6 +549,11 @@ def extras_gpu(device):
                      "frac_tensor": round(tf / tensor_peak(fmt if fmt == wfmt else 0, peaks, False), 3),
                      "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
         del a, w, qa, qws, C
+    # the macro-block-scaled GEMM's cost over the plain MXFP4 GEMM on the same
+    # shape (the MXFP4 paper page's section 4 quotes 6.2% at prefill with
+    # dedicated vector units beside the tensor cores)
+    out["dit_mxfp4_mbs_gemm"]["overhead_vs_mxfp4"] = round(
+        out["dit_mxfp4_mbs_gemm"]["us"] / out["dit_mxfp4_gemm"]["us"] - 1.0, 3)
     # The skinny weight-stream GEMMs as the configuration states them: bf16
     # activations X [M x 8192] ~ N(0, 1), quantized inside the fused call (NVFP4:
     # g from X's amax pre-pass), times pre-quantized weights [28672 x 8192];

@@ -18,6 +18,7 @@
 #include "rotate.cuh"
 #include "gemm_sm100.cuh"
 #include "gemm_pair_sm100.cuh"
+#include "gemm_mbs_sm100.cuh"
 
 namespace {
 
@@ -139,8 +140,10 @@ uint32_t f8f6f4_type(int fmt) {
 }
 // Can A and B be multiplied, and on which kernel: the format's own (same
 // format, 0..3) or the run-time-typed kind::mxf8f6f4 one.
-bool gemm_pair_ok(int fa, int fb) { return (fa == fb && fa <= MX_NVFP4) || (f8f6f4_fmt(fa) && f8f6f4_fmt(fb)); }
-bool gemm_runtime_types(int fa, int fb) { return !(fa == fb && fa <= MX_NVFP4); }
+bool gemm_pair_ok(int fa, int fb) {
+    return (fa == fb && (fa <= MX_NVFP4 || fa == MX_MXFP4_MBS)) || (f8f6f4_fmt(fa) && f8f6f4_fmt(fb));
+}
+bool gemm_runtime_types(int fa, int fb) { return !(fa == fb && (fa <= MX_NVFP4 || fa == MX_MXFP4_MBS)); }
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // --- quantize ------------------------------------------------------------
@@ -468,6 +471,48 @@ mx_status launch_gemm(const mx_tensor *A, const mx_tensor *B, const void *a_code
     }
 }
 
+// MXFP4-MBS x MXFP4-MBS (gemm_mbs_sm100.cuh): one CTA per 128 x 128 tile.
+mx_status launch_gemm_mbs(const mx_tensor *A, const mx_tensor *B, uint16_t *C, int64_t ldc, cudaStream_t st) {
+    using L = MbsLayout;
+    const int64_t M = A->rows, N = B->rows, K = A->cols;
+    const int64_t kbytes = K / 2;
+    const int64_t sf_tiles_k = cdiv(K / 16, 4);
+    CUtensorMap ta, tb, tsa, tsb;
+    if (!make_tmap_u8(&ta, A->codes, M, kbytes, 128)) return MX_ERR_CUDA;
+    if (!make_tmap_u8(&tb, B->codes, N, kbytes, 128)) return MX_ERR_CUDA;
+    if (!make_tmap_sf(&tsa, A->scales, cdiv(M, 128), sf_tiles_k, 4, 1)) return MX_ERR_CUDA;
+    if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, 4, 1)) return MX_ERR_CUDA;
+    if (smem_limit_once(reinterpret_cast<const void *>(gemm_mbs_kernel), L::kAlloc) != cudaSuccess)
+        return MX_ERR_CUDA;
+    MbsParams p{};
+    p.C = C;
+    p.ldc = ldc;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.num_kt = (int)cdiv(kbytes, kStageKBytes);
+    p.n_macro = (int)(K / 128);
+    p.m_blocks = (int)cdiv(M, 128);
+    p.macro_a = A->scales + tile_bytes(MX_MXFP4_MBS, M, K);
+    p.macro_b = B->scales + tile_bytes(MX_MXFP4_MBS, N, K);
+    p.vec_store = (ldc % 8 == 0) && aligned16(C) ? 1 : 0;
+    p.skip_producer = g_skip_producer.load();
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const int64_t tiles = (int64_t)p.m_blocks * cdiv(N, kMbsBN);
+    if (tiles > INT32_MAX) return MX_ERR_UNSUPPORTED_SHAPE;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)tiles, 1, 1);
+    cfg.blockDim = dim3(kMbsThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    if (cudaLaunchKernelEx(&cfg, gemm_mbs_kernel, ta, tb, tsa, tsb, p) != cudaSuccess) return last_launch();
+    return last_launch();
+}
+
 // The fused call's workspace: a header, then X's codes and scales, each
 // starting on a 256-byte boundary.  Header words: [0] g of X (NVFP4), [1]
 // amax(|X|) of the pre-pass, [2] the fused kernel's work counter, [3] unused,
@@ -476,8 +521,7 @@ constexpr size_t kWsBandOffset = 64;
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t fused_ws_header(int64_t M) { return align256(kWsBandOffset + 4 * (size_t)cdiv(M, 128)); }
 size_t fused_ws_bytes(int fmt, int64_t M, int64_t K) {
-    return fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8)) +
-           align256((size_t)(cdiv(M, 128) * 128 * cdiv(K / fmt_block(fmt), 4) * 4));
+    return fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8)) + align256(scales_bytes(fmt, M, K));
 }
 
 // Zero the fused kernel's counters (the work counter and the band counters).
@@ -751,6 +795,7 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
     if (gemm_runtime_types(A->fmt, B->fmt) && ((fmt_bits(A->fmt) < 8 && !aligned32(A->codes)) ||
                                                (fmt_bits(B->fmt) < 8 && !aligned32(B->codes))))
         return MX_ERR_MISALIGNED;
+    if (A->fmt == MX_MXFP4_MBS) return launch_gemm_mbs(A, B, static_cast<uint16_t *>(C_bf16), ldc, st);
     return launch_gemm(A, B, A->codes, A->scales, A->gscale, static_cast<uint16_t *>(C_bf16), ldc, 0, nullptr, st,
                        nullptr);
 }
@@ -789,6 +834,21 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     const float *ga = nullptr;
     const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (fmt == MX_MXFP4_MBS) {
+        // the macro-block GEMM has the plain epilogue only
+        if (epilogue != MX_EPI_NONE || amax_out != nullptr) return MX_ERR_INVALID_ARG;
+        xa.fmt = fmt;
+        xa.reserved = 0;
+        xa.rows = M;
+        xa.cols = K;
+        xa.codes = ws + fused_ws_header(M);
+        xa.scales = ws + fused_ws_header(M) + align256((size_t)(M * K / 2));
+        xa.gscale = nullptr;
+        launch_quantize_mbs(X, M, K, ldx, &xa, st);
+        s = last_launch();
+        if (s != MX_OK) return s;
+        return launch_gemm_mbs(&xa, W, static_cast<uint16_t *>(C_bf16), ldc, st);
+    }
     int mode = g_fused_mode.load();
     // a single 128-row band is written only when the whole quantize is: no band
     // of it to start early on, so the pipelined mode would only add its counter

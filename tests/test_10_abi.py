@@ -101,7 +101,7 @@ def test_host_checks_reject_bad_arguments(L):
     assert mx.mx_quantize(4, 0x1000, 4, 48, 48, _t(4, 4, 48), None, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
     # MXFP4 with macro-block scaling: K a multiple of 128; not a GEMM or rotation format
     assert mx.mx_quantize(5, 0x1000, 4, 64, 64, _t(5, 4, 64), None, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
-    assert mx.mx_gemm(_t(5, 8, 256), _t(5, 8, 256), 0x4000, 8, None) == mx.MX_ERR_INVALID_ARG
+    assert mx.mx_gemm(_t(5, 8, 256), _t(2, 8, 256), 0x4000, 8, None) == mx.MX_ERR_INVALID_ARG   # MBS x MXFP4
     assert mx.mx_quantize_rht(5, 0x1000, 4, 256, 256, _t(5, 4, 256), None, None) == mx.MX_ERR_INVALID_ARG
     assert mx.mx_dequantize(_t(5, 4, 64), 0x4000, 64, None) == mx.MX_ERR_UNSUPPORTED_SHAPE
     assert mx.mx_gemm(A, _t(0, 8, 128), 0x4000, 8, None) == mx.MX_ERR_INVALID_ARG               # K mismatch

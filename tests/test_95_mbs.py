@@ -79,8 +79,12 @@ def test_mbs_qsnr_sums_and_gap_to_nvfp4():
     assert got[1] < s4[1] / 1.5                     # well above plain MXFP4
 
 
-def test_gemm_rejects_mbs_operands():
+def test_gemm_rejects_mbs_with_another_format():
+    """MXFP4-MBS multiplies only with MXFP4-MBS (tests/test_96_mbs_gemm.py)."""
     bits = synth.gaussian_weights(100, 128, 256)
     q = quantize_dev(bits, MBS)
-    C = torch.empty((128, 128), dtype=torch.bfloat16, device="cuda")
-    assert mx.mx_gemm(q.c(), q.c(), C.data_ptr(), 128, None) == mx.MX_ERR_INVALID_ARG
+    for other in (0, 2, 3):
+        o = quantize_dev(bits, other)
+        C = torch.empty((128, 128), dtype=torch.bfloat16, device="cuda")
+        assert mx.mx_gemm(q.c(), o.c(), C.data_ptr(), 128, None) == mx.MX_ERR_INVALID_ARG
+        assert mx.mx_gemm(o.c(), q.c(), C.data_ptr(), 128, None) == mx.MX_ERR_INVALID_ARG
