@@ -74,6 +74,9 @@ def _load():
                 "orc_amax_bf16": (d, [P, i64, i64, i64]),
                 "orc_quantize": (i32, [i32, P, i64, i64, i64, P, P, P, i32]),
                 "orc_quantize_oas": (i32, [P, i64, i64, i64, P, P]),
+                "orc_quantize_mbs_dynamic": (i32, [P, i64, i64, i64, P, P]),
+                "orc_mbs_macro_sse": (d, [P, i32]),
+                "orc_mbs_dynamic_mantissa": (i32, [P]),
                 "orc_quantize_f32": (i32, [i32, P, i64, i64, i64, P, P, P, i32]),
                 "orc_rht32_f32": (i32, [P, i64, i64, i64, P]),
                 "orc_qsnr_db": (d, [P, i64, i64, i64, P, P]),
@@ -209,6 +212,34 @@ def quantize_oas(src_bits: np.ndarray):
     if rc != 0:
         raise ValueError(f"oracle quantize_oas failed with code {rc}")
     return codes, scales
+
+
+def quantize_mbs_dynamic(src_bits: np.ndarray):
+    """MXFP4 with dynamic macro-block scaling (reading R21: per 128 elements the
+    macro mantissa of the smallest squared error) -> (codes, scales), in
+    MXFP4-MBS storage (macro bytes after the scale tiles)."""
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    M, K = src.shape
+    codes = np.zeros(codes_bytes(MXFP4_MBS, M, K), dtype=np.uint8)
+    scales = np.zeros(scales_bytes(MXFP4_MBS, M, K), dtype=np.uint8)
+    rc = _load().orc_quantize_mbs_dynamic(_ptr(src), M, K, K, _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise ValueError(f"oracle quantize_mbs_dynamic failed with code {rc}")
+    return codes, scales
+
+
+def mbs_macro_sse(block_values: np.ndarray, m: int) -> float:
+    """fp64 squared error of one 128-value macro block quantized with macro
+    mantissa m (reading R21's sum, in element order)."""
+    v = np.ascontiguousarray(block_values, dtype=np.float64)
+    assert v.shape == (128,)
+    return float(_load().orc_mbs_macro_sse(_ptr(v), int(m)))
+
+
+def mbs_dynamic_mantissa(block_values: np.ndarray) -> int:
+    v = np.ascontiguousarray(block_values, dtype=np.float64)
+    assert v.shape == (128,)
+    return int(_load().orc_mbs_dynamic_mantissa(_ptr(v)))
 
 
 def rht32(src_bits: np.ndarray) -> np.ndarray:

@@ -17,6 +17,7 @@ off-by-one in the scale rule, a transposed operand) shows up as a mismatch:
 """
 from __future__ import annotations
 
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -182,6 +183,41 @@ def mbs_static_mantissa(block: list[Fraction]) -> int:
         if alpha / (1 + Fraction(m, 256)) <= 6 * Fraction(2) ** e:
             return m
     return 0
+
+
+def mbs_quantize_macro(block: list[Fraction], m: int, negative: list[bool]):
+    """One macro block (128 exact values) quantized with macro mantissa m:
+    per 16 the smallest E with every |x| / ((1 + m/256) 2^(E-127)) <= 6, the
+    nearest E2M1 value of each quotient (ties to the even code).  Returns
+    (codes[128], exponents[8], values xhat[128])."""
+    f = 1 + Fraction(m, 256)
+    codes, exps, xhat = [], [], []
+    for jb in range(8):
+        blk = block[jb * 16:(jb + 1) * 16]
+        amax = max(abs(x) for x in blk)
+        # the smallest E with amax <= 6 f 2^(E-127): a float estimate, settled exactly
+        E = 0 if amax == 0 else min(254, max(0, math.ceil(math.log2(float(amax / (6 * f)))) + 127))
+        while E > 0 and amax <= 6 * f * Fraction(2) ** (E - 1 - 127):
+            E -= 1
+        while E < 254 and amax > 6 * f * Fraction(2) ** (E - 127):
+            E += 1
+        exps.append(E)
+        denom = f * Fraction(2) ** (E - 127)
+        for i, x in enumerate(blk):
+            c = round_to_grid(x / denom, E2M1_GRID, 0x8, negative[jb * 16 + i])
+            codes.append(c)
+            xhat.append(e2m1(c) * denom)
+    return codes, exps, xhat
+
+
+def mbs_dynamic_choice(block: list[Fraction], negative: list[bool]):
+    """Every macro mantissa's exact squared error of the block: a list of 256
+    Fractions sum (x - xhat)^2."""
+    out = []
+    for m in range(256):
+        _, _, xhat = mbs_quantize_macro(block, m, negative)
+        out.append(sum(((x - h) ** 2 for x, h in zip(block, xhat)), Fraction(0)))
+    return out
 
 
 def quantize_mbs(bits: np.ndarray):

@@ -56,6 +56,14 @@
  *       (0 if alpha == 0 or none suffices).  Each base block then takes the MX
  *       rule on x / (1 + m/256) and RNE elements of that quotient.  The
  *       macro bytes are stored after the scale tiles, row-major [rows][K/128].
+ *   R21 MXFP4 with dynamic macro-block scaling [OAS/MBS page, section B, the
+ *       variant whose macro factor minimises the squared error]: the same
+ *       storage and per-m quantization as R20, with m = the byte in [0, 255]
+ *       whose quantization of the macro block has the smallest sum of squared
+ *       errors sum_i (x_i - xhat_i)^2, the terms (each exact in fp64) added in
+ *       element order in fp64; ties go to the smallest m.  (The page names a
+ *       lookup table computed to minimise the error; an exhaustive search is
+ *       the error-minimising choice that table stands for.)
  */
 #include <math.h>
 #include <stdint.h>
@@ -440,6 +448,8 @@ static uint8_t e2m1_encode_quotient(double x, double denom) {
     return (uint8_t)(c | (signbit(x) ? 0x8 : 0));
 }
 
+int orc_mbs_dynamic_mantissa(const double *mac);
+
 /* Quantize a dense row-major [M x K] matrix of exactly-held values xv (fp64).
  * codes: orc_codes_bytes bytes; scales: orc_scales_bytes bytes (fully written,
  * padding 0).  NVFP4: if gscale_given, *gscale is used as g, else g is computed
@@ -447,7 +457,7 @@ static uint8_t e2m1_encode_quotient(double x, double denom) {
  * |x| is mapped at or below by the MX scale (the format's largest element for
  * the OCP rule). */
 static int quantize_core(int fmt, double mx_threshold, const double *xv, int64_t M, int64_t K, uint8_t *codes,
-                         uint8_t *scales, float *gscale, int gscale_given) {
+                         uint8_t *scales, float *gscale, int gscale_given, int mbs_dynamic) {
     build_tables();
     int bs = fmt_block(fmt);
     int64_t sf_cols = K / bs;
@@ -466,17 +476,23 @@ static int quantize_core(int fmt, double mx_threshold, const double *xv, int64_t
         }
     }
     if (fmt == ORC_MXFP4_MBS) {
-        /* [reading R20]: macro mantissa per 128 elements, then 16-element
-         * blocks on x / (1 + m/256), elements decided by exact comparisons
-         * with the quotient's E2M1 midpoints (denominator (256+m) 2^(E-135)). */
+        /* [reading R20]: macro mantissa per 128 elements (R21: by error
+         * search), then 16-element blocks on x / (1 + m/256), elements decided
+         * by exact comparisons with the quotient's E2M1 midpoints (denominator
+         * (256+m) 2^(E-135)). */
         #pragma omp parallel for schedule(static)
         for (int64_t r = 0; r < M; ++r) {
             for (int64_t mb = 0; mb < K / 128; ++mb) {
                 const double *mac = xv + r * K + mb * 128;
-                double alpha = 0.0;
-                for (int i = 0; i < 128; ++i)
-                    if (fabs(mac[i]) > alpha) alpha = fabs(mac[i]);
-                int m = orc_mbs_static_mantissa(alpha);
+                int m;
+                if (mbs_dynamic) {
+                    m = orc_mbs_dynamic_mantissa(mac);
+                } else {
+                    double alpha = 0.0;
+                    for (int i = 0; i < 128; ++i)
+                        if (fabs(mac[i]) > alpha) alpha = fabs(mac[i]);
+                    m = orc_mbs_static_mantissa(alpha);
+                }
                 scales[orc_mbs_macro_offset(M, K, r, mb)] = (uint8_t)m;
                 for (int jb = 0; jb < 8; ++jb) {
                     const double *blk = mac + jb * 16;
@@ -527,9 +543,48 @@ static int quantize_core(int fmt, double mx_threshold, const double *xv, int64_t
     return ORC_OK;
 }
 
+/* [reading R21] the squared error of one macro block (128 values) quantized
+ * with macro mantissa m: per 16-element base block the exponent of R20, each
+ * element's E2M1 value times (256 + m) 2^(E - 135) as xhat; every term
+ * (x - xhat)^2 is exact in fp64 (xhat is 0 or within a factor of 3 of |x|, so
+ * x - xhat has at most 22 significant bits), added in element order. */
+double orc_mbs_macro_sse(const double *mac, int m) {
+    double sse = 0.0;
+    for (int jb = 0; jb < 8; ++jb) {
+        const double *blk = mac + jb * 16;
+        double amax = 0.0;
+        for (int i = 0; i < 16; ++i)
+            if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
+        int E = orc_mbs_block_exponent(amax, m);
+        double denom = ldexp((double)(256 + m), E - 135);
+        for (int i = 0; i < 16; ++i) {
+            uint8_t q = e2m1_encode_quotient(blk[i], denom);
+            double xhat = orc_e2m1_decode(q) * denom;
+            double d = blk[i] - xhat;
+            sse = sse + d * d;
+        }
+    }
+    return sse;
+}
+
+/* [reading R21] the macro mantissa of the smallest squared error (ties: the
+ * smallest m). */
+int orc_mbs_dynamic_mantissa(const double *mac) {
+    int best = 0;
+    double best_sse = orc_mbs_macro_sse(mac, 0);
+    for (int m = 1; m < 256; ++m) {
+        double e = orc_mbs_macro_sse(mac, m);
+        if (e < best_sse) {
+            best_sse = e;
+            best = m;
+        }
+    }
+    return best;
+}
+
 /* bf16 source with row pitch ld: checks, widening to fp64 (exact), quantize. */
 static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
-                         uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
+                         uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given, int mbs_dynamic) {
     int bs = fmt_block(fmt);
     if (!fmt_ok(fmt) || M < 0 || K < 0 || K % bs != 0 || ld < K) return ORC_EINVAL;
     if (fmt == ORC_MXFP4_MBS && K % 128 != 0) return ORC_EINVAL;
@@ -544,7 +599,7 @@ static int quantize_impl(int fmt, double mx_threshold, const uint16_t *src, int6
             }
             xv[r * K + k] = x;
         }
-    int rc = quantize_core(fmt, mx_threshold, xv, M, K, codes, scales, gscale, gscale_given);
+    int rc = quantize_core(fmt, mx_threshold, xv, M, K, codes, scales, gscale, gscale_given, mbs_dynamic);
     free(xv);
     return rc;
 }
@@ -566,7 +621,7 @@ int orc_quantize_f32(int fmt, const float *src, int64_t M, int64_t K, int64_t ld
             }
             xv[r * K + k] = x;
         }
-    int rc = quantize_core(fmt, fmt_maxelem(fmt), xv, M, K, codes, scales, gscale, gscale_given);
+    int rc = quantize_core(fmt, fmt_maxelem(fmt), xv, M, K, codes, scales, gscale, gscale_given, 0);
     free(xv);
     return rc;
 }
@@ -602,7 +657,14 @@ int orc_rht32_f32(const uint16_t *src, int64_t M, int64_t K, int64_t ld, float *
 
 int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
                  uint8_t *codes, uint8_t *scales, float *gscale, int gscale_given) {
-    return quantize_impl(fmt, fmt_maxelem(fmt), src, M, K, ld, codes, scales, gscale, gscale_given);
+    return quantize_impl(fmt, fmt_maxelem(fmt), src, M, K, ld, codes, scales, gscale, gscale_given, 0);
+}
+
+/* MXFP4 with dynamic macro-block scaling [reading R21]: MXFP4-MBS storage,
+ * the macro mantissa of each 128 elements chosen by the squared-error search. */
+int orc_quantize_mbs_dynamic(const uint16_t *src, int64_t M, int64_t K, int64_t ld, uint8_t *codes,
+                             uint8_t *scales) {
+    return quantize_impl(ORC_MXFP4_MBS, 6.0, src, M, K, ld, codes, scales, NULL, 0, 1);
 }
 
 /* MXFP4 with overflow-aware scaling [OAS page, section 2.A]: the block scale
@@ -610,7 +672,7 @@ int orc_quantize(int fmt, const uint16_t *src, int64_t M, int64_t K, int64_t ld,
  * E = ceil(log2(max_val / 7)) + 127; elements above 6 after scaling saturate
  * to 6 as any E2M1 value does.  Same storage as MXFP4. */
 int orc_quantize_oas(const uint16_t *src, int64_t M, int64_t K, int64_t ld, uint8_t *codes, uint8_t *scales) {
-    return quantize_impl(ORC_MXFP4, 7.0, src, M, K, ld, codes, scales, NULL, 0);
+    return quantize_impl(ORC_MXFP4, 7.0, src, M, K, ld, codes, scales, NULL, 0, 0);
 }
 
 /* Quantization SNR in dB [OAS page, section 3: "QSNR"]: 10 log10(sum x^2 /
