@@ -358,7 +358,8 @@ def qsnr_table(device):
         row = {}
         for label, quant in (("mxfp8_e4m3", lambda: mx.quantize(x, 0)), ("mxfp4", lambda: mx.quantize(x, 2)),
                              ("mxfp4_oas", lambda: mx.quantize_oas(x)), ("nvfp4", lambda: mx.quantize(x, 3)),
-                             ("mxfp6_e3m2", lambda: mx.quantize(x, 4)), ("mxfp4_mbs", lambda: mx.quantize(x, 5))):
+                             ("mxfp6_e3m2", lambda: mx.quantize(x, 4)), ("mxfp4_mbs", lambda: mx.quantize(x, 5)),
+                             ("mxfp4_mbs_dynamic", lambda: mx.quantize_mbs_dynamic(x))):
             s = mx.qsnr_sums(quant(), x).cpu().numpy()
             row[label] = round(float(10.0 * np.log10(s[0] / s[1])), 3)
         for label, fmt in (("mxfp4_rht32", 2), ("nvfp4_rht32", 3)):
@@ -511,6 +512,16 @@ def extras_gpu(device):
         sweep[f"{name}_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
                                  "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
         del qs
+    # MXFP4 with dynamic macro-block scaling: an exhaustive search over the 256
+    # macro mantissas of every macro block (compute-bound; same bytes as MBS)
+    Md = 4096
+    xsd = [torch.randn((Md, K), generator=g, device=device).to(torch.bfloat16) for _ in range(2)]
+    qsd = [mx.empty(5, Md, K) for _ in xsd]
+    ms = timed(lambda i: mx.quantize_mbs_dynamic(xsd[i % 2], out=qsd[i % 2]), 2, reps=4)
+    gbs = Md * K * quant_bytes_per_elem(5) / (ms * 1e-3) / 1e9
+    sweep[f"mxfp4_mbs_dynamic_M{Md}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                         "macro_blocks_per_s": round(Md * K / 128 / (ms * 1e-3), 1)}
+    del xsd, qsd
     # Walsh-Hadamard rotation fused with quantization: the same HBM bytes as the plain quantize
     for fmt, name in ((2, "mxfp4_rht32"), (3, "nvfp4_rht32")):
         qs = [mx.empty(fmt, M, K) for _ in xs]

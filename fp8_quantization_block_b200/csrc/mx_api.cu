@@ -685,6 +685,25 @@ mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld
     return last_launch();
 }
 
+mx_status mx_quantize_mbs_dynamic(const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
+                                  void *stream) {
+    if (!dst || dst->fmt != MX_MXFP4_MBS || M < 0 || K < 0) return MX_ERR_INVALID_ARG;
+    if (dst->rows != M || dst->cols != K) return MX_ERR_INVALID_ARG;
+    if (K % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || K == 0) return MX_OK;
+    if (!src_bf16 || !dst->codes || !dst->scales) return MX_ERR_INVALID_ARG;
+    if (ld_src < K || (ld_src & 7) != 0) return MX_ERR_MISALIGNED;
+    if (!aligned16(src_bf16) || !aligned16(dst->codes) || !aligned16(dst->scales)) return MX_ERR_MISALIGNED;
+    if (M > 65535 || K / 128 > INT32_MAX) return MX_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // padding bytes of the scale tiles and of the macro section stay zero
+    if (cudaMemsetAsync(dst->scales, 0, scales_bytes(MX_MXFP4_MBS, M, K), st) != cudaSuccess) return MX_ERR_CUDA;
+    quantize_mbs_dynamic_kernel<<<dim3((unsigned)(K / 128), (unsigned)M, 1), 256, 0, st>>>(
+        static_cast<const uint16_t *>(src_bf16), M, K, ld_src, static_cast<uint8_t *>(dst->codes), dst->scales,
+        cdiv(K / 16, 4), dst->scales + tile_bytes(MX_MXFP4_MBS, M, K));
+    return last_launch();
+}
+
 mx_status mx_quantize_rht(int fmt, const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
                           const float *gscale_in, void *stream) {
     if (!valid_fmt(fmt) || fmt == MX_MXFP4_MBS || !dst || M < 0 || K < 0) return MX_ERR_INVALID_ARG;

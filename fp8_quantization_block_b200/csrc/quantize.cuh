@@ -763,6 +763,128 @@ __global__ void __launch_bounds__(kQThreads) quantize_mbs_kernel(const uint16_t 
     griddep_launch_dependents();
 }
 
+// ------------------------------------------------------------------ MXFP4 with dynamic macro-block scaling
+// Same storage and per-m quantization as quantize_mbs_kernel; the macro
+// mantissa of each 1x128 macro block is the byte m in [0, 255] whose
+// quantization of the block has the smallest sum of squared errors
+// sum_i (x_i - xhat_i)^2, the terms (exact in fp64) added in element order with
+// round-to-nearest fp64 additions; ties go to the smallest m (page "Unveiling
+// the Potential of Quantization with MXFP4", section 2.B: the dynamic variant's
+// factor minimises the error).
+//
+// One CTA of 256 threads per macro block: thread t scores m = t, sequentially
+// over the 128 elements (so its sum is rounded exactly as the definition says),
+// then a (error, m) minimum over the CTA picks m, and threads 0..63 write the
+// block's codes, 0..7 its base-block exponents, thread 0 its macro byte.  The
+// element decision is exact: |x| against each E2M1 midpoint times the divisor
+// (256 + m) 2^(E - 135), products of at most 12 significant bits.  The scale
+// buffer (tiles and macro section) is cleared by the host first, so padding
+// stays zero.
+MX_DEVICE_INLINE uint32_t mbs_dyn_code(double a, double denom) {
+    const double mids[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+    uint32_t c = 0;
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+        const double t = __dmul_rn(mids[k], denom);
+        if (a > t) c = (uint32_t)k + 1u;
+        else {
+            if (a == t) c = (k & 1) ? (uint32_t)k + 1u : (uint32_t)k;   // tie: the even code
+            break;
+        }
+    }
+    return c;
+}
+
+__global__ void __launch_bounds__(256) quantize_mbs_dynamic_kernel(const uint16_t *__restrict__ src, int64_t M,
+                                                                  int64_t K, int64_t ld,
+                                                                  uint8_t *__restrict__ codes,
+                                                                  uint8_t *__restrict__ scales, int64_t sf_tiles_k,
+                                                                  uint8_t *__restrict__ macro_out) {
+    __shared__ double xs[128];
+    __shared__ uint32_t amax_bits[8];
+    __shared__ double red_e[8];
+    __shared__ uint32_t red_m[8];
+    __shared__ uint32_t chosen;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int64_t row = blockIdx.y, mb = blockIdx.x;
+    const uint16_t *x = src + row * ld + mb * 128;
+    griddep_wait();
+    if (t < 128) {
+        xs[t] = (double)__uint_as_float((uint32_t)x[t] << 16);
+        // base-block maxima of the magnitude bits (16 lanes per block)
+        uint32_t mbits = (uint32_t)x[t] & 0x7FFFu;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mbits = max(mbits, __shfl_xor_sync(0xffffffffu, mbits, o));
+        if ((t & 15) == 0) amax_bits[t >> 4] = mbits;
+    }
+    __syncthreads();
+    // score m = t
+    const uint32_t m = (uint32_t)t;
+    double sse = 0.0;
+    for (int jb = 0; jb < 8; ++jb) {
+        const uint32_t E = mbs_block_exponent(amax_bits[jb], m);
+        const double denom = ldexp((double)(256u + m), (int)E - 135);
+        for (int i = 0; i < 16; ++i) {
+            const double v = xs[jb * 16 + i];
+            const double a = fabs(v);
+            const uint32_t c = mbs_dyn_code(a, denom);
+            const double mag = __dmul_rn((double)e2m1_mag(c), denom);
+            const double d = __dsub_rn(a, mag);    // |x - xhat| (same sign on both)
+            sse = __dadd_rn(sse, __dmul_rn(d, d));
+        }
+    }
+    // (error, m) minimum: within the warp, then over the 8 warps
+    uint32_t bm = m;
+    double be = sse;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double oe = __shfl_xor_sync(0xffffffffu, be, o);
+        const uint32_t om = __shfl_xor_sync(0xffffffffu, bm, o);
+        if (oe < be || (oe == be && om < bm)) {
+            be = oe;
+            bm = om;
+        }
+    }
+    if (lane == 0) {
+        red_e[warp] = be;
+        red_m[warp] = bm;
+    }
+    __syncthreads();
+    if (t == 0) {
+        double e = red_e[0];
+        uint32_t mm = red_m[0];
+        for (int w = 1; w < 8; ++w)
+            if (red_e[w] < e || (red_e[w] == e && red_m[w] < mm)) {
+                e = red_e[w];
+                mm = red_m[w];
+            }
+        chosen = mm;
+        macro_out[row * (K / 128) + mb] = (uint8_t)mm;
+    }
+    __syncthreads();
+    const uint32_t mc = chosen;
+    if (t < 64) {
+        // elements 2t and 2t + 1 (one byte of codes)
+        const int jb = (2 * t) >> 4;
+        const uint32_t E = mbs_block_exponent(amax_bits[jb], mc);
+        const double denom = ldexp((double)(256u + mc), (int)E - 135);
+        uint32_t byte = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const double v = xs[2 * t + h];
+            const uint32_t c = mbs_dyn_code(fabs(v), denom) | (signbit(v) ? 8u : 0u);
+            byte |= c << (4 * h);
+        }
+        codes[row * (K / 2) + mb * 64 + t] = (uint8_t)byte;
+    } else if (t < 72) {
+        const int jb = t - 64;
+        const int64_t j = mb * 8 + jb;   // base-block column
+        const uint32_t E = mbs_block_exponent(amax_bits[jb], mc);
+        scales[((row >> 7) * sf_tiles_k + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3)] =
+            (uint8_t)E;
+    }
+}
+
 // max |x| over a bf16 tensor -> atomicMax on the float bits of *amax (init 0).
 // Persistent: CTA b walks the 128 x 128 tiles n-1-b, n-1-b-G, ... (G CTAs), a
 // thread issuing its 8 16-byte loads of a tile (4 rows x 16 columns, as in

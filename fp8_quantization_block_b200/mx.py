@@ -35,7 +35,7 @@ EXPORTED = [
     "mx_codes_bytes", "mx_scales_bytes", "mx_block_size", "mx_quantize", "mx_dequantize", "mx_gemm",
     "mx_gemm_fused_act", "mx_fused_workspace_bytes", "mx_check_device_error", "mx_status_string",
     "mx_version", "mx_debug_set", "mx_gemm_fused_act_noalloc", "mx_quantize_oas", "mx_qsnr",
-    "mx_quantize_rht",
+    "mx_quantize_rht", "mx_quantize_mbs_dynamic",
 ]
 MX_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
                 "mx_quantize": (i32, [i32, P, i64, i64, i64, T, P, P]),
                 "mx_dequantize": (i32, [T, P, i64, P]),
                 "mx_quantize_oas": (i32, [P, i64, i64, i64, T, P]),
+                "mx_quantize_mbs_dynamic": (i32, [P, i64, i64, i64, T, P]),
                 "mx_quantize_rht": (i32, [i32, P, i64, i64, i64, T, P, P]),
                 "mx_qsnr": (i32, [T, P, i64, P, P]),
                 "mx_gemm": (i32, [T, T, P, i64, P]),
@@ -110,6 +111,10 @@ def mx_quantize(fmt, src_ptr, M, K, ld, dst: MxTensorC, gscale_in_ptr, stream) -
 
 def mx_quantize_oas(src_ptr, M, K, ld, dst: MxTensorC, stream) -> int:
     return int(lib().mx_quantize_oas(src_ptr, M, K, ld, ctypes.byref(dst), stream))
+
+
+def mx_quantize_mbs_dynamic(src_ptr, M, K, ld, dst: MxTensorC, stream) -> int:
+    return int(lib().mx_quantize_mbs_dynamic(src_ptr, M, K, ld, ctypes.byref(dst), stream))
 
 
 def mx_quantize_rht(fmt, src_ptr, M, K, ld, dst: MxTensorC, gscale_in_ptr, stream) -> int:
@@ -222,6 +227,16 @@ def quantize_oas(x: torch.Tensor, out: MxTensor | None = None, stream=None) -> M
     M, K = x.shape
     out = out if out is not None else empty(MX_MXFP4, M, K, x.device)
     check(mx_quantize_oas(x.data_ptr(), M, K, x.stride(0), out.c(), _stream(stream)), "mx_quantize_oas")
+    return out
+
+
+def quantize_mbs_dynamic(x: torch.Tensor, out: MxTensor | None = None, stream=None) -> MxTensor:
+    """bf16 [M, K] CUDA tensor -> MXFP4-MBS MxTensor whose macro factors minimise the squared error."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    out = out if out is not None else empty(MX_MXFP4_MBS, M, K, x.device)
+    check(mx_quantize_mbs_dynamic(x.data_ptr(), M, K, x.stride(0), out.c(), _stream(stream)),
+          "mx_quantize_mbs_dynamic")
     return out
 
 

@@ -46,11 +46,13 @@ extern "C" {
 
 /* Element formats.  Block size 32 with an E8M0 scale for the four MX formats;
  * block size 16 with an E4M3 scale plus one FP32 per-tensor scale for NVFP4;
- * MXFP4_MBS ([OAS] section B, macro block scaling, static variant): E2M1 in
- * blocks of 16 with E8M0 scales, plus one byte m per 128 elements (a factor
- * 1 + m/256 on the whole macro block).  MXFP4_MBS is a storage and fidelity
- * format: quantize, dequantize and QSNR take it; the GEMM does not (the tensor
- * core applies only E8M0 / E4M3 block scales).
+ * MXFP4_MBS ([OAS] section B, macro block scaling): E2M1 in blocks of 16 with
+ * E8M0 scales, plus one byte m per 128 elements (a factor 1 + m/256 on the
+ * whole macro block), m from the block maximum (mx_quantize, the static
+ * variant) or by error search (mx_quantize_mbs_dynamic).  mx_gemm multiplies
+ * two MXFP4_MBS operands: the tensor core sums each macro block's products
+ * with the base-block scales, and the macro factors are applied to that
+ * partial sum on the CUDA cores.
  * E3M2 ([MX] format table, MXFP6): sign, 3 exponent bits with bias 3, 2
  * mantissa bits, no infinities or NaN, largest magnitude 28. */
 typedef enum {
@@ -143,6 +145,20 @@ mx_status mx_dequantize(const mx_tensor *src, void *dst_bf16, int64_t ld_dst, vo
  * consume it unchanged.  Same requirements as mx_quantize. */
 mx_status mx_quantize_oas(const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
                           void *stream);
+
+/* MXFP4 with dynamic macro-block scaling ([OAS] section 2.B, the variant whose
+ * macro factor minimises the quantization error): as mx_quantize(MX_MXFP4_MBS,
+ * ...) except that each 128-element macro block's mantissa byte m is the one
+ * in [0, 255] whose quantization of the block (base-block exponents and
+ * elements exactly as for the static variant, given m) has the smallest sum
+ * of squared errors sum (x - xhat)^2, the terms added in element order in
+ * fp64 (round to nearest); ties go to the smallest m.  dst is an ordinary
+ * MXFP4_MBS tensor (dst->fmt == MX_MXFP4_MBS): mx_dequantize, mx_qsnr and
+ * mx_gemm consume it unchanged.  K % 128 == 0, M <= 65535; otherwise as
+ * mx_quantize.  An exhaustive search: 256 candidates per macro block, a few
+ * hundred times the work of the static variant. */
+mx_status mx_quantize_mbs_dynamic(const void *src_bf16, int64_t M, int64_t K, int64_t ld_src, mx_tensor *dst,
+                                  void *stream);
 
 /* Walsh-Hadamard rotation fused with quantization ([MX] section "Técnicas de
  * preservação de acurácia": Hadamard rotations spread a block's outlier
