@@ -780,7 +780,7 @@ METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
 # kernel sources still hash to `src`, i.e. the counters were taken on the code
 # that runs.
 NCU_TRAFFIC = {
-    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6>", "bytes": 22812160 + 20224, "src": "f677cdba00e4c32f"},
+    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6, 256>", "bytes": 22812160 + 20224, "src": "f677cdba00e4c32f"},
 }
 
 
@@ -802,15 +802,18 @@ def traffic_bytes(workload_key: str, kernel: str):
     return rec["bytes"]
 
 
-def gemm_kernel_name(fmt: int, M: int, N: int) -> str:
+def gemm_kernel_name(fmt: int, M: int, N: int, gelu: bool = False) -> str:
     """The GEMM kernel mx_gemm dispatches to for this shape (both operands in
-    format fmt), named as ncu shows it: CTA pairs for M > 128 and N > 128 (5
-    stages for the FP4 kinds, 6 otherwise; MXFP6 runs on the run-time-typed
+    format fmt), named as ncu shows it: CTA pairs for M > 128 and N > 128
+    (256 x 256 tiles with 5 stages for the FP4 kinds, 6 otherwise; with the GELU
+    epilogue 256 x 128 tiles and 7 stages; MXFP6 runs on the run-time-typed
     kernel, template format 4), else one CTA with 128-wide N tiles for
     N <= 128, 32-row A tiles and 5 stages for M <= 32, 128 x 256 tiles
     otherwise."""
     if M > 128 and N > 128:
-        return f"gemm_pair_kernel<{fmt}, {5 if fmt in (2, 3) else 6}>"
+        if gelu:
+            return f"gemm_pair_kernel<{fmt}, 7, 128>"
+        return f"gemm_pair_kernel<{fmt}, {5 if fmt in (2, 3) else 6}, 256>"
     if N <= 128:
         return f"gemm_kernel<{fmt}, 128, 4, 128>"
     if M <= 32:

@@ -3,16 +3,19 @@
 // Same computation as gemm_sm100.cuh (C = A_dq * B_dq^T in bf16; page
 // "Microscaling MXFP4/NVFP4 on Blackwell", section "Arquitetura Blackwell SM100
 // e aceleração nativa de NVFP4"), for M > 128.  Two CTAs on neighbouring SMs
-// (a cluster of 2) compute a 256 x 256 output tile with M = 256 MMAs: each CTA
-// loads its own 128 rows of A and its own 128-row half of B, and the tensor
+// (a cluster of 2) compute a 256 x BN output tile with M = 256 MMAs: each CTA
+// loads its own 128 rows of A and its own BN/2-row half of B, and the tensor
 // core reads B from both CTAs' shared memory.  Per SM that is half the B
-// traffic of a 128 x 256 tile for the same MMA work.  No load is multicast.
+// traffic of a 128 x BN tile for the same MMA work.  No load is multicast.
+// BN = 256, or 128 for the GELU epilogue: then the two accumulators and the
+// scale slots fit TMEM without sharing columns, so a tile's GELU drain
+// overlaps the next tile's MMAs entirely.
 //
 // Roles per CTA (12 warps), as in the single-CTA kernel:
 //   warp 0     code-tile producer: own A rows and B half, completion counted
 //              on the leader CTA's barrier;
 //   warp 10    scale-tile producer: own A band and both B bands (this CTA's
-//              TMEM needs the scales of all 256 B rows), local barriers;
+//              TMEM needs the scales of all BN B rows), local barriers;
 //   warps 6-9  scale warps: this CTA's TMEM slot, then an arrive on the
 //              leader's slot barrier (8 arrivals: both CTAs' scale warps);
 //   warp 11    leader CTA only: gate, counts the stages whose code tiles (both
@@ -28,18 +31,21 @@
 
 namespace mx {
 
-// Per CTA: 128 rows of A and 128 rows of B in smem per stage, scale tiles of
-// two B bands, a 256-column accumulator.
-template <int FMT, int STAGES>
-using PairSmem = GemmLayout<FMT, 2, 128, STAGES>;
+// Per CTA: 128 rows of A and BN/2 rows of B in smem per stage, scale tiles of
+// BN/128 B bands, a BN-column accumulator.
+template <int FMT, int STAGES, int BN = 256>
+using PairSmem = GemmLayout<FMT, BN / 128, BN / 2, STAGES>;
 
-template <int FMT, int STAGES>
+template <int FMT, int STAGES, int BN = 256>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSfa,
                      const __grid_constant__ CUtensorMap tmSfb, GemmParams p) {
     using F = GemmFmt<FMT>;
-    using L = PairSmem<FMT, STAGES>;
+    using L = PairSmem<FMT, STAGES, BN>;
+    // with GELU the scale warps help drain the accumulator columns the next
+    // tile shares, if any
+    constexpr bool kHelp = gelu_help_chunks<BN, L::kAccStride>() > 0;
     static_assert(sizeof(FusedQuantSmem) <= L::kEpiAreaBytes, "fused quantize scratch in the staging buffers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -57,7 +63,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs)
-    const int num_tiles = p.m_blocks * p.n_blocks;  // 256 x 256 tiles
+    const int num_tiles = p.m_blocks * p.n_blocks;  // 256 x BN tiles
     const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
 
     if (threadIdx.x == 0) {
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         // both CTAs' epilogue warps (with GELU, their scale warps too)
-        mbar_init(acc_empty, (p.epilogue == 1 ? 4 : 2) * kEpiWarps);
+        mbar_init(acc_empty, (p.epilogue == 1 && kHelp ? 4 : 2) * kEpiWarps);
         mbar_init(mma_done, 1);
         for (int i = 0; i < L::kSlots; ++i) mbar_init(&sf_full[i], 8);
         *abort_flag = 0;
@@ -110,8 +116,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int ready_band = -1;   // fused quantize: the last A band known to be written
             for (int tile = pair; tile < num_tiles && !stop; tile += npairs) {
                 int m0, n0;
-                tile_coords(p, tile, m0, n0, 256, 256);
-                const int my_m = m0 + 128 * (int)rank, my_n = n0 + 128 * (int)rank;
+                tile_coords(p, tile, m0, n0, 256, BN);
+                const int my_m = m0 + 128 * (int)rank, my_n = n0 + (BN / 2) * (int)rank;
                 if (p.fused && my_m / 128 != ready_band) {
                     if (!wait_band_ready(p, my_m / 128, lane, abort_flag)) break;
                     ready_band = my_m / 128;
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, pair, npairs, num_tiles,
                                 [&](int tile, int &a_band, int &b_band) {
                                     int m0, n0;
-                                    tile_coords(p, tile, m0, n0, 256, 256);
+                                    tile_coords(p, tile, m0, n0, 256, BN);
                                     a_band = m0 / 128 + (int)rank;
                                     b_band = n0 / 128;
                                 },
@@ -179,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // scale slot once they have completed.
                 auto run_stage = [&](int k, uint32_t acc) {
                     const uint32_t t_sfa = tmem + (uint32_t)(L::kTmemSf + slot * L::kSfSlotCols);
-                    issue_stage<FMT, true, 256, 8>(k + 1 < p.num_kt ? 4 : last_n_mma, t_acc, ad0 + (uint64_t)(s * (L::kABytes >> 4)),
+                    issue_stage<FMT, true, BN, 4 * L::kBBands>(k + 1 < p.num_kt ? 4 : last_n_mma, t_acc, ad0 + (uint64_t)(s * (L::kABytes >> 4)),
                         bd0 + (uint64_t)(s * (L::kBBytes >> 4)), t_sfa, t_sfa + 4 * F::kChunks, acc, leader, ab);
                     tc_commit_pair_if(&empty[s], 0x3, leader);
                     s = (s + 1 == STAGES) ? 0 : s + 1;
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         uint32_t amax = 0;
         auto rows_of = [&](int t, int &m0, int &n0) {
-            tile_coords(p, pair + t * npairs, m0, n0, 256, 256);
+            tile_coords(p, pair + t * npairs, m0, n0, 256, BN);
             m0 += 128 * (int)rank;
         };
         // GELU: this warp's share of the shared columns of tile t (all but the
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait_bounded(&acc_full[b], (t >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag))
                 return false;
             tc_fence_after();
-            help_drain_t<256, L::kAccStride, FMT == 3>(
+            help_drain_t<BN, L::kAccStride, FMT == 3>(
                 p, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride), b, m0 + 32 * q, n0, lane, amax,
                 scale);
             tc_fence_before();
@@ -262,13 +268,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                               my_tiles, lane, abort_flag,
                               [&](int slot) { mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot); },
                               [&](int kg) -> bool {
-                                  if (p.epilogue != 1) return true;
+                                  if (p.epilogue != 1 || !kHelp) return true;
                                   for (; help_next < my_tiles - 1 && kg - L::kSlots >= (help_next + 1) * p.num_kt;
                                        ++help_next)
                                       if (!help(help_next)) return false;
                                   return true;
                               });
-        if (p.epilogue == 1 && !*abort_flag)
+        if (p.epilogue == 1 && kHelp && !*abort_flag)
             for (; help_next < my_tiles - 1; ++help_next)
                 if (!help(help_next)) break;
         // then the upper half of the columns of this CTA's rows of the last tile
@@ -287,7 +293,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
                 uint32_t nstore = 0;
                 epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
-                                                       m0 + 32 * q, n0, 4, 8, lane, bufs, nstore, amax, scale);
+                                                       m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs, nstore, amax,
+                                                       scale);
             }
         }
         epilogue_finish(p, lane, amax);
@@ -304,7 +311,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             int m0, n0;
-            tile_coords(p, tile, m0, n0, 256, 256);
+            tile_coords(p, tile, m0, n0, 256, BN);
             m0 += 128 * (int)rank;
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
@@ -313,11 +320,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (tile + npairs >= num_tiles) {
                 // the last tile: the lower half of the columns (the scale warp of
                 // this quadrant drains the upper half); nothing waits for its release
-                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, 0, 4, lane, bufs, nstore, amax,
-                                                       scale);
+                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, 0, BN / 64, lane, bufs, nstore,
+                                                       amax, scale);
                 break;
             }
-            epilogue_tile<256, L::kAccStride, L::kEpiBufs, FMT == 3>(
+            epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(
                 p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
                 [&] {
                     if (lane == 0) mbar_arrive_cluster(acc_empty_leader);

@@ -180,7 +180,12 @@ struct GemmLayout {
     // stages (one scale chunk) with 6 or more smem stages take 6 slots; the
     // FP4 kinds, whose slots are 2-4x wider, keep 4 so that TMEM still holds
     // the two accumulators.
-    static constexpr int kSlots = (F::kChunks == 1 && STAGES >= 6) ? 6 : kSfSlots;
+    static constexpr int kSlots = (F::kChunks == 1 && STAGES >= 6)
+                                      ? 6
+                                      // FP4 kinds: 6 slots where they fit beside two whole accumulators
+                                      : ((STAGES >= 6 && 2 * 128 * B_BANDS + 6 * 4 * F::kChunks * (1 + B_BANDS) <= 512)
+                                             ? 6
+                                             : kSfSlots);
     // full[S], empty[S], sfload[G], sfree[G], acc_full[2], acc_empty, mma_done, sf_full[slots]
     static constexpr int bytes_for(int groups, int bufs) {
         return STAGES * (kABytes + kBBytes) + groups * (kSfaGroupBytes + kSfbGroupBytes) +
@@ -243,11 +248,11 @@ MX_DEVICE_INLINE void gemm_mma_if(uint32_t d, uint64_t a, uint64_t b, uint32_t i
     else tc_mma_nvf4_if(d, a, b, idesc, sfa, sfb, acc, issue);
 }
 
-// Instruction descriptor of the CTA-pair MMA (M = 256 over two CTAs, N = 256).
-template <int FMT>
+// Instruction descriptor of the CTA-pair MMA (M = 256 over two CTAs, N = BN).
+template <int FMT, int BN = 256>
 MX_DEVICE_INLINE uint32_t pair_idesc(uint32_t sf_id) {
     using F = GemmFmt<FMT>;
-    return (sf_id << 4) | (F::kAFmt << 7) | (F::kAFmt << 10) | ((uint32_t)(256 >> 3) << 17) |
+    return (sf_id << 4) | (F::kAFmt << 7) | (F::kAFmt << 10) | ((uint32_t)(BN >> 3) << 17) |
            (F::kScaleUE8M0 << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
 }
 
@@ -275,7 +280,7 @@ MX_DEVICE_INLINE void issue_one(int j, uint32_t t_acc, uint64_t ad, uint64_t bd,
     const uint32_t sf_id = (uint32_t)((j % F::kMmaPerChunk) * F::kSfPerMma);
     const uint32_t a = acc | (j > 0 ? 1u : 0u);
     if (PAIR)
-        pair_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, pair_idesc<FMT>(sf_id) | ab, t_sfa + 4 * chunk,
+        pair_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, pair_idesc<FMT, BN>(sf_id) | ab, t_sfa + 4 * chunk,
                          t_sfb + SFB_STEP * chunk, a, issue);
     else
         gemm_mma_if<FMT>(t_acc, ad + 2u * j, bd + 2u * j, gemm_idesc<FMT, BN>(sf_id) | ab, t_sfa + 4 * chunk,

@@ -374,12 +374,12 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     return last_launch();
 }
 
-// CTA-pair kernel: 256 x 256 tiles on clusters of two CTAs (M > 128).
-template <int FMT, int STAGES>
+// CTA-pair kernel: 256 x BN tiles on clusters of two CTAs (M > 128).
+template <int FMT, int STAGES, int BN = 256>
 mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                              const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out,
                              cudaStream_t st, const FusedX *fx) {
-    using L = PairSmem<FMT, STAGES>;
+    using L = PairSmem<FMT, STAGES, BN>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
     const int64_t kbytes = K / GemmFmt<FMT>::kElemPerByte;   // shared-memory bytes of a row's K
@@ -387,18 +387,18 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     CUtensorMap ta, tb, tc, tsa, tsb;
     if (FMT == kGemmRuntimeTypes) {
         if (!make_tmap_codes_f8f6f4(&ta, A->fmt, a_codes, M, K, 128)) return MX_ERR_CUDA;
-        if (!make_tmap_codes_f8f6f4(&tb, B->fmt, B->codes, N, K, 128)) return MX_ERR_CUDA;
+        if (!make_tmap_codes_f8f6f4(&tb, B->fmt, B->codes, N, K, BN / 2)) return MX_ERR_CUDA;
     } else {
         if (!make_tmap_u8(&ta, a_codes, M, kbytes, 128)) return MX_ERR_CUDA;
-        if (!make_tmap_u8(&tb, B->codes, N, kbytes, 128)) return MX_ERR_CUDA;
+        if (!make_tmap_u8(&tb, B->codes, N, kbytes, BN / 2)) return MX_ERR_CUDA;
     }
     if (!make_tmap_sf(&tsa, a_scales, cdiv(M, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 1)) return MX_ERR_CUDA;
-    if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, 2))
+    if (!make_tmap_sf(&tsb, B->scales, cdiv(N, 128), sf_tiles_k, kSfGroup * GemmFmt<FMT>::kChunks, BN / 128))
         return MX_ERR_CUDA;
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
-    if (smem_limit_once(reinterpret_cast<const void *>(gemm_pair_kernel<FMT, STAGES>), L::kAlloc) != cudaSuccess)
+    if (smem_limit_once(reinterpret_cast<const void *>(gemm_pair_kernel<FMT, STAGES, BN>), L::kAlloc) != cudaSuccess)
         return MX_ERR_CUDA;
     GemmParams p{};
     p.sf_tiles_k = sf_tiles_k;
@@ -409,7 +409,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     p.K = (int)K;
     p.num_kt = (int)cdiv(kbytes, kStageKBytes);
     p.m_blocks = (int)cdiv(M, 256);
-    p.n_blocks = (int)cdiv(N, 256);
+    p.n_blocks = (int)cdiv(N, BN);
     p.ga = ga;
     p.gb = B->gscale;
     p.amax_out = amax_out;
@@ -417,8 +417,8 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     p.use_tma_store = tma_store ? 1 : 0;
     p.skip_producer = g_skip_producer.load();
     p.ab_types = (f8f6f4_type(A->fmt) << 7) | (f8f6f4_type(B->fmt) << 10);
-    // both CTAs' copies (128 rows of A and 128 of B each) report to the leader's barrier
-    p.stage_tx = (uint32_t)(2 * kStageKBytes * 128 * (fmt_bits(A->fmt) + fmt_bits(B->fmt)) / 8);
+    // both CTAs' copies (128 rows of A and BN/2 of B each) report to the leader's barrier
+    p.stage_tx = (uint32_t)(2 * kStageKBytes * (128 * fmt_bits(A->fmt) + (BN / 2) * fmt_bits(B->fmt)) / 8);
     p.wait_limit_ns = g_wait_limit_ns.load();
     set_fused(p, fx, a_codes, a_scales, M, K);
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
@@ -438,7 +438,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1 + (unsigned)pdl_attr(&attr[1]);
-    if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES, BN>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
         return last_launch();
     return last_launch();
 }
@@ -447,9 +447,14 @@ template <int FMT>
 mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                           const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st,
                           const FusedX *fx) {
-    if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load())
+    if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load()) {
+        // GELU: 256 x 128 tiles, whose two accumulators need no shared TMEM
+        // columns, so each tile's GELU drain overlaps the next tile's MMAs
+        if (epi == MX_EPI_GELU)
+            return launch_gemm_pair_t<FMT, 7, 128>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
         return launch_gemm_pair_t<FMT, (FMT == 2 || FMT == 3) ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi,
                                                                        amax_out, st, fx);
+    }
     if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
     // at most 32 rows of A (decode-like activations): the weight stream gets a
     // fifth stage from the shared memory a 128-row A tile would take
