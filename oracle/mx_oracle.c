@@ -767,8 +767,11 @@ int orc_gemm_f64(const double *A, const double *B, const int64_t *rows, int64_t 
 }
 
 /* GELU with the exact erf form (the pages give no GELU; PyTorch's default form
- * is taken): 0.5 * x * (1 + erf(x / sqrt(2))). */
-double orc_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }
+ * is taken): 0.5 * x * (1 + erf(x / sqrt(2))), evaluated as
+ * 0.5 * x * erfc(-x / sqrt(2)), the same function (1 + erf(y) = erfc(-y)) without
+ * the cancellation that leaves nothing of the negative tail (x <= -8.5 would
+ * come out as -0 where GELU is about -1e-18 at -9, a normal bf16 value). */
+double orc_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }
 
 void orc_gelu_array(const double *x, double *y, int64_t n) {
     #pragma omp parallel for schedule(static)

@@ -374,6 +374,33 @@ def test_gelu_against_normal_cdf():
     assert np.allclose(y - oracle.gelu(-x), x, rtol=0, atol=1e-14)      # GELU(x) - GELU(-x) = x
 
 
+def test_gelu_negative_tail_relative():
+    """Far in the negative tail GELU(x) = x Phi(x) is tiny but far above the
+    bf16 range's floor (about -1.0e-18 at x = -9), so it must keep its relative
+    accuracy there, not cancel to zero.  Pinned by Laplace's asymptotic series
+    of the normal tail, Phi(-t) = phi(t)/t * sum_n (-1)^n (2n-1)!! / t^(2n),
+    summed to its smallest term (below 1e-15 of the sum for t >= 9), and by
+    scipy's ndtr away from it."""
+    from scipy.special import ndtr
+    for t in (9.0, 9.5, 10.0, 12.0, 16.0, 20.0, 26.0, 30.0, 37.0):
+        term, total, n = 1.0, 1.0, 0
+        while True:
+            nxt = -term * (2 * n + 1) / (t * t)
+            if abs(nxt) >= abs(term):
+                break
+            term, n = nxt, n + 1
+            total += term
+        assert abs(term) < 1e-15
+        phi = np.exp(-t * t / 2) / np.sqrt(2 * np.pi)
+        want = -t * phi / t * total
+        got = float(oracle.gelu(np.array([-t]))[0])
+        assert got == pytest.approx(want, rel=1e-12), (t, got, want)
+    # the rounding of x / sqrt(2) reaches the result multiplied by about x^2
+    # (the log-derivative of exp(-x^2 / 2)): 1369 * 2^-52 = 3e-13 at x = -37
+    x = np.linspace(-37, -1, 3601)
+    assert np.all(np.abs(oracle.gelu(x) / (x * ndtr(x)) - 1) <= 4 * x * x * 2.0 ** -52)
+
+
 def test_gelu_lipschitz_constant_of_the_fused_tolerance():
     """The fused GEMM tests bound GELU's error by 1.13 x the GEMM bound: the
     largest |GELU'| is Phi(sqrt 2) + sqrt 2 phi(sqrt 2) = 1.128904, below 1.13.
