@@ -732,6 +732,9 @@ PROFILE_CASES = {
     "quant_nvfp4_32768x4096": ("quant", 3, 32768, 0, 4096),
     "quant_mxfp8_dit_4096x3072": ("quant", 0, 4096, 0, 3072),
     "fused_gelu_mlp1_nvfp4": ("fused_gelu", 3, 4608, 12288, 3072),
+    "fused_dit_mxfp8": ("fused", 0, 4096, 3072, 3072),
+    "gemm_dit_mxfp4_mbs": ("gemm", 5, 4096, 3072, 3072),
+    "quant_mbs_dynamic_1024x4096": ("quant_mbs_dynamic", 5, 1024, 0, 4096),
 }
 
 
@@ -755,6 +758,17 @@ def run_profile_case(name: str, reps: int = 4):
         gs = mx.quantize_rht(x, fmt, out=q).gscale.clone() if fmt == 3 else None
         for _ in range(reps):
             mx.quantize_rht(x, fmt, out=q, gscale=gs)
+    elif kind == "quant_mbs_dynamic":
+        q = mx.empty(fmt, M, K)
+        for _ in range(reps):
+            mx.quantize_mbs_dynamic(x, out=q)
+    elif kind == "fused":
+        w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        qw = mx.quantize(w, wfmt)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = mx.fused_workspace(fmt, M, K)
+        for _ in range(reps):
+            mx.gemm_fused_act(x, qw, out=C, workspace=ws)
     elif kind == "fused_gelu":
         w = (torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
         qw = mx.quantize(w, wfmt)

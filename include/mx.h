@@ -228,10 +228,11 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  *              that overlap on the GPU must not share one.
  *   epilogue : MX_EPI_NONE, or MX_EPI_GELU: the exact-erf form x Phi(x) =
  *              0.5 x erfc(-x / sqrt 2), applied in FP32 before the bf16
- *              rounding, with erfc from the Chebyshev fit of Numerical Recipes
- *              (relative error < 1.2e-7) and the hardware's approximate
- *              reciprocal and exponential: within one bf16 ulp of the form
- *              evaluated with erff.
+ *              rounding, with erfc(z) = t exp(-z^2 + P(t)), t = 1/(1 + z/2),
+ *              P a degree-5 polynomial fitted to it (erfc's relative error
+ *              below 7.7e-6), and the hardware's approximate reciprocal and
+ *              base-2 exponential: within one bf16 ulp of the correctly
+ *              rounded GELU.
  *   amax_out : NULL, or a device float that receives max |C| over the bf16
  *              outputs (it is zeroed by this call first).  Feeding it to the
  *              next call's x_amax chains two NVFP4 GEMMs without a host sync.
