@@ -595,6 +595,38 @@ def extras_gpu(device):
         del qws
         torch.cuda.empty_cache()
     out["skinny_fused"] = {"points": skinny, "call": "mx_gemm_fused_act(X bf16 [M x 8192], W [28672 x 8192])"}
+    # Few output tiles and a long K (a decode-time down projection, W [8192 x
+    # 28672]: 32 tiles of 256 columns for 148 SMs): the fused call splits the
+    # tiles along K over all SMs (its default plan); the same call with the
+    # split turned off beside it.
+    down = {}
+    N, K = 8192, 28672
+    for wfmt in (3, 2):
+        w = (torch.randn((N, K), generator=g, device=device) * 0.02).to(torch.bfloat16)
+        wbytes = mx.mx_codes_bytes(wfmt, N, K) + mx.mx_scales_bytes(wfmt, N, K)
+        nw = max(2, int(np.ceil(2 * L2_BYTES / wbytes)))
+        qws = [mx.quantize(w, wfmt) for _ in range(nw)]
+        del w
+        for M in (1, 16, 128):
+            x = torch.randn((M, K), generator=g, device=device).to(torch.bfloat16)
+            C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            ws = mx.fused_workspace(wfmt, M, K, device)
+            xq = mx.mx_codes_bytes(wfmt, M, K) + mx.mx_scales_bytes(wfmt, M, K)
+            nbytes = wbytes + 2 * M * K + 2 * xq + 2 * M * N
+            r = {}
+            for key, mode in (("split", mx.MX_K_SPLIT_AUTO), ("whole_tiles", mx.MX_K_SPLIT_NEVER)):
+                mx.check(mx.mx_debug_set(mx.MX_DEBUG_K_SPLIT, mode), "mx_debug_set")
+                ms = timed(lambda i: mx.gemm_fused_act(x, qws[i % nw], out=C, workspace=ws), nw)
+                gbs = nbytes / (ms * 1e-3) / 1e9
+                r[key] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+            mx.check(mx.mx_debug_set(mx.MX_DEBUG_K_SPLIT, mx.MX_K_SPLIT_AUTO), "mx_debug_set")
+            r["speedup"] = round(r["whole_tiles"]["us"] / r["split"]["us"], 3)
+            r["algorithmic_bytes"] = nbytes
+            down[f"{FMT_NAMES[wfmt]}_M{M}"] = r
+            del x, C, ws
+        del qws
+        torch.cuda.empty_cache()
+    out["down_proj_split_fused"] = {"points": down, "call": "mx_gemm_fused_act(X bf16 [M x 28672], W [8192 x 28672])"}
     # The DiT step in each mode of the fused call (same results bit for bit)
     M, N, K = 4096, 3072, 3072
     n = 6
@@ -794,7 +826,7 @@ METRIC = "NVFP4/MXFP8 block-scaled GEMM TFLOPS + quantize GB/s, % of roofline"
 # kernel sources still hash to `src`, i.e. the counters were taken on the code
 # that runs.
 NCU_TRAFFIC = {
-    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6, 256>", "bytes": 22812160 + 20224, "src": "f677cdba00e4c32f"},
+    "dit_mxfp8": {"kernel": "gemm_pair_kernel<0, 6, 256, false>", "bytes": 22812160 + 20224, "src": "f677cdba00e4c32f"},
 }
 
 
@@ -816,23 +848,25 @@ def traffic_bytes(workload_key: str, kernel: str):
     return rec["bytes"]
 
 
-def gemm_kernel_name(fmt: int, M: int, N: int, gelu: bool = False) -> str:
+def gemm_kernel_name(fmt: int, M: int, N: int, gelu: bool = False, split: bool = False) -> str:
     """The GEMM kernel mx_gemm dispatches to for this shape (both operands in
     format fmt), named as ncu shows it: CTA pairs for M > 128 and N > 128
     (256 x 256 tiles with 5 stages for the FP4 kinds, 6 otherwise; with the GELU
     epilogue 256 x 128 tiles and 7 stages; MXFP6 runs on the run-time-typed
     kernel, template format 4), else one CTA with 128-wide N tiles for
     N <= 128, 32-row A tiles and 5 stages for M <= 32, 128 x 256 tiles
-    otherwise."""
+    otherwise.  split: the variant compiled for a K split of the tiles (the
+    fused call's plan; never with GELU)."""
+    sp = "true" if split and not gelu else "false"
     if M > 128 and N > 128:
         if gelu:
-            return f"gemm_pair_kernel<{fmt}, 7, 128>"
-        return f"gemm_pair_kernel<{fmt}, {5 if fmt in (2, 3) else 6}, 256>"
+            return f"gemm_pair_kernel<{fmt}, 7, 128, false>"
+        return f"gemm_pair_kernel<{fmt}, {5 if fmt in (2, 3) else 6}, 256, {sp}>"
     if N <= 128:
-        return f"gemm_kernel<{fmt}, 128, 4, 128>"
+        return f"gemm_kernel<{fmt}, 128, 4, 128, {sp}>"
     if M <= 32:
-        return f"gemm_kernel<{fmt}, 256, 5, 32>"
-    return f"gemm_kernel<{fmt}, 256, 4, 128>"
+        return f"gemm_kernel<{fmt}, 256, 5, 32, {sp}>"
+    return f"gemm_kernel<{fmt}, 256, 4, 128, {sp}>"
 
 
 def gemm_bytes(fmt: int, M: int, N: int, K: int) -> int:

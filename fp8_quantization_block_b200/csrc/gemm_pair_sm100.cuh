@@ -36,7 +36,7 @@ namespace mx {
 template <int FMT, int STAGES, int BN = 256>
 using PairSmem = GemmLayout<FMT, BN / 128, BN / 2, STAGES>;
 
-template <int FMT, int STAGES, int BN = 256>
+template <int FMT, int STAGES, int BN = 256, bool SPLIT = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSfa,
@@ -63,8 +63,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs)
-    const int num_tiles = p.m_blocks * p.n_blocks;  // 256 x BN tiles
-    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+    const int pair = (int)(blockIdx.x >> 1);        // the worker: units of 256 x BN tiles
+    const int n_units = unit_count<SPLIT>(p, pair);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -114,15 +114,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t ph = 0;
             bool stop = false;
             int ready_band = -1;   // fused quantize: the last A band known to be written
-            for (int tile = pair; tile < num_tiles && !stop; tile += npairs) {
+            for (int u = 0; u < n_units && !stop; ++u) {
+                const KUnit U = unit_at<SPLIT>(p, pair, u);
                 int m0, n0;
-                tile_coords(p, tile, m0, n0, 256, BN);
+                tile_coords(p, U.tile, m0, n0, 256, BN);
                 const int my_m = m0 + 128 * (int)rank, my_n = n0 + (BN / 2) * (int)rank;
                 if (p.fused && my_m / 128 != ready_band) {
                     if (!wait_band_ready(p, my_m / 128, lane, abort_flag)) break;
                     ready_band = my_m / 128;
                 }
-                for (int kt = 0; kt < p.num_kt; ++kt) {
+                for (int kt = U.kb; kt < U.ke; ++kt) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY, abort_flag)) {
                         stop = true;
                         break;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == kSfWarp) {
         // ------------------------------------------------------------ scale-tile producer
         if (!p.skip_producer)
-            sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, pair, npairs, num_tiles,
+            sf_producer_role<L, SPLIT>(p, &tmSfa, &tmSfb, smem, sfload, sfree, pair,
                                 [&](int tile, int &a_band, int &b_band) {
                                     int m0, n0;
                                     tile_coords(p, tile, m0, n0, 256, BN);
@@ -178,8 +179,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t kg = 0;      // stages consumed
             uint32_t avail = 0;   // stages the gate warp has reported ready
             bool stop = false;
-            int it = 0;
-            for (int tile = pair; tile < num_tiles && !stop; tile += npairs, ++it) {
+            for (int it = 0; it < n_units && !stop; ++it) {
+                const KUnit U = unit_at<SPLIT>(p, pair, it);
                 const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
                 // One stage: its MMAs, then a commit that frees the smem stage and the
                 // scale slot once they have completed.
@@ -194,8 +195,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 };
                 // Two stages per iteration: the loop's own instructions then fall between
                 // MMAs only every other stage.
-                for (int kt = 0; kt < p.num_kt; kt += 2) {
-                    const bool two = kt + 1 < p.num_kt;
+                for (int kt = U.kb; kt < U.ke; kt += 2) {
+                    const bool two = kt + 1 < U.ke;
                     // the gate warp publishes how many stages have their code tiles and
                     // scale slots in; read it only when the stages known ready run out
                     const uint32_t need = kg + (two ? 1u : 0u);
@@ -207,7 +208,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                         tc_fence_after();
                     }
-                    if (kt == 0 && it > 0) {
+                    if (kt == U.kb && it > 0) {
                         // the epilogue has released the columns this accumulator shares
                         if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY, abort_flag)) {
                             stop = true;
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                         tc_fence_after();
                     }
-                    run_stage(kt, kt > 0 ? 1u : 0u);
+                    run_stage(kt, kt > U.kb ? 1u : 0u);
                     if (two) run_stage(kt + 1, 1u);
                 }
                 if (!stop) tc_commit_pair_if(&acc_full[it & 1], 0x3, leader);
@@ -226,22 +227,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == kGateWarp) {
         // ------------------------------------------------------------ gate (leader)
         if (rank == 0) {
-            int my_tiles = 0;
-            for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
-            gate_role<STAGES, L::kSlots>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
+            gate_role<STAGES, L::kSlots>(p, full, sf_full, ready_count, unit_stages<SPLIT>(p, pair), lane, abort_flag);
         }
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps
         const int q = warp & 3;
         const uint32_t sf_full_leader0 = mapa_shared(smem_u32(&sf_full[0]), 0);
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-        int my_tiles = 0;
-        for (int tile = pair; tile < num_tiles; tile += npairs) ++my_tiles;
+        const int my_tiles = n_units;
         float scale = 1.0f;
         if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         uint32_t amax = 0;
         auto rows_of = [&](int t, int &m0, int &n0) {
-            tile_coords(p, pair + t * npairs, m0, n0, 256, BN);
+            tile_coords(p, unit_at<SPLIT>(p, pair, t).tile, m0, n0, 256, BN);
             m0 += 128 * (int)rank;
         };
         // GELU: this warp's share of the shared columns of tile t (all but the
@@ -264,8 +262,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
             return true;
         };
-        scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
-                              my_tiles, lane, abort_flag,
+        scale_role<L, STAGES, SPLIT>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
+                              pair, lane, abort_flag,
                               [&](int slot) { mbar_arrive_cluster(sf_full_leader0 + 8u * (uint32_t)slot); },
                               [&](int kg) -> bool {
                                   if (p.epilogue != 1 || !kHelp) return true;
@@ -292,9 +290,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_fence_after();
                 uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
                 uint32_t nstore = 0;
-                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
-                                                       m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs, nstore, amax,
-                                                       scale);
+                const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
+                const KUnit U = unit_at<SPLIT>(p, pair, it);
+                if (U.kind == kUnitPartial)
+                    ks_partial_drain<BN, L::kAccStride>(p, pair, 2, (int)rank, t_acc, b, m0 + 32 * q, n0, q, lane,
+                                                        false, BN / 64, BN / 32, 1u, [] {});
+                else if (U.kind == kUnitWhole ||
+                         ks_finish_fold<L, STAGES>(p, smem, 2 * q + 1, U, pair, 2, (int)rank, t_acc, m0 + 32 * q, n0,
+                                                   q, lane, BN / 64, BN / 32, abort_flag))
+                    epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs,
+                                                           nstore, amax, scale);
             }
         }
         epilogue_finish(p, lane, amax);
@@ -308,27 +313,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t amax = 0, nstore = 0;
         float scale = 1.0f;
         if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
-        int it = 0;
-        for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+        auto release = [&] {
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        };
+        for (int it = 0; it < n_units; ++it) {
+            const KUnit U = unit_at<SPLIT>(p, pair, it);
             int m0, n0;
-            tile_coords(p, tile, m0, n0, 256, BN);
+            tile_coords(p, U.tile, m0, n0, 256, BN);
             m0 += 128 * (int)rank;
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
-            if (tile + npairs >= num_tiles) {
+            const bool last = it + 1 == n_units;
+            // a piece of a split tile (this CTA's 128 rows): on the last unit
+            // the lower half of the columns (the scale warp takes the upper
+            // half), else all of them
+            if (U.kind == kUnitPartial) {
+                ks_partial_drain<BN, L::kAccStride>(p, pair, 2, (int)rank, t_acc, b, m0 + 32 * q, n0, q, lane, !last,
+                                                    0, last ? BN / 64 : BN / 32, last ? 1u : 2u, release);
+                if (last) break;
+                continue;
+            }
+            if (U.kind == kUnitFinish &&
+                !ks_finish_fold<L, STAGES>(p, smem, 2 * q, U, pair, 2, (int)rank, t_acc, m0 + 32 * q, n0, q, lane, 0,
+                                           last ? BN / 64 : BN / 32, abort_flag))
+                break;
+            if (last) {
                 // the last tile: the lower half of the columns (the scale warp of
                 // this quadrant drains the upper half); nothing waits for its release
                 epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, 0, BN / 64, lane, bufs, nstore,
                                                        amax, scale);
                 break;
             }
-            epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(
-                p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs, nstore, amax, scale,
-                [&] {
-                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-                });
+            epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs,
+                                                                     nstore, amax, scale, release);
         }
         epilogue_finish(p, lane, amax);
     }

@@ -6,8 +6,9 @@
 // NVFP4": the 5th-generation tensor core consumes the block codes directly and
 // applies the block scale during FP32 accumulation).
 //
-// Persistent kernel: one CTA per SM walks output tiles of 128 x BN (tile t,
-// t + gridDim.x, ...) with six warp roles:
+// Persistent kernel: one CTA per SM walks its work units (ksplit.cuh: output
+// tiles of 128 x BN, t, t + gridDim.x, ..., and with a split plan pieces of
+// the last wave's tiles along K) with six warp roles:
 //   warp 0     TMA producer of the code tiles of A and B (128-byte swizzled,
 //              K-major) into a STAGES-deep smem ring that runs continuously
 //              across tiles;
@@ -39,6 +40,7 @@
 // S + BN up.  Every mbarrier wait is bounded (mx_common.cuh).
 #pragma once
 
+#include "ksplit.cuh"
 #include "mx_common.cuh"
 #include "quantize.cuh"
 
@@ -136,6 +138,14 @@ struct GemmParams {
     uint8_t *xq_scales;
     uint32_t *band_ready;
     uint32_t *next_item;
+    // Work schedule (ksplit.cuh): whole tiles, and with ks.on the tiles of
+    // the last wave split along K.  Partial sums go to ks_partials, slot
+    // worker (x 2 + rank on CTA pairs), in 4 KB blocks (ks_block);
+    // ks_flags[slot] reaches kSplitSlotDone once the slot is written.
+    KSplitPlan ks;
+    float *ks_partials;
+    uint32_t *ks_flags;
+    int ks_slot_quads;    // 32-row quadrants of a slot (of the rows that exist)
 };
 
 // gA of an NVFP4 A operand (the epilogue multiplies by gA * gB).
@@ -395,24 +405,52 @@ MX_DEVICE_INLINE void stage_scales_to_tmem(const uint8_t *sfa_stage, const uint8
     tmem_wait_st();
 }
 
+// ---------------------------------------------------------------- work units
+// The work units of worker c (ksplit.cuh).  Kernels compiled without SPLIT
+// run whole tiles c, c + workers, ... with K stages [0, num_kt): constant
+// bounds, and none of the split's branches in their loops.
+template <bool SPLIT>
+MX_DEVICE_INLINE int unit_count(const GemmParams &p, int c) {
+    if (SPLIT) return ks_units(p.ks, c);
+    return c < p.ks.tiles ? (p.ks.tiles - c + p.ks.workers - 1) / p.ks.workers : 0;
+}
+template <bool SPLIT>
+MX_DEVICE_INLINE KUnit unit_at(const GemmParams &p, int c, int u) {
+    if (SPLIT) return ks_unit(p.ks, c, u);
+    KUnit r;
+    r.tile = c + u * p.ks.workers;
+    r.kb = 0;
+    r.ke = p.num_kt;
+    r.kind = kUnitWhole;
+    r.first = c;
+    return r;
+}
+template <bool SPLIT>
+MX_DEVICE_INLINE int unit_stages(const GemmParams &p, int c) {
+    return SPLIT ? ks_stages(p.ks, c) : unit_count<false>(p, c) * p.num_kt;
+}
+
 // ---------------------------------------------------------------- scale-tile roles
-// Producer of scale tiles (one warp; lane 0 issues): for each tile of this CTA
-// (bands_of(tile, a_band, b_band)), one 3D TMA copy per operand and group of
-// kSfGroup stages into ring slot g, once the scale warps have freed it.
+// Producer of scale tiles (one warp; lane 0 issues): for each work unit of
+// this worker (bands_of(tile, a_band, b_band)), one 3D TMA copy per operand
+// and group of kSfGroup stages into ring slot g, once the scale warps have
+// freed it.
 // Coordinates past the scale buffer (a ragged K or N) read zeros.
-template <typename L, typename BandsOf>
+template <typename L, bool SPLIT, typename BandsOf>
 MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *tmSfa, const CUtensorMap *tmSfb,
-                                       uint8_t *smem, uint64_t *sfload, uint64_t *sfree, int tile0, int tile_step,
-                                       int num_tiles, BandsOf bands_of, int lane, volatile int *abort_flag) {
+                                       uint8_t *smem, uint64_t *sfload, uint64_t *sfree, int worker,
+                                       BandsOf bands_of, int lane, volatile int *abort_flag) {
     constexpr int NG = L::kSfGroups;
     constexpr int kChunks = L::F::kChunks;
     int used = 0, g = 0;
     uint32_t ph = 0;
     bool stop = false;
     int ready_band = -1;   // fused quantize: the last A band known to be written
-    for (int tile = tile0; tile < num_tiles && !stop; tile += tile_step) {
+    const int n_units = unit_count<SPLIT>(p, worker);
+    for (int u = 0; u < n_units && !stop; ++u) {
+        const KUnit U = unit_at<SPLIT>(p, worker, u);
         int a_band, b_band;
-        bands_of(tile, a_band, b_band);
+        bands_of(U.tile, a_band, b_band);
         if (p.fused && a_band != ready_band) {
             if (!wait_band_ready(p, a_band, lane, abort_flag)) {
                 stop = true;
@@ -420,7 +458,7 @@ MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *t
             }
             ready_band = a_band;
         }
-        for (int kt0 = 0; kt0 < p.num_kt; kt0 += kSfGroup) {
+        for (int kt0 = U.kb; kt0 < U.ke; kt0 += kSfGroup) {   // U.kb is even
             if (!mbar_wait_bounded(&sfree[g], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_SF_FREE, abort_flag)) {
                 stop = true;
                 break;
@@ -444,7 +482,7 @@ MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *t
 }
 
 // Scale warps (one per TMEM lane quadrant; lane r handles TMEM lane 32q + r):
-// for every stage of this CTA's tiles, wait for its scale group in smem and
+// for every stage of this worker's units, wait for its scale group in smem and
 // for the MMAs that last read the TMEM slot (stage kg - L::kSlots, whose
 // commit completes empty[]), then write the slot and report it with
 // arrive_full(slot).  After a group's last stage the warp frees the group.
@@ -453,9 +491,9 @@ MX_DEVICE_INLINE void sf_producer_role(const GemmParams &p, const CUtensorMap *t
 // latency it hides.)  before_wait(kg) runs just before the wait for stage
 // kg - L::kSlots; the kernels use it to drain accumulator columns whose
 // release that stage's MMAs may be waiting for.
-template <typename L, int STAGES, typename ArriveFull, typename BeforeWait>
+template <typename L, int STAGES, bool SPLIT, typename ArriveFull, typename BeforeWait>
 MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *sfload, uint64_t *sfree, uint64_t *empty,
-                                 uint32_t t_sf0, int my_tiles, int lane, volatile int *abort_flag,
+                                 uint32_t t_sf0, int worker, int lane, volatile int *abort_flag,
                                  ArriveFull arrive_full, BeforeWait before_wait) {
     constexpr int NG = L::kSfGroups;
     constexpr int kChunks = L::F::kChunks;
@@ -463,8 +501,10 @@ MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *s
     uint32_t gph = 0, eph = 0;
     int kg = 0;
     bool stop = false;
-    for (int t = 0; t < my_tiles && !stop; ++t) {
-        for (int kt = 0; kt < p.num_kt; ++kt, ++kg) {
+    const int n_units = unit_count<SPLIT>(p, worker);
+    for (int u = 0; u < n_units && !stop; ++u) {
+        const KUnit U = unit_at<SPLIT>(p, worker, u);
+        for (int kt = U.kb; kt < U.ke; ++kt, ++kg) {
             const int gi = kt % kSfGroup;
             if (gi == 0 && !mbar_wait_bounded(&sfload[g], gph, p.wait_limit_ns, SITE_GEMM_SF_LOAD, abort_flag)) {
                 stop = true;
@@ -492,7 +532,7 @@ MX_DEVICE_INLINE void scale_role(const GemmParams &p, uint8_t *smem, uint64_t *s
             __syncwarp();
             if (lane == 0) arrive_full(slot);
             slot = (slot + 1 == L::kSlots) ? 0 : slot + 1;
-            if (gi == kSfGroup - 1 || kt == p.num_kt - 1) {
+            if (gi == kSfGroup - 1 || kt == U.ke - 1) {
                 if (lane == 0) mbar_arrive(&sfree[g]);
                 if (++g == NG) {
                     g = 0;
@@ -614,30 +654,28 @@ MX_DEVICE_INLINE void fused_quantize_role(const GemmParams &p, FusedQuantSmem *f
     }
 }
 
-// Gate warp: for every stage of this CTA's tiles, in order, wait for its code
-// tiles (full) and its scale slot (sf_full), then publish the number of
-// stages ready so far.
+// Gate warp: for every stage of this CTA's work units (my_stages in all), in
+// order, wait for its code tiles (full) and its scale slot (sf_full), then
+// publish the number of stages ready so far.
 template <int STAGES, int SLOTS>
-MX_DEVICE_INLINE void gate_role(const GemmParams &p, uint64_t *full, uint64_t *sf_full, uint32_t *ready, int my_tiles,
-                                int lane, volatile int *abort_flag) {
+MX_DEVICE_INLINE void gate_role(const GemmParams &p, uint64_t *full, uint64_t *sf_full, uint32_t *ready,
+                                int my_stages, int lane, volatile int *abort_flag) {
     int s = 0, slot = 0;
     uint32_t fph = 0, sph = 0, k = 0;
-    for (int t = 0; t < my_tiles; ++t) {
-        for (int kt = 0; kt < p.num_kt; ++kt) {
-            if (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
-                !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))
-                return;
-            ++k;
-            __syncwarp();
-            if (lane == 0) st_release_shared(ready, k);
-            if (++s == STAGES) {
-                s = 0;
-                fph ^= 1u;
-            }
-            if (++slot == SLOTS) {
-                slot = 0;
-                sph ^= 1u;
-            }
+    for (int kt = 0; kt < my_stages; ++kt) {
+        if (!mbar_wait_bounded(&full[s], fph, p.wait_limit_ns, SITE_GEMM_MMA_FULL, abort_flag) ||
+            !mbar_wait_bounded(&sf_full[slot], sph, p.wait_limit_ns, SITE_GEMM_MMA_SF, abort_flag))
+            return;
+        ++k;
+        __syncwarp();
+        if (lane == 0) st_release_shared(ready, k);
+        if (++s == STAGES) {
+            s = 0;
+            fph ^= 1u;
+        }
+        if (++slot == SLOTS) {
+            slot = 0;
+            sph ^= 1u;
         }
     }
 }
@@ -855,7 +893,218 @@ MX_DEVICE_INLINE void epilogue_finish(const GemmParams &p, int lane, uint32_t am
     }
 }
 
-template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
+// ---------------------------------------------------------------- K split
+// The counter of a partial-sum slot reaches kSplitSlotDone once every warp
+// that writes part of the slot has published: the four epilogue warps with 2
+// each, or, on the worker's last unit (whose columns the scale warps share),
+// the four epilogue and four scale warps with 1 each.
+constexpr uint32_t kSplitSlotDone = 8;
+
+// A partial-sum slot is 8 chunks x ks_slot_quads quadrants of 4 KB blocks;
+// block (chunk c, quadrant q) holds rows 32q .. 32q + 31 and columns 32c ..
+// 32c + 31 as [c4 = 0 .. 7][row 0 .. 31][4 fp32]: a warp's store of four
+// columns is 512 contiguous bytes, and the finishing warp brings the block
+// into shared memory with one bulk copy, each lane then reading its row's
+// 16-byte groups without bank conflicts.
+constexpr int kSplitBlockBytes = 4096;
+MX_DEVICE_INLINE float4 *ks_block(const GemmParams &p, int slot, int chunk, int q) {
+    return reinterpret_cast<float4 *>(p.ks_partials) + ((size_t)(slot * 8 + chunk) * p.ks_slot_quads + q) * 256;
+}
+
+// One 32-column chunk of this warp's accumulator quadrant into its block of
+// a partial-sum slot (L2-only stores: another SM reads them).
+MX_DEVICE_INLINE void ks_store_chunk(const GemmParams &p, uint32_t t_addr, int slot, int chunk, int q, int lane) {
+    uint32_t r[32];
+    tmem_ld32(t_addr, r);
+    tmem_wait_ld();
+    float4 *d = ks_block(p, slot, chunk, q) + lane;
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+        __stcg(d + 32 * v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                       __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+}
+
+// Publish this warp's share of a written slot: every lane's stores are made
+// visible at gpu scope (and to the async proxy) before lane 0 adds to the
+// slot's counter.
+MX_DEVICE_INLINE void ks_publish(const GemmParams &p, int slot, uint32_t share, int lane) {
+    __threadfence();
+    fence_proxy_async_global();   // the finishing warp reads the slot with bulk copies
+    __syncwarp();
+    if (lane == 0) red_release_gpu_add(p.ks_flags + slot, share);
+}
+
+// Wait (lane 0 polls, bounded) until the n slots slot0, slot0 + step, ... are
+// written; lane 0 then issues the bulk copies that read them (the wait ends
+// with an async-proxy fence).
+MX_DEVICE_INLINE bool ks_wait(const GemmParams &p, int slot0, int n, int step, int lane, volatile int *abort_flag) {
+    bool ok = true;
+    if (lane == 0)
+        for (int j = 0; j < n && ok; ++j)
+            ok = wait_global_at_least(p.ks_flags + slot0 + j * step, kSplitSlotDone, p.wait_limit_ns,
+                                      SITE_KSPLIT_PARTIAL, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __threadfence();
+    return ok;
+}
+
+// This warp's part of a partial piece of worker `worker` (its slot is worker
+// * ranks + rank): TMEM quadrant q of the accumulator t_acc (rows m0q .. m0q +
+// 31 of C, local rows 32q ..) into the slot, then `share` added to the slot's
+// counter.  ordered: all chunks, those the next unit's accumulator shares
+// (buffer b's) first, then release() and the rest; otherwise chunks
+// [c_begin, c_end) and no release (the worker's last unit).
+template <int BN, int ACC_STRIDE, typename Release>
+MX_DEVICE_INLINE void ks_partial_drain(const GemmParams &p, int worker, int ranks, int rank, uint32_t t_acc, int b,
+                                       int m0q, int n0, int q, int lane, bool ordered, int c_begin, int c_end,
+                                       uint32_t share, Release release) {
+    constexpr int kChunks = BN / 32;
+    constexpr int kOv = (BN - ACC_STRIDE) / 32;
+    const int n_valid = p.N - n0;
+    const int slot = worker * ranks + rank;
+    const bool any_rows = m0q < p.M;  // warp-uniform; a quadrant without rows has no block
+    const int n_chunks = ordered ? kChunks : c_end - c_begin;
+#pragma unroll 1
+    for (int idx = 0; idx < n_chunks; ++idx) {
+        int col;
+        if (ordered) {
+            if (idx == kOv) {
+                tc_fence_before();
+                __syncwarp();
+                release();
+            }
+            col = 32 * ((b == 0) ? (idx + (kChunks - kOv)) % kChunks : idx);
+        } else {
+            col = 32 * (c_begin + idx);
+        }
+        if (any_rows && col < n_valid) ks_store_chunk(p, t_acc + (uint32_t)col, slot, col / 32, q, lane);
+    }
+    if (ordered && kOv == kChunks) {
+        tc_fence_before();
+        __syncwarp();
+        release();
+    }
+    ks_publish(p, slot, share, lane);
+}
+
+// Shared memory of a finishing piece's fold (the worker's last unit, whose
+// MMAs have completed, so the stage rings are idle): for each draining warp
+// (two per TMEM lane quadrant: area 2q for the epilogue warp, 2q + 1 for the
+// scale warp) a ring of 4 KB buffers and their mbarriers, carved from the B
+// ring past the scale warps' staging buffers and from the A ring; the ring is
+// as deep as the areas of the quadrants that hold rows allow (2 to 16
+// buffers: 16 in the decode-shape kernel, where only one quadrant does).
+template <typename L, int STAGES>
+struct FoldPlan {
+    static constexpr int kStaging = kEpiWarps * L::kEpiBufs * kEpiChunkBytes;
+    static constexpr int kAPiece = STAGES * L::kABytes, kBPiece = STAGES * L::kBBytes - kStaging;
+    __host__ __device__ static constexpr int area_bytes(int nb) { return nb * kSplitBlockBytes + 128; }
+    __host__ __device__ static constexpr int fits(int nb) { return kBPiece / area_bytes(nb) + kAPiece / area_bytes(nb); }
+    // the deepest ring (at most 16 buffers) that n_areas areas allow
+    __host__ __device__ static constexpr int bufs_for(int n_areas) {
+        int nb = 16;
+        while (nb > 2 && fits(nb) < n_areas) --nb;
+        return nb;
+    }
+    static_assert(fits(2) >= 2 * kEpiWarps, "fold areas in the stage rings");
+};
+// Area `area` of n_areas (2 per TMEM lane quadrant with rows): its buffers.
+template <typename L, int STAGES>
+MX_DEVICE_INLINE uint8_t *ks_fold_area(uint8_t *smem, int area, int nbufs) {
+    using F = FoldPlan<L, STAGES>;
+    const int a = F::area_bytes(nbufs), in_b = F::kBPiece / a;
+    return area < in_b ? smem + L::kOffB + F::kStaging + area * a : smem + L::kOffA + (area - in_b) * a;
+}
+
+// This warp's part of a finishing piece, before its epilogue: wait for the
+// partial sums of workers U.first .. worker - 1 (bounded), then add them,
+// in that order, to chunks [c_begin, c_end) of quadrant q of the accumulator
+// (read, added to and written back to TMEM for the ordinary epilogue).  The
+// 4 KB blocks, partial sum by partial sum and chunk by chunk, stream through
+// the warp's ring by bulk copies, so that the L2 round trips overlap.  Only a
+// worker's last unit finishes a tile.
+template <typename L, int STAGES>
+MX_DEVICE_INLINE bool ks_finish_fold(const GemmParams &p, uint8_t *smem, int area, const KUnit &U, int worker,
+                                     int ranks, int rank, uint32_t t_acc, int m0q, int n0, int q, int lane,
+                                     int c_begin, int c_end, volatile int *abort_flag) {
+    if (m0q >= p.M) return true;  // no rows in this quadrant (warp-uniform)
+    const int n = worker - U.first;
+    const int slot0 = U.first * ranks + rank;
+    if (!ks_wait(p, slot0, n, ranks, lane, abort_flag)) return false;
+    int nc = 0;
+    while (c_begin + nc < c_end && 32 * (c_begin + nc) < p.N - n0) ++nc;
+    const int nb = nc * n;
+    if (nb == 0) return true;
+    // with fewer quadrants holding rows, fewer warps fold, each with a deeper ring
+    constexpr int kBufs2 = FoldPlan<L, STAGES>::bufs_for(2), kBufs4 = FoldPlan<L, STAGES>::bufs_for(4),
+                  kBufs6 = FoldPlan<L, STAGES>::bufs_for(6), kBufs8 = FoldPlan<L, STAGES>::bufs_for(8);
+    const int kBufs = p.ks_slot_quads == 1 ? kBufs2 : p.ks_slot_quads == 2 ? kBufs4
+                                                     : p.ks_slot_quads == 3 ? kBufs6 : kBufs8;
+    uint8_t *const buf = ks_fold_area<L, STAGES>(smem, area, kBufs);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(buf + kBufs * kSplitBlockBytes);
+    // blocks in order: partial sum j (slot slot0 + j * ranks), then chunk
+    // c_begin + c; lane 0 issues them ahead of the warp into ring buffer ik
+    const float4 *blk0 = ks_block(p, slot0, c_begin, q);
+    const size_t slot_step = (size_t)ranks * 8 * p.ks_slot_quads * 256, chunk_step = (size_t)p.ks_slot_quads * 256;
+    int ij = 0, ic = 0, ik = 0, issued = 0;
+    auto issue_next = [&]() {  // lane 0
+        mbar_arrive_expect_tx(&bar[ik], kSplitBlockBytes);
+        bulk_load(buf + ik * kSplitBlockBytes, blk0 + (size_t)ij * slot_step + (size_t)ic * chunk_step,
+                  kSplitBlockBytes, &bar[ik]);
+        if (++ic == nc) ic = 0, ++ij;
+        if (++ik == kBufs) ik = 0;
+        ++issued;
+    };
+    if (lane == 0) {
+        for (int k = 0; k < kBufs; ++k) mbar_init(&bar[k], 1);
+        fence_barrier_init();
+        while (issued < kBufs && ij < n) issue_next();
+    }
+    __syncwarp();
+    int k = 0, consumed = 0;
+    uint32_t ph = 0;
+    for (int j = 0; j < n; ++j) {
+        for (int c = 0; c < nc; ++c) {
+            if (!mbar_wait_bounded(&bar[k], ph, p.wait_limit_ns, SITE_KSPLIT_PARTIAL, abort_flag)) {
+                // copies still in flight into this ring: let them land first
+                if (lane == 0)
+                    for (int x = consumed; x < issued; ++x)
+                        mbar_wait_bounded(&bar[x % kBufs], (uint32_t)((x / kBufs) & 1), p.wait_limit_ns,
+                                          SITE_GEMM_TAIL, nullptr);
+                __syncwarp();
+                return false;
+            }
+            const uint32_t ta = t_acc + (uint32_t)(32 * (c_begin + c));
+            const float4 *src = reinterpret_cast<const float4 *>(buf + k * kSplitBlockBytes) + lane;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t r[16];
+                tmem_ld16(ta + 16 * h, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 a = src[32 * (4 * h + v)];
+                    r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + a.x);
+                    r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + a.y);
+                    r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + a.z);
+                    r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + a.w);
+                }
+                tmem_st16(ta + 16 * h, r);
+            }
+            tmem_wait_st();  // the next partial sum reads these columns again
+            __syncwarp();    // every lane has read buffer k
+            ++consumed;
+            if (lane == 0 && ij < n) {
+                fence_proxy_async_smem();
+                issue_next();
+            }
+            if (++k == kBufs) k = 0, ph ^= 1u;
+        }
+    }
+    return true;
+}
+
+template <int FMT, int BN, int STAGES, int A_ROWS = kBM, bool SPLIT = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSfa,
@@ -878,7 +1127,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t *ready_count = reinterpret_cast<uint32_t *>(smem + L::kOffMisc + 8);  // gate -> MMA issuer
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = p.m_blocks * p.n_blocks;
+    const int worker = (int)blockIdx.x;
+    const int n_units = unit_count<SPLIT>(p, worker);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -928,14 +1178,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t ph = 0;
             bool stop = false;
             int ready_band = -1;   // fused quantize: the last A band known to be written
-            for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+            for (int u = 0; u < n_units && !stop; ++u) {
+                const KUnit U = unit_at<SPLIT>(p, worker, u);
                 int m0, n0;
-                tile_coords(p, tile, m0, n0, kBM, BN);
+                tile_coords(p, U.tile, m0, n0, kBM, BN);
                 if (p.fused && m0 / kBM != ready_band) {
                     if (!wait_band_ready(p, m0 / kBM, lane, abort_flag)) break;
                     ready_band = m0 / kBM;
                 }
-                for (int kt = 0; kt < p.num_kt; ++kt) {
+                for (int kt = U.kb; kt < U.ke; ++kt) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.wait_limit_ns, SITE_GEMM_PRODUCER_EMPTY, abort_flag)) {
                         stop = true;
                         break;
@@ -963,7 +1214,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == kSfWarp) {
         // ------------------------------------------------------------ scale-tile producer
         if (!p.skip_producer)
-            sf_producer_role<L>(p, &tmSfa, &tmSfb, smem, sfload, sfree, blockIdx.x, gridDim.x, num_tiles,
+            sf_producer_role<L, SPLIT>(p, &tmSfa, &tmSfb, smem, sfload, sfree, worker,
                                 [&](int tile, int &a_band, int &b_band) {
                                     int m0, n0;
                                     tile_coords(p, tile, m0, n0, kBM, BN);
@@ -989,8 +1240,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t kg = 0;      // stages consumed
         uint32_t avail = 0;   // stages the gate warp has reported ready
         bool stop = false;
-        int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++it) {
+        for (int it = 0; it < n_units && !stop; ++it) {
+            const KUnit U = unit_at<SPLIT>(p, worker, it);
             const uint32_t t_acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
             // One stage: its MMAs, then a commit that frees the smem stage and the
             // scale slot once they have completed.
@@ -1005,8 +1256,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             };
             // Two stages per iteration: the loop's own instructions then fall between
             // MMAs only every other stage.
-            for (int kt = 0; kt < p.num_kt; kt += 2) {
-                const bool two = kt + 1 < p.num_kt;
+            for (int kt = U.kb; kt < U.ke; kt += 2) {
+                const bool two = kt + 1 < U.ke;
                 // the gate warp publishes how many stages have their code tiles and
                 // scale slots in; read it only when the stages known ready run out
                 const uint32_t need = kg + (two ? 1u : 0u);
@@ -1018,7 +1269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     tc_fence_after();
                 }
-                if (kt == 0 && it > 0) {
+                if (kt == U.kb && it > 0) {
                     // the epilogue has released the columns this accumulator shares
                     if (!mbar_wait_bounded(acc_empty, (it - 1) & 1, p.wait_limit_ns, SITE_GEMM_MMA_ACC_EMPTY, abort_flag)) {
                         stop = true;
@@ -1026,7 +1277,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     tc_fence_after();
                 }
-                run_stage(kt, kt > 0 ? 1u : 0u);
+                run_stage(kt, kt > U.kb ? 1u : 0u);
                 if (two) run_stage(kt + 1, 1u);
             }
             if (!stop) tc_commit_if(&acc_full[it & 1], leader);
@@ -1035,14 +1286,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else if (warp == kGateWarp) {
         // ------------------------------------------------------------ gate
-        int my_tiles = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
-        gate_role<STAGES, L::kSlots>(p, full, sf_full, ready_count, my_tiles, lane, abort_flag);
+        gate_role<STAGES, L::kSlots>(p, full, sf_full, ready_count, unit_stages<SPLIT>(p, worker), lane, abort_flag);
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps
         const int q = warp & 3;
-        int my_tiles = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) ++my_tiles;
+        const int my_tiles = n_units;
         float scale = 1.0f;
         if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
         uint32_t amax = 0;
@@ -1052,7 +1300,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int help_next = 0;
         auto help = [&](int t) -> bool {
             int m0, n0;
-            tile_coords(p, blockIdx.x + t * gridDim.x, m0, n0, kBM, BN);
+            tile_coords(p, unit_at<SPLIT>(p, worker, t).tile, m0, n0, kBM, BN);
             const int b = t & 1;
             if (!mbar_wait_bounded(&acc_full[b], (t >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag))
                 return false;
@@ -1065,8 +1313,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (lane == 0) mbar_arrive(acc_empty);
             return true;
         };
-        scale_role<L, STAGES>(p, smem, sfload, sfree, empty, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf,
-                              my_tiles, lane, abort_flag, [&](int slot) { mbar_arrive(&sf_full[slot]); },
+        scale_role<L, STAGES, SPLIT>(p, smem, sfload, sfree, empty,
+                                     tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)L::kTmemSf, worker, lane, abort_flag,
+                                     [&](int slot) { mbar_arrive(&sf_full[slot]); },
                               [&](int kg) -> bool {
                                   if (p.epilogue != 1) return true;
                                   for (; help_next < my_tiles - 1 && kg - L::kSlots >= (help_next + 1) * p.num_kt;
@@ -1081,8 +1330,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // completed, so the B stage ring is free for the staging buffers)
         if (my_tiles > 0 && !*abort_flag) {
             const int it = my_tiles - 1, b = it & 1;
+            const KUnit U = unit_at<SPLIT>(p, worker, it);
             int m0, n0;
-            tile_coords(p, blockIdx.x + it * gridDim.x, m0, n0, kBM, BN);
+            tile_coords(p, U.tile, m0, n0, kBM, BN);
             // mma_done (one phase) rather than acc_full[b]: without GELU this warp
             // may finish its slots several tiles ahead of the MMAs, and a parity
             // wait on acc_full[b], whose phases alternate every second tile,
@@ -1091,8 +1341,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_fence_after();
                 uint8_t *bufs = smem + L::kOffB + (warp - 6) * L::kEpiBufs * kEpiChunkBytes;
                 uint32_t nstore = 0;
-                epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride),
-                                                       m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs, nstore, amax, scale);
+                const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
+                if (U.kind == kUnitPartial)
+                    ks_partial_drain<BN, L::kAccStride>(p, worker, 1, 0, t_acc, b, m0 + 32 * q, n0, q, lane, false,
+                                                        BN / 64, BN / 32, 1u, [] {});
+                else if (U.kind == kUnitWhole ||
+                         ks_finish_fold<L, STAGES>(p, smem, 2 * q + 1, U, worker, 1, 0, t_acc, m0 + 32 * q, n0, q, lane,
+                                                   BN / 64, BN / 32, abort_flag))
+                    epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, BN / 64, BN / 32, lane, bufs,
+                                                           nstore, amax, scale);
             }
         }
         epilogue_finish(p, lane, amax);
@@ -1105,15 +1362,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t amax = 0, nstore = 0;
         float scale = 1.0f;
         if (FMT == 3) scale = gemm_ga(p) * (*p.gb);
-        int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        auto release = [&] {
+            if (lane == 0) mbar_arrive(acc_empty);
+        };
+        for (int it = 0; it < n_units; ++it) {
+            const KUnit U = unit_at<SPLIT>(p, worker, it);
             int m0, n0;
-            tile_coords(p, tile, m0, n0, kBM, BN);
+            tile_coords(p, U.tile, m0, n0, kBM, BN);
             const int b = it & 1;
             if (!mbar_wait_bounded(&acc_full[b], (it >> 1) & 1, p.wait_limit_ns, SITE_GEMM_EPI_ACC, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * L::kAccStride);
-            if (tile + (int)gridDim.x >= num_tiles) {
+            const bool last = it + 1 == n_units;
+            // a piece of a split tile: on the last unit the lower half of the
+            // columns (the scale warp takes the upper half), else all of them
+            if (U.kind == kUnitPartial) {
+                ks_partial_drain<BN, L::kAccStride>(p, worker, 1, 0, t_acc, b, m0 + 32 * q, n0, q, lane, !last, 0,
+                                                    last ? BN / 64 : BN / 32, last ? 1u : 2u, release);
+                if (last) break;
+                continue;
+            }
+            if (U.kind == kUnitFinish &&
+                !ks_finish_fold<L, STAGES>(p, smem, 2 * q, U, worker, 1, 0, t_acc, m0 + 32 * q, n0, q, lane, 0,
+                                           last ? BN / 64 : BN / 32, abort_flag))
+                break;
+            if (last) {
                 // the last tile: the lower half of the columns (the scale warp of
                 // this quadrant drains the upper half); nothing waits for its release
                 epilogue_chunks<L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, m0 + 32 * q, n0, 0, BN / 64, lane, bufs, nstore,
@@ -1121,9 +1394,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             epilogue_tile<BN, L::kAccStride, L::kEpiBufs, FMT == 3>(p, &tmC, t_acc, b, m0 + 32 * q, n0, lane, bufs,
-                                                                     nstore, amax, scale, [&] {
-                                                                         if (lane == 0) mbar_arrive(acc_empty);
-                                                                     });
+                                                                     nstore, amax, scale, release);
         }
         epilogue_finish(p, lane, amax);
     }

@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -30,6 +31,7 @@ std::atomic<int> g_pair_enabled{1};
 std::atomic<int> g_pdl_enabled{1};
 std::atomic<int> g_max_gemm_ctas{0};  // 0: one CTA (or CTA pair) per SM pair of the device
 std::atomic<int> g_fused_mode{MX_FUSED_PIPELINED};  // how mx_gemm_fused_act runs (MX_DEBUG_FUSED_MODE)
+std::atomic<int> g_ksplit_mode{0};  // MX_DEBUG_K_SPLIT: 0 auto, 1 never, 2 whenever possible
 
 // Launch attributes shared by the kernels that may overlap the previous kernel
 // in the stream (they call griddep_wait() before reading any input).
@@ -150,7 +152,7 @@ bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) ==
 template <int FMT, int RULE = RULE_OCP>
 mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
                           const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0,
-                          uint32_t *band_ready = nullptr) {
+                          uint32_t *band_ready = nullptr, uint32_t *clear = nullptr, int n_clear = 0) {
     if (M == 0 || K == 0) return MX_OK;
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
     cudaLaunchConfig_t cfg;
@@ -162,7 +164,7 @@ mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld,
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
     if (cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes),
-                           dst->scales, sf_tiles_k, g_in, g_out, g_from_amax, band_ready) != cudaSuccess)
+                           dst->scales, sf_tiles_k, g_in, g_out, g_from_amax, band_ready, clear, n_clear) != cudaSuccess)
         return last_launch();
     return MX_OK;
 }
@@ -280,6 +282,63 @@ cudaError_t smem_limit_once(const void *fn, int bytes) {
 
 // The activation of a fused call: bf16 x quantized inside the GEMM kernel (see
 // GemmParams::fused); A's codes and scales are its destination.
+// Room for the K split's partial sums (ksplit.cuh): the fused call's
+// workspace provides it when it is large enough.
+struct SplitRoom {
+    float *partials;   // kSplitSlots slots of 8 x slot_quads 4 KB blocks
+    uint32_t *flags;   // kSplitSlots counters, zero at the start of the GEMM
+    int slot_quads;
+};
+
+// How many CTA pairs of this kernel the device holds at once (0 if unknown);
+// a split schedule needs every worker resident, since a finishing piece waits
+// for the partial sums of other workers.
+int coresident_pairs(const void *kernel, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(kernel, dev);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
+
+// The work schedule's plan and grid for a launch (fills p.ks and the slot
+// pointers): a split needs the room, no GELU (the finishing piece's epilogue
+// is the plain one) and every worker resident.
+void plan_split(GemmParams &p, int64_t tiles, int workers, int ranks, const SplitRoom *room) {
+    const bool can = room != nullptr && p.epilogue == MX_EPI_NONE && workers * ranks <= kSplitSlots;
+    // the fused call walks its tiles band-major in every mode, so that the
+    // same tiles are split (and summed in the same order) whichever mode runs
+    if (room != nullptr) p.band_major = 1;
+    p.ks = ks_plan(tiles, workers, p.num_kt, g_ksplit_mode.load(), can);
+    if (p.ks.on) {
+        p.ks_partials = room->partials;
+        p.ks_flags = room->flags;
+        p.ks_slot_quads = room->slot_quads;
+    }
+}
+
 struct FusedX {
     int mode;            // GemmParams::fused: 1 in-kernel quantize, 2 quantize kernel feeding bands
     const uint16_t *x;
@@ -313,7 +372,7 @@ void set_fused(GemmParams &p, const FusedX *fx, const void *a_codes, const uint8
 template <int FMT, int BN, int STAGES, int A_ROWS = kBM>
 mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                         const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out, cudaStream_t st,
-                        const FusedX *fx) {
+                        const FusedX *fx, const SplitRoom *room) {
     using L = GemmSmem<FMT, BN, STAGES, A_ROWS>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
@@ -333,8 +392,10 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
-    if (smem_limit_once(reinterpret_cast<const void *>(gemm_kernel<FMT, BN, STAGES, A_ROWS>), L::kAlloc) !=
-        cudaSuccess)
+    if (smem_limit_once(reinterpret_cast<const void *>(gemm_kernel<FMT, BN, STAGES, A_ROWS, false>), L::kAlloc) !=
+            cudaSuccess ||
+        smem_limit_once(reinterpret_cast<const void *>(gemm_kernel<FMT, BN, STAGES, A_ROWS, true>), L::kAlloc) !=
+            cudaSuccess)
         return MX_ERR_CUDA;
     GemmParams p{};
     p.sf_tiles_k = sf_tiles_k;
@@ -357,9 +418,11 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     p.wait_limit_ns = g_wait_limit_ns.load();
     set_fused(p, fx, a_codes, a_scales, M, K);
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    if (tiles > INT32_MAX) return MX_ERR_UNSUPPORTED_SHAPE;
     const int cap = g_max_gemm_ctas.load();
-    const int64_t max_ctas = cap > 0 && cap < num_sms() ? cap : num_sms();
-    const unsigned grid = (unsigned)(tiles < max_ctas ? tiles : max_ctas);
+    const int max_ctas = cap > 0 && cap < num_sms() ? cap : num_sms();
+    plan_split(p, tiles, max_ctas, 1, room);
+    const unsigned grid = (unsigned)p.ks.workers;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(grid, 1, 1);
@@ -369,8 +432,9 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     cudaLaunchAttribute attr[1];
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, BN, STAGES, A_ROWS>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
-        return last_launch();
+    // the kernel compiled for the split runs only when the plan splits
+    const auto kern = p.ks.on ? gemm_kernel<FMT, BN, STAGES, A_ROWS, true> : gemm_kernel<FMT, BN, STAGES, A_ROWS, false>;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tsa, tsb, p) != cudaSuccess) return last_launch();
     return last_launch();
 }
 
@@ -378,7 +442,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
 template <int FMT, int STAGES, int BN = 256>
 mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                              const float *ga, uint16_t *C, int64_t ldc, int epilogue, float *amax_out,
-                             cudaStream_t st, const FusedX *fx) {
+                             cudaStream_t st, const FusedX *fx, const SplitRoom *room) {
     using L = PairSmem<FMT, STAGES, BN>;
     static_assert(L::kAlloc <= kSmemLimit, "shared memory budget");
     const int64_t M = A->rows, N = B->rows, K = A->cols;
@@ -398,7 +462,13 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     const bool tma_store = (ldc % 8 == 0) && aligned16(C);
     memset(&tc, 0, sizeof(tc));
     if (tma_store && !make_tmap_c(&tc, C, M, N, ldc)) return MX_ERR_CUDA;
-    if (smem_limit_once(reinterpret_cast<const void *>(gemm_pair_kernel<FMT, STAGES, BN>), L::kAlloc) != cudaSuccess)
+    // only the 256-wide tiles (no GELU) have a variant compiled for the split
+    constexpr bool kCanSplit = BN == 256;
+    using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+    const Kern kern_whole = gemm_pair_kernel<FMT, STAGES, BN, false>;
+    const Kern kern_split = kCanSplit ? gemm_pair_kernel<FMT, STAGES, BN, kCanSplit> : kern_whole;
+    if (smem_limit_once(reinterpret_cast<const void *>(kern_whole), L::kAlloc) != cudaSuccess ||
+        smem_limit_once(reinterpret_cast<const void *>(kern_split), L::kAlloc) != cudaSuccess)
         return MX_ERR_CUDA;
     GemmParams p{};
     p.sf_tiles_k = sf_tiles_k;
@@ -422,9 +492,15 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     p.wait_limit_ns = g_wait_limit_ns.load();
     set_fused(p, fx, a_codes, a_scales, M, K);
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    if (tiles > INT32_MAX) return MX_ERR_UNSUPPORTED_SHAPE;
     const int cap = g_max_gemm_ctas.load();
-    const int64_t max_pairs = cap > 0 && cap < num_sms() ? (cap + 1) / 2 : num_sms() / 2;
-    const unsigned pairs = (unsigned)(tiles < max_pairs ? tiles : max_pairs);
+    const int max_pairs = cap > 0 && cap < num_sms() ? (cap + 1) / 2 : num_sms() / 2;
+    // a split plan runs only on pairs that are all resident at once
+    const int resident =
+        room != nullptr && kCanSplit ? coresident_pairs(reinterpret_cast<const void *>(kern_split), L::kAlloc) : 0;
+    plan_split(p, tiles, resident > 0 && resident < max_pairs ? resident : max_pairs, 2, resident > 0 ? room : nullptr);
+    if (!p.ks.on) p.ks = ks_plan(tiles, max_pairs, p.num_kt, 1, false);
+    const unsigned pairs = (unsigned)p.ks.workers;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(2 * pairs, 1, 1);
@@ -438,7 +514,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1 + (unsigned)pdl_attr(&attr[1]);
-    if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<FMT, STAGES, BN>, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, p.ks.on ? kern_split : kern_whole, ta, tb, tc, tsa, tsb, p) != cudaSuccess)
         return last_launch();
     return last_launch();
 }
@@ -446,33 +522,34 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
 template <int FMT>
 mx_status launch_gemm_fmt(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                           const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st,
-                          const FusedX *fx) {
+                          const FusedX *fx, const SplitRoom *room) {
     if (A->rows > 128 && B->rows > 128 && g_pair_enabled.load()) {
         // GELU: 256 x 128 tiles, whose two accumulators need no shared TMEM
         // columns, so each tile's GELU drain overlaps the next tile's MMAs
         if (epi == MX_EPI_GELU)
-            return launch_gemm_pair_t<FMT, 7, 128>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+            return launch_gemm_pair_t<FMT, 7, 128>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
         return launch_gemm_pair_t<FMT, (FMT == 2 || FMT == 3) ? 5 : 6>(A, B, a_codes, a_scales, ga, C, ldc, epi,
-                                                                       amax_out, st, fx);
+                                                                       amax_out, st, fx, room);
     }
-    if (B->rows <= 128) return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+    if (B->rows <= 128)
+        return launch_gemm_t<FMT, 128, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
     // at most 32 rows of A (decode-like activations): the weight stream gets a
     // fifth stage from the shared memory a 128-row A tile would take
     if (A->rows <= 32)
-        return launch_gemm_t<FMT, 256, 5, 32>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
-    return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+        return launch_gemm_t<FMT, 256, 5, 32>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
+    return launch_gemm_t<FMT, 256, 4>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
 }
 
 mx_status launch_gemm(const mx_tensor *A, const mx_tensor *B, const void *a_codes, const uint8_t *a_scales,
                       const float *ga, uint16_t *C, int64_t ldc, int epi, float *amax_out, cudaStream_t st,
-                      const FusedX *fx = nullptr) {
+                      const FusedX *fx = nullptr, const SplitRoom *room = nullptr) {
     if (gemm_runtime_types(A->fmt, B->fmt))
-        return launch_gemm_fmt<kGemmRuntimeTypes>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+        return launch_gemm_fmt<kGemmRuntimeTypes>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
     switch (A->fmt) {
-    case MX_MXFP8_E4M3: return launch_gemm_fmt<0>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
-    case MX_MXFP8_E5M2: return launch_gemm_fmt<1>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
-    case MX_MXFP4: return launch_gemm_fmt<2>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
-    default: return launch_gemm_fmt<3>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx);
+    case MX_MXFP8_E4M3: return launch_gemm_fmt<0>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
+    case MX_MXFP8_E5M2: return launch_gemm_fmt<1>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
+    case MX_MXFP4: return launch_gemm_fmt<2>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
+    default: return launch_gemm_fmt<3>(A, B, a_codes, a_scales, ga, C, ldc, epi, amax_out, st, fx, room);
     }
 }
 
@@ -518,15 +595,23 @@ mx_status launch_gemm_mbs(const mx_tensor *A, const mx_tensor *B, uint16_t *C, i
     return last_launch();
 }
 
-// The fused call's workspace: a header, then X's codes and scales, each
-// starting on a 256-byte boundary.  Header words: [0] g of X (NVFP4), [1]
-// amax(|X|) of the pre-pass, [2] the fused kernel's work counter, [3] unused,
-// [16 ..] one ready counter per 128-row band of X.
+// The fused call's workspace: a header, then X's codes and scales, then
+// (optional) the K split's partial-sum slots, each starting on a 256-byte
+// boundary.  Header words: [0] g of X (NVFP4), [1] amax(|X|) of the pre-pass,
+// [2] the fused kernel's work counter, [3] unused, [16 ..] one ready counter
+// per 128-row band of X, then kSplitSlots counters of the partial-sum slots.
 constexpr size_t kWsBandOffset = 64;
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-size_t fused_ws_header(int64_t M) { return align256(kWsBandOffset + 4 * (size_t)cdiv(M, 128)); }
+size_t fused_ws_flags(int64_t M) { return kWsBandOffset + 4 * (size_t)cdiv(M, 128); }
+size_t fused_ws_header(int64_t M) { return align256(fused_ws_flags(M) + 4 * (size_t)kSplitSlots); }
 size_t fused_ws_bytes(int fmt, int64_t M, int64_t K) {
     return fused_ws_header(M) + align256((size_t)(M * K * fmt_bits(fmt) / 8)) + align256(scales_bytes(fmt, M, K));
+}
+// 32-row quadrants of a partial-sum slot: those of a CTA's accumulator rows
+// that exist (a slot holds 8 column chunks of 4 KB per quadrant)
+size_t fused_split_quads(int64_t M) { return (size_t)(M < 128 ? cdiv(M, 32) : 4); }
+size_t fused_ws_split_bytes(int fmt, int64_t M, int64_t K) {
+    return fused_ws_bytes(fmt, M, K) + (size_t)kSplitSlots * 8 * fused_split_quads(M) * 4096;
 }
 
 // Zero the fused kernel's counters (the work counter and the band counters).
@@ -557,7 +642,8 @@ mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st) {
 // device pointer of X's g (NVFP4) through *ga.
 mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int64_t ldx, uint8_t *ws,
                            const float *x_gscale, const float *x_amax, mx_tensor *xa, const float **ga,
-                           cudaStream_t st, uint32_t *band_ready = nullptr) {
+                           cudaStream_t st, uint32_t *band_ready = nullptr, uint32_t *clear = nullptr,
+                           int n_clear = 0) {
     float *g_slot = reinterpret_cast<float *>(ws);
     float *amax_slot = reinterpret_cast<float *>(ws + 4);
     xa->fmt = fmt;
@@ -570,13 +656,13 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
     *ga = nullptr;
     mx_status s = MX_OK;
     switch (fmt) {
-    case MX_MXFP8_E4M3: s = launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
-    case MX_MXFP8_E5M2: s = launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
-    case MX_MXFP4: s = launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
-    case MX_MXFP6_E3M2: s = launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready); break;
+    case MX_MXFP8_E4M3: s = launch_quantize<0>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready, clear, n_clear); break;
+    case MX_MXFP8_E5M2: s = launch_quantize<1>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready, clear, n_clear); break;
+    case MX_MXFP4: s = launch_quantize<2>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready, clear, n_clear); break;
+    case MX_MXFP6_E3M2: s = launch_quantize<4>(X, M, K, ldx, xa, nullptr, nullptr, st, 0, band_ready, clear, n_clear); break;
     default:
         if (x_gscale != nullptr) {
-            s = launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st, 0, band_ready);
+            s = launch_quantize<3>(X, M, K, ldx, xa, x_gscale, nullptr, st, 0, band_ready, clear, n_clear);
             *ga = x_gscale;
         } else {
             const float *amax = x_amax;
@@ -586,7 +672,7 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
                     X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
                 amax = amax_slot;
             }
-            s = launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1, band_ready);
+            s = launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1, band_ready, clear, n_clear);
             *ga = g_slot;
         }
     }
@@ -635,6 +721,10 @@ mx_status mx_debug_set(int key, uint64_t value) {
     case MX_DEBUG_FUSED_MODE:
         if (value > MX_FUSED_TWO_KERNELS) return MX_ERR_INVALID_ARG;
         g_fused_mode.store((int)value);
+        return MX_OK;
+    case MX_DEBUG_K_SPLIT:
+        if (value > MX_K_SPLIT_ALWAYS) return MX_ERR_INVALID_ARG;
+        g_ksplit_mode.store((int)value);
         return MX_OK;
     default: return MX_ERR_INVALID_ARG;
     }
@@ -825,8 +915,32 @@ mx_status mx_gemm(const mx_tensor *A, const mx_tensor *B, void *C_bf16, int64_t 
 }
 
 size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K) {
-    if (!valid_fmt(fmt) || M < 0 || K < 0) return 0;
+    if (!valid_fmt(fmt) || M < 0 || K < 0 || M > INT32_MAX || K > INT32_MAX) return 0;
     return fused_ws_bytes(fmt, M, K);
+}
+
+size_t mx_fused_split_workspace_bytes(int fmt, int64_t M, int64_t K) {
+    if (!valid_fmt(fmt) || M < 0 || K < 0 || M > INT32_MAX || K > INT32_MAX) return 0;
+    return fused_ws_split_bytes(fmt, M, K);
+}
+
+int mx_debug_split_units(int64_t tiles, int workers, int kt, int mode, int worker, int32_t *out, int max_units,
+                         int *n_workers) {
+    if (tiles < 0 || tiles > INT32_MAX || workers < 1 || kt < 1 || mode < 0 || mode > MX_K_SPLIT_ALWAYS || worker < 0)
+        return -1;
+    const KSplitPlan plan = ks_plan(tiles, workers, kt, mode, true);
+    if (n_workers) *n_workers = plan.workers;
+    if (worker >= plan.workers) return 0;
+    const int n = ks_units(plan, worker);
+    for (int u = 0; u < n && u < max_units && out; ++u) {
+        const KUnit x = ks_unit(plan, worker, u);
+        out[5 * u] = x.tile;
+        out[5 * u + 1] = x.kb;
+        out[5 * u + 2] = x.ke;
+        out[5 * u + 3] = x.kind;
+        out[5 * u + 4] = x.first;
+    }
+    return n;
 }
 
 mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx, const mx_tensor *W,
@@ -873,17 +987,28 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
         if (s != MX_OK) return s;
         return launch_gemm_mbs(&xa, W, static_cast<uint16_t *>(C_bf16), ldc, st);
     }
+    // room for the K split's partial sums (the GEMM decides whether to split)
+    SplitRoom room;
+    const SplitRoom *roomp = nullptr;
+    if (workspace_bytes >= fused_ws_split_bytes(fmt, M, K) && epilogue == MX_EPI_NONE) {
+        room.partials = reinterpret_cast<float *>(ws + fused_ws_bytes(fmt, M, K));
+        room.flags = reinterpret_cast<uint32_t *>(ws + fused_ws_flags(M));
+        room.slot_quads = (int)fused_split_quads(M);
+        roomp = &room;
+    }
     int mode = g_fused_mode.load();
     // a single 128-row band is written only when the whole quantize is: no band
     // of it to start early on, so the pipelined mode would only add its counter
     // reset
     if (mode == MX_FUSED_PIPELINED && M <= kQTileRows) mode = MX_FUSED_TWO_KERNELS;
     if (mode == MX_FUSED_TWO_KERNELS) {
-        // quantize_kernel into the workspace, then the plain GEMM in stream order
-        s = fused_quantize_x(fmt, X, M, K, ldx, ws, x_gscale, x_amax, &xa, &ga, st);
+        // quantize_kernel into the workspace (clearing the slot counters, with
+        // split room), then the plain GEMM in stream order
+        s = fused_quantize_x(fmt, X, M, K, ldx, ws, x_gscale, x_amax, &xa, &ga, st, nullptr,
+                             roomp != nullptr ? room.flags : nullptr, kSplitSlots);
         if (s != MX_OK) return s;
         return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out,
-                           st);
+                           st, nullptr, roomp);
     }
     // X quantized by the GEMM kernel itself (MX_FUSED_IN_KERNEL) or by the
     // quantize kernel, band by band, with the GEMM starting on the bands already
@@ -923,7 +1048,7 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
             ga = x_amax_src;
         }
     }
-    // words 2 .. 15 and the band counters
+    // words 2 .. 15, the band counters and the slot counters
     s = launch_fused_reset(reinterpret_cast<uint32_t *>(ws + 8), (int)((fused_ws_header(M) - 8) / 4), st);
     if (s != MX_OK) return s;
     if (fx.mode == 2) {
@@ -933,7 +1058,8 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
         if (s != MX_OK) return s;
     }
     return launch_gemm(&xa, W, xa.codes, xa.scales, ga, static_cast<uint16_t *>(C_bf16), ldc, epilogue, amax_out, st,
-                       &fx);}
+                       &fx, roomp);
+}
 
 }  // extern "C"
 

@@ -37,6 +37,7 @@ enum : unsigned {
     SITE_GEMM_SF_FREE = 12,
     SITE_GEMM_MMA_READY = 13,
     SITE_FUSED_BAND_READY = 14,   // a TMA producer waiting for a band of the fused quantize
+    SITE_KSPLIT_PARTIAL = 15,     // a finishing piece waiting for the partial sums of its tile
 };
 
 // {flags, first site, first block, count}
@@ -252,6 +253,15 @@ MX_DEVICE_INLINE void tma_load_2d(void *smem_dst, const void *tmap, int32_t x, i
         : "memory");
 }
 
+// Untiled bulk copy (no multicast) of `bytes` from global memory into this
+// CTA's shared memory; both addresses 16-byte aligned, bytes a multiple of 16.
+MX_DEVICE_INLINE void bulk_load(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // 3D tiled TMA load (no multicast) into this CTA's shared memory.
 MX_DEVICE_INLINE void tma_load_3d(void *smem_dst, const void *tmap, int32_t x, int32_t y, int32_t z, uint64_t *bar) {
     asm volatile(
@@ -324,6 +334,15 @@ MX_DEVICE_INLINE void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, ui
 }
 
 // Load 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one row per thread).
+MX_DEVICE_INLINE void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
 MX_DEVICE_INLINE void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "

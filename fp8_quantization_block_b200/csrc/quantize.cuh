@@ -547,7 +547,9 @@ MX_DEVICE_INLINE void tile_quantize(const TileRegs<NT, ROWS> &r, int64_t M, int6
 // is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
 // if gscale_out != nullptr, CTA 0 also stores g there.  band_ready (nullable):
 // each CTA adds one to its 128-row band's counter once its codes and scales
-// are written (release, gpu scope).
+// are written (release, gpu scope).  clear (nullable): n_clear words that CTA
+// 0 zeroes once the previous kernel in the stream has completed (the partial-
+// sum counters of the fused call's GEMM, which runs after this grid).
 // CTAs per SM that the register allocation of quantize_kernel<FMT> targets,
 // chosen by timing 2^28-element inputs: the FP8 and FP4 MX casts run fastest
 // with the registers left free (1), NVFP4 with four resident CTAs (the
@@ -563,7 +565,8 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
                                                              const float *__restrict__ gscale_in,
                                                              float *__restrict__ gscale_out, int g_from_amax,
-                                                             uint32_t *__restrict__ band_ready) {
+                                                             uint32_t *__restrict__ band_ready,
+                                                             uint32_t *__restrict__ clear, int n_clear) {
     constexpr int kPasses = kQTileRows / 32;               // 32 rows per pass (8 warps x 4 rows)
     __shared__ __align__(16) uint8_t sf_tile[quantize_sf_bytes<FMT>()];
 
@@ -581,6 +584,8 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
     // kernel in the stream may take SMs as this grid's CTAs leave them (it still
     // waits for this grid's completion before reading anything).
     griddep_launch_dependents();
+    if (clear != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < n_clear; i += blockDim.x) clear[i] = 0u;
     if (FMT == FMT_NVFP4) {
         const float g = nv_g_from(gscale_in, g_from_amax);
         if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;

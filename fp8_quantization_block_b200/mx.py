@@ -30,12 +30,15 @@ MX_DEBUG_WAIT_LIMIT_NS, MX_DEBUG_SKIP_PRODUCER, MX_DEBUG_PAIR_GEMM, MX_DEBUG_OVE
 MX_DEBUG_MAX_GEMM_CTAS = 5
 MX_DEBUG_FUSED_MODE = 6
 MX_FUSED_PIPELINED, MX_FUSED_IN_KERNEL, MX_FUSED_TWO_KERNELS = 0, 1, 2
+MX_DEBUG_K_SPLIT = 7
+MX_K_SPLIT_AUTO, MX_K_SPLIT_NEVER, MX_K_SPLIT_ALWAYS = 0, 1, 2
+KUNIT_WHOLE, KUNIT_PARTIAL, KUNIT_FINISH = 0, 1, 2
 
 EXPORTED = [
     "mx_codes_bytes", "mx_scales_bytes", "mx_block_size", "mx_quantize", "mx_dequantize", "mx_gemm",
     "mx_gemm_fused_act", "mx_fused_workspace_bytes", "mx_check_device_error", "mx_status_string",
     "mx_version", "mx_debug_set", "mx_gemm_fused_act_noalloc", "mx_quantize_oas", "mx_qsnr",
-    "mx_quantize_rht", "mx_quantize_mbs_dynamic",
+    "mx_quantize_rht", "mx_quantize_mbs_dynamic", "mx_fused_split_workspace_bytes", "mx_debug_split_units",
 ]
 MX_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -78,6 +81,8 @@ def lib() -> ctypes.CDLL:
                 "mx_gemm": (i32, [T, T, P, i64, P]),
                 "mx_gemm_fused_act": (i32, [i32, P, i64, i64, i64, T, P, i64, i32, P, P, P, P, sz, P]),
                 "mx_fused_workspace_bytes": (sz, [i32, i64, i64]),
+                "mx_fused_split_workspace_bytes": (sz, [i32, i64, i64]),
+                "mx_debug_split_units": (i32, [i64, i32, i32, i32, i32, P, i32, P]),
                 "mx_gemm_fused_act_noalloc": (i32, [i32, P, i64, i64, i64, T, P, i64, i32, P, P, P, P]),
                 "mx_check_device_error": (i32, [P, ctypes.POINTER(ctypes.c_uint32)]),
                 "mx_status_string": (ctypes.c_char_p, [i32]),
@@ -148,6 +153,22 @@ def mx_gemm_fused_act_noalloc(fmt, X_ptr, M, K, ldx, W: MxTensorC, C_ptr, ldc, e
 
 def mx_fused_workspace_bytes(fmt: int, M: int, K: int) -> int:
     return int(lib().mx_fused_workspace_bytes(fmt, M, K))
+
+
+def mx_fused_split_workspace_bytes(fmt: int, M: int, K: int) -> int:
+    return int(lib().mx_fused_split_workspace_bytes(fmt, M, K))
+
+
+def split_units(tiles: int, workers: int, kt: int, mode: int, worker: int):
+    """The GEMM work schedule of one worker (host only): (grid workers, [(tile,
+    kb, ke, kind, first), ...])."""
+    n_workers = ctypes.c_int(0)
+    n = int(lib().mx_debug_split_units(tiles, workers, kt, mode, worker, None, 0, ctypes.byref(n_workers)))
+    if n < 0:
+        raise MxError(MX_ERR_INVALID_ARG, "mx_debug_split_units")
+    buf = (ctypes.c_int32 * (5 * max(n, 1)))()
+    lib().mx_debug_split_units(tiles, workers, kt, mode, worker, buf, n, None)
+    return n_workers.value, [tuple(buf[5 * u:5 * u + 5]) for u in range(n)]
 
 
 def mx_check_device_error(stream=None):
@@ -289,9 +310,11 @@ def gemm_fused_act(x: torch.Tensor, W: MxTensor, out: torch.Tensor | None = None
     return out
 
 
-def fused_workspace(fmt: int, M: int, K: int, device="cuda") -> torch.Tensor:
-    """A workspace for gemm_fused_act (torch's allocator hands out 256-B aligned blocks)."""
-    return torch.empty(mx_fused_workspace_bytes(fmt, M, K), dtype=torch.uint8, device=device)
+def fused_workspace(fmt: int, M: int, K: int, device="cuda", split: bool = True) -> torch.Tensor:
+    """A workspace for gemm_fused_act (torch's allocator hands out 256-B aligned
+    blocks); split: with room for the K split of the last wave."""
+    n = mx_fused_split_workspace_bytes(fmt, M, K) if split else mx_fused_workspace_bytes(fmt, M, K)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def check_device_error(stream=None) -> None:

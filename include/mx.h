@@ -225,7 +225,19 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  * also the amax pre-pass).
  *   workspace: device buffer of at least mx_fused_workspace_bytes(fmt, M, K)
  *              bytes, 256-byte aligned; its contents are scratch, and calls
- *              that overlap on the GPU must not share one.
+ *              that overlap on the GPU must not share one.  With at least
+ *              mx_fused_split_workspace_bytes(fmt, M, K) bytes and no
+ *              epilogue function, the GEMM may also split its last wave of
+ *              output tiles along K so that every SM has work: when the tile
+ *              count leaves more than 15% of the SMs (CTA pairs) without a
+ *              tile in the last wave, those tiles' K stages are shared evenly
+ *              over all of them, each piece's fp32 partial sum goes to the
+ *              workspace, and the worker holding a tile's last stages adds the
+ *              others' partial sums to its own, in a fixed order, before the
+ *              epilogue.  Results then differ from mx_gemm's only in the fp32
+ *              summation order (within the same accuracy contract); they are
+ *              the same from call to call for one shape, device and workspace
+ *              size.
  *   epilogue : MX_EPI_NONE, or MX_EPI_GELU: the exact-erf form x Phi(x) =
  *              0.5 x erfc(-x / sqrt 2), applied in FP32 before the bf16
  *              rounding, with erfc(z) = t exp(-z^2 + P(t)), t = 1/(1 + z/2),
@@ -246,9 +258,14 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
                             float *amax_out, const float *x_gscale, const float *x_amax,
                             void *workspace, size_t workspace_bytes, void *stream);
 /* Workspace bytes mx_gemm_fused_act needs for an [M x K] activation of format
- * fmt (a header of 64 bytes plus 4 per 128-row band, rounded up to 256, then
- * X's codes and scales); 0 for a bad format. */
+ * fmt (a header of 64 bytes, 4 per 128-row band and 4 per partial-sum slot,
+ * rounded up to 256, then X's codes and scales); 0 for a bad format or size. */
 size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K);
+/* Workspace bytes with which mx_gemm_fused_act may also split its last wave
+ * along K: mx_fused_workspace_bytes plus 148 partial-sum slots of 32 KB per
+ * 32 rows of min(M, 128) (fp32 sums of 256 columns; 19.4 MB for M > 96); 0
+ * for a bad format or size. */
+size_t mx_fused_split_workspace_bytes(int fmt, int64_t M, int64_t K);
 
 /* mx_gemm_fused_act without a workspace argument, for callers that cannot
  * allocate device memory: code inside an inference engine's enqueue or plugin
@@ -264,6 +281,10 @@ size_t mx_fused_workspace_bytes(int fmt, int64_t M, int64_t K);
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, once per device, with that device current); make
  *   that first call before any stream capture.
+ *   The GEMM splits its last wave along K (see workspace above) only where
+ *   the array also holds mx_fused_split_workspace_bytes(fmt, M, K), i.e. for
+ *   small M; a workspace call with a workspace of MX_NOALLOC_SCRATCH_BYTES
+ *   gives the same results bit for bit.
  *   Every call uses the same array and leaves its contents behind (whatever
  *   must start at zero is cleared by the call).  Calls that overlap on the GPU
  *   -- on different streams, or from several host threads -- race on it and
@@ -306,7 +327,9 @@ int mx_version(void);
  *                            CTA walks several tiles even on small shapes;
  *                            0 (default) = one CTA per SM.  The result does
  *                            not depend on it (each tile is summed in the
- *                            same order wherever it runs).
+ *                            same order wherever it runs), except where the
+ *                            fused call splits tiles along K (the split
+ *                            follows the grid).
  *   MX_DEBUG_FUSED_MODE    : how mx_gemm_fused_act runs (same results bit for
  *                            bit in every mode):
  *                            MX_FUSED_PIPELINED (default): the quantize kernel
@@ -320,14 +343,22 @@ int mx_version(void);
  *                            X band by band before their first tile;
  *                            MX_FUSED_TWO_KERNELS: the quantize kernel, then the
  *                            GEMM kernel after it has completed.
- * Returns MX_ERR_INVALID_ARG for an unknown key. */
+ *   MX_DEBUG_K_SPLIT       : when the fused call splits its last wave along K
+ *                            (given the workspace room): MX_K_SPLIT_AUTO
+ *                            (default, when the last wave would leave more than
+ *                            15% of the workers idle), MX_K_SPLIT_NEVER, or
+ *                            MX_K_SPLIT_ALWAYS (whenever the tile count is not
+ *                            a multiple of the workers and each worker gets at
+ *                            least two K stages).
+ * Returns MX_ERR_INVALID_ARG for an unknown key or value. */
 typedef enum {
     MX_DEBUG_WAIT_LIMIT_NS = 1,
     MX_DEBUG_SKIP_PRODUCER = 2,
     MX_DEBUG_PAIR_GEMM = 3,
     MX_DEBUG_OVERLAP_LAUNCH = 4,
     MX_DEBUG_MAX_GEMM_CTAS = 5,
-    MX_DEBUG_FUSED_MODE = 6
+    MX_DEBUG_FUSED_MODE = 6,
+    MX_DEBUG_K_SPLIT = 7
 } mx_debug_key;
 /* Values of MX_DEBUG_FUSED_MODE. */
 typedef enum {
@@ -335,7 +366,25 @@ typedef enum {
     MX_FUSED_IN_KERNEL = 1,
     MX_FUSED_TWO_KERNELS = 2
 } mx_fused_mode;
+/* Values of MX_DEBUG_K_SPLIT. */
+typedef enum {
+    MX_K_SPLIT_AUTO = 0,
+    MX_K_SPLIT_NEVER = 1,
+    MX_K_SPLIT_ALWAYS = 2
+} mx_k_split_mode;
 mx_status mx_debug_set(int key, uint64_t value);
+
+/* The GEMM kernels' work schedule, for tests (host only, no GPU needed): the
+ * plan for `tiles` output tiles of `kt` K stages each on at most `workers`
+ * workers (CTAs, or CTA pairs) under split mode `mode` (mx_k_split_mode, with
+ * room for the partial sums), and the work units of worker `worker` in the
+ * order it runs them: out[5u .. 5u + 4] = {tile, first K stage, end K stage,
+ * kind (0 whole tile, 1 partial piece, 2 finishing piece), the first worker
+ * holding a partial sum of the tile (kind 2)}, for up to max_units units.
+ * *n_workers (if non-NULL) receives the grid's worker count.  Returns the
+ * worker's number of units, or -1 for invalid arguments. */
+int mx_debug_split_units(int64_t tiles, int workers, int kt, int mode, int worker, int32_t *out, int max_units,
+                         int *n_workers);
 
 #ifdef __cplusplus
 }

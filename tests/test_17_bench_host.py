@@ -45,17 +45,21 @@ SHAPES = [(4096, 3072), (4608, 12288), (16, 28672), (1, 300), (32, 257), (33, 40
 def test_kernel_names_are_built_kernels(bench, kernel_symbols, fmt):
     for M, N in SHAPES:
         for gelu in (False, True):
-            assert bench.gemm_kernel_name(fmt, M, N, gelu) in kernel_symbols, (fmt, M, N, sorted(kernel_symbols))
+            for split in (False, True):
+                name = bench.gemm_kernel_name(fmt, M, N, gelu, split)
+                assert name in kernel_symbols, (fmt, M, N, name, sorted(kernel_symbols))
 
 
 def test_kernel_choice_by_shape(bench):
-    assert bench.gemm_kernel_name(0, 4096, 3072) == "gemm_pair_kernel<0, 6, 256>"
-    assert bench.gemm_kernel_name(3, 4608, 12288) == "gemm_pair_kernel<3, 5, 256>"
-    assert bench.gemm_kernel_name(3, 4608, 12288, gelu=True) == "gemm_pair_kernel<3, 7, 128>"
-    assert bench.gemm_kernel_name(4, 4096, 3072) == "gemm_pair_kernel<4, 6, 256>"
-    assert bench.gemm_kernel_name(3, 16, 28672) == "gemm_kernel<3, 256, 5, 32>"
-    assert bench.gemm_kernel_name(3, 128, 28672) == "gemm_kernel<3, 256, 4, 128>"
-    assert bench.gemm_kernel_name(2, 300, 100) == "gemm_kernel<2, 128, 4, 128>"
+    assert bench.gemm_kernel_name(0, 4096, 3072) == "gemm_pair_kernel<0, 6, 256, false>"
+    assert bench.gemm_kernel_name(3, 4608, 12288) == "gemm_pair_kernel<3, 5, 256, false>"
+    assert bench.gemm_kernel_name(3, 4608, 12288, gelu=True) == "gemm_pair_kernel<3, 7, 128, false>"
+    assert bench.gemm_kernel_name(3, 4608, 12288, gelu=True, split=True) == "gemm_pair_kernel<3, 7, 128, false>"
+    assert bench.gemm_kernel_name(4, 4096, 3072) == "gemm_pair_kernel<4, 6, 256, false>"
+    assert bench.gemm_kernel_name(3, 16, 28672) == "gemm_kernel<3, 256, 5, 32, false>"
+    assert bench.gemm_kernel_name(3, 16, 8192, split=True) == "gemm_kernel<3, 256, 5, 32, true>"
+    assert bench.gemm_kernel_name(3, 128, 28672) == "gemm_kernel<3, 256, 4, 128, false>"
+    assert bench.gemm_kernel_name(2, 300, 100) == "gemm_kernel<2, 128, 4, 128, false>"
 
 
 def test_roofline_bound_follows_arithmetic_intensity(bench):
@@ -111,7 +115,7 @@ def test_result_line_keeps_the_contract(bench):
         assert line["higher_is_better"] is True and line["vs_baseline"] is None
         assert line["config"]["workload"] == wl["name"]
         roof = line["roofline"]
-        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6, 256> (fused quantize)"
+        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6, 256, false> (fused quantize)"
         assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"], rel=1e-3)
         assert roof["peak"] == pytest.approx(bench.tensor_peak(0, bench.measured_peaks()[0], False), rel=1e-3)
         assert roof["clock_normalised_kernel_us"] == pytest.approx(40.5 * 1762 / 1965, abs=0.01)
@@ -126,7 +130,7 @@ def test_result_line_keeps_the_contract(bench):
     args.workload = "skinny_nvfp4"
     line = bench.result_line(args, bench.WORKLOADS["skinny_nvfp4"], dict(r, f_ms=[0.025] * 50), 1)
     assert line["roofline"]["bound"] == "hbm" and line["roofline"]["unit"] == "GB/s"
-    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32> (fused quantize)"
+    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32, false> (fused quantize)"
     assert line["gpu_launches"] == 3 * 50
     json_line = __import__("json").dumps(line)
     assert "\n" not in json_line

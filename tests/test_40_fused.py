@@ -29,7 +29,8 @@ def test_fused_equals_unfused(fmt, M, N, K):
     W_bits = synth.gaussian_weights(400 + N, N, K)
     X, Wt = to_dev(X_bits), to_dev(W_bits)
     W = mx.quantize(Wt, fmt)
-    C_f = mx.gemm_fused_act(X, W)
+    # without room for the K split, whose partial sums change the fp32 order
+    C_f = mx.gemm_fused_act(X, W, workspace=mx.fused_workspace(fmt, M, K, split=False))
     C_u = mx.gemm(mx.quantize(X, fmt), W)
     torch.cuda.synchronize()
     mx.check_device_error()
@@ -126,7 +127,7 @@ def test_nvfp4_mlp_chain_without_host_sync():
     W2 = mx.quantize(to_dev(synth.gaussian_weights(72, D, F)), 3)
     aH = torch.empty(1, device="cuda")
     H = mx.gemm_fused_act(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=aH)
-    Y = mx.gemm_fused_act(H, W2, x_amax=aH)
+    Y = mx.gemm_fused_act(H, W2, x_amax=aH, workspace=mx.fused_workspace(3, M, F, split=False))
     torch.cuda.synchronize()
     mx.check_device_error()
     # the same chain unfused: quantize H (g from its own amax) then GEMM
@@ -177,7 +178,7 @@ def test_nvfp4_mlp_pair_full_size_sampled_rows():
     X = to_dev(X_bits)
     aH = torch.empty(1, device="cuda")
     H = mx.gemm_fused_act(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=aH)
-    Y = mx.gemm_fused_act(H, W2, x_amax=aH)
+    Y = mx.gemm_fused_act(H, W2, x_amax=aH, workspace=mx.fused_workspace(3, M, F, split=False))
     qX = mx.quantize(X, 3)
     qH = mx.quantize(H, 3)
     Y_u = mx.gemm(qH, W2)

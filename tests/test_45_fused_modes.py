@@ -166,7 +166,8 @@ def test_workspace_dirty_and_reused(fmt, mode):
 def test_workspace_holds_mx_quantize_output(fmt, mode):
     """X's codes and scales, as the GEMM kernel wrote them into the workspace,
     equal mx_quantize's (the workspace layout is the header, then the codes,
-    then the scales, each on a 256-byte boundary)."""
+    then the scales, each on a 256-byte boundary; the header holds 64 bytes,
+    a counter per 128-row band and the 148 partial-sum slot counters)."""
     M, N, K = 333, 384, 1024
     X = to_dev(synth.sweep_tensor(670, M, K))
     W = mx.quantize(to_dev(synth.gaussian_weights(671, N, K)), 4 if fmt == 4 else fmt)
@@ -175,7 +176,7 @@ def test_workspace_holds_mx_quantize_output(fmt, mode):
         mx.gemm_fused_act(X, W, workspace=ws, x_fmt=fmt)
     q = mx.quantize(X, fmt)
     torch.cuda.synchronize()
-    header = ((64 + 4 * ((M + 127) // 128)) + 255) // 256 * 256
+    header = ((64 + 4 * ((M + 127) // 128) + 4 * 148) + 255) // 256 * 256
     nc, ns = mx.mx_codes_bytes(fmt, M, K), mx.mx_scales_bytes(fmt, M, K)
     codes = ws[header:header + nc]
     so = header + (nc + 255) // 256 * 256

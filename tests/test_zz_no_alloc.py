@@ -30,6 +30,12 @@ def library():
     mx.lib()
 
 
+def _scratch_sized() -> torch.Tensor:
+    """A workspace of exactly the scratch array's size: the workspace entry then
+    makes the same choices (the K split needs room) as the no-allocation one."""
+    return torch.empty(mx.MX_NOALLOC_SCRATCH_BYTES, dtype=torch.uint8, device="cuda")
+
+
 def _noalloc(x: torch.Tensor, W: mx.MxTensor, **kw) -> torch.Tensor:
     M, K = x.shape
     out = torch.empty((M, W.rows), dtype=torch.bfloat16, device=x.device)
@@ -50,7 +56,7 @@ def test_noalloc_matches_workspace_entry_two_calls(fmt):
         X_bits = synth.student_t(seed + fmt, M, K)
         X = synth.bits_to_tensor(X_bits).cuda()
         got = _noalloc(X, W)
-        want = mx.gemm_fused_act(X, W)
+        want = mx.gemm_fused_act(X, W, workspace=_scratch_sized())
         torch.cuda.synchronize()
         mx.check_device_error()
         assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"call {call}"
@@ -71,8 +77,8 @@ def test_noalloc_epilogue_and_amax_chain():
     a1, a2 = torch.empty(1, device="cuda"), torch.empty(1, device="cuda")
     H1 = _noalloc(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=a1)
     Y1 = _noalloc(H1, W2, x_amax=a1)
-    H2 = mx.gemm_fused_act(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=a2)
-    Y2 = mx.gemm_fused_act(H2, W2, x_amax=a2)
+    H2 = mx.gemm_fused_act(X, W1, epilogue=mx.MX_EPI_GELU, amax_out=a2, workspace=_scratch_sized())
+    Y2 = mx.gemm_fused_act(H2, W2, x_amax=a2, workspace=_scratch_sized())
     torch.cuda.synchronize()
     mx.check_device_error()
     assert torch.equal(H1.view(torch.int16), H2.view(torch.int16))
@@ -111,7 +117,7 @@ def test_noalloc_largest_shape_runs_and_the_next_is_rejected(fmt):
     # the largest accepted shape fills the array to its end: bit for bit the workspace entry
     X = synth.bits_to_tensor(synth.sweep_tensor(913 + fmt, M, K)).cuda()
     got = _noalloc(X, W)
-    want = mx.gemm_fused_act(X, W)
+    want = mx.gemm_fused_act(X, W, workspace=_scratch_sized())
     torch.cuda.synchronize()
     mx.check_device_error()
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
@@ -131,7 +137,7 @@ for _ in range(2):
                                      torch.cuda.current_stream().cuda_stream)
     mx.check(s, "mx_gemm_fused_act_noalloc")
     outs.append(out)
-want = mx.gemm_fused_act(X, W)
+want = mx.gemm_fused_act(X, W, workspace=torch.empty(mx.MX_NOALLOC_SCRATCH_BYTES, dtype=torch.uint8, device="cuda"))
 torch.cuda.synchronize()
 mx.check_device_error()
 for o in outs:
