@@ -767,6 +767,8 @@ PROFILE_CASES = {
     "fused_dit_mxfp8": ("fused", 0, 4096, 3072, 3072),
     "gemm_dit_mxfp4_mbs": ("gemm", 5, 4096, 3072, 3072),
     "quant_mbs_dynamic_1024x4096": ("quant_mbs_dynamic", 5, 1024, 0, 4096),
+    "quant_nvfp4_prepass_32768x4096": ("quant_prepass", 3, 32768, 0, 4096),
+    "fused_down_nvfp4_16x8192x28672": ("fused", 3, 16, 8192, 28672),
 }
 
 
@@ -790,6 +792,10 @@ def run_profile_case(name: str, reps: int = 4):
         gs = mx.quantize_rht(x, fmt, out=q).gscale.clone() if fmt == 3 else None
         for _ in range(reps):
             mx.quantize_rht(x, fmt, out=q, gscale=gs)
+    elif kind == "quant_prepass":
+        q = mx.empty(fmt, M, K)
+        for _ in range(reps):
+            mx.quantize(x, fmt, out=q)      # NVFP4 without g: the amax pre-pass, then the quantize
     elif kind == "quant_mbs_dynamic":
         q = mx.empty(fmt, M, K)
         for _ in range(reps):
@@ -934,6 +940,18 @@ def add_clock_normalised(extras: dict, clocks: dict) -> None:
 FMT_NAMES = {0: "mxfp8_e4m3", 1: "mxfp8_e5m2", 2: "mxfp4", 3: "nvfp4", 4: "mxfp6_e3m2", 5: "mxfp4_mbs"}
 
 
+def fused_launches(fmt: int, M: int) -> int:
+    """Kernels one mx_gemm_fused_act call launches in its default mode (no g
+    or amax of X given): with more than one 128-row band of X, the kernel that
+    clears the workspace counters, the quantize kernel and the GEMM kernel
+    launched to overlap it (NVFP4: the amax pre-pass after the clear); with
+    one band, the quantize kernel and the GEMM after it (NVFP4: first a
+    one-block kernel that clears the amax slot, then the pre-pass)."""
+    if fmt != 3:
+        return 3 if M > 128 else 2
+    return 4
+
+
 def result_line(args, wl: dict, r: dict, world: int) -> dict:
     """The JSON line of the GPU arm from run_gpu's measurements r (device
     times in ms, already the maximum over ranks)."""
@@ -958,7 +976,8 @@ def result_line(args, wl: dict, r: dict, world: int) -> dict:
         "vs_baseline": None, "dtype": FMT_NAMES[fmt], "data": "synthetic",
         "config": {"workload": wl["name"], "format": FMT_NAMES[fmt], "M": M, "N": N, "K": K,
                    "step": "mx_gemm_fused_act(X bf16, Wq pre-quantized): X quantized to "
-                           f"{FMT_NAMES[fmt]} inside the GEMM kernel, then the block-scaled GEMM to bf16 C",
+                           f"{FMT_NAMES[fmt]} band by band into the workspace while the block-scaled GEMM, "
+                           "launched to overlap the quantize, starts on the bands already written; bf16 C",
                    "timed_as": "one replay of a CUDA graph holding the K steps' launches",
                    "ms_per_step_eager": round(r["eager_ms"] / args.steps, 4),
                    "l2": f"inputs larger than L2: {r['n_sets']} rotating input sets x {r['per_set'] / 2**20:.1f} MB",
@@ -972,9 +991,8 @@ def result_line(args, wl: dict, r: dict, world: int) -> dict:
                      "kernel_us_isolated": round(f_iso * 1e3, 2),
                      "timing": "CUDA events on the launching stream around one graph replay of the K fused calls "
                                "(the timed steps' inputs, back to back), right after the timed replay; each call is "
-                               "the GEMM kernel with the quantize inside and a one-block kernel clearing the "
-                               "workspace counters; kernel_us_isolated: events around each call of a further eager "
-                               "pass"},
+                               "the kernels of the fused call (see gpu_launches), the GEMM overlapping the "
+                               "quantize; kernel_us_isolated: events around each call of a further eager pass"},
         "two_kernel_split": {
             "step_us": round(r["two_ms"] * 1e3, 2),
             "quantize_kernel": f"quantize_kernel<{FMT_NAMES[fmt]}>", "quantize_us": round(r["q_ms"] * 1e3, 2),
@@ -986,9 +1004,7 @@ def result_line(args, wl: dict, r: dict, world: int) -> dict:
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"], "path": "pinned host X -> H2D -> mx_gemm_fused_act -> D2H C, upload / compute / download on three "
                         "streams with double buffers (consecutive steps overlap)"},
-        # per step: the GEMM kernel (with the quantize inside) and the kernel that
-        # clears the workspace counters; NVFP4 without a given g adds the amax pre-pass
-        "gpu_launches": (3 if fmt == 3 else 2) * args.steps,
+        "gpu_launches": fused_launches(fmt, M) * args.steps,
         "clocks": r["clocks"],
     }
 

@@ -638,6 +638,22 @@ mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st) {
     return MX_OK;
 }
 
+// amax(|X|) into *slot by the persistent amax kernel, launched to overlap the
+// previous kernel in the stream (the counter reset that zeroed the slot).
+mx_status launch_amax_overlapped(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float *slot, cudaStream_t st) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)amax_grid(M, K, num_sms()), 1, 1);
+    cfg.blockDim = dim3(kQThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    if (cudaLaunchKernelEx(&cfg, amax_kernel, X, M, K, ldx, reinterpret_cast<unsigned int *>(slot)) != cudaSuccess)
+        return last_launch();
+    return MX_OK;
+}
+
 // Quantize X into the workspace as the A operand of the GEMM.  Returns the
 // device pointer of X's g (NVFP4) through *ga.
 mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int64_t ldx, uint8_t *ws,
@@ -667,9 +683,12 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
         } else {
             const float *amax = x_amax;
             if (amax == nullptr) {
-                if (cudaMemsetAsync(amax_slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
-                amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(
-                    X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
+                // the amax pre-pass into the header's slot, zeroed by a one-block
+                // kernel just before it (both overlap their predecessors' tails)
+                s = launch_fused_reset(reinterpret_cast<uint32_t *>(amax_slot), 1, st);
+                if (s != MX_OK) return s;
+                s = launch_amax_overlapped(X, M, K, ldx, amax_slot, st);
+                if (s != MX_OK) return s;
                 amax = amax_slot;
             }
             s = launch_quantize<3>(X, M, K, ldx, xa, amax, g_slot, st, /*g_from_amax=*/1, band_ready, clear, n_clear);
@@ -1034,23 +1053,29 @@ mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, i
     // pipelined GEMM may run before that store is visible), always its source
     float *amax_slot = reinterpret_cast<float *>(ws + 4);
     const float *x_amax_src = x_amax;
+    bool prepass = false;
     if (fmt == MX_NVFP4) {
         if (x_gscale != nullptr) {
             ga = x_gscale;
         } else {
             fx.ga_from_amax = 1;
             if (x_amax == nullptr) {
-                if (cudaMemsetAsync(amax_slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
-                amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(
-                    X, M, K, ldx, reinterpret_cast<unsigned int *>(amax_slot));
+                prepass = true;
                 x_amax_src = amax_slot;
             }
             ga = x_amax_src;
         }
     }
-    // words 2 .. 15, the band counters and the slot counters
-    s = launch_fused_reset(reinterpret_cast<uint32_t *>(ws + 8), (int)((fused_ws_header(M) - 8) / 4), st);
+    // words 2 .. 15, the band counters and the slot counters (and word 1, the
+    // amax slot, before the pre-pass), then the pre-pass: each kernel of the
+    // chain overlaps the tail of the one before it
+    const int w0 = prepass ? 1 : 2;
+    s = launch_fused_reset(reinterpret_cast<uint32_t *>(ws + 4 * w0), (int)(fused_ws_header(M) / 4 - w0), st);
     if (s != MX_OK) return s;
+    if (prepass) {
+        s = launch_amax_overlapped(X, M, K, ldx, amax_slot, st);
+        if (s != MX_OK) return s;
+    }
     if (fx.mode == 2) {
         mx_tensor xq;
         const float *unused = nullptr;

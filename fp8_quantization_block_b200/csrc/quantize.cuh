@@ -898,6 +898,12 @@ __global__ void __launch_bounds__(256) quantize_mbs_dynamic_kernel(const uint16_
 // the quantize kernel that follows reads those rows first.
 __global__ void __launch_bounds__(kQThreads) amax_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
                                                          int64_t ld, unsigned int *__restrict__ amax_bits) {
+    // src and the zeroed slot may come from the previous kernel in the stream
+    // (launched with programmatic serialization, this kernel starts early);
+    // the quantize kernel that follows may launch now and waits for this
+    // grid's completion itself
+    griddep_wait();
+    griddep_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t tiles_x = (K + kQTileCols - 1) / kQTileCols;
     const int64_t n_tiles = tiles_x * ((M + kQTileRows - 1) / kQTileRows);
