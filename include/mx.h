@@ -281,10 +281,10 @@ size_t mx_fused_split_workspace_bytes(int fmt, int64_t M, int64_t K);
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, once per device, with that device current); make
  *   that first call before any stream capture.
- *   The GEMM splits its last wave along K (see workspace above) only where
- *   the array also holds mx_fused_split_workspace_bytes(fmt, M, K), i.e. for
- *   small M; a workspace call with a workspace of MX_NOALLOC_SCRATCH_BYTES
- *   gives the same results bit for bit.
+ *   The array is smaller than any workspace with room for the K split (the
+ *   partial-sum slots alone take 148 x 32 KB), so this call never splits its
+ *   tiles along K: a workspace call with a workspace of
+ *   MX_NOALLOC_SCRATCH_BYTES bytes gives the same results bit for bit.
  *   Every call uses the same array and leaves its contents behind (whatever
  *   must start at zero is cleared by the call).  Calls that overlap on the GPU
  *   -- on different streams, or from several host threads -- race on it and
