@@ -155,8 +155,7 @@ mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld,
                           uint32_t *band_ready = nullptr, uint32_t *clear = nullptr, int n_clear = 0) {
     if (M == 0 || K == 0) return MX_OK;
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows), 1);
     cfg.blockDim = dim3(kQThreads, 1, 1);
     cfg.stream = st;
@@ -173,8 +172,7 @@ template <int FMT>
 void launch_quantize_rht(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst,
                          const float *g_in, float *g_out, cudaStream_t st, int g_from_amax = 0) {
     const int64_t sf_tiles_k = cdiv(K / fmt_block(FMT), 4);
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cdiv(K, kQTileCols), (unsigned)cdiv(M, kQTileRows), 1);
     cfg.blockDim = dim3(kQThreads, 1, 1);
     cfg.stream = st;
@@ -186,8 +184,7 @@ void launch_quantize_rht(const uint16_t *src, int64_t M, int64_t K, int64_t ld, 
 }
 
 void launch_quantize_mbs(const uint16_t *src, int64_t M, int64_t K, int64_t ld, const mx_tensor *dst, cudaStream_t st) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(K / kQTileCols), (unsigned)cdiv(M, kQTileRows), 1);
     cfg.blockDim = dim3(kQThreads, 1, 1);
     cfg.stream = st;
@@ -302,8 +299,7 @@ int coresident_pairs(const void *kernel, size_t smem) {
     const auto key = std::make_pair(kernel, dev);
     const auto it = cache.find(key);
     if (it != cache.end()) return it->second;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
@@ -423,8 +419,7 @@ mx_status launch_gemm_t(const mx_tensor *A, const mx_tensor *B, const void *a_co
     const int max_ctas = cap > 0 && cap < num_sms() ? cap : num_sms();
     plan_split(p, tiles, max_ctas, 1, room);
     const unsigned grid = (unsigned)p.ks.workers;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kAlloc;
@@ -501,8 +496,7 @@ mx_status launch_gemm_pair_t(const mx_tensor *A, const mx_tensor *B, const void 
     plan_split(p, tiles, resident > 0 && resident < max_pairs ? resident : max_pairs, 2, resident > 0 ? room : nullptr);
     if (!p.ks.on) p.ks = ks_plan(tiles, max_pairs, p.num_kt, 1, false);
     const unsigned pairs = (unsigned)p.ks.workers;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs, 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kAlloc;
@@ -582,8 +576,7 @@ mx_status launch_gemm_mbs(const mx_tensor *A, const mx_tensor *B, uint16_t *C, i
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (int64_t)p.m_blocks * cdiv(N, kMbsBN);
     if (tiles > INT32_MAX) return MX_ERR_UNSUPPORTED_SHAPE;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)tiles, 1, 1);
     cfg.blockDim = dim3(kMbsThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kAlloc;
@@ -626,8 +619,7 @@ __global__ void fused_reset_kernel(uint32_t *__restrict__ words, int n) {
 }
 
 mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, 1);
     cfg.blockDim = dim3(128, 1, 1);
     cfg.stream = st;
@@ -641,8 +633,7 @@ mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st) {
 // amax(|X|) into *slot by the persistent amax kernel, launched to overlap the
 // previous kernel in the stream (the counter reset that zeroed the slot).
 mx_status launch_amax_overlapped(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float *slot, cudaStream_t st) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)amax_grid(M, K, num_sms()), 1, 1);
     cfg.blockDim = dim3(kQThreads, 1, 1);
     cfg.stream = st;
