@@ -115,10 +115,13 @@ def test_result_line_keeps_the_contract(bench):
         assert line["higher_is_better"] is True and line["vs_baseline"] is None
         assert line["config"]["workload"] == wl["name"]
         roof = line["roofline"]
-        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6, 256, false> (fused quantize)"
+        assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_pair_kernel<0, 6, 256, false>"
+        assert roof["kernel_us"] == pytest.approx(42.0)                  # the GEMM's own launches
         assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"], rel=1e-3)
         assert roof["peak"] == pytest.approx(bench.tensor_peak(0, bench.measured_peaks()[0], False), rel=1e-3)
-        assert roof["clock_normalised_kernel_us"] == pytest.approx(40.5 * 1762 / 1965, abs=0.01)
+        assert roof["clock_normalised_kernel_us"] == pytest.approx(42.0 * 1762 / 1965, abs=0.01)
+        assert roof["fused_call"]["us"] == pytest.approx(40.5)
+        assert roof["fused_call"]["frac"] == pytest.approx(flops / 40.5e-6 / 1e12 / roof["peak"], rel=1e-3)
         assert "traffic" in roof
         assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
         assert line["e2e"]["h2d_bytes_per_step"] == r["h2d"]
@@ -131,7 +134,7 @@ def test_result_line_keeps_the_contract(bench):
     args.workload = "skinny_nvfp4"
     line = bench.result_line(args, bench.WORKLOADS["skinny_nvfp4"], dict(r, f_ms=[0.025] * 50), 1)
     assert line["roofline"]["bound"] == "hbm" and line["roofline"]["unit"] == "GB/s"
-    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32, false> (fused quantize)"
+    assert line["roofline"]["kernel"] == "gemm_kernel<3, 256, 5, 32, false>"
     # one band of X: the amax slot's clear, the amax pre-pass, the quantize kernel, the GEMM
     assert line["gpu_launches"] == 4 * 50
     json_line = __import__("json").dumps(line)
