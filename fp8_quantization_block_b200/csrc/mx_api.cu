@@ -162,8 +162,13 @@ mx_status launch_quantize(const uint16_t *src, int64_t M, int64_t K, int64_t ld,
     cudaLaunchAttribute attr[1];
     cfg.attrs = attr;
     cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
-    if (cudaLaunchKernelEx(&cfg, quantize_kernel<FMT, RULE>, src, M, K, ld, static_cast<uint8_t *>(dst->codes),
-                           dst->scales, sf_tiles_k, g_in, g_out, g_from_amax, band_ready, clear, n_clear) != cudaSuccess)
+    // g_from_amax == 2: a tiny NVFP4 tensor whose amax every CTA takes itself
+    auto kernel = quantize_kernel<FMT, RULE>;
+    if constexpr (FMT == 3) {
+        if (g_from_amax == 2) kernel = quantize_kernel<FMT, RULE, true>;
+    }
+    if (cudaLaunchKernelEx(&cfg, kernel, src, M, K, ld, static_cast<uint8_t *>(dst->codes), dst->scales, sf_tiles_k,
+                           g_in, g_out, g_from_amax, band_ready, clear, n_clear) != cudaSuccess)
         return last_launch();
     return MX_OK;
 }
@@ -673,6 +678,14 @@ mx_status fused_quantize_x(int fmt, const uint16_t *X, int64_t M, int64_t K, int
             *ga = x_gscale;
         } else {
             const float *amax = x_amax;
+            if (amax == nullptr && M * K <= kTinyAmaxElements) {
+                // a tiny X: each quantize CTA takes amax(|X|) itself, no pre-pass
+                s = launch_quantize<3>(X, M, K, ldx, xa, nullptr, g_slot, st, /*g_from_amax=*/2, band_ready, clear,
+                                       n_clear);
+                *ga = g_slot;
+                if (s != MX_OK) return s;
+                return last_launch();
+            }
             if (amax == nullptr) {
                 // the amax pre-pass into the header's slot, zeroed by a one-block
                 // kernel just before it (both overlap their predecessors' tails)
@@ -761,7 +774,10 @@ mx_status mx_quantize(int fmt, const void *src_bf16, int64_t M, int64_t K, int64
     case MX_MXFP6_E3M2: s = launch_quantize<4>(src, M, K, ld_src, dst, nullptr, nullptr, st); break;
     case MX_MXFP4_MBS: launch_quantize_mbs(src, M, K, ld_src, dst, st); break;
     default: {
-        if (gscale_in == nullptr) {
+        if (gscale_in == nullptr && M * K <= kTinyAmaxElements) {
+            // a tiny tensor: each CTA takes amax(|src|) itself, no pre-pass
+            s = launch_quantize<3>(src, M, K, ld_src, dst, nullptr, dst->gscale, st, /*g_from_amax=*/2);
+        } else if (gscale_in == nullptr) {
             s = nvfp4_gscale_prepass(src, M, K, ld_src, dst->gscale, st);
             if (s != MX_OK) return s;
             s = launch_quantize<3>(src, M, K, ld_src, dst, dst->gscale, nullptr, st);

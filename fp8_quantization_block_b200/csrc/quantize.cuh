@@ -542,10 +542,50 @@ MX_DEVICE_INLINE void tile_quantize(const TileRegs<NT, ROWS> &r, int64_t M, int6
     }
 }
 
+// amax(|x|) of a whole bf16 tensor of at most kTinyAmaxElements elements,
+// computed by every thread of one CTA (which all receive it): each thread
+// issues the loads of its four 16-element segments (row-aligned, as the
+// quantize tiles and amax_kernel cut them) at once, and the segment maxima
+// reduce exactly as in amax_kernel, so the value is the one its pre-pass
+// would store.  For an NVFP4 quantize of a tensor this small, every CTA
+// computing the maximum itself costs one read of at most 32 KB from L2, less
+// than the two kernels of the pre-pass (the slot reset and amax_kernel).
+constexpr int64_t kTinyAmaxElements = 16 * 4 * kQThreads;   // 16384
+MX_DEVICE_INLINE float tiny_tensor_amax(const uint16_t *__restrict__ src, int64_t M, int64_t K, int64_t ld) {
+    __shared__ uint32_t red[kQThreads / 32];
+    const int64_t segs_row = K / 16, n = M * segs_row;   // K % 16 == 0
+    uint4 v[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t sg = threadIdx.x + (int64_t)i * kQThreads;
+        if (sg < n) {
+            const uint16_t *p = src + (sg / segs_row) * ld + (sg % segs_row) * 16;
+            v[i][0] = ldg_stream(p);
+            v[i][1] = ldg_stream(p + 8);
+        } else {
+            v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = max(m, absmax16(v[i][0], v[i][1]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kQThreads / 32; ++w) m = max(m, red[w]);
+    return __uint_as_float(m << 16);   // bf16 magnitude -> fp32 (0 for an all-zero tensor)
+}
+
 // src bf16 [M x K] (row pitch ld).  codes / scales as in mx.h.  sf_tiles_k =
 // ceil((K / block) / 4) 512-byte tiles per 128-row band.  NVFP4: *gscale_in
 // is g, or amax(|src|) when g_from_amax (then g = RU(amax / 2688), 1 for 0);
-// if gscale_out != nullptr, CTA 0 also stores g there.  band_ready (nullable):
+// SELF_AMAX (tensors of at most kTinyAmaxElements elements): every CTA
+// computes amax(|src|) itself, gscale_in unused (a separate instantiation, so
+// that the common kernel's code is unchanged).  If gscale_out != nullptr, CTA
+// 0 also stores g there.  band_ready (nullable):
 // each CTA adds one to its 128-row band's counter once its codes and scales
 // are written (release, gpu scope).  clear (nullable): n_clear words that CTA
 // 0 zeroes once the previous kernel in the stream has completed (the partial-
@@ -559,7 +599,7 @@ constexpr int quantize_min_blocks() {
     return FMT == FMT_NVFP4 ? 4 : (FMT == FMT_MXFP6 ? 5 : 1);
 }
 
-template <int FMT, int RULE = RULE_OCP>
+template <int FMT, int RULE = RULE_OCP, bool SELF_AMAX = false>
 __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantize_kernel(const uint16_t *__restrict__ src, int64_t M, int64_t K,
                                                              int64_t ld, uint8_t *__restrict__ codes,
                                                              uint8_t *__restrict__ scales, int64_t sf_tiles_k,
@@ -587,7 +627,13 @@ __global__ void __launch_bounds__(kQThreads, quantize_min_blocks<FMT>()) quantiz
     if (clear != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
         for (int i = threadIdx.x; i < n_clear; i += blockDim.x) clear[i] = 0u;
     if (FMT == FMT_NVFP4) {
-        const float g = nv_g_from(gscale_in, g_from_amax);
+        float g;
+        if (SELF_AMAX) {
+            const float amax = tiny_tensor_amax(src, M, K, ld);
+            g = nv_g_from(&amax, 1);
+        } else {
+            g = nv_g_from(gscale_in, g_from_amax);
+        }
         if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
         ns = nv_scale_setup(g);
         if (threadIdx.x < 128) nv_tables_fill(&nvt, threadIdx.x);

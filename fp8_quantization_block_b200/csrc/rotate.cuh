@@ -125,29 +125,18 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_rht_kernel(const uint16
 
     float g = 1.0f, rg_lo = 1.0f, rg_hi = 1.0f, inv6g = 1.0f, sc = 1.0f;
     __shared__ NvTables nvt;
-    griddep_wait();
-    if (FMT == FMT_NVFP4) {
-        g = *gscale_in;
-        if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;
-        if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
-        // as in quantize_kernel: a tiny g is handled as (y 2^64) / (g 2^64)
-        if (g < 0x1p-100f) {
-            sc = 0x1p64f;
-            g *= sc;
-        }
-        rg_lo = __frcp_rd(g);
-        rg_hi = __frcp_ru(g);
-        inv6g = 1.0f / (6.0f * g);
-        if (threadIdx.x < 128) {
-            const uint32_t c = threadIdx.x;
-            const float v = (c == 0u || c == 127u) ? 0.0f : e4m3_pos_value(c);
-            nvt.val[c] = v;
-            nvt.inv_lo[c] = v > 0.0f ? __frcp_rd(v) : 0.0f;
-            nvt.inv_hi[c] = v > 0.0f ? __frcp_ru(v) : 0.0f;
-        }
-        __syncthreads();
+    // the NVFP4 tables are constants: filled while the previous kernel in the
+    // stream finishes
+    if (FMT == FMT_NVFP4 && threadIdx.x < 128) {
+        const uint32_t c = threadIdx.x;
+        const float v = (c == 0u || c == 127u) ? 0.0f : e4m3_pos_value(c);
+        nvt.val[c] = v;
+        nvt.inv_lo[c] = v > 0.0f ? __frcp_rd(v) : 0.0f;
+        nvt.inv_hi[c] = v > 0.0f ? __frcp_ru(v) : 0.0f;
     }
+    griddep_wait();
 
+    // the tile's loads first, so that they are in flight while g is read
     uint4 v[kPasses][2];
 #pragma unroll
     for (int i = 0; i < kPasses; ++i) {
@@ -160,6 +149,20 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_rht_kernel(const uint16
         } else {
             v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
         }
+    }
+    if (FMT == FMT_NVFP4) {
+        g = *gscale_in;
+        if (g_from_amax) g = g > 0.0f ? __fdiv_ru(g, 2688.0f) : 1.0f;
+        if (gscale_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gscale_out = g;
+        // as in quantize_kernel: a tiny g is handled as (y 2^64) / (g 2^64)
+        if (g < 0x1p-100f) {
+            sc = 0x1p64f;
+            g *= sc;
+        }
+        rg_lo = __frcp_rd(g);
+        rg_hi = __frcp_ru(g);
+        inv6g = 1.0f / (6.0f * g);
+        __syncthreads();  // the tables
     }
 
 #pragma unroll

@@ -115,7 +115,8 @@ int mx_block_size(int fmt);
  *     E4M3 / E5M2 / E2M1 / E3M2).
  *   NVFP4: g = the FP32 value *gscale_in if gscale_in != NULL, else
  *     amax(|src|) / 2688 rounded up to FP32 (1.0 for an all-zero tensor),
- *     computed on the device (an extra read of src).  g is written to
+ *     computed on the device (an extra read of src: a pre-pass, or, for
+ *     M*K <= 16384, inside every CTA of the quantize kernel).  g is written to
  *     *dst->gscale.  Block scale s = smallest positive finite E4M3 with
  *     max|x| <= 6*g*s (0 for an all-zero block); element = RNE of the exact
  *     quotient x / (g*s) onto E2M1, saturating at 6.
@@ -222,7 +223,8 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  * W_dq^T as in mx_gemm.  X's quantized form is not an output of this call.
  * Launches: a one-thread-block kernel that clears the workspace's counters,
  * the quantize kernel and the GEMM kernel (NVFP4 without x_gscale or x_amax:
- * also the amax pre-pass).
+ * also the amax pre-pass, except for M*K <= 16384, where the quantize kernel
+ * computes amax(|X|) itself).
  *   workspace: device buffer of at least mx_fused_workspace_bytes(fmt, M, K)
  *              bytes, 256-byte aligned; its contents are scratch, and calls
  *              that overlap on the GPU must not share one.  With at least
@@ -251,7 +253,8 @@ typedef enum { MX_EPI_NONE = 0, MX_EPI_GELU = 1 } mx_epilogue;
  *   NVFP4 only, how g of X is found (first non-NULL wins):
  *     x_gscale : device float holding g itself;
  *     x_amax   : device float holding amax(|X|); g = RU_fp32(amax / 2688);
- *     neither  : amax(|X|) is computed by a pre-pass over X.
+ *     neither  : amax(|X|) is computed on the device: by a pre-pass over X,
+ *                or, for M*K <= 16384, by every CTA of the quantize kernel.
  * K % 128 == 0, ldx % 8 == 0. */
 mx_status mx_gemm_fused_act(int fmt, const void *X_bf16, int64_t M, int64_t K, int64_t ldx,
                             const mx_tensor *W, void *C_bf16, int64_t ldc, int epilogue,
