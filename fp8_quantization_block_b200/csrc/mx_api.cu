@@ -215,12 +215,26 @@ int num_sms() {
     return n;
 }
 
-// amax(|src|) -> slot (float bits), then g = RU(amax / 2688) in place.
+mx_status launch_fused_reset(uint32_t *words, int n, cudaStream_t st);
+mx_status launch_amax_overlapped(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float *slot, cudaStream_t st);
+
+// amax(|src|) -> slot (float bits), then g = RU(amax / 2688) in place: the
+// slot's reset, the amax pass and the conversion are kernels launched with
+// programmatic serialization, each launched while its predecessor runs and
+// waiting for it before it touches the slot.
 mx_status nvfp4_gscale_prepass(const uint16_t *src, int64_t M, int64_t K, int64_t ld, float *slot, cudaStream_t st) {
-    if (cudaMemsetAsync(slot, 0, sizeof(float), st) != cudaSuccess) return MX_ERR_CUDA;
-    amax_kernel<<<(unsigned)amax_grid(M, K, num_sms()), kQThreads, 0, st>>>(src, M, K, ld,
-                                                                           reinterpret_cast<unsigned int *>(slot));
-    gscale_from_amax_kernel<<<1, 1, 0, st>>>(slot);
+    mx_status s = launch_fused_reset(reinterpret_cast<uint32_t *>(slot), 1, st);
+    if (s != MX_OK) return s;
+    s = launch_amax_overlapped(src, M, K, ld, slot, st);
+    if (s != MX_OK) return s;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(1, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)pdl_attr(&attr[0]);
+    if (cudaLaunchKernelEx(&cfg, gscale_from_amax_kernel, slot) != cudaSuccess) return last_launch();
     return last_launch();
 }
 

@@ -992,7 +992,11 @@ inline int64_t amax_grid(int64_t M, int64_t K, int num_sms) {
 }
 
 // g = RU_fp32(amax / 2688), 1 for an all-zero tensor; in place (amax bits -> g).
+// Launched with programmatic serialization, it waits for the amax pass before
+// reading the slot, and lets the quantize kernel launch at once.
 __global__ void gscale_from_amax_kernel(float *__restrict__ slot) {
+    griddep_wait();
+    griddep_launch_dependents();
     const float amax = *slot;
     *slot = amax > 0.0f ? __fdiv_ru(amax, 2688.0f) : 1.0f;
 }
