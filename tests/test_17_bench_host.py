@@ -141,6 +141,16 @@ def test_result_line_keeps_the_contract(bench):
     assert "\n" not in json_line
 
 
+def test_fused_launch_counts(bench):
+    # MX formats: counter reset + quantize + GEMM with several bands, quantize + GEMM with one
+    assert bench.fused_launches(0, 4096, 3072) == 3 and bench.fused_launches(2, 128, 8192) == 2
+    # NVFP4 without g: the amax pre-pass (slot clear + amax) before the quantize ...
+    assert bench.fused_launches(3, 16, 8192) == 4 and bench.fused_launches(3, 4608, 3072) == 4
+    # ... except for an X of at most 16384 elements, whose amax the quantize kernel takes itself
+    assert bench.fused_launches(3, 1, 8192) == 2 and bench.fused_launches(3, 1, 16384) == 2
+    assert bench.fused_launches(3, 2, 16384) == 4
+
+
 def test_extras_get_clock_normalised_fractions(bench):
     ex = {"mlp_nvfp4_gemm1": {"us": 81.5, "frac_tensor": 0.647}, "quantize_sweep": {"x": {"frac_hbm": 0.8}}}
     bench.add_clock_normalised(ex, {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0})
